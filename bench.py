@@ -1,0 +1,417 @@
+"""Throughput of the compressed-expert routed MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one forward of the layer (route/bucket, gate/up + SwiGLU, down +
+weighted combine, final cast) over one batch of synthetic tokens, with the
+weights and the step's inputs already resident in HBM.  The default workload
+is the single-token MXFP4 decode of the MiMo-shaped layer (hidden 4096,
+inter 2048, 256 experts, top-8).  Every rank runs its own replica on its own
+tokens (the path partitions by batch; no collective on the data path), so
+``value`` is the total over ranks and ``scaling`` is "weak".
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the oracle (the f64
+CPU restatement) on the host cores instead, on a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# workload -> (config name, overrides)
+WORKLOADS = {
+    "decode_mxfp4": ("decode_mxfp4", {}),
+    "decode_vq_t1": ("decode_vq", dict(T=1)),
+    "decode_vq_t4": ("decode_vq", dict(T=4)),
+    "decode_vq_t8": ("decode_vq", dict(T=8)),
+    "decode_vq_t1_r0": ("decode_vq", dict(T=1, fmt="vq13")),
+    "decode_vq_t8_r0": ("decode_vq", dict(T=8, fmt="vq13")),
+    "prefill_mxfp4_zipf": ("prefill_mxfp4_zipf", {}),
+    "prefill_vq_overflow": ("prefill_vq_overflow", {}),
+}
+
+
+def workload_cfg(name):
+    base, over = WORKLOADS[name]
+    return synth.get_cfg(base, **over)
+
+
+def is_decode(cfg):
+    return cfg.T <= 8
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def proj_bytes(cfg, p):
+    """Compressed bytes of one expert's projection p."""
+    N, K = cfg.shape(p)
+    if cfg.fmt == "mxfp4":
+        return N * (K // 2 + K // 32)
+    b = N * synth.idx13_row_bytes(K)
+    if cfg.fmt == "vq13r8":
+        b += N * (K // 8)
+    if cfg.gains:
+        b += 2 * N
+    return b
+
+
+def book_bytes(cfg):
+    return 0 if cfg.fmt == "mxfp4" else 8192 * 16 + (256 * 16 if cfg.fmt == "vq13r8" else 0)
+
+
+def flops(cfg, n_routes):
+    return 2 * n_routes * 3 * cfg.H * cfg.I
+
+
+# ------------------------------------------------------------------ inputs
+
+def step_inputs(cfg, n_steps, seed=0):
+    """Per-step routings and activations.  Single-token decode rotates 32
+    disjoint expert sets so no expert's weights are reused within 32 steps
+    (3.4 GB of MXFP4 weights stream between reuses: larger than L2);
+    multi-token decode draws a fresh routing per step; prefill reuses one
+    batch (each step streams 2-3.4 GB of weights, larger than L2)."""
+    if cfg.T == 1:
+        ids, w = synth.gen_disjoint_routing_schedule(cfg, n_steps, seed=seed)
+        xs = np.stack([synth.gen_activations(cfg, seed=seed + 1 + i) for i in range(min(n_steps, 64))])
+        xs = xs[np.arange(n_steps) % len(xs)]
+        how = "inputs larger than L2: 32 disjoint expert sets rotate, a set recurs after 31 others"
+    elif is_decode(cfg):
+        ids = np.empty((n_steps, cfg.T, cfg.k), np.int32)
+        w = np.empty((n_steps, cfg.T, cfg.k), np.float32)
+        xs = []
+        for i in range(n_steps):
+            ids[i], w[i] = synth.gen_routing(cfg, seed=seed + 1 + i)
+            xs.append(synth.gen_activations(cfg, seed=seed + 1 + i))
+        xs = np.stack(xs)
+        how = "inputs larger than L2: a fresh routing per step (~30-60 experts, 150-470 MB of weights)"
+    else:
+        i0, w0 = synth.gen_routing(cfg, seed=seed)
+        x0 = synth.gen_activations(cfg, seed=seed)
+        ids = np.broadcast_to(i0, (n_steps,) + i0.shape)
+        w = np.broadcast_to(w0, (n_steps,) + w0.shape)
+        xs = np.broadcast_to(x0, (n_steps,) + x0.shape)
+        how = "inputs larger than L2: every step streams all routed experts' weights (GBs)"
+    return xs, ids, w, how
+
+
+# ------------------------------------------------------------------ clocks
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") \
+            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/moeq_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def run_reference(args, cfg):
+    import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    L = synth.gen_layer(cfg)
+    n_total = args.warmup + args.steps
+    xs, ids, w, how = step_inputs(cfg, n_total)
+    # size each step's sample so the whole run stays within ~150 s of CPU time
+    probe_t = time.perf_counter()
+    oracle.forward(L, xs[0][:1], ids[0][:1], w[0][:1])
+    per_token = time.perf_counter() - probe_t
+    budget = 150.0 / n_total
+    tok_per_step = int(max(1, min(cfg.T, budget // max(per_token, 1e-6))))
+    times = []
+    for i in range(n_total):
+        tok = np.arange(tok_per_step, dtype=np.int32) + (i * tok_per_step) % max(1, cfg.T - tok_per_step + 1)
+        tok = tok % cfg.T
+        t0 = time.perf_counter()
+        oracle.forward(L, xs[i], ids[i], w[i], tokens=tok)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = tok_per_step * args.steps / total
+    sample = f"{tok_per_step} of {cfg.T} tokens per step (all their routes), steps {args.steps}"
+    line = {
+        "impl": "reference", "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_obj(args, cfg, how),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_obj(args, cfg, how):
+    return {"workload": args.workload, "hidden": cfg.H, "inter": cfg.I, "experts": cfg.E, "top_k": cfg.k,
+            "tokens_per_step": cfg.T, "format": cfg.fmt, "act": cfg.act, "routing": cfg.routing,
+            "seed": 0, "l2": how, "parallelism": f"replicas x{args.gpus} (one per GPU, no collective)"}
+
+
+# ------------------------------------------------------------------ cpu baseline (our arm)
+
+def cpu_baseline(cfg, L, xs, ids, w, seconds=12.0):
+    import oracle
+    done_tok, t_used, i = 0, 0.0, 0
+    per_call = max(1, min(cfg.T, 2))
+    while t_used < seconds and i < 10000:
+        tok = (np.arange(per_call, dtype=np.int32) + i * per_call) % cfg.T
+        t0 = time.perf_counter()
+        oracle.forward(L, xs[i % len(xs)], ids[i % len(ids)], w[i % len(w)], tokens=tok)
+        t_used += time.perf_counter() - t0
+        done_tok += per_call
+        i += 1
+    return {"value": done_tok / t_used, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{done_tok} tokens ({i} calls of {per_call} token(s) with all their routes), "
+                      f"{t_used:.1f} s on the host"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="decode_mxfp4", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    cfg = workload_cfg(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import torch
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    from bit_quantized_moe_routed_b200 import moeq
+
+    L = synth.gen_layer(cfg)
+    lay = moeq.Layer(cfg.H, cfg.I, cfg.E, cfg.k, cfg.T, cfg.fmt, cfg.act, device=local)
+    lay.upload(L)
+    n_total = args.warmup + args.steps
+    xs_h, ids_h, w_h, how = step_inputs(cfg, n_total, seed=rank)
+    dev = torch.device("cuda", local)
+    to_x = (lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)) \
+        if cfg.act == "bf16" else (lambda a: torch.from_numpy(np.ascontiguousarray(a)))
+    uniq = 1 if not is_decode(cfg) else n_total
+    xs = to_x(xs_h[:uniq]).to(dev)
+    ids = torch.from_numpy(np.ascontiguousarray(ids_h[:uniq])).to(dev)
+    ws = torch.from_numpy(np.ascontiguousarray(w_h[:uniq])).to(dev)
+    outs = torch.empty((uniq, cfg.T, cfg.H), dtype=xs.dtype, device=dev)
+
+    def step(i, out=None):
+        j = i % uniq
+        lay.forward(xs[j], ids[j], ws[j], out=outs[j] if out is None else out)
+
+    # warm-up: W eager steps
+    l0 = lay.kernel_launches()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    launches_per_step = (lay.kernel_launches() - l0) // args.warmup
+
+    # capture the K timed steps as one CUDA graph
+    cap = torch.cuda.Stream(device=dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for i in range(args.warmup, n_total):
+            step(i)
+    g.replay()                      # untimed: graph upload
+    torch.cuda.synchronize()
+
+    # clock soak (~1 s of the same work), then the timed replay
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        g.replay()
+        torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(cap)
+    g.replay()
+    e1.record(cap)
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+
+    # per-phase kernel durations over the same K steps (a second graph with
+    # phase events between the kernels)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=cap):
+        for n, i in enumerate(range(args.warmup, n_total)):
+            j = i % uniq
+            lay.forward_profiled(xs[j], ids[j], ws[j], outs[j], ev[n])
+    g2.replay()
+    torch.cuda.synchronize()
+    g2.replay()
+    torch.cuda.synchronize()
+    phase_ms = [sum(ev[n][p].elapsed_time(ev[n][p + 1]) for n in range(args.steps)) / args.steps
+                for p in range(4)]
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    xh = torch.from_numpy(np.ascontiguousarray(xs_h[0])).pin_memory()
+    ih = torch.from_numpy(np.ascontiguousarray(ids_h[0])).pin_memory()
+    wh = torch.from_numpy(np.ascontiguousarray(w_h[0])).pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    h_bytes = xh.numel() * xh.element_size() + ih.numel() * 4 + wh.numel() * 4
+    d_bytes = oh.numel() * oh.element_size()
+    e2e_steps = min(args.steps, 200)
+    for _ in range(3):
+        lay.forward_host_ptr(xh.data_ptr(), ih.data_ptr(), wh.data_ptr(), cfg.T, oh.data_ptr())
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        lay.forward_host_ptr(xh.data_ptr(), ih.data_ptr(), wh.data_ptr(), cfg.T, oh.data_ptr())
+    e2e_s = time.perf_counter() - t0
+
+    # max over ranks
+    if world > 1:
+        tt = torch.tensor([ms, e2e_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, e2e_s = float(tt[0]), float(tt[1])
+
+    if rank == 0:
+        peaks = FALLBACK_PEAKS
+        peak_src = "fallback"
+        if os.path.exists(PEAKS_FILE):
+            peaks = json.load(open(PEAKS_FILE))
+            peak_src = "measured"
+        ms_step = ms / args.steps
+        value = world * cfg.T * args.steps / (ms / 1e3)
+        n_routes = int(((ids_h[args.warmup:] >= 0) & (ids_h[args.warmup:] < cfg.E)).sum()) / args.steps
+        if is_decode(cfg):
+            # dominant kernel: gate/up + SwiGLU; algorithmic bytes = distinct
+            # experts per step x compressed gate+up bytes per expert (+ books)
+            d_mean = float(np.mean([len(np.unique(ids_h[i])) for i in range(args.warmup, n_total)]))
+            bytes_gu = d_mean * (proj_bytes(cfg, 0) + proj_bytes(cfg, 1)) + book_bytes(cfg)
+            achieved = bytes_gu / (phase_ms[1] / 1e3) / 1e9
+            peak = float(peaks["hbm_gbs"])
+            roof = {"kernel": "gate/up + SwiGLU", "bound": "hbm", "achieved": achieved, "peak": peak,
+                    "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                    "peak_source": f"{peak_src} hbm_gbs",
+                    "per_launch_bytes": bytes_gu, "launch_ms": phase_ms[1]}
+            d_all = float(np.mean([len(np.unique(ids_h[i])) for i in range(args.warmup, n_total)]))
+            step_bytes = d_all * sum(proj_bytes(cfg, p) for p in range(3)) + book_bytes(cfg)
+            extra = {"step_weight_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                     "step_hbm_frac": step_bytes / (ms_step / 1e3) / 1e9 / peak}
+        else:
+            fl_gu = 2 * n_routes * 2 * cfg.H * cfg.I
+            achieved = fl_gu / (phase_ms[1] / 1e3) / 1e12
+            peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+            roof = {"kernel": "gate/up + SwiGLU", "bound": "tensor", "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                    "peak_source": f"{peak_src} bf16_tflops_sustained",
+                    "per_launch_flops": fl_gu, "launch_ms": phase_ms[1]}
+            extra = {"step_tflops": flops(cfg, n_routes) / (ms_step / 1e3) / 1e12,
+                     "step_tensor_frac": flops(cfg, n_routes) / (ms_step / 1e3) / 1e12 / peak}
+        line = {
+            "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.act == "bf16" else "f32",
+            "data": "synthetic", "config": config_obj(args, cfg, how),
+            "roofline": roof, "phase_ms": dict(zip(["route", "gateup", "down_combine", "cast"], phase_ms)),
+            "step": extra,
+            "e2e": {"value": world * cfg.T * e2e_steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h_bytes,
+                    "d2h_bytes_per_step": d_bytes, "steps": e2e_steps,
+                    "how": "moeq_forward_host per step: pinned H2D of x/ids/w, forward, D2H of out, sync"},
+            "gpu_launches": int(launches_per_step * args.steps),
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg, L, xs_h, ids_h, w_h)
+        print(json.dumps(line), flush=True)
+    del g, g2
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    lay.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

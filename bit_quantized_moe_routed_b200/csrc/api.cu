@@ -1,0 +1,334 @@
+// api.cu -- the extern "C" entry points of libmoeq (declared in moeq.h):
+// argument validation, device memory ownership and kernel dispatch.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "internal.cuh"
+
+using namespace moeq;
+
+// The opaque handle of moeq.h is the library's layer object.
+struct moeq_layer : moeq::Layer {};
+
+namespace {
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+    int prev = -1;
+    cudaError_t err = cudaSuccess;
+    explicit DeviceGuard(int dev) {
+        cudaGetDevice(&prev);
+        if (prev != dev) err = cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        cudaGetDevice(&cur);
+        if (prev >= 0 && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+moeq_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MOEQ_OK;
+    if (e == cudaErrorMemoryAllocation) return MOEQ_ERR_OUT_OF_MEMORY;
+    return MOEQ_ERR_CUDA;
+}
+
+// Host-side fault injection for tests: MOEQ_TEST_FAIL_ALLOC=n makes the
+// n-th device allocation of this process (1-based) report out-of-memory.
+long g_alloc_count = 0;
+cudaError_t dev_alloc(void **p, size_t bytes) {
+    static long fail_at = [] {
+        const char *s = std::getenv("MOEQ_TEST_FAIL_ALLOC");
+        return s ? std::atol(s) : 0L;
+    }();
+    ++g_alloc_count;
+    if (fail_at > 0 && g_alloc_count == fail_at) {
+        *p = nullptr;
+        return cudaErrorMemoryAllocation;
+    }
+    return cudaMalloc(p, bytes ? bytes : 16);
+}
+
+size_t row_bytes(int fmt, int plane, int K) {
+    // plane 0: codes / idx13; plane 1: scales / idx8
+    if (fmt == MOEQ_FMT_MXFP4) return plane == 0 ? (size_t)K / 2 : (size_t)K / 32;
+    return plane == 0 ? (size_t)K * 13 / 64 : (size_t)K / 8;
+}
+
+void free_layer(moeq_layer *L) {
+    if (!L) return;
+    for (int p = 0; p < 3; ++p) {
+        cudaFree(L->w.codes[p]);
+        cudaFree(L->w.scales[p]);
+        cudaFree(L->w.idx13[p]);
+        cudaFree(L->w.idx8[p]);
+        cudaFree(L->w.gain[p]);
+    }
+    cudaFree(L->w.book13);
+    cudaFree(L->w.book8);
+    cudaFree(L->b.offsets);
+    cudaFree(L->b.perm);
+    cudaFree(L->b.active);
+    cudaFree(L->h);
+    cudaFree(L->acc);
+    cudaFree(L->status);
+    cudaFree(L->x_stage);
+    cudaFree(L->out_stage);
+    cudaFree(L->ids_stage);
+    cudaFree(L->w_stage);
+    delete L;
+}
+
+bool desc_valid(const moeq_layer_desc *d) {
+    if (d->hidden <= 0 || d->inter <= 0 || d->n_experts <= 0 || d->top_k <= 0 || d->max_tokens <= 0)
+        return false;
+    if (d->n_experts > kMaxExperts || d->top_k > d->n_experts || d->top_k > kMaxTopK) return false;
+    if (d->act != MOEQ_ACT_F32 && d->act != MOEQ_ACT_BF16) return false;
+    if (d->fmt == MOEQ_FMT_MXFP4) {
+        if (d->hidden % 32 || d->inter % 32) return false;
+    } else if (d->fmt == MOEQ_FMT_VQ13 || d->fmt == MOEQ_FMT_VQ13_R8) {
+        if (d->hidden % 64 || d->inter % 64) return false;
+    } else {
+        return false;
+    }
+    // sizes that must fit the kernels' 32-bit index arithmetic
+    if ((long long)d->max_tokens * d->top_k > (1LL << 30)) return false;
+    return true;
+}
+
+moeq_status launch_forward(moeq_layer *L, const void *x, const int32_t *ids, const float *w, int32_t T,
+                           void *out, cudaStream_t s, const cudaEvent_t *ev = nullptr) {
+    if (ev) cudaEventRecord(ev[0], s);
+    cudaError_t e = launch_route_bucket(*L, ids, T * L->d.top_k, L->b.offsets, L->b.perm, L->b.active, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (ev) cudaEventRecord(ev[1], s);
+    e = launch_ffn_simt(*L, x, w, T, out, s, ev);
+    return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moeq_status_string(moeq_status s) {
+    switch (s) {
+        case MOEQ_OK: return "ok";
+        case MOEQ_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case MOEQ_ERR_UNSUPPORTED: return "unsupported";
+        case MOEQ_ERR_OUT_OF_MEMORY: return "out of device memory";
+        case MOEQ_ERR_CUDA: return "CUDA error";
+        case MOEQ_ERR_NOT_UPLOADED: return "weights not uploaded";
+        case MOEQ_ERR_ROUTE_OUT_OF_RANGE: return "route id outside [-1, n_experts)";
+        case MOEQ_ERR_TIMEOUT: return "a bounded device wait timed out";
+    }
+    return "unknown status";
+}
+
+moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
+    if (!out) return MOEQ_ERR_INVALID_ARGUMENT;
+    *out = nullptr;
+    if (!desc || !desc_valid(desc)) return MOEQ_ERR_INVALID_ARGUMENT;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || desc->device < 0 || desc->device >= ndev)
+        return MOEQ_ERR_CUDA;
+    DeviceGuard g(desc->device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    moeq_layer *L = new (std::nothrow) moeq_layer();
+    if (!L) return MOEQ_ERR_OUT_OF_MEMORY;
+    L->d = *desc;
+    cudaDeviceGetAttribute(&L->sm_count, cudaDevAttrMultiProcessorCount, desc->device);
+    const int E = desc->n_experts, H = desc->hidden, I = desc->inter, k = desc->top_k;
+    const size_t M = (size_t)desc->max_tokens;
+    const int fmt = desc->fmt;
+    cudaError_t e = cudaSuccess;
+#define ALLOC(ptr, bytes)                                              \
+    do {                                                               \
+        if (e == cudaSuccess) e = dev_alloc((void **)&(ptr), (bytes)); \
+    } while (0)
+    for (int p = 0; p < 3; ++p) {
+        const int N = (p == MOEQ_DOWN) ? H : I, K = (p == MOEQ_DOWN) ? I : H;
+        const size_t rows = (size_t)E * N;
+        if (fmt == MOEQ_FMT_MXFP4) {
+            ALLOC(L->w.codes[p], rows * row_bytes(fmt, 0, K));
+            ALLOC(L->w.scales[p], rows * row_bytes(fmt, 1, K));
+        } else {
+            ALLOC(L->w.idx13[p], rows * row_bytes(fmt, 0, K));
+            if (fmt == MOEQ_FMT_VQ13_R8) ALLOC(L->w.idx8[p], rows * row_bytes(fmt, 1, K));
+            ALLOC(L->w.gain[p], rows * sizeof(uint16_t));
+        }
+    }
+    if (fmt != MOEQ_FMT_MXFP4) {
+        ALLOC(L->w.book13, sizeof(uint16_t) * kBook13Rows * 8);
+        if (fmt == MOEQ_FMT_VQ13_R8) ALLOC(L->w.book8, sizeof(uint16_t) * kBook8Rows * 8);
+    }
+    ALLOC(L->b.offsets, sizeof(int32_t) * (E + 1));
+    ALLOC(L->b.active, sizeof(int32_t) * (E + 1));
+    ALLOC(L->b.perm, sizeof(int32_t) * M * k);
+    ALLOC(L->h, sizeof(float) * M * k * I);
+    ALLOC(L->acc, sizeof(float) * M * H);
+    ALLOC(L->status, sizeof(uint32_t));
+    ALLOC(L->x_stage, (size_t)L->elem_bytes() * M * H);
+    ALLOC(L->out_stage, (size_t)L->elem_bytes() * M * H);
+    ALLOC(L->ids_stage, sizeof(int32_t) * M * k);
+    ALLOC(L->w_stage, sizeof(float) * M * k);
+#undef ALLOC
+    if (e == cudaSuccess) e = cudaMemset(L->status, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) {
+        free_layer(L);
+        cudaGetLastError();  // clear a sticky allocation error
+        return from_cuda(e);
+    }
+    *out = L;
+    return MOEQ_OK;
+}
+
+void moeq_layer_destroy(moeq_layer_t layer) {
+    if (!layer) return;
+    DeviceGuard g(layer->d.device);
+    cudaDeviceSynchronize();
+    free_layer(layer);
+}
+
+moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *stream) {
+    if (!L || !w) return MOEQ_ERR_INVALID_ARGUMENT;
+    const int fmt = L->d.fmt, E = L->d.n_experts, H = L->d.hidden, I = L->d.inter;
+    const bool mx = fmt == MOEQ_FMT_MXFP4, r8 = fmt == MOEQ_FMT_VQ13_R8;
+    // presence / absence of every plane
+    int n_gain = 0;
+    for (int p = 0; p < 3; ++p) {
+        if (mx != (w->codes[p] != nullptr) || mx != (w->scales[p] != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
+        if (mx == (w->idx13[p] != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
+        if (r8 != (w->idx8[p] != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
+        if (w->gain[p]) {
+            if (mx) return MOEQ_ERR_INVALID_ARGUMENT;
+            ++n_gain;
+        }
+    }
+    if (n_gain != 0 && n_gain != 3) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (mx == (w->book13 != nullptr) || r8 != (w->book8 != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
+    // E8M0 255 is NaN and not a valid scale
+    if (mx) {
+        for (int p = 0; p < 3; ++p) {
+            const int N = (p == MOEQ_DOWN) ? H : I, K = (p == MOEQ_DOWN) ? I : H;
+            size_t n = (size_t)E * N * row_bytes(fmt, 1, K);
+            if (std::memchr(w->scales[p], 0xFF, n)) return MOEQ_ERR_INVALID_ARGUMENT;
+        }
+    }
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    for (int p = 0; p < 3 && e == cudaSuccess; ++p) {
+        const int N = (p == MOEQ_DOWN) ? H : I, K = (p == MOEQ_DOWN) ? I : H;
+        const size_t rows = (size_t)E * N;
+        if (mx) {
+            e = cudaMemcpyAsync(L->w.codes[p], w->codes[p], rows * row_bytes(fmt, 0, K), cudaMemcpyHostToDevice, s);
+            if (e == cudaSuccess)
+                e = cudaMemcpyAsync(L->w.scales[p], w->scales[p], rows * row_bytes(fmt, 1, K), cudaMemcpyHostToDevice, s);
+        } else {
+            e = cudaMemcpyAsync(L->w.idx13[p], w->idx13[p], rows * row_bytes(fmt, 0, K), cudaMemcpyHostToDevice, s);
+            if (e == cudaSuccess && r8)
+                e = cudaMemcpyAsync(L->w.idx8[p], w->idx8[p], rows * row_bytes(fmt, 1, K), cudaMemcpyHostToDevice, s);
+            if (e == cudaSuccess && n_gain)
+                e = cudaMemcpyAsync(L->w.gain[p], w->gain[p], rows * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
+        }
+    }
+    if (e == cudaSuccess && !mx)
+        e = cudaMemcpyAsync(L->w.book13, w->book13, sizeof(uint16_t) * kBook13Rows * 8, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && r8)
+        e = cudaMemcpyAsync(L->w.book8, w->book8, sizeof(uint16_t) * kBook8Rows * 8, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return from_cuda(e);
+    L->w.has_gain = n_gain == 3;
+    L->uploaded = true;
+    return MOEQ_OK;
+}
+
+moeq_status moeq_forward(moeq_layer_t L, const void *x, const int32_t *ids, const float *w, int32_t T,
+                         void *out, void *stream) {
+    if (!L) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (T < 0 || T > L->d.max_tokens) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (T == 0) return MOEQ_OK;
+    if (!x || !ids || !w || !out) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (!L->uploaded) return MOEQ_ERR_NOT_UPLOADED;
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    return launch_forward(L, x, ids, w, T, out, (cudaStream_t)stream);
+}
+
+moeq_status moeq_forward_profiled(moeq_layer_t L, const void *x, const int32_t *ids, const float *w,
+                                  int32_t T, void *out, void *stream, void *const *events) {
+    if (!L || !events) return MOEQ_ERR_INVALID_ARGUMENT;
+    for (int i = 0; i < 5; ++i)
+        if (!events[i]) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (T < 0 || T > L->d.max_tokens) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (T == 0) return MOEQ_OK;
+    if (!x || !ids || !w || !out) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (!L->uploaded) return MOEQ_ERR_NOT_UPLOADED;
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    cudaEvent_t ev[5];
+    for (int i = 0; i < 5; ++i) ev[i] = (cudaEvent_t)events[i];
+    return launch_forward(L, x, ids, w, T, out, (cudaStream_t)stream, ev);
+}
+
+moeq_status moeq_route(moeq_layer_t L, const int32_t *ids, int32_t T, int32_t *offsets_out,
+                       int32_t *perm_out, void *stream) {
+    if (!L || !ids || !offsets_out || !perm_out || T < 1 || T > L->d.max_tokens)
+        return MOEQ_ERR_INVALID_ARGUMENT;
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    return from_cuda(launch_route_bucket(*L, ids, T * L->d.top_k, offsets_out, perm_out, L->b.active,
+                                         (cudaStream_t)stream));
+}
+
+moeq_status moeq_forward_host(moeq_layer_t L, const void *x, const int32_t *ids, const float *w,
+                              int32_t T, void *out, void *stream) {
+    if (!L) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (T < 0 || T > L->d.max_tokens) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (T == 0) return MOEQ_OK;
+    if (!x || !ids || !w || !out) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (!L->uploaded) return MOEQ_ERR_NOT_UPLOADED;
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t xb = (size_t)L->elem_bytes() * T * L->d.hidden;
+    const size_t rb = (size_t)T * L->d.top_k;
+    cudaError_t e = cudaMemcpyAsync(L->x_stage, x, xb, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(L->ids_stage, ids, rb * sizeof(int32_t), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(L->w_stage, w, rb * sizeof(float), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    moeq_status st = launch_forward(L, L->x_stage, L->ids_stage, L->w_stage, T, L->out_stage, s);
+    if (st != MOEQ_OK) return st;
+    e = cudaMemcpyAsync(out, L->out_stage, xb, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return from_cuda(e);
+}
+
+moeq_status moeq_dequant(moeq_layer_t L, int32_t expert, int32_t proj, float *out, void *stream) {
+    if (!L || !out || expert < 0 || expert >= L->d.n_experts || proj < 0 || proj > 2)
+        return MOEQ_ERR_INVALID_ARGUMENT;
+    if (!L->uploaded) return MOEQ_ERR_NOT_UPLOADED;
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    return from_cuda(launch_dequant(*L, expert, proj, out, (cudaStream_t)stream));
+}
+
+int64_t moeq_kernel_launches(moeq_layer_t L) { return L ? (int64_t)L->launches : -1; }
+
+moeq_status moeq_layer_status(moeq_layer_t L, int32_t clear) {
+    if (!L) return MOEQ_ERR_INVALID_ARGUMENT;
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    uint32_t v = 0;
+    cudaError_t e = cudaMemcpy(&v, L->status, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && clear) e = cudaMemset(L->status, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) return from_cuda(e);
+    if (v & FLAG_ROUTE_RANGE) return MOEQ_ERR_ROUTE_OUT_OF_RANGE;
+    if (v & FLAG_TIMEOUT) return MOEQ_ERR_TIMEOUT;
+    return MOEQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,86 @@
+// dequant.cu -- decode one expert projection to f32 [N][K], bit-exact.
+//
+// MXFP4 ("MiMo-V2.6-Flash-RL GGUF for a single DGX Spark", "Architecture
+// notes"): w = e2m1(nibble) * 2^(scale-127); the product of an E2M1 value
+// and a power of two is exact in f32 unless it overflows (then +-inf under
+// round-to-nearest), so one f32 multiply gives the defined value.
+// VQ ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): w[8j+i] =
+// (B13[idx13_j][i] + R8[idx8_j][i]) * gain, each step one IEEE f32
+// operation in that order (__fadd_rn / __fmul_rn, never contracted).
+// The library is built without flush-to-zero, so f32 subnormals survive.
+#include "internal.cuh"
+
+namespace moeq {
+namespace {
+
+// One thread per 32 consecutive weights of a row.
+__global__ void dequant_mxfp4_kernel(const uint8_t *__restrict__ codes,
+                                     const uint8_t *__restrict__ scales, int N, int K,
+                                     float *__restrict__ out) {
+    const int units_per_row = K / 32;
+    long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= (long long)N * units_per_row) return;
+    int n = (int)(u / units_per_row), b = (int)(u % units_per_row);
+    const uint8_t *c = codes + (size_t)n * (K / 2) + (size_t)b * 16;
+    float sc = e8m0_to_f32(scales[(size_t)n * units_per_row + b]);
+    float *o = out + (size_t)n * K + (size_t)b * 32;
+    uint4 raw = *reinterpret_cast<const uint4 *>(c);
+    uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t nib = (words[q] >> (4 * i)) & 0xFu;
+            o[q * 8 + i] = __fmul_rn(e2m1_to_f32(nib), sc);
+        }
+    }
+}
+
+__global__ void dequant_vq_kernel(const uint8_t *__restrict__ idx13, const uint8_t *__restrict__ idx8,
+                                  const uint16_t *__restrict__ book13,
+                                  const uint16_t *__restrict__ book8,
+                                  const uint16_t *__restrict__ gain, int N, int K,
+                                  float *__restrict__ out) {
+    const int groups = K / 8;
+    long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= (long long)N * groups) return;
+    int n = (int)(u / groups), j = (int)(u % groups);
+    const uint8_t *row13 = idx13 + (size_t)n * (K / 8) * 13 / 8;
+    uint32_t i13 = idx13_at(row13, j);
+    const uint16_t *b = book13 + (size_t)i13 * 8;
+    const uint16_t *r = idx8 ? book8 + (size_t)idx8[(size_t)n * groups + j] * 8 : nullptr;
+    float g = gain ? f16_bits_to_f32(gain[n]) : 1.0f;
+    float *o = out + (size_t)n * K + (size_t)j * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float v = bf16_bits_to_f32(b[i]);
+        if (r) v = __fadd_rn(v, bf16_bits_to_f32(r[i]));
+        if (gain) v = __fmul_rn(v, g);
+        o[i] = v;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_dequant(const Layer &L, int expert, int proj, float *out, cudaStream_t s) {
+    ProjView v = L.view(proj);
+    L.count_launches(1);
+    const int threads = 256;
+    if (L.d.fmt == MOEQ_FMT_MXFP4) {
+        long long units = (long long)v.N * (v.K / 32);
+        const uint8_t *c = v.codes + (size_t)expert * v.N * (v.K / 2);
+        const uint8_t *sc = v.scales + (size_t)expert * v.N * (v.K / 32);
+        dequant_mxfp4_kernel<<<(unsigned)((units + threads - 1) / threads), threads, 0, s>>>(
+            c, sc, v.N, v.K, out);
+    } else {
+        long long units = (long long)v.N * (v.K / 8);
+        const uint8_t *i13 = v.idx13 + (size_t)expert * v.N * (v.K / 8) * 13 / 8;
+        const uint8_t *i8 = v.idx8 ? v.idx8 + (size_t)expert * v.N * (v.K / 8) : nullptr;
+        const uint16_t *g = v.gain ? v.gain + (size_t)expert * v.N : nullptr;
+        dequant_vq_kernel<<<(unsigned)((units + threads - 1) / threads), threads, 0, s>>>(
+            i13, i8, v.book13, v.book8, g, v.N, v.K, out);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moeq

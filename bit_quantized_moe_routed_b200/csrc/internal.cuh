@@ -1,0 +1,133 @@
+// internal.cuh -- shared declarations of the moeq CUDA library (not part of
+// the public ABI; see include/moeq.h for that).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moeq.h"
+
+namespace moeq {
+
+// Device status-word flags (atomicOr'ed by kernels, read by moeq_layer_status).
+enum : uint32_t { FLAG_ROUTE_RANGE = 1u, FLAG_TIMEOUT = 2u };
+
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 64;
+constexpr int kBook13Rows = 8192;
+constexpr int kBook8Rows = 256;
+
+// Device copies of the compressed weights.  Layout is the logical one of
+// moeq_weights (row-major [E][N][...] per projection).
+struct DevWeights {
+    uint8_t *codes[3] = {nullptr, nullptr, nullptr};
+    uint8_t *scales[3] = {nullptr, nullptr, nullptr};
+    uint8_t *idx13[3] = {nullptr, nullptr, nullptr};
+    uint8_t *idx8[3] = {nullptr, nullptr, nullptr};
+    uint16_t *gain[3] = {nullptr, nullptr, nullptr};
+    uint16_t *book13 = nullptr;
+    uint16_t *book8 = nullptr;
+    bool has_gain = false;
+};
+
+// Routing tables produced by the route/bucket kernel for one forward.
+struct Buckets {
+    int32_t *offsets = nullptr;  // [E+1] exclusive scan of per-expert route counts
+    int32_t *perm = nullptr;     // [T*k] route ids r = t*k+s, sorted by (expert, r)
+    int32_t *active = nullptr;   // [E+1] active[0] = #experts with routes, then their ids ascending
+};
+
+// Everything one projection kernel needs to find and decode a matrix.
+struct ProjView {
+    const uint8_t *codes;   // MXFP4 nibbles          [E][N][K/2]
+    const uint8_t *scales;  // MXFP4 E8M0 bytes       [E][N][K/32]
+    const uint8_t *idx13;   // VQ 13-bit stream       [E][N][K*13/64]
+    const uint8_t *idx8;    // VQ residual indices    [E][N][K/8] or null
+    const uint16_t *gain;   // f16 row gains          [E][N] or null
+    const uint16_t *book13; // bf16 [8192][8]
+    const uint16_t *book8;  // bf16 [256][8] or null
+    int32_t N, K;
+};
+
+struct Layer {
+    moeq_layer_desc d{};
+    DevWeights w;
+    Buckets b;
+    float *h = nullptr;        // [max_tokens*k][I] SwiGLU intermediates, route-sorted order
+    float *acc = nullptr;      // [max_tokens][H] f32 combine accumulator
+    uint32_t *status = nullptr;
+    // staging for moeq_forward_host
+    void *x_stage = nullptr;
+    void *out_stage = nullptr;
+    int32_t *ids_stage = nullptr;
+    float *w_stage = nullptr;
+    bool uploaded = false;
+    int sm_count = 0;
+    // kernels launched (or captured into a graph) by this layer so far
+    mutable long long launches = 0;
+    void count_launches(int n) const { launches += n; }
+
+    ProjView view(int p) const {
+        ProjView v{};
+        v.codes = w.codes[p];
+        v.scales = w.scales[p];
+        v.idx13 = w.idx13[p];
+        v.idx8 = (d.fmt == MOEQ_FMT_VQ13_R8) ? w.idx8[p] : nullptr;
+        v.gain = w.has_gain ? w.gain[p] : nullptr;
+        v.book13 = w.book13;
+        v.book8 = (d.fmt == MOEQ_FMT_VQ13_R8) ? w.book8 : nullptr;
+        v.N = (p == MOEQ_DOWN) ? d.hidden : d.inter;
+        v.K = (p == MOEQ_DOWN) ? d.inter : d.hidden;
+        return v;
+    }
+    int elem_bytes() const { return d.act == MOEQ_ACT_F32 ? 4 : 2; }
+};
+
+// ---- launchers (each returns cudaGetLastError() of its launch) ----
+cudaError_t launch_route_bucket(const Layer &L, const int32_t *topk_ids, int32_t n_routes,
+                                int32_t *offsets, int32_t *perm, int32_t *active, cudaStream_t s);
+cudaError_t launch_dequant(const Layer &L, int expert, int proj, float *out, cudaStream_t s);
+// ev: null, or the 5 phase events of moeq_forward_profiled (ev[0] and ev[1]
+// are recorded by the caller around routing).
+cudaError_t launch_ffn_simt(const Layer &L, const void *x, const float *topk_w, int32_t n_tokens,
+                            void *out, cudaStream_t s, const cudaEvent_t *ev);
+
+// ---- small device helpers shared by the kernels ----
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+__device__ __forceinline__ float f16_bits_to_f32(uint16_t b) {
+    return __half2float(__ushort_as_half(b));
+}
+
+// E2M1 code (4 bits) -> f32.  Exponent field e (bias 1) and mantissa m:
+// e > 0 gives 2^(e-1) (1 + m/2), whose f32 pattern is ((126+e)<<23)|(m<<22)
+// = (code&7)<<22 + (126<<23); e == 0 gives 0 or 0.5.
+__device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
+    uint32_t mag = c & 7u;
+    uint32_t bits = (mag >= 2u) ? ((mag << 22) + (126u << 23)) : (mag ? 0x3F000000u : 0u);
+    return __uint_as_float(bits | ((c & 8u) << 28));
+}
+
+// E8M0 byte -> f32 2^(b-127): b<<23 for b >= 1, the subnormal 2^-127 for
+// b == 0, NaN for 255 (rejected at upload).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
+    return __uint_as_float(b == 0u ? 0x00400000u : (b == 255u ? 0x7FC00000u : (b << 23)));
+}
+
+// 13-bit index j of a row's little-endian index stream.  Reads the third
+// byte only when the field reaches it, so the last index of the last row
+// never reads past the array.
+__device__ __forceinline__ uint32_t idx13_at(const uint8_t *row, int j) {
+    uint32_t bit = 13u * (uint32_t)j;
+    const uint8_t *p = row + (bit >> 3);
+    uint32_t sh = bit & 7u;
+    uint32_t win = (uint32_t)p[0] | ((uint32_t)p[1] << 8);
+    if (sh > 3u) win |= (uint32_t)p[2] << 16;
+    return (win >> sh) & 0x1FFFu;
+}
+
+__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + expf(-g)); }
+
+}  // namespace moeq

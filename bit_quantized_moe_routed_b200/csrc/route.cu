@@ -1,0 +1,128 @@
+// route.cu -- route/bucket kernel: groups the T*k routes of a forward by
+// expert.
+//
+// The layer sends each token to k experts ("MiMo-V2.6-Flash-RL GGUF for a
+// single DGX Spark", "Architecture notes": 8 of 256 routed experts), and the
+// expert matmuls want all of an expert's tokens together ("Speed": at a
+// micro-batch of 512 each of the 256 experts sees too few tokens per matmul).
+// This kernel produces, for one forward:
+//   offsets[E+1]  exclusive scan of the per-expert route counts
+//   perm[n_valid] route ids r = t*k + s, ordered by (expert, r) -- stable, so
+//                 the order is fully determined by the input
+//   active[E+1]   active[0] = number of experts with at least one route,
+//                 active[1..] = those experts in ascending order
+// Route ids of -1 are "no route"; any other id outside [0, E) is skipped and
+// raises FLAG_ROUTE_RANGE in the status word.
+//
+// One CTA of 1024 threads does it all: a shared-memory histogram, a scan,
+// then the routes in tiles of 1024 in index order, each route's rank among
+// equal experts found with __match_any_sync inside a warp and per-warp
+// counts across warps.
+#include "internal.cuh"
+
+namespace moeq {
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+
+__global__ void __launch_bounds__(kThreads, 1)
+route_bucket_kernel(const int32_t *__restrict__ ids, int32_t n_routes, int32_t E,
+                    int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+                    int32_t *__restrict__ active, uint32_t *__restrict__ status) {
+    extern __shared__ int32_t smem[];
+    int32_t *cnt = smem;                 // [E]
+    int32_t *base = smem + E;            // [E]
+    int32_t *wcnt = smem + 2 * E;        // [kWarps][E]
+    __shared__ int32_t s_total;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    for (int i = tid; i < E * (2 + kWarps); i += kThreads) smem[i] = 0;
+    __syncthreads();
+
+    // 1. histogram
+    bool bad = false;
+    for (int r = tid; r < n_routes; r += kThreads) {
+        int32_t e = ids[r];
+        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+        else if (e != -1) bad = true;
+    }
+    if (__syncthreads_or(bad) && tid == 0) atomicOr(status, FLAG_ROUTE_RANGE);
+
+    // 2. exclusive scan of counts and compaction of active experts (warp 0)
+    if (warp == 0) {
+        int32_t run = 0, nact = 0;
+        for (int c0 = 0; c0 < E; c0 += 32) {
+            int e = c0 + lane;
+            int32_t v = (e < E) ? cnt[e] : 0;
+            int32_t incl = v;
+            for (int o = 1; o < 32; o <<= 1) {
+                int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            uint32_t act = __ballot_sync(0xffffffffu, v > 0);
+            if (e < E) {
+                offsets[e] = run + incl - v;
+                base[e] = run + incl - v;
+                if (v > 0) active[1 + nact + __popc(act & ((1u << lane) - 1u))] = e;
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
+            nact += __popc(act);
+        }
+        if (lane == 0) {
+            offsets[E] = run;
+            active[0] = nact;
+            s_total = run;
+        }
+    }
+    __syncthreads();
+
+    // 3. stable scatter, one tile of kThreads routes at a time
+    for (int t0 = 0; t0 < n_routes; t0 += kThreads) {
+        int r = t0 + tid;
+        int32_t e = (r < n_routes) ? ids[r] : -1;
+        bool valid = (e >= 0 && e < E);
+        int32_t key = valid ? e : -1 - lane;  // invalid lanes match nobody
+        uint32_t same = __match_any_sync(0xffffffffu, key);
+        int rank = __popc(same & ((1u << lane) - 1u));
+        bool leader = rank == 0;
+        if (valid && leader) wcnt[warp * E + e] = __popc(same);
+        __syncthreads();
+        int pos = 0;
+        if (valid) {
+            pos = base[e] + rank;
+            for (int w2 = 0; w2 < warp; ++w2) pos += wcnt[w2 * E + e];
+            perm[pos] = r;
+        }
+        __syncthreads();
+        if (valid && leader) {
+            atomicAdd(&base[e], __popc(same));
+            wcnt[warp * E + e] = 0;
+        }
+        __syncthreads();
+    }
+    (void)s_total;
+}
+
+}  // namespace
+
+cudaError_t launch_route_bucket(const Layer &L, const int32_t *topk_ids, int32_t n_routes,
+                                int32_t *offsets, int32_t *perm, int32_t *active, cudaStream_t s) {
+    const int E = L.d.n_experts;
+    size_t smem = sizeof(int32_t) * (size_t)E * (2 + kWarps);
+    static bool attr_set[64] = {};
+    int dev = L.d.device;
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t err = cudaFuncSetAttribute(route_bucket_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)(sizeof(int32_t) * kMaxExperts * (2 + kWarps)));
+        if (err != cudaSuccess) return err;
+        attr_set[dev] = true;
+    }
+    L.count_launches(1);
+    route_bucket_kernel<<<1, kThreads, smem, s>>>(topk_ids, n_routes, E, offsets, perm, active,
+                                                  L.status);
+    return cudaGetLastError();
+}
+
+}  // namespace moeq

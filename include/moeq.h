@@ -1,0 +1,223 @@
+/*
+ * moeq.h -- C ABI of the compressed-expert routed MoE layer for NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer is the routed-expert FFN of a MiMo-V2.6-Flash-shaped MoE block:
+ * every token t is sent to k experts e = topk_ids[t][s] with weights
+ * topk_w[t][s], and
+ *
+ *     out[t] = sum_s topk_w[t][s] * W_down,e ( silu(W_gate,e x[t]) * (W_up,e x[t]) )
+ *
+ * with silu(z) = z / (1 + e^-z).  The expert matrices stay compressed in
+ * device memory and are decoded inside the matrix products.  Sources (page
+ * title, section):
+ *   - "MiMo-V2.6-Flash-RL GGUF for a single DGX Spark", "Architecture notes":
+ *     256 routed experts, 8 active per token, no shared expert; experts stored
+ *     as MXFP4, one E8M0 exponent per 32 values.
+ *   - "MiMo-V2.6-Flash-RL Mixed-Quant GGUF", "Why this model needs an
+ *     asymmetric layout": packed MXFP4, two weights per byte; gate/up and down
+ *     projections per expert.
+ *   - "MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe" and "Why 13 bits plus
+ *     an 8-bit residual": each 8 consecutive weights of an expert row are one
+ *     13-bit index into the layer's 8192x8 codebook (shared by all experts and
+ *     gate/up/down), times an f16 row gain; an optional second 256x8 book codes
+ *     the first stage's residual with 8 more bits per 8 weights; the kernels
+ *     keep the layer's whole codebook in shared memory while they decode every
+ *     selected expert.
+ *   - "MiMo-V2.6-Flash-RL GGUF for a single DGX Spark", "Recipe": a 32-value
+ *     expert-intermediate sum can pass f16's 65504, so intermediates are kept
+ *     in a type with f32's exponent range.
+ *
+ * Conventions
+ *   - Every call returns a moeq_status; no exception or signal crosses the ABI.
+ *   - Projection p: MOEQ_GATE [inter][hidden], MOEQ_UP [inter][hidden],
+ *     MOEQ_DOWN [hidden][inter].  Rows are output features; the reduction axis
+ *     K is contiguous in memory.
+ *   - A "stream" argument is a cudaStream_t passed as void* (NULL = the legacy
+ *     default stream).  Device pointers must be on the layer's device.
+ *   - One layer's workspace is not re-entrant: calls on one layer must be
+ *     ordered (one stream, or explicit events).  Distinct layers are
+ *     independent and may be used from different host threads.
+ */
+#ifndef MOEQ_H
+#define MOEQ_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOEQ_API __attribute__((visibility("default")))
+#else
+#define MOEQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOEQ_OK = 0,
+    MOEQ_ERR_INVALID_ARGUMENT = 1,  /* bad pointer, size, enum or weight byte  */
+    MOEQ_ERR_UNSUPPORTED = 2,       /* valid but not implemented combination   */
+    MOEQ_ERR_OUT_OF_MEMORY = 3,     /* a device allocation failed              */
+    MOEQ_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed    */
+    MOEQ_ERR_NOT_UPLOADED = 5,      /* forward/dequant before upload_weights   */
+    MOEQ_ERR_ROUTE_OUT_OF_RANGE = 6,/* device flag: an id outside [-1, E) seen */
+    MOEQ_ERR_TIMEOUT = 7            /* device flag: a bounded wait gave up     */
+} moeq_status;
+
+typedef enum { MOEQ_FMT_MXFP4 = 0, MOEQ_FMT_VQ13 = 1, MOEQ_FMT_VQ13_R8 = 2 } moeq_format;
+typedef enum { MOEQ_ACT_F32 = 0, MOEQ_ACT_BF16 = 1 } moeq_dtype;
+typedef enum { MOEQ_GATE = 0, MOEQ_UP = 1, MOEQ_DOWN = 2 } moeq_proj;
+
+typedef struct {
+    int32_t hidden;      /* H: model width (K of gate/up, N of down)              */
+    int32_t inter;       /* I: expert intermediate width                          */
+    int32_t n_experts;   /* E, 1..1024                                            */
+    int32_t top_k;       /* k, 1..min(E, 64)                                      */
+    int32_t max_tokens;  /* largest n_tokens any forward will pass, >= 1          */
+    int32_t fmt;         /* moeq_format                                           */
+    int32_t act;         /* moeq_dtype of x and out                               */
+    int32_t device;      /* CUDA device ordinal                                   */
+} moeq_layer_desc;
+
+typedef struct moeq_layer *moeq_layer_t;
+
+/*
+ * Host copy of a layer's compressed weights, logical layout, one array per
+ * projection p (index = moeq_proj).  N, K are the projection's rows and
+ * reduction length.
+ *
+ * MXFP4 ("Architecture notes" above):
+ *   codes[p]   uint8 [E][N][K/2]  element k of a row is the low nibble of byte
+ *                                 k/2 when k is even, the high nibble when odd;
+ *                                 nibble = E2M1 (sign, 2 exponent bits with
+ *                                 bias 1, 1 mantissa bit)
+ *   scales[p]  uint8 [E][N][K/32] E8M0 byte b: weight = e2m1 * 2^(b-127);
+ *                                 b = 255 (NaN) is rejected
+ * VQ13 / VQ13_R8 ("Recipe" above):
+ *   idx13[p]   uint8 [E][N][K*13/64]  per row, the K/8 indices as one
+ *                                 little-endian bitstream: index j is bits
+ *                                 13j..13j+12, bit q of the stream is bit q%8
+ *                                 of byte q/8
+ *   idx8[p]    uint8 [E][N][K/8]  residual index per 8-vector (VQ13_R8 only)
+ *   book13     uint16 bf16 [8192][8]  base codebook; entry dimension i is K
+ *                                 offset 8j+i of group j
+ *   book8      uint16 bf16 [256][8]   residual codebook (VQ13_R8 only)
+ *   gain[p]    uint16 f16 [E][N] or NULL (gain 1)
+ *   weight[n][8j+i] = (book13[idx13][i] + book8[idx8][i]) * gain[n], each
+ *   operation IEEE f32 round-to-nearest-even, in that order.
+ * Arrays not used by the format must be NULL.
+ */
+typedef struct {
+    const uint8_t *codes[3];
+    const uint8_t *scales[3];
+    const uint8_t *idx13[3];
+    const uint8_t *idx8[3];
+    const uint16_t *book13;
+    const uint16_t *book8;
+    const uint16_t *gain[3];
+} moeq_weights;
+
+/* Create a layer on desc->device and allocate, on that device, its weight
+ * storage and a workspace sized for desc->max_tokens.  The library owns all
+ * of it until moeq_layer_destroy.
+ * Errors: INVALID_ARGUMENT (NULL pointer; a non-positive size; top_k > E or
+ * > 64; E > 1024; hidden or inter not a multiple of 32 for MXFP4 or of 64
+ * for VQ; unknown fmt/act), CUDA (bad device), OUT_OF_MEMORY.  On error *out
+ * is set to NULL and nothing is left allocated. */
+MOEQ_API moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out);
+
+/* Copy the host arrays of w into the layer (the library may store them in a
+ * different internal order).  Validates first: every array the format needs
+ * is non-NULL, arrays it does not use are NULL, no E8M0 byte is 255.  Uses
+ * `stream` for the copies and synchronizes it before returning, so the
+ * caller may free w's arrays as soon as the call returns.
+ * Errors: INVALID_ARGUMENT (validation), CUDA. */
+MOEQ_API moeq_status moeq_upload_weights(moeq_layer_t layer, const moeq_weights *w, void *stream);
+
+/* out[t] for t < n_tokens, as defined at the top of this file.
+ *   x         device, act dtype, [n_tokens][hidden], row-major
+ *   topk_ids  device int32 [n_tokens][top_k]; -1 = no route (contributes 0);
+ *             any other id outside [0, E) is skipped and raises
+ *             MOEQ_ERR_ROUTE_OUT_OF_RANGE in the layer status word
+ *   topk_w    device f32 [n_tokens][top_k]; any values (need not sum to 1)
+ *   out       device, act dtype, [n_tokens][hidden]; overwritten
+ * Asynchronous on `stream`: all pointers must stay valid until the stream
+ * reaches the end of the call.  The sum over routes is accumulated in f32
+ * and rounded once (RNE) to the output dtype; the order in which routes are
+ * added is not specified.  n_tokens == 0 is a no-op.
+ * Errors (synchronous): INVALID_ARGUMENT (NULL pointer, n_tokens < 0 or >
+ * max_tokens), NOT_UPLOADED, CUDA (launch). */
+MOEQ_API moeq_status moeq_forward(moeq_layer_t layer, const void *x, const int32_t *topk_ids,
+                         const float *topk_w, int32_t n_tokens, void *out, void *stream);
+
+/* moeq_forward with HOST buffers (same shapes and dtypes): copies x,
+ * topk_ids and topk_w to the layer's device staging area, runs the forward
+ * and copies out back, all on `stream`, and synchronizes the stream before
+ * returning.  Host buffers may be pageable or pinned.
+ * Errors: as moeq_forward, and CUDA for a failed copy or synchronize. */
+MOEQ_API moeq_status moeq_forward_host(moeq_layer_t layer, const void *x_host, const int32_t *topk_ids_host,
+                              const float *topk_w_host, int32_t n_tokens, void *out_host,
+                              void *stream);
+
+/* The route/bucket step of moeq_forward on its own: groups the routes of
+ * topk_ids (device int32 [n_tokens][top_k]) by expert.
+ *   offsets_out  device int32 [E+1]: offsets_out[e] = number of valid routes
+ *                whose expert is below e (valid: id in [0, E))
+ *   perm_out     device int32 [n_tokens*top_k]: its first offsets_out[E]
+ *                entries are the valid route ids r = t*top_k + s, expert by
+ *                expert, ascending r within an expert (a stable sort)
+ * Ids of -1 are skipped; other ids outside [0, E) are skipped and raise
+ * MOEQ_ERR_ROUTE_OUT_OF_RANGE in the status word.  Asynchronous on
+ * `stream`; uses the layer's workspace (ordered like moeq_forward).
+ * Source: "MiMo-V2.6-Flash-RL GGUF for a single DGX Spark", "Speed" (each
+ * expert's tokens are gathered into one matmul) and "Architecture notes"
+ * (k of E experts per token).
+ * Errors: INVALID_ARGUMENT (NULL pointer, n_tokens < 1 or > max_tokens),
+ * CUDA. */
+MOEQ_API moeq_status moeq_route(moeq_layer_t layer, const int32_t *topk_ids, int32_t n_tokens,
+                                int32_t *offsets_out, int32_t *perm_out, void *stream);
+
+/* moeq_forward that also records five caller-created CUDA events (passed
+ * as cudaEvent_t cast to void*) on `stream` at its phase boundaries:
+ * events[0] before the first launch, [1] after route/bucket, [2] after the
+ * gate/up + SwiGLU kernel, [3] after the down projection and combine, [4]
+ * after the final cast.  Where a phase is fused into another, its two
+ * events are recorded back to back.  For measuring kernel durations; the
+ * results are those of moeq_forward.  Errors: as moeq_forward, and
+ * INVALID_ARGUMENT for a NULL events array. */
+MOEQ_API moeq_status moeq_forward_profiled(moeq_layer_t layer, const void *x, const int32_t *topk_ids,
+                                           const float *topk_w, int32_t n_tokens, void *out, void *stream,
+                                           void *const *events);
+
+/* Decode projection `proj` of expert `expert` into out, device f32 [N][K],
+ * logical layout.  Bit-exact: every element equals the f32 weight defined
+ * by the format above (signed zeros, f32 subnormals and +-inf overflow of
+ * an E8M0 x E2M1 product included).  Asynchronous on `stream`.
+ * Errors: INVALID_ARGUMENT (expert or proj out of range, NULL out),
+ * NOT_UPLOADED, CUDA. */
+MOEQ_API moeq_status moeq_dequant(moeq_layer_t layer, int32_t expert, int32_t proj, float *out, void *stream);
+
+/* The layer's device status word, read after synchronizing the device:
+ * MOEQ_OK, or the first-raised device flag (MOEQ_ERR_ROUTE_OUT_OF_RANGE,
+ * MOEQ_ERR_TIMEOUT).  clear != 0 resets it.  Errors: INVALID_ARGUMENT,
+ * CUDA. */
+MOEQ_API moeq_status moeq_layer_status(moeq_layer_t layer, int32_t clear);
+
+/* Number of kernels the layer has launched so far (a launch captured into
+ * a CUDA graph counts once, at capture); -1 for a NULL layer.  Lets a caller
+ * check that the work ran in this library's kernels. */
+MOEQ_API int64_t moeq_kernel_launches(moeq_layer_t layer);
+
+/* Static description of a status code; never NULL. */
+MOEQ_API const char *moeq_status_string(moeq_status s);
+
+/* Free everything the layer owns (synchronizes its device first).
+ * NULL is a no-op. */
+MOEQ_API void moeq_layer_destroy(moeq_layer_t layer);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEQ_H */

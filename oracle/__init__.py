@@ -14,4 +14,5 @@ from .oracle import (  # noqa: F401
     dequant,
     forward,
     num_threads,
+    route_bucket,
 )

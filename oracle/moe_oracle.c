@@ -294,3 +294,29 @@ int orc_num_threads(void)
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------ */
+/* Route bucketing                                                     */
+/* ------------------------------------------------------------------ */
+
+/* Group the n_routes = T*k routes of a forward by expert [SPK "Speed": the
+ * expert matmuls want each expert's tokens together; "Architecture notes":
+ * k of E experts per token].  offsets[E+1]: offsets[e] = number of valid
+ * routes with an expert below e.  perm: the valid route ids r (= t*k + s)
+ * listed expert by expert, ascending r within an expert.  -1 is "no route";
+ * other ids outside [0, E) are dropped.  Returns the number of dropped ids
+ * other than -1. */
+int64_t orc_route_bucket(const int32_t *ids, int64_t n_routes, int32_t E,
+                         int32_t *offsets, int32_t *perm)
+{
+    int64_t invalid = 0, pos = 0;
+    for (int64_t r = 0; r < n_routes; ++r)
+        if (ids[r] != -1 && (ids[r] < 0 || ids[r] >= E)) ++invalid;
+    for (int32_t e = 0; e < E; ++e) {
+        offsets[e] = (int32_t)pos;
+        for (int64_t r = 0; r < n_routes; ++r)
+            if (ids[r] == e) perm[pos++] = (int32_t)r;
+    }
+    offsets[E] = (int32_t)pos;
+    return invalid;
+}

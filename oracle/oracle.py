@@ -65,6 +65,8 @@ def lib():
         L.orc_forward.argtypes = [C.POINTER(_Layer), C.c_void_p, C.c_void_p, C.c_void_p,
                                   C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]
         L.orc_num_threads.restype = C.c_int
+        L.orc_route_bucket.restype = C.c_int64
+        L.orc_route_bucket.argtypes = [C.c_void_p, C.c_int64, C.c_int32, C.c_void_p, C.c_void_p]
         _lib = L
     return _lib
 
@@ -88,6 +90,15 @@ def f16_to_f64(bits: int) -> float:
 def idx13(stream: np.ndarray, j: int) -> int:
     s = np.ascontiguousarray(stream, dtype=np.uint8)
     return int(lib().orc_idx13(s.ctypes.data, j))
+
+
+def route_bucket(topk_ids, E: int):
+    """(offsets int32 [E+1], perm int32 [n_valid], n_invalid) of the routes."""
+    ids = np.ascontiguousarray(topk_ids, dtype=np.int32).ravel()
+    offsets = np.empty(E + 1, np.int32)
+    perm = np.empty(len(ids), np.int32)
+    bad = lib().orc_route_bucket(ids.ctypes.data, len(ids), E, offsets.ctypes.data, perm.ctypes.data)
+    return offsets, perm[: offsets[E]].copy(), int(bad)
 
 
 def num_threads() -> int:

@@ -1,0 +1,149 @@
+"""moeq_forward against the oracle on small and medium layers, plus the
+invariants the pages fix (unrouted experts contribute nothing, no-route ids,
+linearity in the routing weights, slot order, the host-buffer entry point)."""
+import numpy as np
+import pytest
+
+from _gpu_util import (TOL, assert_close, dev_layer, oracle, oracle_ref, out_to_f64, rel_err_per_token, run,
+                       synth, to_dev_inputs, torch_mod)
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_mxfp4_f32_config():
+    cfg = synth.get_cfg("tiny_mxfp4")
+    L = synth.gen_layer(cfg)
+    x = synth.gen_activations(cfg)
+    ids, w = synth.gen_routing(cfg)
+    lay = dev_layer(L)
+    out = run(lay, cfg, x, ids, w)
+    assert_close(out, oracle_ref(L, x, ids, w), "f32", "tiny")
+
+
+# medium layers: several 128-row tiles, ragged token counts, every format
+MEDIUM = [
+    dict(H=512, I=256, E=32, k=4, T=37),
+    dict(H=1024, I=384, E=8, k=2, T=300),
+]
+
+
+@pytest.mark.parametrize("shape", MEDIUM, ids=["m37", "m300"])
+@pytest.mark.parametrize("fmt,act,gains", [("mxfp4", "bf16", False), ("mxfp4", "f32", False),
+                                           ("vq13", "bf16", False), ("vq13r8", "bf16", True),
+                                           ("vq13r8", "f32", False)])
+def test_medium_layers(shape, fmt, act, gains):
+    cfg = synth.get_cfg("tiny_mxfp4", fmt=fmt, act=act, gains=gains, scale_exp=(-9, -5), **shape)
+    L = synth.gen_layer(cfg, seed=21)
+    x = synth.gen_activations(cfg, seed=21)
+    ids, w = synth.gen_routing(cfg, seed=21)
+    lay = dev_layer(L)
+    out = run(lay, cfg, x, ids, w)
+    assert_close(out, oracle_ref(L, x, ids, w), act, f"{fmt}/{act}/{shape}")
+
+
+def _cfg_small():
+    return synth.get_cfg("tiny_mxfp4", H=512, I=256, E=32, k=4, T=37, act="bf16", scale_exp=(-9, -5))
+
+
+def test_unrouted_experts_do_not_change_the_output():
+    torch = torch_mod()
+    cfg = _cfg_small()
+    L = synth.gen_layer(cfg, seed=3)
+    x = synth.gen_activations(cfg, seed=3)
+    ids, w = synth.gen_routing(cfg, seed=3)
+    ids[:, 0] = -1                      # some no-route slots too
+    used = set(ids.ravel().tolist())
+    lay = dev_layer(L)
+    out1 = run(lay, cfg, x, ids, w)
+    L2 = synth.gen_layer(cfg, seed=3)
+    rng = np.random.default_rng(5)
+    n_pert = 0
+    for e in range(cfg.E):
+        if e not in used:
+            n_pert += 1
+            for p in range(3):
+                L2.codes[p][e] = rng.integers(0, 256, size=L2.codes[p][e].shape, dtype=np.uint8)
+    assert n_pert > 0
+    lay2 = dev_layer(L2)
+    out2 = run(lay2, cfg, x, ids, w)
+    assert np.array_equal(out1, out2)
+    assert_close(out1, oracle_ref(L, x, ids, w), "bf16")
+    torch.cuda.synchronize()
+
+
+def test_no_route_and_out_of_range_ids():
+    from bit_quantized_moe_routed_b200 import moeq
+    cfg = _cfg_small()
+    L = synth.gen_layer(cfg, seed=4)
+    x = synth.gen_activations(cfg, seed=4)
+    ids, w = synth.gen_routing(cfg, seed=4)
+    lay = dev_layer(L)
+    ids2 = ids.copy()
+    ids2[2, 1] = -1
+    ids2[5, 3] = cfg.E
+    ids2[7, 0] = -100
+    out = run(lay, cfg, x, ids2, w)
+    assert lay.status(clear=True) == moeq.ROUTE_OUT_OF_RANGE
+    w2 = w.copy()
+    w2[2, 1] = w2[5, 3] = w2[7, 0] = 0.0
+    assert_close(out, oracle_ref(L, x, ids, w2), "bf16")
+    # a token with every slot empty gets exactly zero
+    ids3 = ids.copy()
+    ids3[0, :] = -1
+    out3 = run(lay, cfg, x, ids3, w)
+    assert not out3[0].any()
+    assert lay.status() == moeq.OK
+
+
+def test_linear_in_weights_and_slot_permutation():
+    cfg = _cfg_small().replace(fmt="vq13r8")
+    L = synth.gen_layer(cfg, seed=6)
+    x = synth.gen_activations(cfg, seed=6)
+    ids, w = synth.gen_routing(cfg, seed=6)
+    lay = dev_layer(L)
+    ref = oracle_ref(L, x, ids, w)
+    out1 = run(lay, cfg, x, ids, w)
+    out2 = run(lay, cfg, x, ids, 2 * w)
+    out3 = run(lay, cfg, x, ids[:, ::-1], w[:, ::-1])
+    assert_close(out1, ref, "bf16")
+    assert_close(out2, 2 * ref, "bf16")
+    assert_close(out3, ref, "bf16")
+
+
+def test_forward_host_and_profiled_match_forward():
+    torch = torch_mod()
+    cfg = _cfg_small()
+    L = synth.gen_layer(cfg, seed=7)
+    x = synth.gen_activations(cfg, seed=7)
+    ids, w = synth.gen_routing(cfg, seed=7)
+    lay = dev_layer(L)
+    ref = run(lay, cfg, x, ids, w)
+    oh = lay.forward_host(x, ids, w)
+    outh = out_to_f64(torch.from_numpy(oh.view(np.int16)).view(torch.bfloat16))
+    assert_close(outh, oracle_ref(L, x, ids, w), "bf16")
+    xt, it, wt = to_dev_inputs(cfg, x, ids, w)
+    out = torch.empty_like(xt)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    lay.forward_profiled(xt, it, wt, out, ev)
+    torch.cuda.synchronize()
+    assert_close(out_to_f64(out), oracle_ref(L, x, ids, w), "bf16")
+    times = [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
+    assert all(t >= 0 for t in times)
+    np.testing.assert_allclose(out_to_f64(out), ref, rtol=0, atol=np.abs(ref).max() * 1e-6)
+
+
+def test_zero_tokens_is_a_noop_and_bad_sizes_fail():
+    from bit_quantized_moe_routed_b200 import moeq
+    torch = torch_mod()
+    cfg = _cfg_small()
+    lay = dev_layer(synth.gen_layer(cfg, seed=8))
+    x = torch.zeros(0, cfg.H, dtype=torch.bfloat16, device="cuda")
+    ids = torch.zeros(0, cfg.k, dtype=torch.int32, device="cuda")
+    w = torch.zeros(0, cfg.k, device="cuda")
+    lay.forward(x, ids, w)
+    x = torch.zeros(cfg.T + 1, cfg.H, dtype=torch.bfloat16, device="cuda")
+    ids = torch.zeros(cfg.T + 1, cfg.k, dtype=torch.int32, device="cuda")
+    w = torch.zeros(cfg.T + 1, cfg.k, device="cuda")
+    with pytest.raises(moeq.MoeqError) as ei:
+        lay.forward(x, ids, w)
+    assert ei.value.code == moeq.INVALID_ARGUMENT

@@ -374,3 +374,23 @@ def test_overflow_workload_property_and_finite():
     sums = np.abs(h.reshape(8, cfg.I // 32, 32).sum(-1))
     assert (sums > 65504).any()
     assert np.isfinite(out).all() and np.isfinite(h).all()
+
+
+def test_route_bucket_hand_example():
+    # 3 tokens x 2 slots over 4 experts; -1 = no route, 9 = invalid
+    ids = np.array([[2, 0], [0, -1], [2, 9]], np.int32)
+    offsets, perm, bad = oracle.route_bucket(ids, 4)
+    assert list(offsets) == [0, 2, 2, 4, 4]
+    assert list(perm) == [1, 2, 0, 4]
+    assert bad == 1
+
+
+def test_route_bucket_is_a_stable_sort():
+    # the bucketed order is numpy's stable argsort of the expert ids
+    cfg = synth.get_cfg("prefill_mxfp4_zipf")
+    ids, _ = synth.gen_routing(cfg)
+    offsets, perm, bad = oracle.route_bucket(ids, cfg.E)
+    flat = ids.ravel()
+    assert bad == 0 and np.array_equal(perm, np.argsort(flat, kind="stable"))
+    assert np.array_equal(np.diff(offsets), np.bincount(flat, minlength=cfg.E))
+    assert offsets[13] == offsets[14] and offsets[184] == offsets[185]   # never routed
