@@ -321,6 +321,10 @@ def main():
     # per-phase kernel durations over the same K steps (a second graph with
     # phase events between the kernels)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for row in ev:              # torch creates the CUDA event at its first record
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g2, stream=cap):
         for n, i in enumerate(range(args.warmup, n_total)):

@@ -73,6 +73,9 @@ void free_layer(moeq_layer *L) {
     cudaFree(L->b.active);
     cudaFree(L->h);
     cudaFree(L->acc);
+    cudaFree(L->dec_gmax);
+    cudaFree(L->dec_ybuf);
+    cudaFree(L->dec_counters);
     cudaFree(L->status);
     cudaFree(L->x_stage);
     cudaFree(L->out_stage);
@@ -87,7 +90,7 @@ bool desc_valid(const moeq_layer_desc *d) {
     if (d->n_experts > kMaxExperts || d->top_k > d->n_experts || d->top_k > kMaxTopK) return false;
     if (d->act != MOEQ_ACT_F32 && d->act != MOEQ_ACT_BF16) return false;
     if (d->fmt == MOEQ_FMT_MXFP4) {
-        if (d->hidden % 32 || d->inter % 32) return false;
+        if (d->hidden % 128 || d->inter % 128) return false;
     } else if (d->fmt == MOEQ_FMT_VQ13 || d->fmt == MOEQ_FMT_VQ13_R8) {
         if (d->hidden % 64 || d->inter % 64) return false;
     } else {
@@ -101,6 +104,7 @@ bool desc_valid(const moeq_layer_desc *d) {
 moeq_status launch_forward(moeq_layer *L, const void *x, const int32_t *ids, const float *w, int32_t T,
                            void *out, cudaStream_t s, const cudaEvent_t *ev = nullptr) {
     if (ev) cudaEventRecord(ev[0], s);
+    if (decode_mx_supported(*L, T)) return from_cuda(launch_decode_mx(*L, x, ids, w, T, out, s, ev));
     cudaError_t e = launch_route_bucket(*L, ids, T * L->d.top_k, L->b.offsets, L->b.perm, L->b.active, s);
     if (e != cudaSuccess) return from_cuda(e);
     if (ev) cudaEventRecord(ev[1], s);
@@ -168,6 +172,9 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     ALLOC(L->b.perm, sizeof(int32_t) * M * k);
     ALLOC(L->h, sizeof(float) * M * k * I);
     ALLOC(L->acc, sizeof(float) * M * H);
+    ALLOC(L->dec_gmax, sizeof(float) * kDecMaxGrid * kDecMaxTokens);
+    ALLOC(L->dec_ybuf, sizeof(float) * kDecMaxRoutes * kDecMaxTokens * H);
+    ALLOC(L->dec_counters, sizeof(int) * (H / 32 + 1));
     ALLOC(L->status, sizeof(uint32_t));
     ALLOC(L->x_stage, (size_t)L->elem_bytes() * M * H);
     ALLOC(L->out_stage, (size_t)L->elem_bytes() * M * H);
@@ -175,6 +182,7 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     ALLOC(L->w_stage, sizeof(float) * M * k);
 #undef ALLOC
     if (e == cudaSuccess) e = cudaMemset(L->status, 0, sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMemset(L->dec_counters, 0, sizeof(int) * (H / 32 + 1));
     if (e != cudaSuccess) {
         free_layer(L);
         cudaGetLastError();  // clear a sticky allocation error
@@ -234,6 +242,11 @@ moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *str
             if (e == cudaSuccess && n_gain)
                 e = cudaMemcpyAsync(L->w.gain[p], w->gain[p], rows * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
         }
+    }
+    // MXFP4 codes go to the device layout (64-byte groups word-transposed)
+    for (int p = 0; p < 3 && e == cudaSuccess && mx; ++p) {
+        const int N = (p == MOEQ_DOWN) ? H : I, K = (p == MOEQ_DOWN) ? I : H;
+        e = launch_mx_repack(L->w.codes[p], (size_t)E * N * row_bytes(fmt, 0, K), s);
     }
     if (e == cudaSuccess && !mx)
         e = cudaMemcpyAsync(L->w.book13, w->book13, sizeof(uint16_t) * kBook13Rows * 8, cudaMemcpyHostToDevice, s);

@@ -21,10 +21,10 @@ __global__ void dequant_mxfp4_kernel(const uint8_t *__restrict__ codes,
     long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (u >= (long long)N * units_per_row) return;
     int n = (int)(u / units_per_row), b = (int)(u % units_per_row);
-    const uint8_t *c = codes + (size_t)n * (K / 2) + (size_t)b * 16;
+    const uint8_t *row = codes + (size_t)n * (K / 2);
     float sc = e8m0_to_f32(scales[(size_t)n * units_per_row + b]);
     float *o = out + (size_t)n * K + (size_t)b * 32;
-    uint4 raw = *reinterpret_cast<const uint4 *>(c);
+    uint4 raw = mx_block(row, b);
     uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -60,7 +60,27 @@ __global__ void dequant_vq_kernel(const uint8_t *__restrict__ idx13, const uint8
     }
 }
 
+// In-place 4x4 transpose of the 32-bit words of every 64-byte group (the
+// device layout of MXFP4 codes; see mx_word).
+__global__ void mx_repack_kernel(uint4 *__restrict__ codes, size_t n_groups) {
+    size_t gi = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gi >= n_groups) return;
+    uint4 *g = codes + 4 * gi;
+    uint4 a = g[0], b = g[1], c = g[2], d = g[3];
+    g[0] = make_uint4(a.x, b.x, c.x, d.x);
+    g[1] = make_uint4(a.y, b.y, c.y, d.y);
+    g[2] = make_uint4(a.z, b.z, c.z, d.z);
+    g[3] = make_uint4(a.w, b.w, c.w, d.w);
+}
+
 }  // namespace
+
+cudaError_t launch_mx_repack(uint8_t *codes, size_t bytes, cudaStream_t s) {
+    size_t n_groups = bytes / 64;
+    if (n_groups == 0) return cudaSuccess;
+    mx_repack_kernel<<<(unsigned)((n_groups + 255) / 256), 256, 0, s>>>(reinterpret_cast<uint4 *>(codes), n_groups);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_dequant(const Layer &L, int expert, int proj, float *out, cudaStream_t s) {
     ProjView v = L.view(proj);

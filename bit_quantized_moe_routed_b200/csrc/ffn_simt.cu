@@ -26,7 +26,7 @@ template <int FMT>
 __device__ __forceinline__ void decode_unit(const ProjView &v, int e, int n, int u, float w[32]) {
     const size_t row = (size_t)e * v.N + n;
     if constexpr (FMT == FMT_MX) {
-        uint4 raw = __ldg(reinterpret_cast<const uint4 *>(v.codes + row * (v.K / 2) + (size_t)u * 16));
+        uint4 raw = mx_block(v.codes + row * (v.K / 2), u);
         float sc = e8m0_to_f32(__ldg(v.scales + row * (v.K / 32) + u));
         uint32_t q[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll

@@ -18,6 +18,11 @@ constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 64;
 constexpr int kBook13Rows = 8192;
 constexpr int kBook8Rows = 256;
+// decode fast path: most CTAs a decode kernel launches, routes it handles,
+// tokens it handles
+constexpr int kDecMaxGrid = 1024;
+constexpr int kDecMaxRoutes = 64;
+constexpr int kDecMaxTokens = 8;
 
 // Device copies of the compressed weights.  Layout is the logical one of
 // moeq_weights (row-major [E][N][...] per projection).
@@ -57,6 +62,10 @@ struct Layer {
     Buckets b;
     float *h = nullptr;        // [max_tokens*k][I] SwiGLU intermediates, route-sorted order
     float *acc = nullptr;      // [max_tokens][H] f32 combine accumulator
+    // decode fast path scratch
+    float *dec_gmax = nullptr;     // [kDecMaxGrid][kDecMaxTokens] per-CTA max |w h| per token
+    float *dec_ybuf = nullptr;     // [kDecMaxRoutes][kDecMaxTokens][H] per-expert partial outputs
+    int *dec_counters = nullptr;   // [H/32] per-tile arrival counters, zero between calls
     uint32_t *status = nullptr;
     // staging for moeq_forward_host
     void *x_stage = nullptr;
@@ -91,6 +100,9 @@ cudaError_t launch_route_bucket(const Layer &L, const int32_t *topk_ids, int32_t
 cudaError_t launch_dequant(const Layer &L, int expert, int proj, float *out, cudaStream_t s);
 // ev: null, or the 5 phase events of moeq_forward_profiled (ev[0] and ev[1]
 // are recorded by the caller around routing).
+bool decode_mx_supported(const Layer &L, int T);
+cudaError_t launch_decode_mx(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T,
+                             void *out, cudaStream_t s, const cudaEvent_t *ev);
 cudaError_t launch_ffn_simt(const Layer &L, const void *x, const float *topk_w, int32_t n_tokens,
                             void *out, cudaStream_t s, const cudaEvent_t *ev);
 
@@ -115,6 +127,22 @@ __device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
 __device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
     return __uint_as_float(b == 0u ? 0x00400000u : (b == 255u ? 0x7FC00000u : (b << 23)));
 }
+
+// Device layout of MXFP4 codes.  Each row's bytes come in groups of 64
+// (four 32-weight blocks of 16 bytes); inside a group the 4x4 matrix of
+// 32-bit words is transposed at upload, so that word t of logical block j
+// sits at byte 16*t + 4*j.  A thread that owns bytes 4t..4t+3 of every block
+// (the mma A-fragment slice) then reads four blocks with one 16-byte load.
+// The transpose is its own inverse.
+__device__ __forceinline__ uint32_t mx_word(const uint8_t *row, int blk, int t) {
+    return *reinterpret_cast<const uint32_t *>(row + (blk >> 2) * 64 + 16 * t + 4 * (blk & 3));
+}
+// The 16 logical bytes of block `blk` of a row (as four words, word t =
+// logical bytes 4t..4t+3).
+__device__ __forceinline__ uint4 mx_block(const uint8_t *row, int blk) {
+    return make_uint4(mx_word(row, blk, 0), mx_word(row, blk, 1), mx_word(row, blk, 2), mx_word(row, blk, 3));
+}
+cudaError_t launch_mx_repack(uint8_t *codes, size_t bytes, cudaStream_t s);
 
 // 13-bit index j of a row's little-endian index stream.  Reads the third
 // byte only when the field reaches it, so the last index of the last row

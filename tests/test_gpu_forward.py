@@ -41,13 +41,62 @@ def test_medium_layers(shape, fmt, act, gains):
     assert_close(out, oracle_ref(L, x, ids, w), act, f"{fmt}/{act}/{shape}")
 
 
+# decode-sized MXFP4 layers (1..8 tokens, bf16): the grouped-GEMV path
+DECODE = [
+    dict(H=1024, I=1024, E=16, k=2, T=1),
+    dict(H=2048, I=1024, E=8, k=8, T=8),      # every expert gets 8 routes
+    dict(H=1024, I=2048, E=32, k=8, T=5),
+    dict(H=4096, I=1024, E=64, k=8, T=8),
+]
+
+
+@pytest.mark.parametrize("shape", DECODE, ids=[f"H{s['H']}I{s['I']}E{s['E']}k{s['k']}T{s['T']}" for s in DECODE])
+def test_decode_mxfp4_shapes(shape):
+    cfg = synth.get_cfg("decode_mxfp4", **shape)
+    L = synth.gen_layer(cfg, seed=31)
+    x = synth.gen_activations(cfg, seed=31)
+    ids, w = synth.gen_routing(cfg, seed=31)
+    lay = dev_layer(L)
+    n0 = lay.kernel_launches()
+    out = run(lay, cfg, x, ids, w)
+    assert lay.kernel_launches() - n0 == 2        # the two decode kernels
+    assert_close(out, oracle_ref(L, x, ids, w), "bf16", str(shape))
+    # a second call with another routing (per-tile counters must have reset)
+    ids2, w2 = synth.gen_routing(cfg, seed=32)
+    out2 = run(lay, cfg, x, ids2, w2)
+    assert_close(out2, oracle_ref(L, x, ids2, w2), "bf16", str(shape) + " second call")
+
+
+def test_decode_mxfp4_duplicates_no_routes_and_extreme_activations():
+    from bit_quantized_moe_routed_b200 import moeq
+    cfg = synth.get_cfg("decode_mxfp4", H=1024, I=1024, E=4, k=4, T=8)
+    L = synth.gen_layer(cfg, seed=33)
+    x = synth.gen_activations(cfg, seed=33)
+    rng = np.random.default_rng(33)
+    ids = rng.integers(0, 2, size=(cfg.T, cfg.k)).astype(np.int32)   # ~16 routes per expert, repeats
+    ids[3, :] = -1                                                    # a token with no route
+    ids[5, 2] = -1
+    w = rng.normal(size=(cfg.T, cfg.k)).astype(np.float32)            # any sign, not normalised
+    xf = synth.f32_from_bf16_bits(x)
+    xf[1] = 0.0                                                       # an all-zero token
+    xf[6] *= 2.0 ** 40                                                # a huge one
+    xf[7] *= 2.0 ** -60                                               # a tiny one
+    x = synth.bf16_bits_from_f32(xf)
+    lay = dev_layer(L)
+    out = run(lay, cfg, x, ids, w)
+    ref = oracle_ref(L, x, ids, w)
+    assert not out[1].any() and not out[3].any()
+    assert_close(out, ref, "bf16", "duplicates/extremes")
+    assert lay.status() == moeq.OK
+
+
 def _cfg_small():
     return synth.get_cfg("tiny_mxfp4", H=512, I=256, E=32, k=4, T=37, act="bf16", scale_exp=(-9, -5))
 
 
 def test_unrouted_experts_do_not_change_the_output():
     torch = torch_mod()
-    cfg = _cfg_small()
+    cfg = _cfg_small().replace(E=64, T=8)   # 32 routes over 64 experts: many never routed
     L = synth.gen_layer(cfg, seed=3)
     x = synth.gen_activations(cfg, seed=3)
     ids, w = synth.gen_routing(cfg, seed=3)
