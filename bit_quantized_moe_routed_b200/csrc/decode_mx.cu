@@ -7,34 +7,37 @@
 // top-8 of 256 routed experts, MXFP4 experts with one E8M0 exponent per 32
 // values; "Recipe": expert intermediates stay in a type with f32's range).
 //
-// The products run on the tensor cores through warp-level
-// mma.sync.m16n8k16 (f16 in, f32 accumulate): a decode step is bound by HBM,
-// and the warp MMA lets each thread turn the bytes it loaded straight into
-// A-fragment registers (cvt.rn.f16x2.e2m1x2, exact) without a shared-memory
-// round trip for the weights.  Per 32-weight block the two MMAs accumulate
-// into a fresh fragment that is then folded into the running f32 sum times
-// the block's E8M0 scale, so the scale is applied exactly.  The B operand
-// (activations, or w * h for the down projection) is f16 after a per-token
-// power-of-two prescale that puts the largest magnitude in [2^14, 2^15):
-// f16 cannot overflow, and the scale is undone in f32 afterwards.
+// Memory: a unit is one expert's 16 gate + 16 up rows (gate/up kernel) or 32
+// down rows (down kernel) over the full K.  Its rows are contiguous in HBM,
+// so one warp moves a whole unit into shared memory with 1-D bulk copies
+// (TMA, one per row, rows padded so that the A-fragment reads below hit
+// distinct banks) and signals an mbarrier; a ring of stages keeps the next
+// unit(s) in flight while the current one is computed.  One CTA per SM.
 //
-// Work split: one CTA per SM with two teams of 8 warps.  A unit is one
-// expert's 16 gate+up rows (gate/up kernel) or 32 down rows (down kernel)
-// over the full K; the 8 warps of a team each take K/8 and their partial
-// fragments are summed through shared memory.  The two teams take alternate
-// units so that one team's loads are in flight while the other reduces.
-// The down kernel writes each expert's contribution to its own slice of a
-// scratch buffer; the last unit to finish a 32-row tile (per-tile arrival
-// counter) sums the experts in a fixed order, applies 1/prescale and writes
-// bf16 out, so the result does not depend on unit timing.
+// Math: warp-level mma.sync.m16n8k16 (f16 in, f32 accumulate).  Each thread
+// reads its A-fragment slice of four 32-weight blocks (bytes 4t..4t+3 of
+// each block; the upload transposes the words of each 64-byte group so the
+// slice is one 16-byte word) and decodes it with cvt.rn.f16x2.e2m1x2
+// (exact).  Per block the two MMAs accumulate into a fresh fragment that is
+// folded into the running f32 sum times the block's E8M0 scale, so the scale
+// is applied exactly.  The B operand (activations, or w * h for the down
+// projection) is f16 after a per-token power-of-two prescale that puts the
+// largest magnitude in [2^14, 2^15): f16 cannot overflow, and the scale is
+// undone in f32.  The 16 warps split K; their fragments are summed through
+// shared memory.
+//
+// Combine: the down kernel writes each expert's contribution to its own
+// slice of a scratch buffer; the last unit to finish a 32-row tile
+// (per-tile arrival counter) sums the experts in a fixed order, undoes the
+// prescale and writes bf16 out, so the result does not depend on timing.
+#include "async.cuh"
 #include "internal.cuh"
 
 namespace moeq {
 namespace {
 
-constexpr int kTeamWarps = 8;
-constexpr int kTeams = 2;
-constexpr int kThreads = 32 * kTeamWarps * kTeams;
+constexpr int kWarps = 16;
+constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxT = 8;
 constexpr int kMaxR = 64;
 constexpr int kXPad = 32;  // f16 elements of padding after each staged x row
@@ -164,22 +167,14 @@ __device__ __forceinline__ uint32_t u4get(const uint4 &v, int j) {
     return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
 
-__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-__device__ __forceinline__ uint32_t ldg_nc_u32(const void *p) {
-    uint32_t r;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
-    return r;
-}
-
-// Named barrier for one team (ids 1, 2; 0 is __syncthreads).
-__device__ __forceinline__ void team_sync(int team) {
-    asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(32 * kTeamWarps));
+// After a timed-out wait: wait (bounded again) for the copies of the units
+// after it that were already issued, so none lands in shared memory after
+// the CTA has gone.
+__device__ void drain_stages(uint64_t *full, int n_stages, int j0, int n_units) {
+    for (int j = j0; j < j0 + n_stages - 1; ++j) {
+        if ((int)blockIdx.x + j * (int)gridDim.x >= n_units) break;
+        mbar_wait_bounded(&full[j % n_stages], (uint32_t)((j / n_stages) & 1), 200000000LL);
+    }
 }
 
 // ---------------------------------------------------------------- gate/up
@@ -195,26 +190,80 @@ struct GateUpArgs {
     int T, k, E, H, I;
 };
 
-// NG = groups of 4 blocks per warp slice = H / 1024.
+constexpr int kGUStages = 2;
+constexpr int kRowPad = 64;    // bytes after each staged code row
+constexpr int kScalePad = 16;  // bytes after each staged scale row
+
+struct GULayout {
+    int row_stride, sc_stride, stage_bytes, xs_stride;
+    __host__ __device__ GULayout(int H) {
+        row_stride = H / 2 + kRowPad;
+        sc_stride = H / 32 + kScalePad;
+        stage_bytes = 32 * row_stride + 32 * sc_stride;
+        xs_stride = H + kXPad;
+    }
+    // [stages][stage] [x16: T rows] [red: 16 warps x 32 lanes x 8]
+    __host__ __device__ size_t xs_off() const { return (size_t)kGUStages * stage_bytes; }
+    __host__ __device__ size_t red_off(int T) const { return xs_off() + sizeof(uint16_t) * (size_t)T * xs_stride; }
+    __host__ __device__ size_t bytes(int T) const { return red_off(T) + sizeof(float) * kWarps * 32 * 8; }
+};
+
+// Warp 0: put unit j's 16 gate + 16 up rows and their scale rows in stage j % kGUStages.
+__device__ __forceinline__ void gu_issue(const GateUpArgs &a, const RouteTable &tb, const GULayout &ly,
+                                         uint8_t *stages, uint64_t *full, int j, int n_units) {
+    const int u = blockIdx.x + j * gridDim.x;
+    if (u >= n_units) return;
+    const int lane = threadIdx.x & 31;
+    const int tiles = a.I / 16;
+    const int d = u / tiles, n0 = (u % tiles) * 16;
+    const size_t row0 = (size_t)tb.expert[d] * a.I + n0;
+    uint8_t *st = stages + (size_t)(j % kGUStages) * ly.stage_bytes;
+    uint64_t *bar = full + (j % kGUStages);
+    const uint32_t code_b = a.H / 2, sc_b = a.H / 32;
+    if (lane == 0) mbar_arrive_expect_tx(bar, 32u * (code_b + sc_b));
+    __syncwarp();
+    const int mat = lane >> 4, r = lane & 15;   // lane -> (gate|up, row)
+    const uint8_t *codes = mat ? a.codes_u : a.codes_g;
+    const uint8_t *scales = mat ? a.scales_u : a.scales_g;
+    bulk_g2s(st + (size_t)(mat * 16 + r) * ly.row_stride, codes + (row0 + r) * code_b, code_b, bar);
+    bulk_g2s(st + (size_t)32 * ly.row_stride + (size_t)(mat * 16 + r) * ly.sc_stride, scales + (row0 + r) * sc_b,
+             sc_b, bar);
+}
+
+// NG = groups of four 32-weight blocks per warp's K slice = H / 2048.
 template <int NG>
 __global__ void __launch_bounds__(kThreads, 1) dec_gateup_mx_kernel(GateUpArgs a) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ RouteTable tb;
+    __shared__ __align__(8) uint64_t full[kGUStages];
     __shared__ float xinv[kMaxT];
     __shared__ unsigned cta_max[kMaxT];
     const int H = a.H, I = a.I, T = a.T, k = a.k;
-    const int xs_stride = H + kXPad;
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw);                               // [T][H+pad] f16
-    float *red = reinterpret_cast<float *>(smem_raw + sizeof(uint16_t) * T * xs_stride);  // [2 teams][2][8 warps][32][8]
+    const GULayout ly(H);
+    uint8_t *stages = smem_raw;
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw + ly.xs_off());
+    float *red = reinterpret_cast<float *>(smem_raw + ly.red_off(T));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int team = warp / kTeamWarps, w = warp % kTeamWarps;
     const int g = lane >> 2, t = lane & 3;
 
-    if (warp == 0) build_route_table(tb, a.ids, T * k, a.E, a.status, blockIdx.x == 0);
+    if (tid == 0) {
+        for (int s = 0; s < kGUStages; ++s) mbar_init(&full[s], 1);
+        mbar_fence_init();
+    }
     if (tid < kMaxT) cta_max[tid] = 0u;
-    // stage x as f16 with a per-token power-of-two prescale (warp w <-> token w)
-    if (warp < T) {
-        const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)warp * H);
+    if (warp == 0) build_route_table(tb, a.ids, T * k, a.E, a.status, blockIdx.x == 0);
+    __syncthreads();
+    const int tiles = I / 16;
+    const int n_units = tb.D * tiles;
+    if (warp == 0)
+        for (int j = 0; j < kGUStages; ++j) gu_issue(a, tb, ly, stages, full, j, n_units);
+    // let the down kernel's CTAs launch as SMs free up (they wait for this
+    // grid before reading h)
+    pdl_launch_dependents();
+    // stage x as f16 with a per-token power-of-two prescale (warp w+1 <-> token w)
+    if (warp >= 1 && warp <= T) {
+        const int tk = warp - 1;
+        const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)tk * H);
         float m = 0.f;
         for (int i = lane; i < H / 8; i += 32) {
             uint4 v = xr[i];
@@ -227,14 +276,15 @@ __global__ void __launch_bounds__(kThreads, 1) dec_gateup_mx_kernel(GateUpArgs a
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         const int s = prescale_exp(m);
         const float sc = exp2i(s);
-        if (lane == 0) xinv[warp] = exp2i(-s);
-        uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)warp * xs_stride);
+        if (lane == 0) xinv[tk] = exp2i(-s);
+        uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)tk * ly.xs_stride);
         for (int i = lane; i < H / 8; i += 32) {
             uint4 v = xr[i];
             uint32_t q[4] = {v.x, v.y, v.z, v.w}, o[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                __half2 hv = __floats2half2_rn(__uint_as_float(q[j] << 16) * sc, __uint_as_float(q[j] & 0xFFFF0000u) * sc);
+                __half2 hv = __floats2half2_rn(__uint_as_float(q[j] << 16) * sc,
+                                               __uint_as_float(q[j] & 0xFFFF0000u) * sc);
                 o[j] = *reinterpret_cast<uint32_t *>(&hv);
             }
             dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -242,78 +292,64 @@ __global__ void __launch_bounds__(kThreads, 1) dec_gateup_mx_kernel(GateUpArgs a
     }
     __syncthreads();
 
-    const int tiles = I / 16;
-    const int n_units = tb.D * tiles;
-    const int slice_blocks = 4 * NG;                 // blocks of 32 per warp slice
-    const size_t rowb = (size_t)H / 2, rows = (size_t)H / 32;
-    // let the down kernel's CTAs launch as SMs free up (they wait for this
-    // grid before reading h)
-    asm volatile("griddepcontrol.launch_dependents;");
-    int rc = 0;  // reductions done by this team: picks the red buffer
-    for (int u = blockIdx.x + team * gridDim.x; u < n_units; u += kTeams * gridDim.x) {
-        const int d = u / tiles, tile = u % tiles;
-        const int e = tb.expert[d];
-        const int n0 = tile * 16;
-        const size_t r0 = (size_t)e * I + n0 + g;
-        const uint8_t *pg0 = a.codes_g + r0 * rowb + (size_t)w * slice_blocks * 16 + 16 * t;
-        const uint8_t *pu0 = a.codes_u + r0 * rowb + (size_t)w * slice_blocks * 16 + 16 * t;
-        const uint8_t *sg0 = a.scales_g + r0 * rows + (size_t)w * slice_blocks;
-        const uint8_t *su0 = a.scales_u + r0 * rows + (size_t)w * slice_blocks;
+    for (int j = 0;; ++j) {
+        const int u = blockIdx.x + j * gridDim.x;
+        if (u >= n_units) break;
+        const uint32_t parity = (uint32_t)((j / kGUStages) & 1);
+        const bool ok = mbar_wait_bounded(&full[j % kGUStages], parity);
+        // also keeps red[] from being rewritten before the last unit's readers finish
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(a.status, FLAG_TIMEOUT);
+                drain_stages(full, kGUStages, j + 1, n_units);
+            }
+            break;
+        }
+        const int d = u / tiles, n0 = (u % tiles) * 16;
+        const uint8_t *st = stages + (size_t)(j % kGUStages) * ly.stage_bytes;
         for (int cb = tb.col_beg[d]; cb < tb.col_beg[d + 1]; cb += 8) {
+            if (cb > tb.col_beg[d]) __syncthreads();   // red[] reuse within a unit
             const int ncol = min(8, tb.col_beg[d + 1] - cb);
-            // this thread's B column: column g of the chunk
             const bool live = g < ncol;
             const int tok = live ? tb.route[cb + g] / k : 0;
-            const uint16_t *xrow = xs + (size_t)tok * xs_stride + (size_t)w * slice_blocks * 32 + 8 * t;
-            uint4 cg0[NG], cg8[NG], cu0[NG], cu8[NG];
-            uint32_t qg0[NG], qg8[NG], qu0[NG], qu8[NG];
-#pragma unroll
-            for (int G = 0; G < NG; ++G) {
-                cg0[G] = ldg_nc_v4(pg0 + 64 * G);
-                cg8[G] = ldg_nc_v4(pg0 + 8 * rowb + 64 * G);
-                cu0[G] = ldg_nc_v4(pu0 + 64 * G);
-                cu8[G] = ldg_nc_v4(pu0 + 8 * rowb + 64 * G);
-                qg0[G] = ldg_nc_u32(sg0 + 4 * G);
-                qg8[G] = ldg_nc_u32(sg0 + 8 * rows + 4 * G);
-                qu0[G] = ldg_nc_u32(su0 + 4 * G);
-                qu8[G] = ldg_nc_u32(su0 + 8 * rows + 4 * G);
-            }
+            const uint16_t *xrow = xs + (size_t)tok * ly.xs_stride + 8 * t;
             float aG[4] = {0.f, 0.f, 0.f, 0.f}, aU[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int G = 0; G < NG; ++G) {
+                const int gg = warp * NG + G;   // group index within the row
+                const uint8_t *cp = st + (size_t)g * ly.row_stride + gg * 64 + 16 * t;
+                const uint4 ag0 = lds128(cp), ag8 = lds128(cp + 8 * ly.row_stride);
+                const uint4 au0 = lds128(cp + 16 * ly.row_stride), au8 = lds128(cp + 24 * ly.row_stride);
+                const uint8_t *sp = st + (size_t)32 * ly.row_stride + (size_t)g * ly.sc_stride + gg * 4;
+                const uint32_t sg0 = lds32(sp), sg8 = lds32(sp + 8 * ly.sc_stride);
+                const uint32_t su0 = lds32(sp + 16 * ly.sc_stride), su8 = lds32(sp + 24 * ly.sc_stride);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 xb = live ? *reinterpret_cast<const uint4 *>(xrow + (4 * G + j) * 32)
-                                          : make_uint4(0u, 0u, 0u, 0u);
-                    block_mma(aG, u4get(cg0[G], j), u4get(cg8[G], j), xb, e8m0_byte(qg0[G], j), e8m0_byte(qg8[G], j));
-                    block_mma(aU, u4get(cu0[G], j), u4get(cu8[G], j), xb, e8m0_byte(qu0[G], j), e8m0_byte(qu8[G], j));
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint4 xb = live ? lds128(xrow + (gg * 4 + jj) * 32) : make_uint4(0u, 0u, 0u, 0u);
+                    block_mma(aG, u4get(ag0, jj), u4get(ag8, jj), xb, e8m0_byte(sg0, jj), e8m0_byte(sg8, jj));
+                    block_mma(aU, u4get(au0, jj), u4get(au8, jj), xb, e8m0_byte(su0, jj), e8m0_byte(su8, jj));
                 }
             }
-            // team reduction over the 8 K-slices
-            // (red[rc&1] is rewritten two reductions later, after a team_sync
-            // that every reader of this one has passed)
-            float *rb = red + ((size_t)(team * 2 + (rc & 1)) * kTeamWarps) * 32 * 8;
-            ++rc;
-            float4 *mine = reinterpret_cast<float4 *>(rb + ((size_t)w * 32 + lane) * 8);
+            float4 *mine = reinterpret_cast<float4 *>(red + ((size_t)warp * 32 + lane) * 8);
             mine[0] = make_float4(aG[0], aG[1], aG[2], aG[3]);
             mine[1] = make_float4(aU[0], aU[1], aU[2], aU[3]);
-            team_sync(team);
-            const int ttid = tid - team * 32 * kTeamWarps;
-            if (ttid < 128) {
-                const int row = ttid >> 3, col = ttid & 7;   // 16 rows x 8 columns
+            __syncthreads();
+            // every warp is done reading this stage: refill it with unit j + kGUStages
+            if (warp == 0 && cb + 8 >= tb.col_beg[d + 1]) gu_issue(a, tb, ly, stages, full, j + kGUStages, n_units);
+            if (tid < 128) {
+                const int row = tid >> 3, col = tid & 7;   // 16 rows x 8 columns
                 if (col < ncol) {
                     const int gl = row & 7, hi = row >> 3, tl = col >> 1, cbit = col & 1;
                     const int src_lane = gl * 4 + tl, slot = hi * 2 + cbit;
                     float gs = 0.f, us = 0.f;
 #pragma unroll
-                    for (int ww = 0; ww < kTeamWarps; ++ww) {
-                        gs += rb[((size_t)ww * 32 + src_lane) * 8 + slot];
-                        us += rb[((size_t)ww * 32 + src_lane) * 8 + 4 + slot];
+                    for (int ww = 0; ww < kWarps; ++ww) {
+                        gs += red[((size_t)ww * 32 + src_lane) * 8 + slot];
+                        us += red[((size_t)ww * 32 + src_lane) * 8 + 4 + slot];
                     }
                     const int route = tb.route[cb + col];
                     const float inv = xinv[route / k];
-                    const float gv = gs * inv, uv = us * inv;
-                    const float hv = silu_f32(gv) * uv;
+                    const float hv = silu_f32(gs * inv) * (us * inv);
                     a.h[(size_t)route * I + n0 + row] = hv;
                     const float wh = fabsf(a.topk_w[route] * hv);
                     if (wh > 0.f) atomicMax(&cta_max[route / k], __float_as_uint(isfinite(wh) ? wh : 3.0e38f));
@@ -328,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) dec_gateup_mx_kernel(GateUpArgs a
 // ---------------------------------------------------------------- down
 
 struct DownArgs {
-    const uint8_t *codes, *scales;  // down projection [E][H][I/2], [E][H][I/32]
+    const uint8_t *codes, *scales;  // down projection [E][H][I/2] (device layout), [E][H][I/32]
     const float *h;                 // [T*k][I]
     const float *gmax;              // [n_gmax][kMaxT]
     int n_gmax;
@@ -337,26 +373,74 @@ struct DownArgs {
     float *ybuf;                    // [kMaxR expert slots][kMaxT][H]
     int *counters;                  // [H/32], zero between calls
     uint16_t *out;                  // bf16 [T][H]
+    uint32_t *status;
     int T, k, E, H, I;
 };
 
+constexpr int kDNStages = 4;
+
+struct DNLayout {
+    int row_stride, sc_stride, stage_bytes;
+    __host__ __device__ DNLayout(int I) {
+        row_stride = I / 2 + kRowPad;
+        sc_stride = I / 32 + kScalePad;
+        stage_bytes = 32 * row_stride + 32 * sc_stride;
+    }
+    __host__ __device__ size_t red_off() const { return (size_t)kDNStages * stage_bytes; }
+    __host__ __device__ size_t bytes() const { return red_off() + sizeof(float) * kWarps * 32 * 8; }
+};
+
+__device__ __forceinline__ void dn_issue(const DownArgs &a, const RouteTable &tb, const DNLayout &ly,
+                                         uint8_t *stages, uint64_t *full, int j, int n_units) {
+    const int u = blockIdx.x + j * gridDim.x;
+    if (u >= n_units) return;
+    const int lane = threadIdx.x & 31;
+    const int tiles = a.H / 32;
+    const int d = u / tiles, m0 = (u % tiles) * 32;
+    const size_t row = (size_t)tb.expert[d] * a.H + m0 + lane;
+    uint8_t *st = stages + (size_t)(j % kDNStages) * ly.stage_bytes;
+    uint64_t *bar = full + (j % kDNStages);
+    const uint32_t code_b = a.I / 2, sc_b = a.I / 32;
+    if (lane == 0) mbar_arrive_expect_tx(bar, 32u * (code_b + sc_b));
+    __syncwarp();
+    bulk_g2s(st + (size_t)lane * ly.row_stride, a.codes + row * code_b, code_b, bar);
+    bulk_g2s(st + (size_t)32 * ly.row_stride + (size_t)lane * ly.sc_stride, a.scales + row * sc_b, sc_b, bar);
+}
+
+// NG = groups of four 32-weight blocks per warp's K slice = I / 2048.
 template <int NG>
 __global__ void __launch_bounds__(kThreads, 1) dec_down_mx_kernel(DownArgs a) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ RouteTable tb;
+    __shared__ __align__(8) uint64_t full[kDNStages];
     __shared__ float tok_scale[kMaxT], tok_inv[kMaxT];
     __shared__ float rscale[kMaxR];
-    __shared__ int last_flag[kTeams];
+    __shared__ int last_flag;
     const int H = a.H, I = a.I, T = a.T, k = a.k;
-    float *red = reinterpret_cast<float *>(smem_raw);  // [2 teams][2][8 warps][32][8]
+    const DNLayout ly(I);
+    uint8_t *stages = smem_raw;
+    float *red = reinterpret_cast<float *>(smem_raw + ly.red_off());
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int team = warp / kTeamWarps, w = warp % kTeamWarps;
     const int g = lane >> 2, t = lane & 3;
 
+    if (tid == 0) {
+        for (int s = 0; s < kDNStages; ++s) mbar_init(&full[s], 1);
+        mbar_fence_init();
+    }
     if (warp == 0) build_route_table(tb, a.ids, T * k, a.E, nullptr, false);
-    // h and gmax come from the gate/up kernel (a no-op without PDL)
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (warp >= 1 && warp - 1 < kMaxT) {
+    __syncthreads();
+    const int tiles = H / 32;
+    const int n_units = tb.D * tiles;
+    if (tb.D == 0) {   // no valid route at all: every output is zero
+        for (int i = blockIdx.x * kThreads + tid; i < T * H; i += gridDim.x * kThreads) a.out[i] = 0;
+        return;
+    }
+    // the weights do not depend on the gate/up kernel: start streaming them now
+    if (warp == 0)
+        for (int j = 0; j < kDNStages; ++j) dn_issue(a, tb, ly, stages, full, j, n_units);
+    // h and gmax come from the gate/up kernel
+    pdl_wait_primary();
+    if (warp >= 1 && warp <= kMaxT) {
         const int tk = warp - 1;
         float m = 0.f;
         for (int i = lane; i < a.n_gmax; i += 32) m = fmaxf(m, __ldcg(a.gmax + (size_t)i * kMaxT + tk));
@@ -372,111 +456,113 @@ __global__ void __launch_bounds__(kThreads, 1) dec_down_mx_kernel(DownArgs a) {
     if (tid < T * k) rscale[tid] = a.topk_w[tid] * tok_scale[tid / k];
     __syncthreads();
 
-    const int tiles = H / 32;
-    const int n_units = tb.D * tiles;
-    const int slice_blocks = 4 * NG;
-    const size_t rowb = (size_t)I / 2, rows = (size_t)I / 32;
-    int it = 0;  // units done by this team: picks the red buffer
-    for (int u = blockIdx.x + team * gridDim.x; u < n_units; u += kTeams * gridDim.x, ++it) {
-        const int d = u / tiles, tile = u % tiles;
-        const int e = tb.expert[d];
-        const int m0 = tile * 32;
-        const size_t r0 = (size_t)e * H + m0 + g;
-        const uint8_t *p0 = a.codes + r0 * rowb + (size_t)w * slice_blocks * 16 + 16 * t;
-        const uint8_t *s0 = a.scales + r0 * rows + (size_t)w * slice_blocks;
-        uint4 c[4][NG];
-        uint32_t q[4][NG];
-#pragma unroll
-        for (int G = 0; G < NG; ++G)
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-                c[rr][G] = ldg_nc_v4(p0 + (size_t)(8 * rr) * rowb + 64 * G);
-                q[rr][G] = ldg_nc_u32(s0 + (size_t)(8 * rr) * rows + 4 * G);
-            }
-        // B column g = token g: sum of w * prescale * h over the token's routes to e
+    for (int j = 0;; ++j) {
+        const int u = blockIdx.x + j * gridDim.x;
+        if (u >= n_units) break;
+        const int d = u / tiles, tile = u % tiles, m0 = tile * 32;
+        // B column g = token g: sum over the token's routes to this expert of
+        // w * prescale * h, this warp's K slice (loads issued before the wait)
         const bool live = g < T;
         float bsum[NG][4][8];
 #pragma unroll
         for (int G = 0; G < NG; ++G)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) bsum[G][j][i] = 0.f;
+                for (int i = 0; i < 8; ++i) bsum[G][jj][i] = 0.f;
         if (live) {
             for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) {
                 const int r = tb.route[cc];
                 if (r / k != g) continue;
                 const float rs = rscale[r];
-                const float *hp = a.h + (size_t)r * I + (size_t)w * slice_blocks * 32 + 8 * t;
+                const float *hp = a.h + (size_t)r * I + (size_t)warp * NG * 128 + 8 * t;
 #pragma unroll
                 for (int G = 0; G < NG; ++G)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(hp + (4 * G + j) * 32));
-                        const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(hp + (4 * G + j) * 32 + 4));
-                        bsum[G][j][0] = fmaf(rs, v0.x, bsum[G][j][0]);
-                        bsum[G][j][1] = fmaf(rs, v0.y, bsum[G][j][1]);
-                        bsum[G][j][2] = fmaf(rs, v0.z, bsum[G][j][2]);
-                        bsum[G][j][3] = fmaf(rs, v0.w, bsum[G][j][3]);
-                        bsum[G][j][4] = fmaf(rs, v1.x, bsum[G][j][4]);
-                        bsum[G][j][5] = fmaf(rs, v1.y, bsum[G][j][5]);
-                        bsum[G][j][6] = fmaf(rs, v1.z, bsum[G][j][6]);
-                        bsum[G][j][7] = fmaf(rs, v1.w, bsum[G][j][7]);
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(hp + (4 * G + jj) * 32));
+                        const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(hp + (4 * G + jj) * 32 + 4));
+                        float *bb = bsum[G][jj];
+                        bb[0] = fmaf(rs, v0.x, bb[0]);
+                        bb[1] = fmaf(rs, v0.y, bb[1]);
+                        bb[2] = fmaf(rs, v0.z, bb[2]);
+                        bb[3] = fmaf(rs, v0.w, bb[3]);
+                        bb[4] = fmaf(rs, v1.x, bb[4]);
+                        bb[5] = fmaf(rs, v1.y, bb[5]);
+                        bb[6] = fmaf(rs, v1.z, bb[6]);
+                        bb[7] = fmaf(rs, v1.w, bb[7]);
                     }
             }
         }
+        const uint32_t parity = (uint32_t)((j / kDNStages) & 1);
+        const bool ok = mbar_wait_bounded(&full[j % kDNStages], parity);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(a.status, FLAG_TIMEOUT);
+                drain_stages(full, kDNStages, j + 1, n_units);
+            }
+            break;
+        }
+        const uint8_t *st = stages + (size_t)(j % kDNStages) * ly.stage_bytes;
         float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int G = 0; G < NG; ++G)
+        for (int G = 0; G < NG; ++G) {
+            const int gg = warp * NG + G;
+            const uint8_t *cp = st + (size_t)g * ly.row_stride + gg * 64 + 16 * t;
+            const uint4 c0 = lds128(cp), c1 = lds128(cp + 8 * ly.row_stride);
+            const uint4 c2 = lds128(cp + 16 * ly.row_stride), c3 = lds128(cp + 24 * ly.row_stride);
+            const uint8_t *sp = st + (size_t)32 * ly.row_stride + (size_t)g * ly.sc_stride + gg * 4;
+            const uint32_t q0 = lds32(sp), q1 = lds32(sp + 8 * ly.sc_stride);
+            const uint32_t q2 = lds32(sp + 16 * ly.sc_stride), q3 = lds32(sp + 24 * ly.sc_stride);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int jj = 0; jj < 4; ++jj) {
                 uint4 xb;
-                __half2 h01 = __floats2half2_rn(bsum[G][j][0], bsum[G][j][1]);
-                __half2 h23 = __floats2half2_rn(bsum[G][j][2], bsum[G][j][3]);
-                __half2 h45 = __floats2half2_rn(bsum[G][j][4], bsum[G][j][5]);
-                __half2 h67 = __floats2half2_rn(bsum[G][j][6], bsum[G][j][7]);
+                __half2 h01 = __floats2half2_rn(bsum[G][jj][0], bsum[G][jj][1]);
+                __half2 h23 = __floats2half2_rn(bsum[G][jj][2], bsum[G][jj][3]);
+                __half2 h45 = __floats2half2_rn(bsum[G][jj][4], bsum[G][jj][5]);
+                __half2 h67 = __floats2half2_rn(bsum[G][jj][6], bsum[G][jj][7]);
                 xb.x = *reinterpret_cast<uint32_t *>(&h01);
                 xb.y = *reinterpret_cast<uint32_t *>(&h23);
                 xb.z = *reinterpret_cast<uint32_t *>(&h45);
                 xb.w = *reinterpret_cast<uint32_t *>(&h67);
-                block_mma(acc0, u4get(c[0][G], j), u4get(c[1][G], j), xb, e8m0_byte(q[0][G], j), e8m0_byte(q[1][G], j));
-                block_mma(acc1, u4get(c[2][G], j), u4get(c[3][G], j), xb, e8m0_byte(q[2][G], j), e8m0_byte(q[3][G], j));
+                block_mma(acc0, u4get(c0, jj), u4get(c1, jj), xb, e8m0_byte(q0, jj), e8m0_byte(q1, jj));
+                block_mma(acc1, u4get(c2, jj), u4get(c3, jj), xb, e8m0_byte(q2, jj), e8m0_byte(q3, jj));
             }
-        float *rb = red + ((size_t)(team * 2 + (it & 1)) * kTeamWarps) * 32 * 8;
-        float4 *mine = reinterpret_cast<float4 *>(rb + ((size_t)w * 32 + lane) * 8);
+        }
+        float4 *mine = reinterpret_cast<float4 *>(red + ((size_t)warp * 32 + lane) * 8);
         mine[0] = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
         mine[1] = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
-        team_sync(team);
-        const int ttid = tid - team * 32 * kTeamWarps;   // 0..255: 32 rows x 8 tokens
-        {
-            const int row = ttid >> 3, col = ttid & 7;
+        __syncthreads();
+        if (warp == 0) dn_issue(a, tb, ly, stages, full, j + kDNStages, n_units);
+        if (tid < 256) {
+            const int row = tid >> 3, col = tid & 7;   // 32 rows x 8 tokens
             if (col < T) {
                 const int sub = row >> 4, rl = row & 15;
                 const int gl = rl & 7, hi = rl >> 3, tl = col >> 1, cbit = col & 1;
                 const int src_lane = gl * 4 + tl, slot = sub * 4 + hi * 2 + cbit;
                 float s = 0.f;
 #pragma unroll
-                for (int ww = 0; ww < kTeamWarps; ++ww) s += rb[((size_t)ww * 32 + src_lane) * 8 + slot];
+                for (int ww = 0; ww < kWarps; ++ww) s += red[((size_t)ww * 32 + src_lane) * 8 + slot];
                 __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row, s);
             }
-        }
-        __threadfence();
-        team_sync(team);
-        if (ttid == 0) {
-            const int old = atomicAdd(a.counters + tile, 1);
-            last_flag[team] = (old == tb.D - 1);
-        }
-        team_sync(team);
-        if (last_flag[team]) {
             __threadfence();
-            const int row = ttid >> 3, col = ttid & 7;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const int old = atomicAdd(a.counters + tile, 1);
+            last_flag = (old == tb.D - 1);
+        }
+        __syncthreads();
+        if (last_flag && tid < 256) {
+            __threadfence();
+            const int row = tid >> 3, col = tid & 7;
             if (col < T) {
                 float s = 0.f;
                 for (int dd = 0; dd < tb.D; ++dd) s += __ldcg(a.ybuf + ((size_t)dd * kMaxT + col) * H + m0 + row);
                 __nv_bfloat16 o = __float2bfloat16_rn(s * tok_inv[col]);
                 a.out[(size_t)col * H + m0 + row] = *reinterpret_cast<uint16_t *>(&o);
             }
-            if (ttid == 0) a.counters[tile] = 0;
+            if (tid == 0) a.counters[tile] = 0;
         }
     }
 }
@@ -496,11 +582,27 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
     return cudaLaunchKernelEx(&cfg, kernel, args);
 }
 
+constexpr size_t kMaxDynSmem = 232448 - 4096;   // leave room for the static shared memory
+
 template <int NGU, int NGD>
 cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
                        cudaStream_t s, const cudaEvent_t *ev) {
     const int H = L.d.hidden, I = L.d.inter;
     const int grid = L.sm_count;
+    const GULayout gl(H);
+    const DNLayout dl(I);
+    static bool attr_done[64] = {};
+    const int dev = L.d.device;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(dec_gateup_mx_kernel<NGU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)gl.bytes(kMaxT));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(dec_down_mx_kernel<NGD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)dl.bytes());
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
     GateUpArgs ga;
     ga.codes_g = L.w.codes[MOEQ_GATE];
     ga.codes_u = L.w.codes[MOEQ_UP];
@@ -517,26 +619,11 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     ga.E = L.d.n_experts;
     ga.H = H;
     ga.I = I;
-    const size_t red_bytes = sizeof(float) * kTeams * 2 * kTeamWarps * 32 * 8;
-    const size_t smem_gu = sizeof(uint16_t) * T * (H + kXPad) + red_bytes;
-    static bool attr_done[64] = {};
-    const int dev = L.d.device;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(dec_gateup_mx_kernel<NGU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(sizeof(uint16_t) * kMaxT * (H + kXPad) + red_bytes));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(dec_down_mx_kernel<NGD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)red_bytes);
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
     L.count_launches(2);
-    if (ev) {
-        cudaEventRecord(ev[1], s);   // routing is fused into both kernels' prologues
-    }
-    cudaError_t e = launch_ex(dec_gateup_mx_kernel<NGU>, dim3(grid), dim3(kThreads), smem_gu, s, false, ga);
+    if (ev) record_phase(ev[1], s);   // routing is fused into both kernels' prologues
+    cudaError_t e = launch_ex(dec_gateup_mx_kernel<NGU>, dim3(grid), dim3(kThreads), gl.bytes(T), s, false, ga);
     if (e != cudaSuccess) return e;
-    if (ev) cudaEventRecord(ev[2], s);
+    if (ev) record_phase(ev[2], s);
     DownArgs da;
     da.codes = L.w.codes[MOEQ_DOWN];
     da.scales = L.w.scales[MOEQ_DOWN];
@@ -548,19 +635,20 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     da.ybuf = L.dec_ybuf;
     da.counters = L.dec_counters;
     da.out = reinterpret_cast<uint16_t *>(out);
+    da.status = L.status;
     da.T = T;
     da.k = L.d.top_k;
     da.E = L.d.n_experts;
     da.H = H;
     da.I = I;
-    // programmatic dependent launch: the down kernel's CTAs may start while
-    // the gate/up kernel drains; they wait (cudaGridDependencySynchronize)
-    // before reading h.  Not with phase events between the two launches.
-    e = launch_ex(dec_down_mx_kernel<NGD>, dim3(grid), dim3(kThreads), red_bytes, s, ev == nullptr, da);
+    // programmatic dependent launch: the down kernel's CTAs start streaming
+    // weights while the gate/up kernel drains and wait for it before reading
+    // h.  Not with phase events between the two launches.
+    e = launch_ex(dec_down_mx_kernel<NGD>, dim3(grid), dim3(kThreads), dl.bytes(), s, ev == nullptr, da);
     if (e != cudaSuccess) return e;
     if (ev) {
-        cudaEventRecord(ev[3], s);
-        cudaEventRecord(ev[4], s);
+        record_phase(ev[3], s);
+        record_phase(ev[4], s);
     }
     return cudaSuccess;
 }
@@ -571,21 +659,18 @@ bool decode_mx_supported(const Layer &L, int T) {
     const moeq_layer_desc &d = L.d;
     if (d.fmt != MOEQ_FMT_MXFP4 || d.act != MOEQ_ACT_BF16) return false;
     if (T < 1 || T > kMaxT || T * d.top_k > kMaxR) return false;
-    const bool hk = d.hidden == 1024 || d.hidden == 2048 || d.hidden == 4096 || d.hidden == 8192;
-    const bool ik = d.inter == 1024 || d.inter == 2048 || d.inter == 4096 || d.inter == 8192;
-    return hk && ik && d.inter % 16 == 0 && d.hidden % 32 == 0 && L.sm_count > 0 && L.sm_count <= kDecMaxGrid;
+    if (!((d.hidden == 2048 || d.hidden == 4096) && (d.inter == 2048 || d.inter == 4096))) return false;
+    if (GULayout(d.hidden).bytes(kMaxT) > kMaxDynSmem || DNLayout(d.inter).bytes() > kMaxDynSmem) return false;
+    return L.sm_count > 0 && L.sm_count <= kDecMaxGrid;
 }
 
 cudaError_t launch_decode_mx(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T,
                              void *out, cudaStream_t s, const cudaEvent_t *ev) {
     const int H = L.d.hidden, I = L.d.inter;
-#define MOEQ_DEC(HV, IV)                                                                          \
-    if (H == HV * 1024 && I == IV * 1024) return run_decode<HV, IV>(L, x, ids, topk_w, T, out, s, ev);
-    MOEQ_DEC(1, 1) MOEQ_DEC(1, 2) MOEQ_DEC(1, 4) MOEQ_DEC(1, 8)
-    MOEQ_DEC(2, 1) MOEQ_DEC(2, 2) MOEQ_DEC(2, 4) MOEQ_DEC(2, 8)
-    MOEQ_DEC(4, 1) MOEQ_DEC(4, 2) MOEQ_DEC(4, 4) MOEQ_DEC(4, 8)
-    MOEQ_DEC(8, 1) MOEQ_DEC(8, 2) MOEQ_DEC(8, 4) MOEQ_DEC(8, 8)
-#undef MOEQ_DEC
+    if (H == 2048 && I == 2048) return run_decode<1, 1>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 2048 && I == 4096) return run_decode<1, 2>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 4096 && I == 2048) return run_decode<2, 1>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 4096 && I == 4096) return run_decode<2, 2>(L, x, ids, topk_w, T, out, s, ev);
     return cudaErrorInvalidValue;
 }
 

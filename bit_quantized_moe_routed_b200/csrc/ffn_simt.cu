@@ -197,13 +197,13 @@ cudaError_t run(const Layer &L, const void *x, const float *topk_w, int32_t T, v
     L.count_launches(3);
     gateup_simt_kernel<FMT, BF16><<<dim3((I + kRowsPerCta - 1) / kRowsPerCta, ny), blk, 0, s>>>(
         L.view(MOEQ_GATE), L.view(MOEQ_UP), x, k, L.b.offsets, L.b.perm, L.b.active, L.h);
-    if (ev) cudaEventRecord(ev[2], s);
+    if (ev) record_phase(ev[2], s);
     down_simt_kernel<FMT><<<dim3((H + kRowsPerCta - 1) / kRowsPerCta, ny), blk, 0, s>>>(
         L.view(MOEQ_DOWN), L.h, topk_w, k, L.b.offsets, L.b.perm, L.b.active, L.acc);
-    if (ev) cudaEventRecord(ev[3], s);
+    if (ev) record_phase(ev[3], s);
     long long n = (long long)T * H;
     cast_out_kernel<BF16><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(L.acc, out, n);
-    if (ev) cudaEventRecord(ev[4], s);
+    if (ev) record_phase(ev[4], s);
     return cudaGetLastError();
 }
 

@@ -106,6 +106,11 @@ cudaError_t launch_decode_mx(const Layer &L, const void *x, const int32_t *ids, 
 cudaError_t launch_ffn_simt(const Layer &L, const void *x, const float *topk_w, int32_t n_tokens,
                             void *out, cudaStream_t s, const cudaEvent_t *ev);
 
+// Record a phase event of moeq_forward_profiled.  External, so that under
+// stream capture it becomes an event-record node of the graph (a plain
+// record is only a dependency marker there) and can be timed on replay.
+inline void record_phase(cudaEvent_t e, cudaStream_t s) { cudaEventRecordWithFlags(e, s, cudaEventRecordExternal); }
+
 // ---- small device helpers shared by the kernels ----
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 

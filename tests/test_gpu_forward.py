@@ -43,10 +43,10 @@ def test_medium_layers(shape, fmt, act, gains):
 
 # decode-sized MXFP4 layers (1..8 tokens, bf16): the grouped-GEMV path
 DECODE = [
-    dict(H=1024, I=1024, E=16, k=2, T=1),
-    dict(H=2048, I=1024, E=8, k=8, T=8),      # every expert gets 8 routes
-    dict(H=1024, I=2048, E=32, k=8, T=5),
-    dict(H=4096, I=1024, E=64, k=8, T=8),
+    dict(H=2048, I=2048, E=16, k=2, T=1),
+    dict(H=2048, I=2048, E=8, k=8, T=8),      # every expert gets 8 routes
+    dict(H=2048, I=4096, E=32, k=8, T=5),
+    dict(H=4096, I=2048, E=64, k=8, T=8),
 ]
 
 
@@ -69,7 +69,7 @@ def test_decode_mxfp4_shapes(shape):
 
 def test_decode_mxfp4_duplicates_no_routes_and_extreme_activations():
     from bit_quantized_moe_routed_b200 import moeq
-    cfg = synth.get_cfg("decode_mxfp4", H=1024, I=1024, E=4, k=4, T=8)
+    cfg = synth.get_cfg("decode_mxfp4", H=2048, I=2048, E=4, k=4, T=8)
     L = synth.gen_layer(cfg, seed=33)
     x = synth.gen_activations(cfg, seed=33)
     rng = np.random.default_rng(33)
@@ -88,6 +88,9 @@ def test_decode_mxfp4_duplicates_no_routes_and_extreme_activations():
     assert not out[1].any() and not out[3].any()
     assert_close(out, ref, "bf16", "duplicates/extremes")
     assert lay.status() == moeq.OK
+    # no valid route at all: zeros
+    out0 = run(lay, cfg, x, np.full_like(ids, -1), w)
+    assert not out0.any()
 
 
 def _cfg_small():
@@ -173,6 +176,8 @@ def test_forward_host_and_profiled_match_forward():
     xt, it, wt = to_dev_inputs(cfg, x, ids, w)
     out = torch.empty_like(xt)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    for e in ev:
+        e.record()          # torch creates the CUDA event at its first record
     lay.forward_profiled(xt, it, wt, out, ev)
     torch.cuda.synchronize()
     assert_close(out_to_f64(out), oracle_ref(L, x, ids, w), "bf16")
