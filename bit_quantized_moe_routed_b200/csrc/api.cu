@@ -1,5 +1,6 @@
 // api.cu -- the extern "C" entry points of libmoeq (declared in moeq.h):
 // argument validation, device memory ownership and kernel dispatch.
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -90,7 +91,10 @@ bool desc_valid(const moeq_layer_desc *d) {
     if (d->n_experts > kMaxExperts || d->top_k > d->n_experts || d->top_k > kMaxTopK) return false;
     if (d->act != MOEQ_ACT_F32 && d->act != MOEQ_ACT_BF16) return false;
     if (d->fmt == MOEQ_FMT_MXFP4) {
+        // whole 128-weight groups per row; rows of 1024 or more in whole
+        // 1024-weight chunks (the device layout, MxGeom)
         if (d->hidden % 128 || d->inter % 128) return false;
+        if ((d->hidden > 1024 && d->hidden % 1024) || (d->inter > 1024 && d->inter % 1024)) return false;
     } else if (d->fmt == MOEQ_FMT_VQ13 || d->fmt == MOEQ_FMT_VQ13_R8) {
         if (d->hidden % 64 || d->inter % 64) return false;
     } else {
@@ -155,8 +159,9 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
         const int N = (p == MOEQ_DOWN) ? H : I, K = (p == MOEQ_DOWN) ? I : H;
         const size_t rows = (size_t)E * N;
         if (fmt == MOEQ_FMT_MXFP4) {
-            ALLOC(L->w.codes[p], rows * row_bytes(fmt, 0, K));
-            ALLOC(L->w.scales[p], rows * row_bytes(fmt, 1, K));
+            // codes and scales share one plane in the device layout (MxGeom)
+            ALLOC(L->w.codes[p], (size_t)E * MxGeom(N, K).expert_bytes());
+            (void)rows;
         } else {
             ALLOC(L->w.idx13[p], rows * row_bytes(fmt, 0, K));
             if (fmt == MOEQ_FMT_VQ13_R8) ALLOC(L->w.idx8[p], rows * row_bytes(fmt, 1, K));
@@ -228,13 +233,32 @@ moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *str
     if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaSuccess;
+    // MXFP4: copy the logical planes a batch of experts at a time into
+    // temporary device buffers and pack them into the device layout (MxGeom)
+    uint8_t *tmp_c = nullptr, *tmp_s = nullptr;
+    int batch = 1;
+    if (mx) {
+        const size_t per_expert = (size_t)H * I / 2 + (size_t)H * I / 32;   // largest projection
+        batch = (int)std::max<size_t>(1, ((size_t)64 << 20) / per_expert);
+        batch = std::min(batch, E);
+        e = dev_alloc((void **)&tmp_c, (size_t)batch * H * I / 2);
+        if (e == cudaSuccess) e = dev_alloc((void **)&tmp_s, (size_t)batch * H * I / 32);
+    }
     for (int p = 0; p < 3 && e == cudaSuccess; ++p) {
         const int N = (p == MOEQ_DOWN) ? H : I, K = (p == MOEQ_DOWN) ? I : H;
         const size_t rows = (size_t)E * N;
         if (mx) {
-            e = cudaMemcpyAsync(L->w.codes[p], w->codes[p], rows * row_bytes(fmt, 0, K), cudaMemcpyHostToDevice, s);
-            if (e == cudaSuccess)
-                e = cudaMemcpyAsync(L->w.scales[p], w->scales[p], rows * row_bytes(fmt, 1, K), cudaMemcpyHostToDevice, s);
+            const MxGeom geo(N, K);
+            for (int e0 = 0; e0 < E && e == cudaSuccess; e0 += batch) {
+                const int ne = std::min(batch, E - e0);
+                e = cudaMemcpyAsync(tmp_c, w->codes[p] + (size_t)e0 * N * (K / 2), (size_t)ne * N * (K / 2),
+                                    cudaMemcpyHostToDevice, s);
+                if (e == cudaSuccess)
+                    e = cudaMemcpyAsync(tmp_s, w->scales[p] + (size_t)e0 * N * (K / 32), (size_t)ne * N * (K / 32),
+                                        cudaMemcpyHostToDevice, s);
+                if (e == cudaSuccess)
+                    e = launch_mx_pack(tmp_c, tmp_s, L->w.codes[p] + (size_t)e0 * geo.expert_bytes(), geo, ne, s);
+            }
         } else {
             e = cudaMemcpyAsync(L->w.idx13[p], w->idx13[p], rows * row_bytes(fmt, 0, K), cudaMemcpyHostToDevice, s);
             if (e == cudaSuccess && r8)
@@ -243,16 +267,13 @@ moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *str
                 e = cudaMemcpyAsync(L->w.gain[p], w->gain[p], rows * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
         }
     }
-    // MXFP4 codes go to the device layout (64-byte groups word-transposed)
-    for (int p = 0; p < 3 && e == cudaSuccess && mx; ++p) {
-        const int N = (p == MOEQ_DOWN) ? H : I, K = (p == MOEQ_DOWN) ? I : H;
-        e = launch_mx_repack(L->w.codes[p], (size_t)E * N * row_bytes(fmt, 0, K), s);
-    }
     if (e == cudaSuccess && !mx)
         e = cudaMemcpyAsync(L->w.book13, w->book13, sizeof(uint16_t) * kBook13Rows * 8, cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess && r8)
         e = cudaMemcpyAsync(L->w.book8, w->book8, sizeof(uint16_t) * kBook8Rows * 8, cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaFree(tmp_c);
+    cudaFree(tmp_s);
     if (e != cudaSuccess) return from_cuda(e);
     L->w.has_gain = n_gain == 3;
     L->uploaded = true;

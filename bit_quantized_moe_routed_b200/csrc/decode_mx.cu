@@ -7,24 +7,28 @@
 // top-8 of 256 routed experts, MXFP4 experts with one E8M0 exponent per 32
 // values; "Recipe": expert intermediates stay in a type with f32's range).
 //
-// Memory: a unit is one expert's 16 gate + 16 up rows (gate/up kernel) or 32
-// down rows (down kernel) over the full K.  Its rows are contiguous in HBM,
-// so one warp moves a whole unit into shared memory with 1-D bulk copies
-// (TMA, one per row, rows padded so that the A-fragment reads below hit
-// distinct banks) and signals an mbarrier; a ring of stages keeps the next
-// unit(s) in flight while the current one is computed.  One CTA per SM.
+// Work: a unit is one expert's 16 gate + 16 up rows (gate/up kernel) or 32
+// down rows (down kernel) over the full K; each CTA (one per SM) takes a
+// contiguous, balanced range of units, and each of its 16 consumer warps
+// owns whole units, so no reduction or barrier sits in the main loop.
+//
+// Memory: the device layout (MxGeom) keeps each (16-row tile, 1024-column
+// chunk) block contiguous, so a producer warp streams a chunk of a unit as
+// two 8.7 KB bulk copies (TMA) into a ring of 8 shared-memory stages with
+// full/empty mbarriers, in the order the consumers take them (units in waves
+// of 16, chunk by chunk).  Bulk copies of several KB are what keep HBM busy;
+// the layout also makes the fragment and scale reads bank-conflict free.
 //
 // Math: warp-level mma.sync.m16n8k16 (f16 in, f32 accumulate).  Each thread
 // reads its A-fragment slice of four 32-weight blocks (bytes 4t..4t+3 of
-// each block; the upload transposes the words of each 64-byte group so the
-// slice is one 16-byte word) and decodes it with cvt.rn.f16x2.e2m1x2
-// (exact).  Per block the two MMAs accumulate into a fresh fragment that is
-// folded into the running f32 sum times the block's E8M0 scale, so the scale
-// is applied exactly.  The B operand (activations, or w * h for the down
-// projection) is f16 after a per-token power-of-two prescale that puts the
-// largest magnitude in [2^14, 2^15): f16 cannot overflow, and the scale is
-// undone in f32.  The 16 warps split K; their fragments are summed through
-// shared memory.
+// each block: one 16-byte word in the layout) and decodes it with
+// cvt.rn.f16x2.e2m1x2 (exact).  Per block the two MMAs accumulate into a
+// fresh fragment that is folded into the running f32 sum times the block's
+// E8M0 scale (one packed f32x2 FMA per row pair), so the scale is applied
+// exactly.  The B operand (activations, or w * h for the down projection) is
+// f16 after a per-token power-of-two prescale that puts the largest
+// magnitude in [2^14, 2^15): f16 cannot overflow, and the scale is undone in
+// f32.
 //
 // Combine: the down kernel writes each expert's contribution to its own
 // slice of a scratch buffer; the last unit to finish a 32-row tile
@@ -147,6 +151,29 @@ __device__ __forceinline__ float e8m0_byte(uint32_t word, int j) {
     return __uint_as_float(max(b << 23, 0x00400000u));
 }
 
+// Four E8M0 bytes (one scale word) -> four f32 scales, exact: two
+// cvt.rn.bf16x2.ue8m0x2 (2^(b-127) is a bf16 value, the subnormal 2^-127
+// for b = 0 included), then bf16 -> f32 by position.
+__device__ __forceinline__ void e8m0x4(uint32_t w, float s[4]) {
+    uint32_t lo, hi;
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.bf16x2.ue8m0x2 %0, a;\n\tcvt.rn.bf16x2.ue8m0x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+    s[0] = __uint_as_float(lo << 16);
+    s[1] = __uint_as_float(lo & 0xFFFF0000u);
+    s[2] = __uint_as_float(hi << 16);
+    s[3] = __uint_as_float(hi & 0xFFFF0000u);
+}
+
+// (a0, a1) += s * (b0, b1) with one packed f32x2 FMA.
+__device__ __forceinline__ void ffma2(float &a0, float &a1, float s, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\tmov.b64 ra, {%2, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
+        "mov.b64 rc, {%0, %1};\n\tfma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(s), "f"(b0), "f"(b1));
+}
+
 // One 32-weight block of a 16-row A tile: rows g (word wa) and g+8 (word wb),
 // thread slice bytes 4t..4t+3, against B fragment {x01, x23, x45, x67}.
 // acc += scale_g * blk (rows g) and scale_g8 * blk (rows g+8).
@@ -157,214 +184,288 @@ __device__ __forceinline__ void block_mma(float acc[4], uint32_t wa, uint32_t wb
     float c[4];
     mma_f16_zero(c, a0, b0, a1, b1, xb.x, xb.y);
     mma_f16(c, a2, b2, a3, b3, xb.z, xb.w);
-    acc[0] = fmaf(sa, c[0], acc[0]);
-    acc[1] = fmaf(sa, c[1], acc[1]);
-    acc[2] = fmaf(sb, c[2], acc[2]);
-    acc[3] = fmaf(sb, c[3], acc[3]);
+    ffma2(acc[0], acc[1], sa, c[0], c[1]);
+    ffma2(acc[2], acc[3], sb, c[2], c[3]);
 }
 
 __device__ __forceinline__ uint32_t u4get(const uint4 &v, int j) {
     return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
 
-// After a timed-out wait: wait (bounded again) for the copies of the units
-// after it that were already issued, so none lands in shared memory after
-// the CTA has gone.
-__device__ void drain_stages(uint64_t *full, int n_stages, int j0, int n_units) {
-    for (int j = j0; j < j0 + n_stages - 1; ++j) {
-        if ((int)blockIdx.x + j * (int)gridDim.x >= n_units) break;
-        mbar_wait_bounded(&full[j % n_stages], (uint32_t)((j / n_stages) & 1), 200000000LL);
+constexpr int kCW = 16;   // consumer warps per CTA
+
+// Barrier among the kCW consumer warps (id 1; the producer warp does not join).
+__device__ __forceinline__ void named_sync_consumers() {
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kCW) : "memory");
+}
+
+// ---------------------------------------------------------------- staging
+
+// Warp roles: kCW consumer warps, each owning whole units, plus one producer
+// warp that streams (tile, chunk) blocks into a ring of shared-memory stages.
+constexpr int kWSThreads = 32 * (kCW + 1);
+constexpr int kProducerWarp = kCW;
+constexpr int kKC = 1024;                       // weights of K per chunk (the layout's chunk)
+constexpr int kBlk = 16 * (kKC / 2 + kKC / 32); // one (16-row tile, chunk) block of the device layout
+constexpr int kStageBytes = 2 * kBlk;           // two blocks: gate + up tile, or two down tiles
+constexpr int kMaxStages = 8;
+constexpr int kMaxDynSmem = 232448 - 4096;      // leave room for static shared memory
+
+// Producer (one thread): two contiguous blocks of the device layout into
+// stage `st`, completing `bar`.
+__device__ __forceinline__ void issue_chunk(uint8_t *st, uint64_t *bar, const uint8_t *blk0, const uint8_t *blk1) {
+    mbar_arrive_expect_tx(bar, 2u * kBlk);
+    bulk_g2s(st, blk0, kBlk, bar);
+    bulk_g2s(st + kBlk, blk1, kBlk, bar);
+}
+
+// Shared-memory address of this thread's fragment word (bytes 4t..4t+3 of
+// the four blocks of K-group grp) of staged row r (0..15) of a block.
+__device__ __forceinline__ const uint8_t *frag_ptr(const uint8_t *blk, int r, int grp, int t) {
+    return blk + (size_t)r * (kKC / 2) + ((grp ^ (r & 1)) * 64) + 16 * t;
+}
+// ... and of the scale word (four blocks) of row r, K-group grp.
+__device__ __forceinline__ const uint8_t *scale_ptr(const uint8_t *blk, int r, int grp) {
+    return blk + 16 * (kKC / 2) + grp * 64 + r * 4;
+}
+
+// This CTA's contiguous share [beg, end) of n units.
+__device__ __forceinline__ void my_range(int n, int &beg, int &end) {
+    beg = (int)(((long long)n * blockIdx.x) / gridDim.x);
+    end = (int)(((long long)n * (blockIdx.x + 1)) / gridDim.x);
+}
+
+// Chunk order shared by producer and consumers: units go in waves of kCW
+// (warp w takes unit w of each wave); within a wave, chunk q of every unit
+// comes before chunk q+1.  Returns the global chunk index of (unit j of this
+// CTA's range, chunk q).
+__device__ __forceinline__ int chunk_index(int j, int q, int n_mine, int nch) {
+    const int wave = j / kCW, wbeg = wave * kCW;
+    const int wn = min(kCW, n_mine - wbeg);
+    return wbeg * nch + q * wn + (j - wbeg);
+}
+
+// Producer loop: chunk c of this CTA, in the order above.  After issuing
+// chunk c it publishes issued = c + 1.  Chunk c reuses the stage of chunk
+// c - S only after that chunk's consumer released it, so a consumer that has
+// seen issued > c knows the stage's barrier is in the phase of chunk c; this
+// keeps a warp that runs ahead of the others (it waits on a stage whose
+// previous chunk, another warp's, is still in flight) from matching the
+// parity of a phase two rounds old.
+template <typename BlockOf>
+__device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_t *empty, int S, int n_mine, int nch,
+                                        uint32_t *status, volatile int *issued, BlockOf block_of) {
+    const int lane = threadIdx.x & 31;
+    int c = 0;
+    for (int wbeg = 0; wbeg < n_mine; wbeg += kCW) {
+        const int wn = min(kCW, n_mine - wbeg);
+        for (int q = 0; q < nch; ++q)
+            for (int jj = 0; jj < wn; ++jj, ++c) {
+                const int s = c % S, kk = c / S;
+                if (lane == 0) {
+                    if (kk >= 1 && !mbar_wait_bounded(&empty[s], (uint32_t)((kk - 1) & 1)))
+                        atomicOr(status, FLAG_TIMEOUT);
+                    const uint8_t *b0, *b1;
+                    block_of(wbeg + jj, q, b0, b1);
+                    issue_chunk(stages + (size_t)s * kStageBytes, &full[s], b0, b1);
+                    __threadfence_block();
+                    *issued = c + 1;
+                }
+                __syncwarp();
+            }
     }
+}
+
+// Consumer: wait until chunk c is issued, then for its data.  False on timeout.
+__device__ __forceinline__ bool wait_chunk(uint64_t *full, int S, int c, volatile int *issued) {
+    if (*issued <= c) {
+        const long long t0 = clock64();
+        while (*issued <= c) {
+            if (clock64() - t0 > 2000000000LL) return false;
+            __nanosleep(32);
+        }
+    }
+    __threadfence_block();
+    return mbar_wait_bounded(&full[c % S], (uint32_t)((c / S) & 1));
 }
 
 // ---------------------------------------------------------------- gate/up
 
 struct GateUpArgs {
-    const uint8_t *codes_g, *codes_u, *scales_g, *scales_u;
-    const uint16_t *x;      // bf16 [T][H]
-    const int32_t *ids;     // [T][k]
-    const float *topk_w;    // [T][k]
-    float *h;               // [T*k][I] f32, by route id
-    float *gmax;            // [gridDim.x][kMaxT]: per-CTA max |w h| per token
+    const uint8_t *codes_g, *codes_u;   // gate, up projections in the device layout (MxGeom)
+    const uint16_t *x;                  // bf16 [T][H]
+    const int32_t *ids;                 // [T][k]
+    const float *topk_w;                // [T][k]
+    float *h;                           // [T*k][I] f32, by route id
+    float *gmax;                        // [gridDim.x][kMaxT]: per-CTA max |w h| per token
     uint32_t *status;
-    int T, k, E, H, I;
+    int T, k, E, H, I, n_stages;
 };
 
-constexpr int kGUStages = 2;
-constexpr int kRowPad = 64;    // bytes after each staged code row
-constexpr int kScalePad = 16;  // bytes after each staged scale row
-
-struct GULayout {
-    int row_stride, sc_stride, stage_bytes, xs_stride;
-    __host__ __device__ GULayout(int H) {
-        row_stride = H / 2 + kRowPad;
-        sc_stride = H / 32 + kScalePad;
-        stage_bytes = 32 * row_stride + 32 * sc_stride;
-        xs_stride = H + kXPad;
-    }
-    // [stages][stage] [x16: T rows] [red: 16 warps x 32 lanes x 8]
-    __host__ __device__ size_t xs_off() const { return (size_t)kGUStages * stage_bytes; }
-    __host__ __device__ size_t red_off(int T) const { return xs_off() + sizeof(uint16_t) * (size_t)T * xs_stride; }
-    __host__ __device__ size_t bytes(int T) const { return red_off(T) + sizeof(float) * kWarps * 32 * 8; }
-};
-
-// Warp 0: put unit j's 16 gate + 16 up rows and their scale rows in stage j % kGUStages.
-__device__ __forceinline__ void gu_issue(const GateUpArgs &a, const RouteTable &tb, const GULayout &ly,
-                                         uint8_t *stages, uint64_t *full, int j, int n_units) {
-    const int u = blockIdx.x + j * gridDim.x;
-    if (u >= n_units) return;
-    const int lane = threadIdx.x & 31;
-    const int tiles = a.I / 16;
-    const int d = u / tiles, n0 = (u % tiles) * 16;
-    const size_t row0 = (size_t)tb.expert[d] * a.I + n0;
-    uint8_t *st = stages + (size_t)(j % kGUStages) * ly.stage_bytes;
-    uint64_t *bar = full + (j % kGUStages);
-    const uint32_t code_b = a.H / 2, sc_b = a.H / 32;
-    if (lane == 0) mbar_arrive_expect_tx(bar, 32u * (code_b + sc_b));
-    __syncwarp();
-    const int mat = lane >> 4, r = lane & 15;   // lane -> (gate|up, row)
-    const uint8_t *codes = mat ? a.codes_u : a.codes_g;
-    const uint8_t *scales = mat ? a.scales_u : a.scales_g;
-    bulk_g2s(st + (size_t)(mat * 16 + r) * ly.row_stride, codes + (row0 + r) * code_b, code_b, bar);
-    bulk_g2s(st + (size_t)32 * ly.row_stride + (size_t)(mat * 16 + r) * ly.sc_stride, scales + (row0 + r) * sc_b,
-             sc_b, bar);
+__host__ __device__ inline size_t gu_xs_off(int n_stages) { return (size_t)n_stages * kStageBytes; }
+__host__ __device__ inline size_t gu_bytes(int n_stages, int T, int H) {
+    return gu_xs_off(n_stages) + sizeof(uint16_t) * (size_t)T * (H + kXPad);
 }
 
-// NG = groups of four 32-weight blocks per warp's K slice = H / 2048.
-template <int NG>
-__global__ void __launch_bounds__(kThreads, 1) dec_gateup_mx_kernel(GateUpArgs a) {
+// Unit i -> (expert slot d, column chunk, 16-row tile): experts with more
+// than 8 routes take one pass per 8 columns.
+struct GUItems {
+    int n;
+    int beg[kMaxR + 1];
+};
+
+template <int NCH>   // K chunks per unit = H / kKC
+__global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ RouteTable tb;
-    __shared__ __align__(8) uint64_t full[kGUStages];
+    __shared__ GUItems items;
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
+    __shared__ int issued;   // chunks issued by the producer (see produce)
     __shared__ float xinv[kMaxT];
     __shared__ unsigned cta_max[kMaxT];
-    const int H = a.H, I = a.I, T = a.T, k = a.k;
-    const GULayout ly(H);
+    const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages;
     uint8_t *stages = smem_raw;
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw + ly.xs_off());
-    float *red = reinterpret_cast<float *>(smem_raw + ly.red_off(T));
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw + gu_xs_off(S));
+    const int xs_stride = H + kXPad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
+    const int tiles = I / 16;
+    const MxGeom geo(I, H);
 
     if (tid == 0) {
-        for (int s = 0; s < kGUStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
         mbar_fence_init();
+        issued = 0;
     }
     if (tid < kMaxT) cta_max[tid] = 0u;
-    if (warp == 0) build_route_table(tb, a.ids, T * k, a.E, a.status, blockIdx.x == 0);
+    if (warp == 0) {
+        build_route_table(tb, a.ids, T * k, a.E, a.status, blockIdx.x == 0);
+        __syncwarp();
+        if (lane == 0) {
+            int n = 0;
+            for (int d = 0; d < tb.D; ++d) {
+                items.beg[d] = n;
+                n += ((tb.col_beg[d + 1] - tb.col_beg[d] + 7) / 8) * tiles;
+            }
+            items.beg[tb.D] = n;
+            items.n = n;
+        }
+    }
     __syncthreads();
-    const int tiles = I / 16;
-    const int n_units = tb.D * tiles;
-    if (warp == 0)
-        for (int j = 0; j < kGUStages; ++j) gu_issue(a, tb, ly, stages, full, j, n_units);
-    // let the down kernel's CTAs launch as SMs free up (they wait for this
-    // grid before reading h)
-    pdl_launch_dependents();
-    // stage x as f16 with a per-token power-of-two prescale (warp w+1 <-> token w)
-    if (warp >= 1 && warp <= T) {
-        const int tk = warp - 1;
-        const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)tk * H);
+    int i0, i1;
+    my_range(items.n, i0, i1);
+    const int n_mine = i1 - i0;
+    auto decode_item = [&](int i, int &d, int &rel) {
+        d = 0;
+        while (items.beg[d + 1] <= i) ++d;
+        rel = i - items.beg[d];
+    };
+
+    if (warp == kProducerWarp) {
+        produce(stages, full, empty, S, n_mine, NCH, a.status, &issued, [&](int j, int q, const uint8_t *&b0, const uint8_t *&b1) {
+            int d, rel;
+            decode_item(i0 + j, d, rel);
+            const size_t off = (size_t)tb.expert[d] * geo.expert_bytes() + geo.block_off(rel % tiles, q);
+            b0 = a.codes_g + off;
+            b1 = a.codes_u + off;
+        });
+        return;
+    }
+
+    // ---- consumers: stage x as f16 with a per-token power-of-two prescale
+    // (warp w <-> token w)
+    if (warp < T) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)warp * H);
         float m = 0.f;
         for (int i = lane; i < H / 8; i += 32) {
             uint4 v = xr[i];
-            uint32_t q[4] = {v.x, v.y, v.z, v.w};
+            uint32_t qv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                m = fmaxf(m, fmaxf(fabsf(__uint_as_float(q[j] << 16)), fabsf(__uint_as_float(q[j] & 0xFFFF0000u))));
+                m = fmaxf(m, fmaxf(fabsf(__uint_as_float(qv[j] << 16)), fabsf(__uint_as_float(qv[j] & 0xFFFF0000u))));
         }
 #pragma unroll
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         const int s = prescale_exp(m);
         const float sc = exp2i(s);
-        if (lane == 0) xinv[tk] = exp2i(-s);
-        uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)tk * ly.xs_stride);
+        if (lane == 0) xinv[warp] = exp2i(-s);
+        uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)warp * xs_stride);
         for (int i = lane; i < H / 8; i += 32) {
             uint4 v = xr[i];
-            uint32_t q[4] = {v.x, v.y, v.z, v.w}, o[4];
+            uint32_t qv[4] = {v.x, v.y, v.z, v.w}, o[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                __half2 hv = __floats2half2_rn(__uint_as_float(q[j] << 16) * sc,
-                                               __uint_as_float(q[j] & 0xFFFF0000u) * sc);
+                __half2 hv = __floats2half2_rn(__uint_as_float(qv[j] << 16) * sc,
+                                               __uint_as_float(qv[j] & 0xFFFF0000u) * sc);
                 o[j] = *reinterpret_cast<uint32_t *>(&hv);
             }
             dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
         }
     }
-    __syncthreads();
+    named_sync_consumers();
 
-    for (int j = 0;; ++j) {
-        const int u = blockIdx.x + j * gridDim.x;
-        if (u >= n_units) break;
-        const uint32_t parity = (uint32_t)((j / kGUStages) & 1);
-        const bool ok = mbar_wait_bounded(&full[j % kGUStages], parity);
-        // also keeps red[] from being rewritten before the last unit's readers finish
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) {
-                atomicOr(a.status, FLAG_TIMEOUT);
-                drain_stages(full, kGUStages, j + 1, n_units);
-            }
-            break;
-        }
-        const int d = u / tiles, n0 = (u % tiles) * 16;
-        const uint8_t *st = stages + (size_t)(j % kGUStages) * ly.stage_bytes;
-        for (int cb = tb.col_beg[d]; cb < tb.col_beg[d + 1]; cb += 8) {
-            if (cb > tb.col_beg[d]) __syncthreads();   // red[] reuse within a unit
-            const int ncol = min(8, tb.col_beg[d + 1] - cb);
-            const bool live = g < ncol;
-            const int tok = live ? tb.route[cb + g] / k : 0;
-            const uint16_t *xrow = xs + (size_t)tok * ly.xs_stride + 8 * t;
-            float aG[4] = {0.f, 0.f, 0.f, 0.f}, aU[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int G = 0; G < NG; ++G) {
-                const int gg = warp * NG + G;   // group index within the row
-                const uint8_t *cp = st + (size_t)g * ly.row_stride + gg * 64 + 16 * t;
-                const uint4 ag0 = lds128(cp), ag8 = lds128(cp + 8 * ly.row_stride);
-                const uint4 au0 = lds128(cp + 16 * ly.row_stride), au8 = lds128(cp + 24 * ly.row_stride);
-                const uint8_t *sp = st + (size_t)32 * ly.row_stride + (size_t)g * ly.sc_stride + gg * 4;
-                const uint32_t sg0 = lds32(sp), sg8 = lds32(sp + 8 * ly.sc_stride);
-                const uint32_t su0 = lds32(sp + 16 * ly.sc_stride), su8 = lds32(sp + 24 * ly.sc_stride);
+    bool timed_out = false;
+    for (int j = warp; j < n_mine; j += kCW) {
+        int d, rel;
+        decode_item(i0 + j, d, rel);
+        const int cb = tb.col_beg[d] + (rel / tiles) * 8, n0 = (rel % tiles) * 16;
+        const int ncol = min(8, tb.col_beg[d + 1] - cb);
+        const bool live = g < ncol;
+        const int tok = live ? tb.route[cb + g] / k : 0;
+        const uint16_t *xrow = xs + (size_t)tok * xs_stride + 8 * t;
+        float aG[4] = {0.f, 0.f, 0.f, 0.f}, aU[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int q = 0; q < NCH; ++q) {
+            const int c = chunk_index(j, q, n_mine, NCH), s = c % S;
+            if (!wait_chunk(full, S, c, &issued)) timed_out = true;
+            const uint8_t *st = stages + (size_t)s * kStageBytes;
+#pragma unroll 2
+            for (int gp = 0; gp < kKC / 128; ++gp) {   // K-groups of four 32-weight blocks
+                // stage = [gate block][up block]; rows g and g+8 of each
+                const uint4 ag0 = lds128(frag_ptr(st, g, gp, t)), ag8 = lds128(frag_ptr(st, g + 8, gp, t));
+                const uint4 au0 = lds128(frag_ptr(st + kBlk, g, gp, t));
+                const uint4 au8 = lds128(frag_ptr(st + kBlk, g + 8, gp, t));
+                float sg0[4], sg8[4], su0[4], su8[4];
+                e8m0x4(lds32(scale_ptr(st, g, gp)), sg0);
+                e8m0x4(lds32(scale_ptr(st, g + 8, gp)), sg8);
+                e8m0x4(lds32(scale_ptr(st + kBlk, g, gp)), su0);
+                e8m0x4(lds32(scale_ptr(st + kBlk, g + 8, gp)), su8);
+                const uint16_t *xq = xrow + (size_t)(q * (kKC / 32) + gp * 4) * 32;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const uint4 xb = live ? lds128(xrow + (gg * 4 + jj) * 32) : make_uint4(0u, 0u, 0u, 0u);
-                    block_mma(aG, u4get(ag0, jj), u4get(ag8, jj), xb, e8m0_byte(sg0, jj), e8m0_byte(sg8, jj));
-                    block_mma(aU, u4get(au0, jj), u4get(au8, jj), xb, e8m0_byte(su0, jj), e8m0_byte(su8, jj));
+                    const uint4 xb = live ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
+                    block_mma(aG, u4get(ag0, jj), u4get(ag8, jj), xb, sg0[jj], sg8[jj]);
+                    block_mma(aU, u4get(au0, jj), u4get(au8, jj), xb, su0[jj], su8[jj]);
                 }
             }
-            float4 *mine = reinterpret_cast<float4 *>(red + ((size_t)warp * 32 + lane) * 8);
-            mine[0] = make_float4(aG[0], aG[1], aG[2], aG[3]);
-            mine[1] = make_float4(aU[0], aU[1], aU[2], aU[3]);
-            __syncthreads();
-            // every warp is done reading this stage: refill it with unit j + kGUStages
-            if (warp == 0 && cb + 8 >= tb.col_beg[d + 1]) gu_issue(a, tb, ly, stages, full, j + kGUStages, n_units);
-            if (tid < 128) {
-                const int row = tid >> 3, col = tid & 7;   // 16 rows x 8 columns
-                if (col < ncol) {
-                    const int gl = row & 7, hi = row >> 3, tl = col >> 1, cbit = col & 1;
-                    const int src_lane = gl * 4 + tl, slot = hi * 2 + cbit;
-                    float gs = 0.f, us = 0.f;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);   // this warp is done with the stage
+        }
+        // epilogue: rows (g, g+8) x columns (2t, 2t+1)
 #pragma unroll
-                    for (int ww = 0; ww < kWarps; ++ww) {
-                        gs += red[((size_t)ww * 32 + src_lane) * 8 + slot];
-                        us += red[((size_t)ww * 32 + src_lane) * 8 + 4 + slot];
-                    }
-                    const int route = tb.route[cb + col];
-                    const float inv = xinv[route / k];
-                    const float hv = silu_f32(gs * inv) * (us * inv);
-                    a.h[(size_t)route * I + n0 + row] = hv;
-                    const float wh = fabsf(a.topk_w[route] * hv);
-                    if (wh > 0.f) atomicMax(&cta_max[route / k], __float_as_uint(isfinite(wh) ? wh : 3.0e38f));
-                }
+        for (int e = 0; e < 4; ++e) {
+            const int row = g + 8 * (e >> 1), col = 2 * t + (e & 1);
+            if (col < ncol) {
+                const int route = tb.route[cb + col];
+                const float inv = xinv[route / k];
+                const float hv = silu_f32(aG[e] * inv) * (aU[e] * inv);
+                a.h[(size_t)route * I + n0 + row] = hv;
+                const float wh = fabsf(a.topk_w[route] * hv);
+                if (wh > 0.f) atomicMax(&cta_max[route / k], __float_as_uint(isfinite(wh) ? wh : 3.0e38f));
             }
         }
     }
-    __syncthreads();
+    if (timed_out && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
+    named_sync_consumers();
     if (tid < kMaxT) a.gmax[(size_t)blockIdx.x * kMaxT + tid] = __uint_as_float(cta_max[tid]);
 }
 
 // ---------------------------------------------------------------- down
 
 struct DownArgs {
-    const uint8_t *codes, *scales;  // down projection [E][H][I/2] (device layout), [E][H][I/32]
+    const uint8_t *codes;           // down projection in the device layout (MxGeom)
     const float *h;                 // [T*k][I]
     const float *gmax;              // [n_gmax][kMaxT]
     int n_gmax;
@@ -374,197 +475,210 @@ struct DownArgs {
     int *counters;                  // [H/32], zero between calls
     uint16_t *out;                  // bf16 [T][H]
     uint32_t *status;
-    int T, k, E, H, I;
+    int T, k, E, H, I, n_stages;
 };
 
-constexpr int kDNStages = 4;
+constexpr int kMaxBSlots = 16;   // staged (expert, token) B columns per CTA
 
-struct DNLayout {
-    int row_stride, sc_stride, stage_bytes;
-    __host__ __device__ DNLayout(int I) {
-        row_stride = I / 2 + kRowPad;
-        sc_stride = I / 32 + kScalePad;
-        stage_bytes = 32 * row_stride + 32 * sc_stride;
-    }
-    __host__ __device__ size_t red_off() const { return (size_t)kDNStages * stage_bytes; }
-    __host__ __device__ size_t bytes() const { return red_off() + sizeof(float) * kWarps * 32 * 8; }
-};
-
-__device__ __forceinline__ void dn_issue(const DownArgs &a, const RouteTable &tb, const DNLayout &ly,
-                                         uint8_t *stages, uint64_t *full, int j, int n_units) {
-    const int u = blockIdx.x + j * gridDim.x;
-    if (u >= n_units) return;
-    const int lane = threadIdx.x & 31;
-    const int tiles = a.H / 32;
-    const int d = u / tiles, m0 = (u % tiles) * 32;
-    const size_t row = (size_t)tb.expert[d] * a.H + m0 + lane;
-    uint8_t *st = stages + (size_t)(j % kDNStages) * ly.stage_bytes;
-    uint64_t *bar = full + (j % kDNStages);
-    const uint32_t code_b = a.I / 2, sc_b = a.I / 32;
-    if (lane == 0) mbar_arrive_expect_tx(bar, 32u * (code_b + sc_b));
-    __syncwarp();
-    bulk_g2s(st + (size_t)lane * ly.row_stride, a.codes + row * code_b, code_b, bar);
-    bulk_g2s(st + (size_t)32 * ly.row_stride + (size_t)lane * ly.sc_stride, a.scales + row * sc_b, sc_b, bar);
+__host__ __device__ inline size_t dn_bytes(int n_stages, int I) {
+    return (size_t)n_stages * kStageBytes + sizeof(uint16_t) * (size_t)kMaxBSlots * (I + kXPad);
 }
 
-// NG = groups of four 32-weight blocks per warp's K slice = I / 2048.
-template <int NG>
-__global__ void __launch_bounds__(kThreads, 1) dec_down_mx_kernel(DownArgs a) {
+template <int NCH>   // K chunks per unit = I / kKC
+__global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ RouteTable tb;
-    __shared__ __align__(8) uint64_t full[kDNStages];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
+    __shared__ int issued;   // chunks issued by the producer (see produce)
     __shared__ float tok_scale[kMaxT], tok_inv[kMaxT];
-    __shared__ float rscale[kMaxR];
-    __shared__ int last_flag;
-    const int H = a.H, I = a.I, T = a.T, k = a.k;
-    const DNLayout ly(I);
+    __shared__ int slot_of[kMaxR][kMaxT];   // (expert slot - d_lo, token) -> staged B column, -1 none
+    __shared__ int slot_d[kMaxBSlots], slot_t[kMaxBSlots];
+    __shared__ int n_slots;
+    const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages;
     uint8_t *stages = smem_raw;
-    float *red = reinterpret_cast<float *>(smem_raw + ly.red_off());
+    uint16_t *bs = reinterpret_cast<uint16_t *>(smem_raw + (size_t)S * kStageBytes);   // [slot][I+pad] f16
+    const int bs_stride = I + kXPad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
+    const int tiles = H / 32;
+    const MxGeom geo(H, I);
 
     if (tid == 0) {
-        for (int s = 0; s < kDNStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
         mbar_fence_init();
+        issued = 0;
     }
     if (warp == 0) build_route_table(tb, a.ids, T * k, a.E, nullptr, false);
     __syncthreads();
-    const int tiles = H / 32;
     const int n_units = tb.D * tiles;
     if (tb.D == 0) {   // no valid route at all: every output is zero
-        for (int i = blockIdx.x * kThreads + tid; i < T * H; i += gridDim.x * kThreads) a.out[i] = 0;
+        for (int i = blockIdx.x * kWSThreads + tid; i < T * H; i += gridDim.x * kWSThreads) a.out[i] = 0;
         return;
     }
-    // the weights do not depend on the gate/up kernel: start streaming them now
-    if (warp == 0)
-        for (int j = 0; j < kDNStages; ++j) dn_issue(a, tb, ly, stages, full, j, n_units);
+    int u0, u1;
+    my_range(n_units, u0, u1);
+    const int n_mine = u1 - u0;
+
+    if (warp == kProducerWarp) {
+        // the weights do not depend on the gate/up kernel: stream them at once
+        produce(stages, full, empty, S, n_mine, NCH, a.status, &issued, [&](int j, int q, const uint8_t *&b0, const uint8_t *&b1) {
+            const int u = u0 + j, d = u / tiles, t32 = u % tiles;
+            const uint8_t *eb = a.codes + (size_t)tb.expert[d] * geo.expert_bytes();
+            b0 = eb + geo.block_off(2 * t32, q);
+            b1 = eb + geo.block_off(2 * t32 + 1, q);
+        });
+        return;
+    }
+
+    // the experts this CTA's units touch, and their (expert, token) columns
+    const int d_lo = n_mine > 0 ? u0 / tiles : 0, d_hi = n_mine > 0 ? (u1 - 1) / tiles : -1;
+    if (tid == 0) {
+        int ns = 0;
+        for (int d = d_lo; d <= d_hi; ++d)
+            for (int tk = 0; tk < T; ++tk) {
+                bool used = false;
+                for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) used |= (tb.route[cc] / k == tk);
+                int sl = -1;
+                if (used) {
+                    if (ns < kMaxBSlots) {
+                        slot_d[ns] = d;
+                        slot_t[ns] = tk;
+                    }
+                    sl = ns++;
+                }
+                slot_of[d - d_lo][tk] = sl;
+            }
+        n_slots = ns;
+    }
     // h and gmax come from the gate/up kernel
     pdl_wait_primary();
-    if (warp >= 1 && warp <= kMaxT) {
-        const int tk = warp - 1;
+    if (warp < kMaxT) {
         float m = 0.f;
-        for (int i = lane; i < a.n_gmax; i += 32) m = fmaxf(m, __ldcg(a.gmax + (size_t)i * kMaxT + tk));
+        for (int i = lane; i < a.n_gmax; i += 32) m = fmaxf(m, __ldcg(a.gmax + (size_t)i * kMaxT + warp));
 #pragma unroll
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) {
             const int s = prescale_exp(m);
-            tok_scale[tk] = exp2i(s);
-            tok_inv[tk] = exp2i(-s);
+            tok_scale[warp] = exp2i(s);
+            tok_inv[warp] = exp2i(-s);
         }
     }
-    __syncthreads();
-    if (tid < T * k) rscale[tid] = a.topk_w[tid] * tok_scale[tid / k];
-    __syncthreads();
-
-    for (int j = 0;; ++j) {
-        const int u = blockIdx.x + j * gridDim.x;
-        if (u >= n_units) break;
-        const int d = u / tiles, tile = u % tiles, m0 = tile * 32;
-        // B column g = token g: sum over the token's routes to this expert of
-        // w * prescale * h, this warp's K slice (loads issued before the wait)
-        const bool live = g < T;
-        float bsum[NG][4][8];
-#pragma unroll
-        for (int G = 0; G < NG; ++G)
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) bsum[G][jj][i] = 0.f;
-        if (live) {
+    named_sync_consumers();
+    const bool staged = n_slots <= kMaxBSlots;
+    if (staged) {
+        // B column (d, token) = sum over the token's routes to expert d of
+        // w * prescale * h, as f16 (summed in f32 first)
+        for (int idx = tid; idx < n_slots * (I / 8); idx += 32 * kCW) {
+            const int sl = idx / (I / 8), k8 = (idx % (I / 8)) * 8;
+            const int d = slot_d[sl], tk = slot_t[sl];
+            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) {
                 const int r = tb.route[cc];
-                if (r / k != g) continue;
-                const float rs = rscale[r];
-                const float *hp = a.h + (size_t)r * I + (size_t)warp * NG * 128 + 8 * t;
+                if (r / k != tk) continue;
+                const float rs = a.topk_w[r] * tok_scale[tk];
+                const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(a.h + (size_t)r * I + k8));
+                const float4 h1 = __ldcg(reinterpret_cast<const float4 *>(a.h + (size_t)r * I + k8 + 4));
+                v[0] = fmaf(rs, h0.x, v[0]); v[1] = fmaf(rs, h0.y, v[1]); v[2] = fmaf(rs, h0.z, v[2]);
+                v[3] = fmaf(rs, h0.w, v[3]); v[4] = fmaf(rs, h1.x, v[4]); v[5] = fmaf(rs, h1.y, v[5]);
+                v[6] = fmaf(rs, h1.z, v[6]); v[7] = fmaf(rs, h1.w, v[7]);
+            }
+            __half2 p0 = __floats2half2_rn(v[0], v[1]), p1 = __floats2half2_rn(v[2], v[3]);
+            __half2 p2 = __floats2half2_rn(v[4], v[5]), p3 = __floats2half2_rn(v[6], v[7]);
+            *reinterpret_cast<uint4 *>(bs + (size_t)sl * bs_stride + k8) =
+                make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
+                           *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
+        }
+        named_sync_consumers();
+    }
+
+    bool timed_out = false;
+    for (int j = warp; j < n_mine; j += kCW) {
+        const int u = u0 + j;
+        const int d = u / tiles, tile = u % tiles, m0 = tile * 32;
+        const int my_slot = (g < T) ? slot_of[d - d_lo][g] : -1;   // B column g = token g
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int q = 0; q < NCH; ++q) {
+            const int c = chunk_index(j, q, n_mine, NCH), s = c % S;
+            if (!wait_chunk(full, S, c, &issued)) timed_out = true;
+            const uint8_t *st = stages + (size_t)s * kStageBytes;
+#pragma unroll 2
+            for (int gp = 0; gp < kKC / 128; ++gp) {
+                const int kbase = q * kKC + gp * 128 + 8 * t;   // this thread's first K of block 0
+                uint4 xb[4];
+                if (staged) {
 #pragma unroll
-                for (int G = 0; G < NG; ++G)
+                    for (int jj = 0; jj < 4; ++jj)
+                        xb[jj] = my_slot >= 0 ? lds128(bs + (size_t)my_slot * bs_stride + kbase + jj * 32)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+                } else {
+                    // more columns than staged slots: build B from h in L2
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
-                        const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(hp + (4 * G + jj) * 32));
-                        const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(hp + (4 * G + jj) * 32 + 4));
-                        float *bb = bsum[G][jj];
-                        bb[0] = fmaf(rs, v0.x, bb[0]);
-                        bb[1] = fmaf(rs, v0.y, bb[1]);
-                        bb[2] = fmaf(rs, v0.z, bb[2]);
-                        bb[3] = fmaf(rs, v0.w, bb[3]);
-                        bb[4] = fmaf(rs, v1.x, bb[4]);
-                        bb[5] = fmaf(rs, v1.y, bb[5]);
-                        bb[6] = fmaf(rs, v1.z, bb[6]);
-                        bb[7] = fmaf(rs, v1.w, bb[7]);
+                        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        if (g < T)
+                            for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) {
+                                const int r = tb.route[cc];
+                                if (r / k != g) continue;
+                                const float rs = a.topk_w[r] * tok_scale[g];
+                                const float *hp = a.h + (size_t)r * I + kbase + jj * 32;
+                                const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(hp));
+                                const float4 h1 = __ldcg(reinterpret_cast<const float4 *>(hp + 4));
+                                v[0] = fmaf(rs, h0.x, v[0]); v[1] = fmaf(rs, h0.y, v[1]);
+                                v[2] = fmaf(rs, h0.z, v[2]); v[3] = fmaf(rs, h0.w, v[3]);
+                                v[4] = fmaf(rs, h1.x, v[4]); v[5] = fmaf(rs, h1.y, v[5]);
+                                v[6] = fmaf(rs, h1.z, v[6]); v[7] = fmaf(rs, h1.w, v[7]);
+                            }
+                        __half2 p0 = __floats2half2_rn(v[0], v[1]), p1 = __floats2half2_rn(v[2], v[3]);
+                        __half2 p2 = __floats2half2_rn(v[4], v[5]), p3 = __floats2half2_rn(v[6], v[7]);
+                        xb[jj] = make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
+                                            *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
                     }
-            }
-        }
-        const uint32_t parity = (uint32_t)((j / kDNStages) & 1);
-        const bool ok = mbar_wait_bounded(&full[j % kDNStages], parity);
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) {
-                atomicOr(a.status, FLAG_TIMEOUT);
-                drain_stages(full, kDNStages, j + 1, n_units);
-            }
-            break;
-        }
-        const uint8_t *st = stages + (size_t)(j % kDNStages) * ly.stage_bytes;
-        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+                }
+                // stage = [rows m0..m0+15 block][rows m0+16..m0+31 block]
+                const uint4 c0 = lds128(frag_ptr(st, g, gp, t)), c1 = lds128(frag_ptr(st, g + 8, gp, t));
+                const uint4 c2 = lds128(frag_ptr(st + kBlk, g, gp, t)), c3 = lds128(frag_ptr(st + kBlk, g + 8, gp, t));
+                float s0[4], s1[4], s2[4], s3[4];
+                e8m0x4(lds32(scale_ptr(st, g, gp)), s0);
+                e8m0x4(lds32(scale_ptr(st, g + 8, gp)), s1);
+                e8m0x4(lds32(scale_ptr(st + kBlk, g, gp)), s2);
+                e8m0x4(lds32(scale_ptr(st + kBlk, g + 8, gp)), s3);
 #pragma unroll
-        for (int G = 0; G < NG; ++G) {
-            const int gg = warp * NG + G;
-            const uint8_t *cp = st + (size_t)g * ly.row_stride + gg * 64 + 16 * t;
-            const uint4 c0 = lds128(cp), c1 = lds128(cp + 8 * ly.row_stride);
-            const uint4 c2 = lds128(cp + 16 * ly.row_stride), c3 = lds128(cp + 24 * ly.row_stride);
-            const uint8_t *sp = st + (size_t)32 * ly.row_stride + (size_t)g * ly.sc_stride + gg * 4;
-            const uint32_t q0 = lds32(sp), q1 = lds32(sp + 8 * ly.sc_stride);
-            const uint32_t q2 = lds32(sp + 16 * ly.sc_stride), q3 = lds32(sp + 24 * ly.sc_stride);
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                uint4 xb;
-                __half2 h01 = __floats2half2_rn(bsum[G][jj][0], bsum[G][jj][1]);
-                __half2 h23 = __floats2half2_rn(bsum[G][jj][2], bsum[G][jj][3]);
-                __half2 h45 = __floats2half2_rn(bsum[G][jj][4], bsum[G][jj][5]);
-                __half2 h67 = __floats2half2_rn(bsum[G][jj][6], bsum[G][jj][7]);
-                xb.x = *reinterpret_cast<uint32_t *>(&h01);
-                xb.y = *reinterpret_cast<uint32_t *>(&h23);
-                xb.z = *reinterpret_cast<uint32_t *>(&h45);
-                xb.w = *reinterpret_cast<uint32_t *>(&h67);
-                block_mma(acc0, u4get(c0, jj), u4get(c1, jj), xb, e8m0_byte(q0, jj), e8m0_byte(q1, jj));
-                block_mma(acc1, u4get(c2, jj), u4get(c3, jj), xb, e8m0_byte(q2, jj), e8m0_byte(q3, jj));
+                for (int jj = 0; jj < 4; ++jj) {
+                    block_mma(acc0, u4get(c0, jj), u4get(c1, jj), xb[jj], s0[jj], s1[jj]);
+                    block_mma(acc1, u4get(c2, jj), u4get(c3, jj), xb[jj], s2[jj], s3[jj]);
+                }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
-        float4 *mine = reinterpret_cast<float4 *>(red + ((size_t)warp * 32 + lane) * 8);
-        mine[0] = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
-        mine[1] = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
-        __syncthreads();
-        if (warp == 0) dn_issue(a, tb, ly, stages, full, j + kDNStages, n_units);
-        if (tid < 256) {
-            const int row = tid >> 3, col = tid & 7;   // 32 rows x 8 tokens
-            if (col < T) {
-                const int sub = row >> 4, rl = row & 15;
-                const int gl = rl & 7, hi = rl >> 3, tl = col >> 1, cbit = col & 1;
-                const int src_lane = gl * 4 + tl, slot = sub * 4 + hi * 2 + cbit;
-                float s = 0.f;
+        // this expert's contribution to rows m0..m0+31, tokens 0..T-1
 #pragma unroll
-                for (int ww = 0; ww < kWarps; ++ww) s += red[((size_t)ww * 32 + src_lane) * 8 + slot];
-                __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row, s);
-            }
+        for (int e = 0; e < 8; ++e) {
+            // e < 4: first tile (rows g, g+8), else second tile (rows 16+g, 24+g)
+            const int row = g + 8 * ((e >> 1) & 1) + (e < 4 ? 0 : 16), col = 2 * t + (e & 1);
+            const float v = e < 4 ? acc0[e] : acc1[e - 4];
+            if (col < T) __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row, v);
+        }
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = (atomicAdd(a.counters + tile, 1) == tb.D - 1);
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {   // every expert of this tile is in: sum in expert order, write bf16
             __threadfence();
-        }
-        __syncthreads();
-        if (tid == 0) {
-            const int old = atomicAdd(a.counters + tile, 1);
-            last_flag = (old == tb.D - 1);
-        }
-        __syncthreads();
-        if (last_flag && tid < 256) {
-            __threadfence();
-            const int row = tid >> 3, col = tid & 7;
-            if (col < T) {
-                float s = 0.f;
-                for (int dd = 0; dd < tb.D; ++dd) s += __ldcg(a.ybuf + ((size_t)dd * kMaxT + col) * H + m0 + row);
-                __nv_bfloat16 o = __float2bfloat16_rn(s * tok_inv[col]);
-                a.out[(size_t)col * H + m0 + row] = *reinterpret_cast<uint16_t *>(&o);
+            for (int col = 0; col < T; ++col) {
+                float sum = 0.f;
+                for (int dd = 0; dd < tb.D; ++dd) sum += __ldcg(a.ybuf + ((size_t)dd * kMaxT + col) * H + m0 + lane);
+                __nv_bfloat16 o = __float2bfloat16_rn(sum * tok_inv[col]);
+                a.out[(size_t)col * H + m0 + lane] = *reinterpret_cast<uint16_t *>(&o);
             }
-            if (tid == 0) a.counters[tile] = 0;
+            if (lane == 0) a.counters[tile] = 0;
         }
     }
+    if (timed_out && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
 }
 
 template <typename K, typename A>
@@ -582,32 +696,34 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
     return cudaLaunchKernelEx(&cfg, kernel, args);
 }
 
-constexpr size_t kMaxDynSmem = 232448 - 4096;   // leave room for the static shared memory
+int gu_stages(int T, int H) {
+    int s = (int)((kMaxDynSmem - gu_bytes(0, T, H)) / kStageBytes);
+    return s > kMaxStages ? kMaxStages : s;
+}
+int dn_stages(int I) {
+    int s = (int)((kMaxDynSmem - dn_bytes(0, I)) / kStageBytes);
+    return s > kMaxStages ? kMaxStages : s;
+}
 
-template <int NGU, int NGD>
+template <int NCU, int NCD>
 cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
                        cudaStream_t s, const cudaEvent_t *ev) {
     const int H = L.d.hidden, I = L.d.inter;
     const int grid = L.sm_count;
-    const GULayout gl(H);
-    const DNLayout dl(I);
     static bool attr_done[64] = {};
     const int dev = L.d.device;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(dec_gateup_mx_kernel<NGU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)gl.bytes(kMaxT));
+        cudaError_t e = cudaFuncSetAttribute(dec_gateup_mx_kernel<NCU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kMaxDynSmem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(dec_down_mx_kernel<NGD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)dl.bytes());
+            e = cudaFuncSetAttribute(dec_down_mx_kernel<NCD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
     GateUpArgs ga;
     ga.codes_g = L.w.codes[MOEQ_GATE];
     ga.codes_u = L.w.codes[MOEQ_UP];
-    ga.scales_g = L.w.scales[MOEQ_GATE];
-    ga.scales_u = L.w.scales[MOEQ_UP];
     ga.x = reinterpret_cast<const uint16_t *>(x);
     ga.ids = ids;
     ga.topk_w = topk_w;
@@ -619,14 +735,15 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     ga.E = L.d.n_experts;
     ga.H = H;
     ga.I = I;
+    ga.n_stages = gu_stages(T, H);
     L.count_launches(2);
     if (ev) record_phase(ev[1], s);   // routing is fused into both kernels' prologues
-    cudaError_t e = launch_ex(dec_gateup_mx_kernel<NGU>, dim3(grid), dim3(kThreads), gl.bytes(T), s, false, ga);
+    cudaError_t e = launch_ex(dec_gateup_mx_kernel<NCU>, dim3(grid), dim3(kWSThreads),
+                              gu_bytes(ga.n_stages, T, H), s, false, ga);
     if (e != cudaSuccess) return e;
     if (ev) record_phase(ev[2], s);
     DownArgs da;
     da.codes = L.w.codes[MOEQ_DOWN];
-    da.scales = L.w.scales[MOEQ_DOWN];
     da.h = L.h;
     da.gmax = L.dec_gmax;
     da.n_gmax = grid;
@@ -641,10 +758,12 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     da.E = L.d.n_experts;
     da.H = H;
     da.I = I;
-    // programmatic dependent launch: the down kernel's CTAs start streaming
-    // weights while the gate/up kernel drains and wait for it before reading
-    // h.  Not with phase events between the two launches.
-    e = launch_ex(dec_down_mx_kernel<NGD>, dim3(grid), dim3(kThreads), dl.bytes(), s, ev == nullptr, da);
+    da.n_stages = dn_stages(I);
+    // programmatic dependent launch: the down kernel's producer streams
+    // weights while the gate/up kernel drains; its consumers wait for that
+    // grid before reading h.  Not with phase events between the launches.
+    e = launch_ex(dec_down_mx_kernel<NCD>, dim3(grid), dim3(kWSThreads), dn_bytes(da.n_stages, I), s, ev == nullptr,
+                  da);
     if (e != cudaSuccess) return e;
     if (ev) {
         record_phase(ev[3], s);
@@ -660,17 +779,17 @@ bool decode_mx_supported(const Layer &L, int T) {
     if (d.fmt != MOEQ_FMT_MXFP4 || d.act != MOEQ_ACT_BF16) return false;
     if (T < 1 || T > kMaxT || T * d.top_k > kMaxR) return false;
     if (!((d.hidden == 2048 || d.hidden == 4096) && (d.inter == 2048 || d.inter == 4096))) return false;
-    if (GULayout(d.hidden).bytes(kMaxT) > kMaxDynSmem || DNLayout(d.inter).bytes() > kMaxDynSmem) return false;
+    if (gu_stages(kMaxT, d.hidden) < 2 || dn_stages(d.inter) < 2) return false;
     return L.sm_count > 0 && L.sm_count <= kDecMaxGrid;
 }
 
 cudaError_t launch_decode_mx(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T,
                              void *out, cudaStream_t s, const cudaEvent_t *ev) {
     const int H = L.d.hidden, I = L.d.inter;
-    if (H == 2048 && I == 2048) return run_decode<1, 1>(L, x, ids, topk_w, T, out, s, ev);
-    if (H == 2048 && I == 4096) return run_decode<1, 2>(L, x, ids, topk_w, T, out, s, ev);
-    if (H == 4096 && I == 2048) return run_decode<2, 1>(L, x, ids, topk_w, T, out, s, ev);
-    if (H == 4096 && I == 4096) return run_decode<2, 2>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 2048 && I == 2048) return run_decode<2, 2>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 2048 && I == 4096) return run_decode<2, 4>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 4096 && I == 2048) return run_decode<4, 2>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 4096 && I == 4096) return run_decode<4, 4>(L, x, ids, topk_w, T, out, s, ev);
     return cudaErrorInvalidValue;
 }
 

@@ -13,18 +13,16 @@
 namespace moeq {
 namespace {
 
-// One thread per 32 consecutive weights of a row.
-__global__ void dequant_mxfp4_kernel(const uint8_t *__restrict__ codes,
-                                     const uint8_t *__restrict__ scales, int N, int K,
-                                     float *__restrict__ out) {
-    const int units_per_row = K / 32;
+// One thread per 32 consecutive weights of a row; e = the expert's base in
+// the device layout.
+__global__ void dequant_mxfp4_kernel(const uint8_t *__restrict__ e, MxGeom g, float *__restrict__ out) {
+    const int N = g.N, K = g.K, units_per_row = K / 32;
     long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (u >= (long long)N * units_per_row) return;
     int n = (int)(u / units_per_row), b = (int)(u % units_per_row);
-    const uint8_t *row = codes + (size_t)n * (K / 2);
-    float sc = e8m0_to_f32(scales[(size_t)n * units_per_row + b]);
+    float sc = e8m0_to_f32(mx_scale(e, g, n, b));
     float *o = out + (size_t)n * K + (size_t)b * 32;
-    uint4 raw = mx_block(row, b);
+    uint4 raw = mx_block(e, g, n, b);
     uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -60,25 +58,32 @@ __global__ void dequant_vq_kernel(const uint8_t *__restrict__ idx13, const uint8
     }
 }
 
-// In-place 4x4 transpose of the 32-bit words of every 64-byte group (the
-// device layout of MXFP4 codes; see mx_word).
-__global__ void mx_repack_kernel(uint4 *__restrict__ codes, size_t n_groups) {
-    size_t gi = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gi >= n_groups) return;
-    uint4 *g = codes + 4 * gi;
-    uint4 a = g[0], b = g[1], c = g[2], d = g[3];
-    g[0] = make_uint4(a.x, b.x, c.x, d.x);
-    g[1] = make_uint4(a.y, b.y, c.y, d.y);
-    g[2] = make_uint4(a.z, b.z, c.z, d.z);
-    g[3] = make_uint4(a.w, b.w, c.w, d.w);
+// Logical planes (codes [ne][N][K/2], scales [ne][N][K/32]) -> device
+// layout (MxGeom).  One thread per 32-weight block of a row.
+__global__ void mx_pack_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
+                               uint8_t *__restrict__ dst, MxGeom g, int ne) {
+    const int bpr = g.K / 32;
+    long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= (long long)ne * g.N * bpr) return;
+    const int b = (int)(u % bpr);
+    const long long rowg = u / bpr;          // expert * N + n
+    const int n = (int)(rowg % g.N), e = (int)(rowg / g.N);
+    const uint4 raw = *reinterpret_cast<const uint4 *>(codes + rowg * (g.K / 2) + (size_t)b * 16);
+    uint8_t *de = dst + (size_t)e * g.expert_bytes();
+    *reinterpret_cast<uint32_t *>(de + g.code_word_off(n, b, 0)) = raw.x;
+    *reinterpret_cast<uint32_t *>(de + g.code_word_off(n, b, 1)) = raw.y;
+    *reinterpret_cast<uint32_t *>(de + g.code_word_off(n, b, 2)) = raw.z;
+    *reinterpret_cast<uint32_t *>(de + g.code_word_off(n, b, 3)) = raw.w;
+    de[g.scale_off(n, b)] = scales[rowg * bpr + b];
 }
 
 }  // namespace
 
-cudaError_t launch_mx_repack(uint8_t *codes, size_t bytes, cudaStream_t s) {
-    size_t n_groups = bytes / 64;
-    if (n_groups == 0) return cudaSuccess;
-    mx_repack_kernel<<<(unsigned)((n_groups + 255) / 256), 256, 0, s>>>(reinterpret_cast<uint4 *>(codes), n_groups);
+cudaError_t launch_mx_pack(const uint8_t *codes, const uint8_t *scales, uint8_t *dst, const MxGeom &g, int ne,
+                           cudaStream_t s) {
+    const long long n = (long long)ne * g.N * (g.K / 32);
+    if (n == 0) return cudaSuccess;
+    mx_pack_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(codes, scales, dst, g, ne);
     return cudaGetLastError();
 }
 
@@ -87,11 +92,10 @@ cudaError_t launch_dequant(const Layer &L, int expert, int proj, float *out, cud
     L.count_launches(1);
     const int threads = 256;
     if (L.d.fmt == MOEQ_FMT_MXFP4) {
+        const MxGeom g(v.N, v.K);
         long long units = (long long)v.N * (v.K / 32);
-        const uint8_t *c = v.codes + (size_t)expert * v.N * (v.K / 2);
-        const uint8_t *sc = v.scales + (size_t)expert * v.N * (v.K / 32);
         dequant_mxfp4_kernel<<<(unsigned)((units + threads - 1) / threads), threads, 0, s>>>(
-            c, sc, v.N, v.K, out);
+            v.codes + (size_t)expert * g.expert_bytes(), g, out);
     } else {
         long long units = (long long)v.N * (v.K / 8);
         const uint8_t *i13 = v.idx13 + (size_t)expert * v.N * (v.K / 8) * 13 / 8;

@@ -26,8 +26,10 @@ template <int FMT>
 __device__ __forceinline__ void decode_unit(const ProjView &v, int e, int n, int u, float w[32]) {
     const size_t row = (size_t)e * v.N + n;
     if constexpr (FMT == FMT_MX) {
-        uint4 raw = mx_block(v.codes + row * (v.K / 2), u);
-        float sc = e8m0_to_f32(__ldg(v.scales + row * (v.K / 32) + u));
+        const MxGeom mg(v.N, v.K);
+        const uint8_t *eb = v.codes + (size_t)e * mg.expert_bytes();
+        uint4 raw = mx_block(eb, mg, n, u);
+        float sc = e8m0_to_f32(mx_scale(eb, mg, n, u));
         uint32_t q[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int a = 0; a < 4; ++a)

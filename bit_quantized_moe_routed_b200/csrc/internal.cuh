@@ -109,7 +109,12 @@ cudaError_t launch_ffn_simt(const Layer &L, const void *x, const float *topk_w, 
 // Record a phase event of moeq_forward_profiled.  External, so that under
 // stream capture it becomes an event-record node of the graph (a plain
 // record is only a dependency marker there) and can be timed on replay.
-inline void record_phase(cudaEvent_t e, cudaStream_t s) { cudaEventRecordWithFlags(e, s, cudaEventRecordExternal); }
+inline void record_phase(cudaEvent_t e, cudaStream_t s) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &st);
+    if (st == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+    else cudaEventRecord(e, s);
+}
 
 // ---- small device helpers shared by the kernels ----
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
@@ -133,21 +138,59 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
     return __uint_as_float(b == 0u ? 0x00400000u : (b == 255u ? 0x7FC00000u : (b << 23)));
 }
 
-// Device layout of MXFP4 codes.  Each row's bytes come in groups of 64
-// (four 32-weight blocks of 16 bytes); inside a group the 4x4 matrix of
-// 32-bit words is transposed at upload, so that word t of logical block j
-// sits at byte 16*t + 4*j.  A thread that owns bytes 4t..4t+3 of every block
-// (the mma A-fragment slice) then reads four blocks with one 16-byte load.
-// The transpose is its own inverse.
-__device__ __forceinline__ uint32_t mx_word(const uint8_t *row, int blk, int t) {
-    return *reinterpret_cast<const uint32_t *>(row + (blk >> 2) * 64 + 16 * t + 4 * (blk & 3));
+// Device layout of one MXFP4 projection (codes and scales in one plane).
+// Per expert, the N x K matrix is cut into tiles of 16 rows and chunks of
+// KC = min(K, 1024) columns; the (tile, chunk) blocks follow each other
+// tile by tile, chunk by chunk.  A block is 16 * (KC/2 + KC/32) bytes (8704
+// for KC = 1024) and holds
+//   [16 rows][KC/2 code bytes]            then
+//   [KC/128 groups][16 rows][4 scale bytes]
+// Inside a code row, each 64-byte group carries four 32-weight blocks with
+// its 4x4 matrix of 32-bit words transposed (word t of block j at byte
+// 16t + 4j), and in odd rows the 64-byte groups are swapped in pairs
+// (group g stored at g ^ 1; only when a chunk row has an even number of
+// groups).  With this layout a tensor-core fragment slice
+// (bytes 4t..4t+3 of four consecutive blocks) is one 16-byte word, a whole
+// block is one contiguous bulk copy, and the staged rows and scale words
+// are read from shared memory without bank conflicts.
+struct MxGeom {
+    int N, K, KC, nchunk, block_bytes;
+    __host__ __device__ MxGeom(int n, int k)
+        : N(n), K(k), KC(k < 1024 ? k : 1024), nchunk(k / (k < 1024 ? k : 1024)),
+          block_bytes(16 * ((k < 1024 ? k : 1024) / 2 + (k < 1024 ? k : 1024) / 32)) {}
+    __host__ __device__ size_t expert_bytes() const { return (size_t)(N / 16) * nchunk * block_bytes; }
+    __host__ __device__ size_t block_off(int tile, int chunk) const {
+        return ((size_t)tile * nchunk + chunk) * block_bytes;
+    }
+    // byte offset, inside an expert, of code word t of 32-weight block blk of row n
+    __host__ __device__ size_t code_word_off(int n, int blk, int t) const {
+        const int kb = blk * 16;                     // logical byte of the block in the row
+        const int chunk = kb / (KC / 2), within = kb % (KC / 2);
+        const int r = n % 16, grp = (within / 64) ^ ((KC / 128) % 2 == 0 ? (r & 1) : 0), j = (within % 64) / 16;
+        return block_off(n / 16, chunk) + (size_t)r * (KC / 2) + grp * 64 + 16 * t + 4 * j;
+    }
+    // byte offset, inside an expert, of the E8M0 scale of block blk of row n
+    __host__ __device__ size_t scale_off(int n, int blk) const {
+        const int chunk = blk / (KC / 32), within = blk % (KC / 32);
+        return block_off(n / 16, chunk) + 16 * (KC / 2) + (size_t)(within / 4) * 64 + (n % 16) * 4 + (within % 4);
+    }
+};
+
+// The 16 logical code bytes of 32-weight block blk of row n (word t =
+// logical bytes 4t..4t+3), and its scale byte.  e = the expert's base.
+__device__ __forceinline__ uint4 mx_block(const uint8_t *e, const MxGeom &g, int n, int blk) {
+    return make_uint4(*reinterpret_cast<const uint32_t *>(e + g.code_word_off(n, blk, 0)),
+                      *reinterpret_cast<const uint32_t *>(e + g.code_word_off(n, blk, 1)),
+                      *reinterpret_cast<const uint32_t *>(e + g.code_word_off(n, blk, 2)),
+                      *reinterpret_cast<const uint32_t *>(e + g.code_word_off(n, blk, 3)));
 }
-// The 16 logical bytes of block `blk` of a row (as four words, word t =
-// logical bytes 4t..4t+3).
-__device__ __forceinline__ uint4 mx_block(const uint8_t *row, int blk) {
-    return make_uint4(mx_word(row, blk, 0), mx_word(row, blk, 1), mx_word(row, blk, 2), mx_word(row, blk, 3));
+__device__ __forceinline__ uint32_t mx_scale(const uint8_t *e, const MxGeom &g, int n, int blk) {
+    return e[g.scale_off(n, blk)];
 }
-cudaError_t launch_mx_repack(uint8_t *codes, size_t bytes, cudaStream_t s);
+// Rewrite experts [e0, e0+ne) of a projection from the logical planes (codes
+// [ne][N][K/2], scales [ne][N][K/32], device memory) into the device layout.
+cudaError_t launch_mx_pack(const uint8_t *codes, const uint8_t *scales, uint8_t *dst, const MxGeom &g, int ne,
+                           cudaStream_t s);
 
 // 13-bit index j of a row's little-endian index stream.  Reads the third
 // byte only when the field reaches it, so the last index of the last row

@@ -122,8 +122,9 @@ typedef struct {
  * storage and a workspace sized for desc->max_tokens.  The library owns all
  * of it until moeq_layer_destroy.
  * Errors: INVALID_ARGUMENT (NULL pointer; a non-positive size; top_k > E or
- * > 64; E > 1024; hidden or inter not a multiple of 128 for MXFP4 or of 64
- * for VQ; unknown fmt/act), CUDA (bad device), OUT_OF_MEMORY.  On error *out
+ * > 64; E > 1024; for MXFP4 hidden or inter not a multiple of 128, or
+ * above 1024 and not a multiple of 1024; for VQ not a multiple of 64;
+ * unknown fmt/act), CUDA (bad device), OUT_OF_MEMORY.  On error *out
  * is set to NULL and nothing is left allocated. */
 MOEQ_API moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out);
 
