@@ -108,7 +108,8 @@ bool desc_valid(const moeq_layer_desc *d) {
 moeq_status launch_forward(moeq_layer *L, const void *x, const int32_t *ids, const float *w, int32_t T,
                            void *out, cudaStream_t s, const cudaEvent_t *ev = nullptr) {
     if (ev) record_phase(ev[0], s);
-    if (decode_mx_supported(*L, T)) return from_cuda(launch_decode_mx(*L, x, ids, w, T, out, s, ev));
+    // the decode kernels bulk-copy token rows of x: 16-byte aligned x only
+    if (decode_mx_supported(*L, T) && ((uintptr_t)x & 15u) == 0) return from_cuda(launch_decode_mx(*L, x, ids, w, T, out, s, ev));
     cudaError_t e = launch_route_bucket(*L, ids, T * L->d.top_k, L->b.offsets, L->b.perm, L->b.active, s);
     if (e != cudaSuccess) return from_cuda(e);
     if (ev) record_phase(ev[1], s);

@@ -9,15 +9,20 @@
 //
 // Work: a unit is one expert's 16 gate + 16 up rows (gate/up kernel) or 32
 // down rows (down kernel) over the full K; each CTA (one per SM) takes a
-// contiguous, balanced range of units, and each of its 16 consumer warps
-// owns whole units, so no reduction or barrier sits in the main loop.
+// contiguous, balanced range of units.  The 16 consumer warps form one group
+// per 1024-column chunk of K, so every chunk of a unit is in compute at
+// once; inside a group each warp takes a share of the chunk's 32-weight
+// block columns for both halves (gate and up, or the two 16-row down tiles),
+// i.e. two independent accumulator chains.  Once per unit, after one
+// barrier, threads spread over all warps sum the partial fragments.
 //
 // Memory: the device layout (MxGeom) keeps each (16-row tile, 1024-column
 // chunk) block contiguous, so a producer warp streams a chunk of a unit as
-// two 8.7 KB bulk copies (TMA) into a ring of 8 shared-memory stages with
-// full/empty mbarriers, in the order the consumers take them (units in waves
-// of 16, chunk by chunk).  Bulk copies of several KB are what keep HBM busy;
-// the layout also makes the fragment and scale reads bank-conflict free.
+// two 8.7 KB bulk copies (TMA) into a ring of shared-memory stages with
+// full/empty mbarriers, unit by unit and chunk by chunk; the activations
+// arrive first, one bulk copy per token.  Bulk copies of several KB are what
+// keep HBM busy; the layout also makes the fragment and scale reads
+// bank-conflict free.
 //
 // Math: warp-level mma.sync.m16n8k16 (f16 in, f32 accumulate).  Each thread
 // reads its A-fragment slice of four 32-weight blocks (bytes 4t..4t+3 of
@@ -198,6 +203,8 @@ constexpr int kCW = 16;   // consumer warps per CTA
 __device__ __forceinline__ void named_sync_consumers() {
     asm volatile("bar.sync 1, %0;" ::"r"(32 * kCW) : "memory");
 }
+// Barrier among consumer warps 0..7 (id 2).
+__device__ __forceinline__ void named_sync_readers() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
 
 // ---------------------------------------------------------------- staging
 
@@ -235,45 +242,27 @@ __device__ __forceinline__ void my_range(int n, int &beg, int &end) {
     end = (int)(((long long)n * (blockIdx.x + 1)) / gridDim.x);
 }
 
-// Chunk order shared by producer and consumers: units go in waves of kCW
-// (warp w takes unit w of each wave); within a wave, chunk q of every unit
-// comes before chunk q+1.  Returns the global chunk index of (unit j of this
-// CTA's range, chunk q).
-__device__ __forceinline__ int chunk_index(int j, int q, int n_mine, int nch) {
-    const int wave = j / kCW, wbeg = wave * kCW;
-    const int wn = min(kCW, n_mine - wbeg);
-    return wbeg * nch + q * wn + (j - wbeg);
-}
-
-// Producer loop: chunk c of this CTA, in the order above.  After issuing
-// chunk c it publishes issued = c + 1.  Chunk c reuses the stage of chunk
-// c - S only after that chunk's consumer released it, so a consumer that has
-// seen issued > c knows the stage's barrier is in the phase of chunk c; this
-// keeps a warp that runs ahead of the others (it waits on a stage whose
-// previous chunk, another warp's, is still in flight) from matching the
-// parity of a phase two rounds old.
+// Chunk c of this CTA is chunk c % nch of unit c / nch (units in order).
+// Producer loop: after issuing chunk c it publishes issued = c + 1.  Chunk
+// c reuses the stage of chunk c - S only after every consumer released
+// that chunk, so a consumer that has seen issued > c knows the stage's
+// barrier is in the phase of chunk c; this keeps a warp that runs ahead of
+// the others from matching the parity of a phase two rounds old.
 template <typename BlockOf>
-__device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_t *empty, int S, int n_mine, int nch,
+__device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_t *empty, int S, int n_chunks,
                                         uint32_t *status, volatile int *issued, BlockOf block_of) {
-    const int lane = threadIdx.x & 31;
-    int c = 0;
-    for (int wbeg = 0; wbeg < n_mine; wbeg += kCW) {
-        const int wn = min(kCW, n_mine - wbeg);
-        for (int q = 0; q < nch; ++q)
-            for (int jj = 0; jj < wn; ++jj, ++c) {
-                const int s = c % S, kk = c / S;
-                if (lane == 0) {
-                    if (kk >= 1 && !mbar_wait_bounded(&empty[s], (uint32_t)((kk - 1) & 1)))
-                        atomicOr(status, FLAG_TIMEOUT);
-                    const uint8_t *b0, *b1;
-                    block_of(wbeg + jj, q, b0, b1);
-                    issue_chunk(stages + (size_t)s * kStageBytes, &full[s], b0, b1);
-                    __threadfence_block();
-                    *issued = c + 1;
-                }
-                __syncwarp();
-            }
+    if ((threadIdx.x & 31) == 0) {
+        for (int c = 0; c < n_chunks; ++c) {
+            const int s = c % S, kk = c / S;
+            if (kk >= 1 && !mbar_wait_bounded(&empty[s], (uint32_t)((kk - 1) & 1))) atomicOr(status, FLAG_TIMEOUT);
+            const uint8_t *b0, *b1;
+            block_of(c, b0, b1);
+            issue_chunk(stages + (size_t)s * kStageBytes, &full[s], b0, b1);
+            __threadfence_block();
+            *issued = c + 1;
+        }
     }
+    __syncwarp();
 }
 
 // Consumer: wait until chunk c is issued, then for its data.  False on timeout.
@@ -285,8 +274,34 @@ __device__ __forceinline__ bool wait_chunk(uint64_t *full, int S, int c, volatil
             __nanosleep(32);
         }
     }
-    __threadfence_block();
     return mbar_wait_bounded(&full[c % S], (uint32_t)((c / S) & 1));
+}
+
+// Chunk q of every unit is computed by the 16/NCH warps [q*16/NCH, ...): a
+// chunk is 16 pieces (8 K-groups x 2 halves: gate/up blocks, or the two
+// down tiles) and each of those warps takes NCH of them, K-groups
+// (i*NCH/2 ...) of both halves, so NCH chunks are in compute at once and
+// each warp runs two independent accumulator chains.  Partial fragments go
+// to red[unit parity][warp][lane][8] (half 0 then half 1) and are summed
+// after one barrier per unit.
+constexpr int kRedBytes = 2 * kCW * 32 * 8 * (int)sizeof(float);
+
+// One 32-weight block pair (both halves) of K-group gp of staged chunk `st`
+// against the four B fragments xb[0..3] of that group.
+__device__ __forceinline__ void chunk_group(const uint8_t *st, int g, int t, int gp, const uint4 xb[4], float acc0[4],
+                                            float acc1[4]) {
+    const uint4 a0 = lds128(frag_ptr(st, g, gp, t)), a8 = lds128(frag_ptr(st, g + 8, gp, t));
+    const uint4 b0 = lds128(frag_ptr(st + kBlk, g, gp, t)), b8 = lds128(frag_ptr(st + kBlk, g + 8, gp, t));
+    float sa0[4], sa8[4], sb0[4], sb8[4];
+    e8m0x4(lds32(scale_ptr(st, g, gp)), sa0);
+    e8m0x4(lds32(scale_ptr(st, g + 8, gp)), sa8);
+    e8m0x4(lds32(scale_ptr(st + kBlk, g, gp)), sb0);
+    e8m0x4(lds32(scale_ptr(st + kBlk, g + 8, gp)), sb8);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        block_mma(acc0, u4get(a0, jj), u4get(a8, jj), xb[jj], sa0[jj], sa8[jj]);
+        block_mma(acc1, u4get(b0, jj), u4get(b8, jj), xb[jj], sb0[jj], sb8[jj]);
+    }
 }
 
 // ---------------------------------------------------------------- gate/up
@@ -303,9 +318,10 @@ struct GateUpArgs {
 };
 
 __host__ __device__ inline size_t gu_xs_off(int n_stages) { return (size_t)n_stages * kStageBytes; }
-__host__ __device__ inline size_t gu_bytes(int n_stages, int T, int H) {
+__host__ __device__ inline size_t gu_red_off(int n_stages, int T, int H) {
     return gu_xs_off(n_stages) + sizeof(uint16_t) * (size_t)T * (H + kXPad);
 }
+__host__ __device__ inline size_t gu_bytes(int n_stages, int T, int H) { return gu_red_off(n_stages, T, H) + kRedBytes; }
 
 // Unit i -> (expert slot d, column chunk, 16-row tile): experts with more
 // than 8 routes take one pass per 8 columns.
@@ -319,24 +335,27 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ RouteTable tb;
     __shared__ GUItems items;
-    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], xbar;
     __shared__ int issued;   // chunks issued by the producer (see produce)
     __shared__ float xinv[kMaxT];
     __shared__ unsigned cta_max[kMaxT];
     const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages;
     uint8_t *stages = smem_raw;
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw + gu_xs_off(S));
+    float *red = reinterpret_cast<float *>(smem_raw + gu_red_off(S, T, H));
     const int xs_stride = H + kXPad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int tiles = I / 16;
     const MxGeom geo(I, H);
+    constexpr int WPC = kCW / NCH;   // warps per chunk
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], WPC);
         }
+        mbar_init(&xbar, 1);
         mbar_fence_init();
         issued = 0;
     }
@@ -365,24 +384,30 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     };
 
     if (warp == kProducerWarp) {
-        produce(stages, full, empty, S, n_mine, NCH, a.status, &issued, [&](int j, int q, const uint8_t *&b0, const uint8_t *&b1) {
-            int d, rel;
-            decode_item(i0 + j, d, rel);
-            const size_t off = (size_t)tb.expert[d] * geo.expert_bytes() + geo.block_off(rel % tiles, q);
-            b0 = a.codes_g + off;
-            b1 = a.codes_u + off;
-        });
+        // the activations first (one bulk copy per token row, into padded rows)
+        if (lane == 0) mbar_arrive_expect_tx(&xbar, (uint32_t)(T * H * 2));
+        __syncwarp();
+        if (lane < T) bulk_g2s(xs + (size_t)lane * xs_stride, a.x + (size_t)lane * H, H * 2, &xbar);
+        produce(stages, full, empty, S, n_mine * NCH, a.status, &issued,
+                [&](int c, const uint8_t *&b0, const uint8_t *&b1) {
+                    int d, rel;
+                    decode_item(i0 + c / NCH, d, rel);
+                    const size_t off = (size_t)tb.expert[d] * geo.expert_bytes() + geo.block_off(rel % tiles, c % NCH);
+                    b0 = a.codes_g + off;
+                    b1 = a.codes_u + off;
+                });
         return;
     }
 
-    // ---- consumers: stage x as f16 with a per-token power-of-two prescale
-    // (warp w <-> token w)
+    // ---- consumers: x -> f16 in place, with a per-token power-of-two
+    // prescale (warp w <-> token w)
+    bool timed_out = !mbar_wait_bounded(&xbar, 0);
     if (warp < T) {
-        const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)warp * H);
+        uint4 *row = reinterpret_cast<uint4 *>(xs + (size_t)warp * xs_stride);
         float m = 0.f;
         for (int i = lane; i < H / 8; i += 32) {
-            uint4 v = xr[i];
-            uint32_t qv[4] = {v.x, v.y, v.z, v.w};
+            const uint4 v = row[i];
+            const uint32_t qv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 m = fmaxf(m, fmaxf(fabsf(__uint_as_float(qv[j] << 16)), fabsf(__uint_as_float(qv[j] & 0xFFFF0000u))));
@@ -392,23 +417,23 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
         const int s = prescale_exp(m);
         const float sc = exp2i(s);
         if (lane == 0) xinv[warp] = exp2i(-s);
-        uint4 *dst = reinterpret_cast<uint4 *>(xs + (size_t)warp * xs_stride);
         for (int i = lane; i < H / 8; i += 32) {
-            uint4 v = xr[i];
-            uint32_t qv[4] = {v.x, v.y, v.z, v.w}, o[4];
+            const uint4 v = row[i];
+            const uint32_t qv[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 __half2 hv = __floats2half2_rn(__uint_as_float(qv[j] << 16) * sc,
                                                __uint_as_float(qv[j] & 0xFFFF0000u) * sc);
                 o[j] = *reinterpret_cast<uint32_t *>(&hv);
             }
-            dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+            row[i] = make_uint4(o[0], o[1], o[2], o[3]);
         }
     }
     named_sync_consumers();
 
-    bool timed_out = false;
-    for (int j = warp; j < n_mine; j += kCW) {
+    const int q = warp / WPC, wi = warp % WPC;   // this warp's chunk of every unit and its place in it
+    for (int j = 0; j < n_mine; ++j) {
         int d, rel;
         decode_item(i0 + j, d, rel);
         const int cb = tb.col_beg[d] + (rel / tiles) * 8, n0 = (rel % tiles) * 16;
@@ -417,40 +442,40 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
         const int tok = live ? tb.route[cb + g] / k : 0;
         const uint16_t *xrow = xs + (size_t)tok * xs_stride + 8 * t;
         float aG[4] = {0.f, 0.f, 0.f, 0.f}, aU[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int q = 0; q < NCH; ++q) {
-            const int c = chunk_index(j, q, n_mine, NCH), s = c % S;
+        {
+            const int c = j * NCH + q, s = c % S;
             if (!wait_chunk(full, S, c, &issued)) timed_out = true;
-            const uint8_t *st = stages + (size_t)s * kStageBytes;
-#pragma unroll 2
-            for (int gp = 0; gp < kKC / 128; ++gp) {   // K-groups of four 32-weight blocks
-                // stage = [gate block][up block]; rows g and g+8 of each
-                const uint4 ag0 = lds128(frag_ptr(st, g, gp, t)), ag8 = lds128(frag_ptr(st, g + 8, gp, t));
-                const uint4 au0 = lds128(frag_ptr(st + kBlk, g, gp, t));
-                const uint4 au8 = lds128(frag_ptr(st + kBlk, g + 8, gp, t));
-                float sg0[4], sg8[4], su0[4], su8[4];
-                e8m0x4(lds32(scale_ptr(st, g, gp)), sg0);
-                e8m0x4(lds32(scale_ptr(st, g + 8, gp)), sg8);
-                e8m0x4(lds32(scale_ptr(st + kBlk, g, gp)), su0);
-                e8m0x4(lds32(scale_ptr(st + kBlk, g + 8, gp)), su8);
-                const uint16_t *xq = xrow + (size_t)(q * (kKC / 32) + gp * 4) * 32;
+            const uint8_t *st = stages + (size_t)s * kStageBytes;   // [gate block][up block]
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint4 xb = live ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
-                    block_mma(aG, u4get(ag0, jj), u4get(ag8, jj), xb, sg0[jj], sg8[jj]);
-                    block_mma(aU, u4get(au0, jj), u4get(au8, jj), xb, su0[jj], su8[jj]);
-                }
+            for (int p = 0; p < NCH / 2; ++p) {
+                const int gp = wi * (NCH / 2) + p;
+                const uint16_t *xq = xrow + (size_t)(q * (kKC / 32) + gp * 4) * 32;
+                uint4 xb[4];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) xb[jj] = live ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
+                chunk_group(st, g, t, gp, xb, aG, aU);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);   // this warp is done with the stage
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
-        // epilogue: rows (g, g+8) x columns (2t, 2t+1)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int row = g + 8 * (e >> 1), col = 2 * t + (e & 1);
+        float *rb = red + (size_t)(j & 1) * kCW * 32 * 8;
+        float4 *mine = reinterpret_cast<float4 *>(rb + ((size_t)warp * 32 + lane) * 8);
+        mine[0] = make_float4(aG[0], aG[1], aG[2], aG[3]);
+        mine[1] = make_float4(aU[0], aU[1], aU[2], aU[3]);
+        named_sync_consumers();
+        if ((tid & 3) == 0) {   // 128 readers spread over the warps: 16 rows x 8 columns
+            const int r = tid >> 2, row = r >> 3, col = r & 7;
             if (col < ncol) {
+                const int src = (row & 7) * 4 + (col >> 1), slot = (row >> 3) * 2 + (col & 1);
+                float gs = 0.f, us = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < kCW; ++ww) {
+                    gs += rb[((size_t)ww * 32 + src) * 8 + slot];
+                    us += rb[((size_t)ww * 32 + src) * 8 + 4 + slot];
+                }
                 const int route = tb.route[cb + col];
                 const float inv = xinv[route / k];
-                const float hv = silu_f32(aG[e] * inv) * (aU[e] * inv);
+                const float hv = silu_f32(gs * inv) * (us * inv);
                 a.h[(size_t)route * I + n0 + row] = hv;
                 const float wh = fabsf(a.topk_w[route] * hv);
                 if (wh > 0.f) atomicMax(&cta_max[route / k], __float_as_uint(isfinite(wh) ? wh : 3.0e38f));
@@ -480,9 +505,10 @@ struct DownArgs {
 
 constexpr int kMaxBSlots = 16;   // staged (expert, token) B columns per CTA
 
-__host__ __device__ inline size_t dn_bytes(int n_stages, int I) {
+__host__ __device__ inline size_t dn_red_off(int n_stages, int I) {
     return (size_t)n_stages * kStageBytes + sizeof(uint16_t) * (size_t)kMaxBSlots * (I + kXPad);
 }
+__host__ __device__ inline size_t dn_bytes(int n_stages, int I) { return dn_red_off(n_stages, I) + kRedBytes; }
 
 template <int NCH>   // K chunks per unit = I / kKC
 __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) {
@@ -493,20 +519,22 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
     __shared__ float tok_scale[kMaxT], tok_inv[kMaxT];
     __shared__ int slot_of[kMaxR][kMaxT];   // (expert slot - d_lo, token) -> staged B column, -1 none
     __shared__ int slot_d[kMaxBSlots], slot_t[kMaxBSlots];
-    __shared__ int n_slots;
+    __shared__ int n_slots, last_flag;
     const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages;
     uint8_t *stages = smem_raw;
     uint16_t *bs = reinterpret_cast<uint16_t *>(smem_raw + (size_t)S * kStageBytes);   // [slot][I+pad] f16
+    float *red = reinterpret_cast<float *>(smem_raw + dn_red_off(S, I));
     const int bs_stride = I + kXPad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int tiles = H / 32;
     const MxGeom geo(H, I);
+    constexpr int WPC = kCW / NCH;   // warps per chunk
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], WPC);
         }
         mbar_fence_init();
         issued = 0;
@@ -524,12 +552,13 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
 
     if (warp == kProducerWarp) {
         // the weights do not depend on the gate/up kernel: stream them at once
-        produce(stages, full, empty, S, n_mine, NCH, a.status, &issued, [&](int j, int q, const uint8_t *&b0, const uint8_t *&b1) {
-            const int u = u0 + j, d = u / tiles, t32 = u % tiles;
-            const uint8_t *eb = a.codes + (size_t)tb.expert[d] * geo.expert_bytes();
-            b0 = eb + geo.block_off(2 * t32, q);
-            b1 = eb + geo.block_off(2 * t32 + 1, q);
-        });
+        produce(stages, full, empty, S, n_mine * NCH, a.status, &issued,
+                [&](int c, const uint8_t *&b0, const uint8_t *&b1) {
+                    const int u = u0 + c / NCH, d = u / tiles, t32 = u % tiles, q = c % NCH;
+                    const uint8_t *eb = a.codes + (size_t)tb.expert[d] * geo.expert_bytes();
+                    b0 = eb + geo.block_off(2 * t32, q);
+                    b1 = eb + geo.block_off(2 * t32 + 1, q);
+                });
         return;
     }
 
@@ -594,25 +623,24 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
         named_sync_consumers();
     }
 
+    const int q = warp / WPC, wi = warp % WPC;   // this warp's chunk of every unit and its place in it
     bool timed_out = false;
-    for (int j = warp; j < n_mine; j += kCW) {
+    for (int j = 0; j < n_mine; ++j) {
         const int u = u0 + j;
         const int d = u / tiles, tile = u % tiles, m0 = tile * 32;
         const int my_slot = (g < T) ? slot_of[d - d_lo][g] : -1;   // B column g = token g
         float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int q = 0; q < NCH; ++q) {
-            const int c = chunk_index(j, q, n_mine, NCH), s = c % S;
-            if (!wait_chunk(full, S, c, &issued)) timed_out = true;
-            const uint8_t *st = stages + (size_t)s * kStageBytes;
-#pragma unroll 2
-            for (int gp = 0; gp < kKC / 128; ++gp) {
-                const int kbase = q * kKC + gp * 128 + 8 * t;   // this thread's first K of block 0
-                uint4 xb[4];
+        {
+            uint4 xb[NCH / 2][4];
+#pragma unroll
+            for (int p = 0; p < NCH / 2; ++p) {
+                const int gp = wi * (NCH / 2) + p;
+                const int kbase = q * kKC + gp * 128 + 8 * t;   // this thread's first K of the group's block 0
                 if (staged) {
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj)
-                        xb[jj] = my_slot >= 0 ? lds128(bs + (size_t)my_slot * bs_stride + kbase + jj * 32)
-                                              : make_uint4(0u, 0u, 0u, 0u);
+                        xb[p][jj] = my_slot >= 0 ? lds128(bs + (size_t)my_slot * bs_stride + kbase + jj * 32)
+                                                 : make_uint4(0u, 0u, 0u, 0u);
                 } else {
                     // more columns than staged slots: build B from h in L2
 #pragma unroll
@@ -633,49 +661,48 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
                             }
                         __half2 p0 = __floats2half2_rn(v[0], v[1]), p1 = __floats2half2_rn(v[2], v[3]);
                         __half2 p2 = __floats2half2_rn(v[4], v[5]), p3 = __floats2half2_rn(v[6], v[7]);
-                        xb[jj] = make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
-                                            *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
+                        xb[p][jj] = make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
+                                               *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
                     }
                 }
-                // stage = [rows m0..m0+15 block][rows m0+16..m0+31 block]
-                const uint4 c0 = lds128(frag_ptr(st, g, gp, t)), c1 = lds128(frag_ptr(st, g + 8, gp, t));
-                const uint4 c2 = lds128(frag_ptr(st + kBlk, g, gp, t)), c3 = lds128(frag_ptr(st + kBlk, g + 8, gp, t));
-                float s0[4], s1[4], s2[4], s3[4];
-                e8m0x4(lds32(scale_ptr(st, g, gp)), s0);
-                e8m0x4(lds32(scale_ptr(st, g + 8, gp)), s1);
-                e8m0x4(lds32(scale_ptr(st + kBlk, g, gp)), s2);
-                e8m0x4(lds32(scale_ptr(st + kBlk, g + 8, gp)), s3);
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    block_mma(acc0, u4get(c0, jj), u4get(c1, jj), xb[jj], s0[jj], s1[jj]);
-                    block_mma(acc1, u4get(c2, jj), u4get(c3, jj), xb[jj], s2[jj], s3[jj]);
-                }
             }
+            const int c = j * NCH + q, s = c % S;
+            if (!wait_chunk(full, S, c, &issued)) timed_out = true;
+            const uint8_t *st = stages + (size_t)s * kStageBytes;   // [rows m0..+15 block][rows m0+16..+31 block]
+#pragma unroll
+            for (int p = 0; p < NCH / 2; ++p) chunk_group(st, g, t, wi * (NCH / 2) + p, xb[p], acc0, acc1);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
-        // this expert's contribution to rows m0..m0+31, tokens 0..T-1
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            // e < 4: first tile (rows g, g+8), else second tile (rows 16+g, 24+g)
-            const int row = g + 8 * ((e >> 1) & 1) + (e < 4 ? 0 : 16), col = 2 * t + (e & 1);
-            const float v = e < 4 ? acc0[e] : acc1[e - 4];
-            if (col < T) __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row, v);
-        }
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) last = (atomicAdd(a.counters + tile, 1) == tb.D - 1);
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {   // every expert of this tile is in: sum in expert order, write bf16
-            __threadfence();
-            for (int col = 0; col < T; ++col) {
+        float *rb = red + (size_t)(j & 1) * kCW * 32 * 8;
+        float4 *mine = reinterpret_cast<float4 *>(rb + ((size_t)warp * 32 + lane) * 8);
+        mine[0] = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
+        mine[1] = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
+        named_sync_consumers();
+        if (tid < 256) {   // readers: warps 0..7, one (row, token) each
+            const int row = tid >> 3, col = tid & 7;   // 32 rows x 8 tokens
+            const int tt = row >> 4, rl = row & 15;
+            const int src = (rl & 7) * 4 + (col >> 1), slot = tt * 4 + (rl >> 3) * 2 + (col & 1);
+            if (col < T) {
                 float sum = 0.f;
-                for (int dd = 0; dd < tb.D; ++dd) sum += __ldcg(a.ybuf + ((size_t)dd * kMaxT + col) * H + m0 + lane);
-                __nv_bfloat16 o = __float2bfloat16_rn(sum * tok_inv[col]);
-                a.out[(size_t)col * H + m0 + lane] = *reinterpret_cast<uint16_t *>(&o);
+#pragma unroll
+                for (int ww = 0; ww < kCW; ++ww) sum += rb[((size_t)ww * 32 + src) * 8 + slot];
+                __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row, sum);
             }
-            if (lane == 0) a.counters[tile] = 0;
+            __threadfence();
+            named_sync_readers();
+            if (tid == 0) last_flag = (atomicAdd(a.counters + tile, 1) == tb.D - 1);
+            named_sync_readers();
+            if (last_flag) {   // every expert of this tile is in: sum in expert order, write bf16
+                __threadfence();
+                if (col < T) {
+                    float sum = 0.f;
+                    for (int dd = 0; dd < tb.D; ++dd) sum += __ldcg(a.ybuf + ((size_t)dd * kMaxT + col) * H + m0 + row);
+                    __nv_bfloat16 o = __float2bfloat16_rn(sum * tok_inv[col]);
+                    a.out[(size_t)col * H + m0 + row] = *reinterpret_cast<uint16_t *>(&o);
+                }
+                if (tid == 0) a.counters[tile] = 0;
+            }
         }
     }
     if (timed_out && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);

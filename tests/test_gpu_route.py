@@ -26,7 +26,7 @@ def test_route_prefill_zipf_exact():
     cfg = synth.get_cfg("prefill_mxfp4_zipf", H=64, I=64)   # routing does not depend on H, I
     ids, _ = synth.gen_routing(cfg)
     from bit_quantized_moe_routed_b200 import moeq
-    lay = moeq.Layer(64, 64, cfg.E, cfg.k, cfg.T, "mxfp4", "bf16")
+    lay = moeq.Layer(128, 128, cfg.E, cfg.k, cfg.T, "mxfp4", "bf16")
     assert _check(lay, ids, cfg.E) == 0
     assert lay.status() == moeq.OK
 
@@ -40,7 +40,7 @@ def test_route_random_with_invalid_ids(T, E, k):
     ids[mask < 0.05] = -1
     ids[(mask >= 0.05) & (mask < 0.07)] = E + 3
     ids[(mask >= 0.07) & (mask < 0.08)] = -7
-    lay = moeq.Layer(64, 64, E, k, T, "mxfp4", "bf16")
+    lay = moeq.Layer(128, 128, E, k, T, "mxfp4", "bf16")
     bad = _check(lay, ids, E)
     assert (lay.status(clear=True) == moeq.ROUTE_OUT_OF_RANGE) == (bad > 0)
     assert lay.status() == moeq.OK
@@ -49,6 +49,6 @@ def test_route_random_with_invalid_ids(T, E, k):
 def test_route_all_no_route():
     from bit_quantized_moe_routed_b200 import moeq
     ids = np.full((5, 2), -1, np.int32)
-    lay = moeq.Layer(64, 64, 16, 2, 5, "mxfp4", "bf16")
+    lay = moeq.Layer(128, 128, 16, 2, 5, "mxfp4", "bf16")
     assert _check(lay, ids, 16) == 0
     assert lay.status() == moeq.OK
