@@ -18,6 +18,8 @@
 // then the routes in tiles of 1024 in index order, each route's rank among
 // equal experts found with __match_any_sync inside a warp and per-warp
 // counts across warps.
+#include <mutex>
+
 #include "internal.cuh"
 
 namespace moeq {
@@ -125,4 +127,62 @@ cudaError_t launch_route_bucket(const Layer &L, const int32_t *topk_ids, int32_t
     return cudaGetLastError();
 }
 
+// ------------------------------------------------ allocation-free variant
+//
+// moeq_route_noalloc runs route_bucket_kernel with its scratch (the active
+// list and the status word) in the fixed array below instead of a layer's
+// workspace, for callers that cannot allocate device memory.
+namespace {
+
+constexpr int kNoAllocStatusWord = kMaxExperts + 1;   // after active[0 .. kMaxExperts]
+constexpr int kNoAllocWords = kMaxExperts + 2;        // 4104 bytes
+
+// One copy per device that loads the library.  In host code this name is a
+// host-side stand-in for the array, not its device address: that comes
+// from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) int32_t g_route_scratch[kNoAllocWords];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+int32_t *g_noalloc_scratch[kNoAllocMaxDevices] = {};
+
+// Set-up for the current device `dev` (once): the scratch's device address
+// and the kernel's dynamic shared-memory limit.
+cudaError_t noalloc_scratch(int dev, int32_t **out) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_scratch[dev]) {
+        int32_t *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_route_scratch);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(route_bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(sizeof(int32_t) * kMaxExperts * (2 + kWarps)));
+        if (e != cudaSuccess) return e;
+        g_noalloc_scratch[dev] = p;
+    }
+    *out = g_noalloc_scratch[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
 }  // namespace moeq
+
+extern "C" moeq_status moeq_route_noalloc(const int32_t *topk_ids, int32_t n_tokens, int32_t top_k,
+                                          int32_t n_experts, int32_t *offsets_out, int32_t *perm_out,
+                                          void *stream) {
+    using namespace moeq;
+    if (!topk_ids || !offsets_out || !perm_out || n_tokens < 1 || top_k < 1 || top_k > kMaxTopK ||
+        n_experts < 1 || (long long)n_tokens * top_k > (1LL << 30))
+        return MOEQ_ERR_INVALID_ARGUMENT;
+    if (n_experts > kMaxExperts) return MOEQ_ERR_UNSUPPORTED;   // the scratch holds kMaxExperts + 1 entries
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return MOEQ_ERR_CUDA;
+    int32_t *scratch = nullptr;
+    if (noalloc_scratch(dev, &scratch) != cudaSuccess) return MOEQ_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t *status = reinterpret_cast<uint32_t *>(scratch + kNoAllocStatusWord);
+    if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return MOEQ_ERR_CUDA;
+    const size_t smem = sizeof(int32_t) * (size_t)n_experts * (2 + kWarps);
+    route_bucket_kernel<<<1, kThreads, smem, s>>>(topk_ids, n_tokens * top_k, n_experts, offsets_out, perm_out,
+                                                  scratch, status);
+    return cudaGetLastError() == cudaSuccess ? MOEQ_OK : MOEQ_ERR_CUDA;
+}

@@ -30,7 +30,7 @@ GATE, UP, DOWN = 0, 1, 2
 # every symbol the header declares
 EXPORTS = ("moeq_layer_create", "moeq_upload_weights", "moeq_forward", "moeq_forward_host",
            "moeq_forward_profiled", "moeq_route", "moeq_dequant", "moeq_layer_status",
-           "moeq_status_string", "moeq_layer_destroy", "moeq_kernel_launches")
+           "moeq_status_string", "moeq_layer_destroy", "moeq_kernel_launches", "moeq_route_noalloc")
 
 
 class LayerDesc(C.Structure):
@@ -53,6 +53,7 @@ _lib.moeq_forward_host.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_
 _lib.moeq_forward_profiled.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p,
                                        C.c_void_p, C.POINTER(C.c_void_p)]
 _lib.moeq_route.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]
+_lib.moeq_route_noalloc.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]
 _lib.moeq_dequant.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p]
 _lib.moeq_layer_status.argtypes = [C.c_void_p, C.c_int32]
 _lib.moeq_status_string.argtypes = [C.c_int]
@@ -62,7 +63,7 @@ _lib.moeq_layer_destroy.restype = None
 _lib.moeq_kernel_launches.argtypes = [C.c_void_p]
 _lib.moeq_kernel_launches.restype = C.c_int64
 for _f in ("moeq_layer_create", "moeq_upload_weights", "moeq_forward", "moeq_forward_host", "moeq_dequant",
-           "moeq_layer_status", "moeq_forward_profiled", "moeq_route"):
+           "moeq_layer_status", "moeq_forward_profiled", "moeq_route", "moeq_route_noalloc"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -96,6 +97,18 @@ def _host(a, dtype):
         return None, None
     a = np.ascontiguousarray(a, dtype=dtype)
     return a, a.ctypes.data
+
+
+def route_noalloc(topk_ids, n_experts, offsets_out, perm_out, stream=None):
+    """moeq_route_noalloc: the route/bucket step without a layer and without
+    any device allocation.  topk_ids int32 cuda [T][k]; offsets_out int32
+    cuda [n_experts+1] and perm_out int32 cuda [T*k] are the caller's and
+    are filled as by Layer.route.  The library's fixed scratch is shared by
+    every call on a device: calls that overlap on the GPU race."""
+    T, k = topk_ids.shape
+    _check(_lib.moeq_route_noalloc(C.c_void_p(topk_ids.data_ptr()), T, k, n_experts,
+                                   C.c_void_p(offsets_out.data_ptr()), C.c_void_p(perm_out.data_ptr()),
+                                   _stream_ptr(stream)), "moeq_route_noalloc")
 
 
 class Layer:

@@ -179,6 +179,40 @@ MOEQ_API moeq_status moeq_forward_host(moeq_layer_t layer, const void *x_host, c
 MOEQ_API moeq_status moeq_route(moeq_layer_t layer, const int32_t *topk_ids, int32_t n_tokens,
                                 int32_t *offsets_out, int32_t *perm_out, void *stream);
 
+/* moeq_route for callers that cannot allocate device memory: no layer
+ * handle, and no cudaMalloc, cudaFree or other allocating call, ever.
+ * Meant for code that runs where allocation is not allowed or not wanted:
+ * inside another framework's memory pool that owns the whole device, under
+ * a hard memory budget, or in a context where a device allocation would
+ * synchronize or fail.  No passage of the paper corresponds to it: it is a
+ * packaging of the route/bucket step, not part of the method.
+ *
+ * Arguments and results are those of moeq_route, on the current device:
+ * topk_ids (device int32 [n_tokens][top_k]) in, offsets_out (device int32
+ * [n_experts+1]) and perm_out (device int32 [n_tokens*top_k]) out, all
+ * owned by the caller; asynchronous on `stream`.  Ids of -1 are skipped;
+ * other ids outside [0, n_experts) are skipped too, and this entry point
+ * does not report them (offsets_out[n_experts] counts the valid routes
+ * only; moeq_route reports them through its layer).
+ *
+ * The kernel's scratch (the list of active experts and a status word, 4104
+ * bytes) is one fixed array inside the library, one copy per device that
+ * loads it, held until the process exits.  Limits that follow from it:
+ * n_experts <= 1024; beyond that the call returns MOEQ_ERR_UNSUPPORTED and
+ * launches nothing.  Every call on a device shares that array and it keeps
+ * the last call's contents (the status word is cleared on `stream` before
+ * each launch): calls that overlap on the GPU, from different streams or
+ * threads, race on it and must be ordered by the caller.  The first call on
+ * each device sets up (looks up the array's device address and sets the
+ * kernel's shared-memory limit); make that first call before any stream
+ * capture on that device.
+ * Errors: INVALID_ARGUMENT (NULL pointer, n_tokens < 1, top_k outside
+ * [1, 64], n_experts < 1, n_tokens*top_k > 2^30), UNSUPPORTED (n_experts >
+ * 1024), CUDA. */
+MOEQ_API moeq_status moeq_route_noalloc(const int32_t *topk_ids, int32_t n_tokens, int32_t top_k,
+                                        int32_t n_experts, int32_t *offsets_out, int32_t *perm_out,
+                                        void *stream);
+
 /* moeq_forward that also records five caller-created CUDA events (passed
  * as cudaEvent_t cast to void*) on `stream` at its phase boundaries:
  * events[0] before the first launch, [1] after route/bucket, [2] after the
