@@ -45,8 +45,6 @@
 namespace moeq {
 namespace {
 
-constexpr int kWarps = 16;
-constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxT = 8;
 constexpr int kMaxR = 64;
 constexpr int kXPad = 32;  // f16 elements of padding after each staged x row
@@ -150,12 +148,6 @@ __device__ __forceinline__ void mma_f16(float d[4], uint32_t a0, uint32_t a1, ui
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// E8M0 byte j of `word` -> 2^(b-127) as f32 (b = 0 gives the subnormal 2^-127).
-__device__ __forceinline__ float e8m0_byte(uint32_t word, int j) {
-    uint32_t b = (word >> (8 * j)) & 0xFFu;
-    return __uint_as_float(max(b << 23, 0x00400000u));
-}
-
 // Four E8M0 bytes (one scale word) -> four f32 scales, exact: two
 // cvt.rn.bf16x2.ue8m0x2 (2^(b-127) is a bf16 value, the subnormal 2^-127
 // for b = 0 included), then bf16 -> f32 by position.
@@ -192,7 +184,6 @@ __device__ __forceinline__ void block_mma(float acc[4], uint32_t wa, uint32_t wb
     ffma2(acc[0], acc[1], sa, c[0], c[1]);
     ffma2(acc[2], acc[3], sb, c[2], c[3]);
 }
-
 __device__ __forceinline__ uint32_t u4get(const uint4 &v, int j) {
     return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
@@ -203,28 +194,21 @@ constexpr int kCW = 16;   // consumer warps per CTA
 __device__ __forceinline__ void named_sync_consumers() {
     asm volatile("bar.sync 1, %0;" ::"r"(32 * kCW) : "memory");
 }
-// Barrier among consumer warps 0..7 (id 2).
-__device__ __forceinline__ void named_sync_readers() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
 
 // ---------------------------------------------------------------- staging
 
-// Warp roles: kCW consumer warps, each owning whole units, plus one producer
-// warp that streams (tile, chunk) blocks into a ring of shared-memory stages.
+// Warp roles: kCW consumer warps plus one producer warp that streams
+// (tile, chunk) blocks into a ring of shared-memory stages.
 constexpr int kWSThreads = 32 * (kCW + 1);
 constexpr int kProducerWarp = kCW;
 constexpr int kKC = 1024;                       // weights of K per chunk (the layout's chunk)
 constexpr int kBlk = 16 * (kKC / 2 + kKC / 32); // one (16-row tile, chunk) block of the device layout
-constexpr int kStageBytes = 2 * kBlk;           // two blocks: gate + up tile, or two down tiles
-constexpr int kMaxStages = 8;
+// A stage holds one piece: cps consecutive chunks of a unit, both halves
+// (gate and up tile, or the two down tiles): [half 0: cps blocks][half 1:
+// cps blocks], each half one contiguous run of the device layout.
+__host__ __device__ inline size_t piece_bytes(int cps) { return 2 * (size_t)cps * kBlk; }
+constexpr int kMaxStages = 12;
 constexpr int kMaxDynSmem = 232448 - 4096;      // leave room for static shared memory
-
-// Producer (one thread): two contiguous blocks of the device layout into
-// stage `st`, completing `bar`.
-__device__ __forceinline__ void issue_chunk(uint8_t *st, uint64_t *bar, const uint8_t *blk0, const uint8_t *blk1) {
-    mbar_arrive_expect_tx(bar, 2u * kBlk);
-    bulk_g2s(st, blk0, kBlk, bar);
-    bulk_g2s(st + kBlk, blk1, kBlk, bar);
-}
 
 // Shared-memory address of this thread's fragment word (bytes 4t..4t+3 of
 // the four blocks of K-group grp) of staged row r (0..15) of a block.
@@ -242,61 +226,106 @@ __device__ __forceinline__ void my_range(int n, int &beg, int &end) {
     end = (int)(((long long)n * (blockIdx.x + 1)) / gridDim.x);
 }
 
-// Chunk c of this CTA is chunk c % nch of unit c / nch (units in order).
-// Producer loop: after issuing chunk c it publishes issued = c + 1.  Chunk
-// c reuses the stage of chunk c - S only after every consumer released
-// that chunk, so a consumer that has seen issued > c knows the stage's
-// barrier is in the phase of chunk c; this keeps a warp that runs ahead of
-// the others from matching the parity of a phase two rounds old.
+// Chunk c of this CTA is chunk c % nch of unit c / nch (units in order),
+// and piece p holds chunks [p cps, (p+1) cps).  The producer warp refills G
+// pieces per step: lanes 2i and 2i+1 wait for the stage of piece p0 + i to
+// be released, then each issues the bulk copy of one half of it, so one
+// instruction starts 2G copies of cps blocks each (fewer, larger copies keep
+// more of HBM busy than many small ones).  After a step it publishes issued
+// = p0 + G.  Piece p reuses the stage of piece p - S only after every
+// consumer released that piece, so a consumer that has seen issued > p knows
+// the stage's barrier is in the phase of piece p; this keeps a warp that
+// runs ahead of the others from matching the parity of a phase two rounds
+// old.
 template <typename BlockOf>
-__device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_t *empty, int S, int n_chunks,
-                                        uint32_t *status, volatile int *issued, BlockOf block_of) {
-    if ((threadIdx.x & 31) == 0) {
-        for (int c = 0; c < n_chunks; ++c) {
-            const int s = c % S, kk = c / S;
-            if (kk >= 1 && !mbar_wait_bounded(&empty[s], (uint32_t)((kk - 1) & 1))) atomicOr(status, FLAG_TIMEOUT);
+__device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_t *empty, int S, int cps,
+                                        int n_pieces, uint32_t *status, volatile int *issued, BlockOf block_of) {
+    const int lane = threadIdx.x & 31, i = lane >> 1, half = lane & 1;
+    const int G = min(S, max(1, 4 / cps));
+    const uint32_t half_bytes = (uint32_t)cps * kBlk;
+    for (int p0 = 0; p0 < n_pieces; p0 += G) {
+        const int p = p0 + i;
+        const bool mine = i < G && p < n_pieces;
+        const int s = mine ? p % S : 0;
+        if (mine && half == 0 && p >= S && !mbar_wait_bounded(&empty[s], (uint32_t)((p / S - 1) & 1)))
+            atomicOr(status, FLAG_TIMEOUT);
+        __syncwarp();
+        if (mine && half == 0) mbar_arrive_expect_tx(&full[s], 2u * half_bytes);
+        __syncwarp();
+        if (mine) {
             const uint8_t *b0, *b1;
-            block_of(c, b0, b1);
-            issue_chunk(stages + (size_t)s * kStageBytes, &full[s], b0, b1);
+            block_of(p, b0, b1);
+            bulk_g2s(stages + (size_t)s * piece_bytes(cps) + half * half_bytes, half ? b1 : b0, half_bytes, &full[s]);
+        }
+        __syncwarp();
+        if (lane == 0) {
             __threadfence_block();
-            *issued = c + 1;
+            *issued = min(p0 + G, n_pieces);
         }
     }
-    __syncwarp();
 }
 
-// Consumer: wait until chunk c is issued, then for its data.  False on timeout.
-__device__ __forceinline__ bool wait_chunk(uint64_t *full, int S, int c, volatile int *issued) {
-    if (*issued <= c) {
+// Consumer: wait until piece p is issued, then for its data.  False on timeout.
+__device__ __forceinline__ bool wait_piece(uint64_t *full, int S, int p, volatile int *issued) {
+    if (*issued <= p) {
         const long long t0 = clock64();
-        while (*issued <= c) {
+        while (*issued <= p) {
             if (clock64() - t0 > 2000000000LL) return false;
             __nanosleep(32);
         }
     }
-    return mbar_wait_bounded(&full[c % S], (uint32_t)((c / S) & 1));
+    return mbar_wait_bounded(&full[p % S], (uint32_t)((p / S) & 1));
 }
 
 // Chunk q of every unit is computed by the 16/NCH warps [q*16/NCH, ...): a
 // chunk is 16 pieces (8 K-groups x 2 halves: gate/up blocks, or the two
 // down tiles) and each of those warps takes NCH of them, K-groups
 // (i*NCH/2 ...) of both halves, so NCH chunks are in compute at once and
-// each warp runs two independent accumulator chains.  Partial fragments go
-// to red[unit parity][warp][lane][8] (half 0 then half 1) and are summed
-// after one barrier per unit.
-constexpr int kRedBytes = 2 * kCW * 32 * 8 * (int)sizeof(float);
+// each warp runs two independent accumulator chains.  The partial
+// fragments go to red[unit parity][warp][half][row][column] and are summed
+// in warp order after one barrier per unit.  A unit has at most Tc = min(T,
+// 8) columns, so only those are kept.
+__host__ __device__ inline int red_cols(int T) { return T < kMaxT ? T : kMaxT; }
+__host__ __device__ inline size_t red_bytes(int T) {
+    return 2 * (size_t)kCW * 2 * 16 * red_cols(T) * sizeof(float);
+}
 
-// One 32-weight block pair (both halves) of K-group gp of staged chunk `st`
-// against the four B fragments xb[0..3] of that group.
-__device__ __forceinline__ void chunk_group(const uint8_t *st, int g, int t, int gp, const uint4 xb[4], float acc0[4],
-                                            float acc1[4]) {
-    const uint4 a0 = lds128(frag_ptr(st, g, gp, t)), a8 = lds128(frag_ptr(st, g + 8, gp, t));
-    const uint4 b0 = lds128(frag_ptr(st + kBlk, g, gp, t)), b8 = lds128(frag_ptr(st + kBlk, g + 8, gp, t));
+__device__ __forceinline__ void put_partials(float *rb, int Tc, int warp, int g, int t, const float a0[4],
+                                             const float a1[4]) {
+    float *h0 = rb + (size_t)warp * 2 * 16 * Tc, *h1 = h0 + 16 * Tc;
+    const int c0 = 2 * t, c1 = 2 * t + 1;
+    if (c0 < Tc) {
+        h0[g * Tc + c0] = a0[0];
+        h0[(g + 8) * Tc + c0] = a0[2];
+        h1[g * Tc + c0] = a1[0];
+        h1[(g + 8) * Tc + c0] = a1[2];
+    }
+    if (c1 < Tc) {
+        h0[g * Tc + c1] = a0[1];
+        h0[(g + 8) * Tc + c1] = a0[3];
+        h1[g * Tc + c1] = a1[1];
+        h1[(g + 8) * Tc + c1] = a1[3];
+    }
+}
+__device__ __forceinline__ float sum_partials(const float *rb, int Tc, int half, int row, int col) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCW; ++w) s += rb[((size_t)(w * 2 + half) * 16 + row) * Tc + col];
+    return s;
+}
+
+// One 32-weight block pair (both halves) of K-group gp of a staged chunk
+// (half-0 block st0, half-1 block st1) against the four B fragments
+// xb[0..3] of that group.
+__device__ __forceinline__ void chunk_group(const uint8_t *st0, const uint8_t *st1, int g, int t, int gp,
+                                            const uint4 xb[4], float acc0[4], float acc1[4]) {
+    const uint4 a0 = lds128(frag_ptr(st0, g, gp, t)), a8 = lds128(frag_ptr(st0, g + 8, gp, t));
+    const uint4 b0 = lds128(frag_ptr(st1, g, gp, t)), b8 = lds128(frag_ptr(st1, g + 8, gp, t));
     float sa0[4], sa8[4], sb0[4], sb8[4];
-    e8m0x4(lds32(scale_ptr(st, g, gp)), sa0);
-    e8m0x4(lds32(scale_ptr(st, g + 8, gp)), sa8);
-    e8m0x4(lds32(scale_ptr(st + kBlk, g, gp)), sb0);
-    e8m0x4(lds32(scale_ptr(st + kBlk, g + 8, gp)), sb8);
+    e8m0x4(lds32(scale_ptr(st0, g, gp)), sa0);
+    e8m0x4(lds32(scale_ptr(st0, g + 8, gp)), sa8);
+    e8m0x4(lds32(scale_ptr(st1, g, gp)), sb0);
+    e8m0x4(lds32(scale_ptr(st1, g + 8, gp)), sb8);
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
         block_mma(acc0, u4get(a0, jj), u4get(a8, jj), xb[jj], sa0[jj], sa8[jj]);
@@ -314,14 +343,16 @@ struct GateUpArgs {
     float *h;                           // [T*k][I] f32, by route id
     float *gmax;                        // [gridDim.x][kMaxT]: per-CTA max |w h| per token
     uint32_t *status;
-    int T, k, E, H, I, n_stages;
+    int T, k, E, H, I, n_stages, cps;
 };
 
-__host__ __device__ inline size_t gu_xs_off(int n_stages) { return (size_t)n_stages * kStageBytes; }
-__host__ __device__ inline size_t gu_red_off(int n_stages, int T, int H) {
-    return gu_xs_off(n_stages) + sizeof(uint16_t) * (size_t)T * (H + kXPad);
+__host__ __device__ inline size_t gu_xs_off(int n_stages, int cps) { return (size_t)n_stages * piece_bytes(cps); }
+__host__ __device__ inline size_t gu_red_off(int n_stages, int cps, int T, int H) {
+    return gu_xs_off(n_stages, cps) + sizeof(uint16_t) * (size_t)T * (H + kXPad);
 }
-__host__ __device__ inline size_t gu_bytes(int n_stages, int T, int H) { return gu_red_off(n_stages, T, H) + kRedBytes; }
+__host__ __device__ inline size_t gu_bytes(int n_stages, int cps, int T, int H) {
+    return gu_red_off(n_stages, cps, T, H) + red_bytes(T);
+}
 
 // Unit i -> (expert slot d, column chunk, 16-row tile): experts with more
 // than 8 routes take one pass per 8 columns.
@@ -339,10 +370,10 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     __shared__ int issued;   // chunks issued by the producer (see produce)
     __shared__ float xinv[kMaxT];
     __shared__ unsigned cta_max[kMaxT];
-    const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages;
+    const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages, cps = a.cps, Tc = red_cols(a.T);
     uint8_t *stages = smem_raw;
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw + gu_xs_off(S));
-    float *red = reinterpret_cast<float *>(smem_raw + gu_red_off(S, T, H));
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw + gu_xs_off(S, cps));
+    float *red = reinterpret_cast<float *>(smem_raw + gu_red_off(S, cps, T, H));
     const int xs_stride = H + kXPad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -353,7 +384,7 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], WPC);
+            mbar_init(&empty[s], WPC * cps);
         }
         mbar_init(&xbar, 1);
         mbar_fence_init();
@@ -388,8 +419,9 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
         if (lane == 0) mbar_arrive_expect_tx(&xbar, (uint32_t)(T * H * 2));
         __syncwarp();
         if (lane < T) bulk_g2s(xs + (size_t)lane * xs_stride, a.x + (size_t)lane * H, H * 2, &xbar);
-        produce(stages, full, empty, S, n_mine * NCH, a.status, &issued,
-                [&](int c, const uint8_t *&b0, const uint8_t *&b1) {
+        produce(stages, full, empty, S, cps, n_mine * NCH / cps, a.status, &issued,
+                [&](int p, const uint8_t *&b0, const uint8_t *&b1) {
+                    const int c = p * cps;
                     int d, rel;
                     decode_item(i0 + c / NCH, d, rel);
                     const size_t off = (size_t)tb.expert[d] * geo.expert_bytes() + geo.block_off(rel % tiles, c % NCH);
@@ -443,9 +475,11 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
         const uint16_t *xrow = xs + (size_t)tok * xs_stride + 8 * t;
         float aG[4] = {0.f, 0.f, 0.f, 0.f}, aU[4] = {0.f, 0.f, 0.f, 0.f};
         {
-            const int c = j * NCH + q, s = c % S;
-            if (!wait_chunk(full, S, c, &issued)) timed_out = true;
-            const uint8_t *st = stages + (size_t)s * kStageBytes;   // [gate block][up block]
+            const int c = j * NCH + q, pc = c / cps, s = pc % S;
+            if (!wait_piece(full, S, pc, &issued)) timed_out = true;
+            // [gate blocks of the piece][up blocks of the piece]
+            const uint8_t *st0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c % cps) * kBlk;
+            const uint8_t *st1 = st0 + (size_t)cps * kBlk;
 #pragma unroll
             for (int p = 0; p < NCH / 2; ++p) {
                 const int gp = wi * (NCH / 2) + p;
@@ -453,26 +487,18 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
                 uint4 xb[4];
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) xb[jj] = live ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
-                chunk_group(st, g, t, gp, xb, aG, aU);
+                chunk_group(st0, st1, g, t, gp, xb, aG, aU);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
-        float *rb = red + (size_t)(j & 1) * kCW * 32 * 8;
-        float4 *mine = reinterpret_cast<float4 *>(rb + ((size_t)warp * 32 + lane) * 8);
-        mine[0] = make_float4(aG[0], aG[1], aG[2], aG[3]);
-        mine[1] = make_float4(aU[0], aU[1], aU[2], aU[3]);
+        float *rb = red + (size_t)(j & 1) * kCW * 2 * 16 * Tc;
+        put_partials(rb, Tc, warp, g, t, aG, aU);
         named_sync_consumers();
-        if ((tid & 3) == 0) {   // 128 readers spread over the warps: 16 rows x 8 columns
-            const int r = tid >> 2, row = r >> 3, col = r & 7;
+        if ((lane & 3) == 0) {   // readers spread over the warps: (row, column) = r % 16, r / 16
+            const int r = warp + kCW * (lane >> 2), row = r & 15, col = r >> 4;
             if (col < ncol) {
-                const int src = (row & 7) * 4 + (col >> 1), slot = (row >> 3) * 2 + (col & 1);
-                float gs = 0.f, us = 0.f;
-#pragma unroll
-                for (int ww = 0; ww < kCW; ++ww) {
-                    gs += rb[((size_t)ww * 32 + src) * 8 + slot];
-                    us += rb[((size_t)ww * 32 + src) * 8 + 4 + slot];
-                }
+                const float gs = sum_partials(rb, Tc, 0, row, col), us = sum_partials(rb, Tc, 1, row, col);
                 const int route = tb.route[cb + col];
                 const float inv = xinv[route / k];
                 const float hv = silu_f32(gs * inv) * (us * inv);
@@ -500,15 +526,21 @@ struct DownArgs {
     int *counters;                  // [H/32], zero between calls
     uint16_t *out;                  // bf16 [T][H]
     uint32_t *status;
-    int T, k, E, H, I, n_stages;
+    int T, k, E, H, I, n_stages, cps;
 };
 
-constexpr int kMaxBSlots = 16;   // staged (expert, token) B columns per CTA
-
-__host__ __device__ inline size_t dn_red_off(int n_stages, int I) {
-    return (size_t)n_stages * kStageBytes + sizeof(uint16_t) * (size_t)kMaxBSlots * (I + kXPad);
+// Staged (expert, token) B columns per CTA.  A CTA's contiguous range of
+// units is shorter than one expert's tiles, so it touches at most two
+// experts: 2T columns (capped; beyond the cap B is built from h in L2).
+constexpr int kMaxBSlots = 16;
+constexpr int kMaxTiles = 128;   // H / 32 for H <= 4096
+__host__ __device__ inline int dn_slots(int T) { return 2 * T < kMaxBSlots ? 2 * T : kMaxBSlots; }
+__host__ __device__ inline size_t dn_red_off(int n_stages, int cps, int T, int I) {
+    return (size_t)n_stages * piece_bytes(cps) + sizeof(uint16_t) * (size_t)dn_slots(T) * (I + kXPad);
 }
-__host__ __device__ inline size_t dn_bytes(int n_stages, int I) { return dn_red_off(n_stages, I) + kRedBytes; }
+__host__ __device__ inline size_t dn_bytes(int n_stages, int cps, int T, int I) {
+    return dn_red_off(n_stages, cps, T, I) + red_bytes(T);
+}
 
 template <int NCH>   // K chunks per unit = I / kKC
 __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) {
@@ -519,11 +551,13 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
     __shared__ float tok_scale[kMaxT], tok_inv[kMaxT];
     __shared__ int slot_of[kMaxR][kMaxT];   // (expert slot - d_lo, token) -> staged B column, -1 none
     __shared__ int slot_d[kMaxBSlots], slot_t[kMaxBSlots];
-    __shared__ int n_slots, last_flag;
-    const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages;
+    __shared__ int n_slots, n_last;
+    __shared__ int last_tiles[kMaxTiles];
+    const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages, cps = a.cps, Tc = red_cols(a.T);
+    const int cap = dn_slots(T);
     uint8_t *stages = smem_raw;
-    uint16_t *bs = reinterpret_cast<uint16_t *>(smem_raw + (size_t)S * kStageBytes);   // [slot][I+pad] f16
-    float *red = reinterpret_cast<float *>(smem_raw + dn_red_off(S, I));
+    uint16_t *bs = reinterpret_cast<uint16_t *>(smem_raw + (size_t)S * piece_bytes(cps));   // [slot][I+pad] f16
+    float *red = reinterpret_cast<float *>(smem_raw + dn_red_off(S, cps, T, I));
     const int bs_stride = I + kXPad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -534,10 +568,11 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], WPC);
+            mbar_init(&empty[s], WPC * cps);
         }
         mbar_fence_init();
         issued = 0;
+        n_last = 0;
     }
     if (warp == 0) build_route_table(tb, a.ids, T * k, a.E, nullptr, false);
     __syncthreads();
@@ -552,8 +587,9 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
 
     if (warp == kProducerWarp) {
         // the weights do not depend on the gate/up kernel: stream them at once
-        produce(stages, full, empty, S, n_mine * NCH, a.status, &issued,
-                [&](int c, const uint8_t *&b0, const uint8_t *&b1) {
+        produce(stages, full, empty, S, cps, n_mine * NCH / cps, a.status, &issued,
+                [&](int p, const uint8_t *&b0, const uint8_t *&b1) {
+                    const int c = p * cps;
                     const int u = u0 + c / NCH, d = u / tiles, t32 = u % tiles, q = c % NCH;
                     const uint8_t *eb = a.codes + (size_t)tb.expert[d] * geo.expert_bytes();
                     b0 = eb + geo.block_off(2 * t32, q);
@@ -572,7 +608,7 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
                 for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) used |= (tb.route[cc] / k == tk);
                 int sl = -1;
                 if (used) {
-                    if (ns < kMaxBSlots) {
+                    if (ns < cap) {
                         slot_d[ns] = d;
                         slot_t[ns] = tk;
                     }
@@ -585,8 +621,15 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
     // h and gmax come from the gate/up kernel
     pdl_wait_primary();
     if (warp < kMaxT) {
-        float m = 0.f;
-        for (int i = lane; i < a.n_gmax; i += 32) m = fmaxf(m, __ldcg(a.gmax + (size_t)i * kMaxT + warp));
+        // eight independent loads per lane cover 256 CTAs in one round trip
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int i = lane + 32 * q;
+            v[q] = i < a.n_gmax ? __ldcg(a.gmax + (size_t)i * kMaxT + warp) : 0.f;
+        }
+        float m = fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
+        for (int i = lane + 256; i < a.n_gmax; i += 32) m = fmaxf(m, __ldcg(a.gmax + (size_t)i * kMaxT + warp));
 #pragma unroll
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) {
@@ -596,7 +639,7 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
         }
     }
     named_sync_consumers();
-    const bool staged = n_slots <= kMaxBSlots;
+    const bool staged = n_slots <= cap;
     if (staged) {
         // B column (d, token) = sum over the token's routes to expert d of
         // w * prescale * h, as f16 (summed in f32 first)
@@ -666,44 +709,47 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
                     }
                 }
             }
-            const int c = j * NCH + q, s = c % S;
-            if (!wait_chunk(full, S, c, &issued)) timed_out = true;
-            const uint8_t *st = stages + (size_t)s * kStageBytes;   // [rows m0..+15 block][rows m0+16..+31 block]
+            const int c = j * NCH + q, pc = c / cps, s = pc % S;
+            if (!wait_piece(full, S, pc, &issued)) timed_out = true;
+            // [rows m0..+15: blocks of the piece][rows m0+16..+31: blocks of the piece]
+            const uint8_t *st0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c % cps) * kBlk;
+            const uint8_t *st1 = st0 + (size_t)cps * kBlk;
 #pragma unroll
-            for (int p = 0; p < NCH / 2; ++p) chunk_group(st, g, t, wi * (NCH / 2) + p, xb[p], acc0, acc1);
+            for (int p = 0; p < NCH / 2; ++p) chunk_group(st0, st1, g, t, wi * (NCH / 2) + p, xb[p], acc0, acc1);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
-        float *rb = red + (size_t)(j & 1) * kCW * 32 * 8;
-        float4 *mine = reinterpret_cast<float4 *>(rb + ((size_t)warp * 32 + lane) * 8);
-        mine[0] = make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
-        mine[1] = make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
+        float *rb = red + (size_t)(j & 1) * kCW * 2 * 16 * Tc;
+        put_partials(rb, Tc, warp, g, t, acc0, acc1);
         named_sync_consumers();
-        if (tid < 256) {   // readers: warps 0..7, one (row, token) each
-            const int row = tid >> 3, col = tid & 7;   // 32 rows x 8 tokens
-            const int tt = row >> 4, rl = row & 15;
-            const int src = (rl & 7) * 4 + (col >> 1), slot = tt * 4 + (rl >> 3) * 2 + (col & 1);
-            if (col < T) {
-                float sum = 0.f;
-#pragma unroll
-                for (int ww = 0; ww < kCW; ++ww) sum += rb[((size_t)ww * 32 + src) * 8 + slot];
-                __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row, sum);
-            }
-            __threadfence();
-            named_sync_readers();
-            if (tid == 0) last_flag = (atomicAdd(a.counters + tile, 1) == tb.D - 1);
-            named_sync_readers();
-            if (last_flag) {   // every expert of this tile is in: sum in expert order, write bf16
-                __threadfence();
-                if (col < T) {
-                    float sum = 0.f;
-                    for (int dd = 0; dd < tb.D; ++dd) sum += __ldcg(a.ybuf + ((size_t)dd * kMaxT + col) * H + m0 + row);
-                    __nv_bfloat16 o = __float2bfloat16_rn(sum * tok_inv[col]);
-                    a.out[(size_t)col * H + m0 + row] = *reinterpret_cast<uint16_t *>(&o);
-                }
-                if (tid == 0) a.counters[tile] = 0;
-            }
+        if ((lane & 1) == 0) {   // readers spread over the warps: (row, token) = r % 32, r / 32
+            const int r = warp + kCW * (lane >> 1), row = r & 31, col = r >> 5;
+            if (col < T)
+                __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row,
+                       sum_partials(rb, Tc, row >> 4, row & 15, col));
         }
+    }
+    // Combine: once every expert's slice of a 32-row tile is in, the CTA
+    // whose unit completed it sums the slices in expert order, undoes the
+    // prescale and writes bf16; the order of the sum does not depend on
+    // timing.
+    __threadfence();
+    named_sync_consumers();
+    for (int j = tid; j < n_mine; j += 32 * kCW) {
+        const int tile = (u0 + j) % tiles;
+        if (atomicAdd(a.counters + tile, 1) == tb.D - 1) last_tiles[atomicAdd(&n_last, 1)] = tile;
+    }
+    named_sync_consumers();
+    if (n_last > 0) {
+        __threadfence();
+        for (int idx = tid; idx < n_last * 32 * T; idx += 32 * kCW) {
+            const int row = idx & 31, col = (idx >> 5) % T, m0 = last_tiles[(idx >> 5) / T] * 32;
+            float sum = 0.f;
+            for (int dd = 0; dd < tb.D; ++dd) sum += __ldcg(a.ybuf + ((size_t)dd * kMaxT + col) * H + m0 + row);
+            __nv_bfloat16 o = __float2bfloat16_rn(sum * tok_inv[col]);
+            a.out[(size_t)col * H + m0 + row] = *reinterpret_cast<uint16_t *>(&o);
+        }
+        for (int li = tid; li < n_last; li += 32 * kCW) a.counters[last_tiles[li]] = 0;
     }
     if (timed_out && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
 }
@@ -723,14 +769,22 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
     return cudaLaunchKernelEx(&cfg, kernel, args);
 }
 
-int gu_stages(int T, int H) {
-    int s = (int)((kMaxDynSmem - gu_bytes(0, T, H)) / kStageBytes);
-    return s > kMaxStages ? kMaxStages : s;
+// Stages and chunks per stage (cps, a divisor of the unit's nch chunks) for
+// a kernel whose other shared memory takes `fixed` bytes: the largest pieces
+// that still leave three stages, else one chunk per stage.
+struct StagePlan {
+    int S, cps;
+};
+StagePlan plan_stages(int nch, size_t fixed) {
+    for (int cps = nch; cps >= 1; cps /= 2) {
+        long long s = ((long long)kMaxDynSmem - (long long)fixed) / (long long)piece_bytes(cps);
+        if (s > kMaxStages) s = kMaxStages;
+        if (s >= 3 || cps == 1) return {(int)(s < 0 ? 0 : s), cps};
+    }
+    return {0, 1};
 }
-int dn_stages(int I) {
-    int s = (int)((kMaxDynSmem - dn_bytes(0, I)) / kStageBytes);
-    return s > kMaxStages ? kMaxStages : s;
-}
+StagePlan gu_plan(int T, int H) { return plan_stages(H / kKC, gu_bytes(0, 1, T, H)); }
+StagePlan dn_plan(int T, int I) { return plan_stages(I / kKC, dn_bytes(0, 1, T, I)); }
 
 template <int NCU, int NCD>
 cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
@@ -762,11 +816,13 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     ga.E = L.d.n_experts;
     ga.H = H;
     ga.I = I;
-    ga.n_stages = gu_stages(T, H);
+    const StagePlan gp = gu_plan(T, H);
+    ga.n_stages = gp.S;
+    ga.cps = gp.cps;
     L.count_launches(2);
     if (ev) record_phase(ev[1], s);   // routing is fused into both kernels' prologues
     cudaError_t e = launch_ex(dec_gateup_mx_kernel<NCU>, dim3(grid), dim3(kWSThreads),
-                              gu_bytes(ga.n_stages, T, H), s, false, ga);
+                              gu_bytes(ga.n_stages, ga.cps, T, H), s, false, ga);
     if (e != cudaSuccess) return e;
     if (ev) record_phase(ev[2], s);
     DownArgs da;
@@ -785,11 +841,13 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     da.E = L.d.n_experts;
     da.H = H;
     da.I = I;
-    da.n_stages = dn_stages(I);
+    const StagePlan dp = dn_plan(T, I);
+    da.n_stages = dp.S;
+    da.cps = dp.cps;
     // programmatic dependent launch: the down kernel's producer streams
     // weights while the gate/up kernel drains; its consumers wait for that
     // grid before reading h.  Not with phase events between the launches.
-    e = launch_ex(dec_down_mx_kernel<NCD>, dim3(grid), dim3(kWSThreads), dn_bytes(da.n_stages, I), s, ev == nullptr,
+    e = launch_ex(dec_down_mx_kernel<NCD>, dim3(grid), dim3(kWSThreads), dn_bytes(da.n_stages, da.cps, T, I), s, ev == nullptr,
                   da);
     if (e != cudaSuccess) return e;
     if (ev) {
@@ -806,7 +864,8 @@ bool decode_mx_supported(const Layer &L, int T) {
     if (d.fmt != MOEQ_FMT_MXFP4 || d.act != MOEQ_ACT_BF16) return false;
     if (T < 1 || T > kMaxT || T * d.top_k > kMaxR) return false;
     if (!((d.hidden == 2048 || d.hidden == 4096) && (d.inter == 2048 || d.inter == 4096))) return false;
-    if (gu_stages(kMaxT, d.hidden) < 2 || dn_stages(d.inter) < 2) return false;
+    for (int tt = 1; tt <= kMaxT; ++tt)
+        if (gu_plan(tt, d.hidden).S < 2 || dn_plan(tt, d.inter).S < 2) return false;
     return L.sm_count > 0 && L.sm_count <= kDecMaxGrid;
 }
 
