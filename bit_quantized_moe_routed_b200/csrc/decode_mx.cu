@@ -314,22 +314,37 @@ __device__ __forceinline__ float sum_partials(const float *rb, int Tc, int half,
     return s;
 }
 
-// One 32-weight block pair (both halves) of K-group gp of a staged chunk
-// (half-0 block st0, half-1 block st1) against the four B fragments
-// xb[0..3] of that group.
-__device__ __forceinline__ void chunk_group(const uint8_t *st0, const uint8_t *st1, int g, int t, int gp,
-                                            const uint4 xb[4], float acc0[4], float acc1[4]) {
-    const uint4 a0 = lds128(frag_ptr(st0, g, gp, t)), a8 = lds128(frag_ptr(st0, g + 8, gp, t));
-    const uint4 b0 = lds128(frag_ptr(st1, g, gp, t)), b8 = lds128(frag_ptr(st1, g + 8, gp, t));
+// A warp's share of one K-group of a staged chunk, read into registers so
+// that the stage can be released before the math: the fragment words of
+// rows g and g+8 of both halves (half-0 block st0, half-1 block st1) and
+// their scale words.
+struct GroupFrags {
+    uint4 a0, a8, b0, b8;
+    uint32_t sa0, sa8, sb0, sb8;
+};
+__device__ __forceinline__ void load_group(const uint8_t *st0, const uint8_t *st1, int g, int t, int gp,
+                                           GroupFrags &f) {
+    f.a0 = lds128(frag_ptr(st0, g, gp, t));
+    f.a8 = lds128(frag_ptr(st0, g + 8, gp, t));
+    f.b0 = lds128(frag_ptr(st1, g, gp, t));
+    f.b8 = lds128(frag_ptr(st1, g + 8, gp, t));
+    f.sa0 = lds32(scale_ptr(st0, g, gp));
+    f.sa8 = lds32(scale_ptr(st0, g + 8, gp));
+    f.sb0 = lds32(scale_ptr(st1, g, gp));
+    f.sb8 = lds32(scale_ptr(st1, g + 8, gp));
+}
+// The four 32-weight block pairs of a loaded group against the four B
+// fragments xb[0..3] of that group.
+__device__ __forceinline__ void compute_group(const GroupFrags &f, const uint4 xb[4], float acc0[4], float acc1[4]) {
     float sa0[4], sa8[4], sb0[4], sb8[4];
-    e8m0x4(lds32(scale_ptr(st0, g, gp)), sa0);
-    e8m0x4(lds32(scale_ptr(st0, g + 8, gp)), sa8);
-    e8m0x4(lds32(scale_ptr(st1, g, gp)), sb0);
-    e8m0x4(lds32(scale_ptr(st1, g + 8, gp)), sb8);
+    e8m0x4(f.sa0, sa0);
+    e8m0x4(f.sa8, sa8);
+    e8m0x4(f.sb0, sb0);
+    e8m0x4(f.sb8, sb8);
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
-        block_mma(acc0, u4get(a0, jj), u4get(a8, jj), xb[jj], sa0[jj], sa8[jj]);
-        block_mma(acc1, u4get(b0, jj), u4get(b8, jj), xb[jj], sb0[jj], sb8[jj]);
+        block_mma(acc0, u4get(f.a0, jj), u4get(f.a8, jj), xb[jj], sa0[jj], sa8[jj]);
+        block_mma(acc1, u4get(f.b0, jj), u4get(f.b8, jj), xb[jj], sb0[jj], sb8[jj]);
     }
 }
 
@@ -480,6 +495,12 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
             // [gate blocks of the piece][up blocks of the piece]
             const uint8_t *st0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c % cps) * kBlk;
             const uint8_t *st1 = st0 + (size_t)cps * kBlk;
+            GroupFrags fr[NCH / 2];
+#pragma unroll
+            for (int p = 0; p < NCH / 2; ++p) load_group(st0, st1, g, t, wi * (NCH / 2) + p, fr[p]);
+            // the stage is free again once every warp holds its share
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
 #pragma unroll
             for (int p = 0; p < NCH / 2; ++p) {
                 const int gp = wi * (NCH / 2) + p;
@@ -487,10 +508,8 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
                 uint4 xb[4];
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) xb[jj] = live ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
-                chunk_group(st0, st1, g, t, gp, xb, aG, aU);
+                compute_group(fr[p], xb, aG, aU);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
         }
         float *rb = red + (size_t)(j & 1) * kCW * 2 * 16 * Tc;
         put_partials(rb, Tc, warp, g, t, aG, aU);
@@ -714,10 +733,14 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
             // [rows m0..+15: blocks of the piece][rows m0+16..+31: blocks of the piece]
             const uint8_t *st0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c % cps) * kBlk;
             const uint8_t *st1 = st0 + (size_t)cps * kBlk;
+            GroupFrags fr[NCH / 2];
 #pragma unroll
-            for (int p = 0; p < NCH / 2; ++p) chunk_group(st0, st1, g, t, wi * (NCH / 2) + p, xb[p], acc0, acc1);
+            for (int p = 0; p < NCH / 2; ++p) load_group(st0, st1, g, t, wi * (NCH / 2) + p, fr[p]);
+            // the stage is free again once every warp holds its share
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+            for (int p = 0; p < NCH / 2; ++p) compute_group(fr[p], xb[p], acc0, acc1);
         }
         float *rb = red + (size_t)(j & 1) * kCW * 2 * 16 * Tc;
         put_partials(rb, Tc, warp, g, t, acc0, acc1);
