@@ -82,6 +82,7 @@ void free_layer(moeq_layer *L) {
     cudaFree(L->out_stage);
     cudaFree(L->ids_stage);
     cudaFree(L->w_stage);
+    prefill_mx_free(*L);
     delete L;
 }
 
@@ -110,6 +111,9 @@ moeq_status launch_forward(moeq_layer *L, const void *x, const int32_t *ids, con
     if (ev) record_phase(ev[0], s);
     // the decode kernels bulk-copy token rows of x: 16-byte aligned x only
     if (decode_mx_supported(*L, T) && ((uintptr_t)x & 15u) == 0) return from_cuda(launch_decode_mx(*L, x, ids, w, T, out, s, ev));
+    // the prefill kernels read x rows as 16-byte vectors
+    if (prefill_mx_supported(*L, T) && ((uintptr_t)x & 15u) == 0)
+        return from_cuda(launch_prefill_mx(*L, x, ids, w, T, out, s, ev));
     cudaError_t e = launch_route_bucket(*L, ids, T * L->d.top_k, L->b.offsets, L->b.perm, L->b.active, s);
     if (e != cudaSuccess) return from_cuda(e);
     if (ev) record_phase(ev[1], s);
@@ -187,6 +191,7 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     ALLOC(L->ids_stage, sizeof(int32_t) * M * k);
     ALLOC(L->w_stage, sizeof(float) * M * k);
 #undef ALLOC
+    if (e == cudaSuccess) e = prefill_mx_create(*L);
     if (e == cudaSuccess) e = cudaMemset(L->status, 0, sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMemset(L->dec_counters, 0, sizeof(int) * (H / 32 + 1));
     if (e != cudaSuccess) {
@@ -259,6 +264,7 @@ moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *str
                                         cudaMemcpyHostToDevice, s);
                 if (e == cudaSuccess)
                     e = launch_mx_pack(tmp_c, tmp_s, L->w.codes[p] + (size_t)e0 * geo.expert_bytes(), geo, ne, s);
+                if (e == cudaSuccess) e = prefill_mx_upload(*L, p, tmp_c, tmp_s, e0, ne, s);
             }
         } else {
             e = cudaMemcpyAsync(L->w.idx13[p], w->idx13[p], rows * row_bytes(fmt, 0, K), cudaMemcpyHostToDevice, s);
@@ -273,6 +279,7 @@ moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *str
     if (e == cudaSuccess && r8)
         e = cudaMemcpyAsync(L->w.book8, w->book8, sizeof(uint16_t) * kBook8Rows * 8, cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess && mx) e = prefill_mx_finish_upload(*L);
     cudaFree(tmp_c);
     cudaFree(tmp_s);
     if (e != cudaSuccess) return from_cuda(e);

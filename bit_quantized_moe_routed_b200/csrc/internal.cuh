@@ -2,6 +2,7 @@
 // the public ABI; see include/moeq.h for that).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -56,8 +57,26 @@ struct ProjView {
     int32_t N, K;
 };
 
+// Prefill path for MXFP4 (prefill_mx.cu): a second copy of the weights in the
+// logical layout for tensor copies, scale atoms, activation workspaces and the
+// tensor maps over them.
+struct PrefillMx {
+    CUtensorMap map_w[3];          // codes [E*N][K] as 4-bit elements
+    CUtensorMap map_x[2];          // activation terms [route position][H]
+    CUtensorMap map_h[2];          // intermediate terms [route position][I]
+    uint8_t *codes[3] = {nullptr, nullptr, nullptr};      // [E*N][K/2], logical layout
+    uint8_t *sf_atoms[3] = {nullptr, nullptr, nullptr};   // [E][N/128][K/128][512]
+    int32_t *tile_base = nullptr;  // [E+1]
+    uint8_t *xq[2] = {nullptr, nullptr};
+    uint8_t *sfx = nullptr;
+    uint8_t *hq[2] = {nullptr, nullptr};
+    uint8_t *sfh = nullptr;
+    bool maps_ready = false;
+};
+
 struct Layer {
     moeq_layer_desc d{};
+    PrefillMx *pf = nullptr;
     DevWeights w;
     Buckets b;
     float *h = nullptr;        // [max_tokens*k][I] SwiGLU intermediates, route-sorted order
@@ -103,6 +122,15 @@ cudaError_t launch_dequant(const Layer &L, int expert, int proj, float *out, cud
 bool decode_mx_supported(const Layer &L, int T);
 cudaError_t launch_decode_mx(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T,
                              void *out, cudaStream_t s, const cudaEvent_t *ev);
+bool prefill_mx_supported(const Layer &L, int T);
+cudaError_t prefill_mx_create(Layer &L);
+void prefill_mx_free(Layer &L);
+// experts [e0, e0+ne) of projection p from logical planes already on the device
+cudaError_t prefill_mx_upload(Layer &L, int p, const uint8_t *codes, const uint8_t *scales, int e0, int ne,
+                              cudaStream_t s);
+cudaError_t prefill_mx_finish_upload(Layer &L);
+cudaError_t launch_prefill_mx(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
+                              cudaStream_t s, const cudaEvent_t *ev);
 cudaError_t launch_ffn_simt(const Layer &L, const void *x, const float *topk_w, int32_t n_tokens,
                             void *out, cudaStream_t s, const cudaEvent_t *ev);
 

@@ -1,0 +1,809 @@
+// prefill_mx.cu -- MXFP4 routed-expert FFN at prefill sizes (more than 8
+// tokens, bf16 activations) on the 5th-generation tensor cores.
+//
+// Layer: out[t] = sum_s w[t,s] W_down,e (silu(W_gate,e x_t) * (W_up,e x_t))
+// ("MiMo-V2.6-Flash-RL GGUF for a single DGX Spark", "Architecture notes":
+// 8 of 256 routed experts per token, MXFP4 experts with one E8M0 exponent per
+// 32 values; "Speed": prefill runs in micro-batches of 2048 tokens and each
+// expert's tokens are gathered into one matmul; "Recipe": intermediates keep
+// f32's range).
+//
+// The weights never pass through the SM's arithmetic: tcgen05.mma
+// kind::mxf8f6f4.block_scale multiplies the E2M1 codes as stored, with their
+// E8M0 block scales in tensor memory.  The other operand must be an 8-bit
+// (or narrower) float with its own E8M0 scale per 32 values, so every
+// activation block is written as x = 2^s (q1 + q2), q1 = RN_E4M3(x 2^-s),
+// q2 = RN_E4M3(x 2^-s - q1), s chosen so that max|x| 2^-s lies in [128,
+// 256).  For bf16 x (8 significant bits) q1 + q2 is exact (q1 keeps 4 bits,
+// the remainder has at most 4); for the f32 intermediates h it keeps about
+// 8 bits.  Two MMAs (one per term) accumulate into the same f32 tensor-
+// memory tile, so the products are exact and the sums are f32.
+//
+// Steps of one forward (all on the stream, no host synchronisation):
+//   route/bucket (route.cu)  -> offsets[E+1], perm (route ids by expert)
+//   pf_tiles_kernel          -> tile_base[E+1]: expert e's routes form
+//                               ceil(n_e/128) tiles of up to 128 routes
+//   pf_quant_x_kernel        -> q1, q2 [route position][H] and their scale
+//                               atoms, one row per route (a gather of x)
+//   pf_gateup_kernel         -> per (route tile, 128 rows of I): gate and up
+//                               tiles in tensor memory, SwiGLU in f32, h
+//                               quantised the same way for the down matmul
+//   pf_down_kernel           -> per (route tile, 128 rows of H): y tile,
+//                               weighted by w[t,s] and added into acc[T][H]
+//   pf_cast_kernel           -> out = bf16(acc)
+//
+// Data in HBM: each projection's codes in their logical layout [E*N][K/2]
+// (read by TMA tensor copies that widen each 16-value packet to 16 bytes in
+// shared memory, as the MMA wants E2M1 operands), and its scales re-laid
+// into 512-byte atoms [E][N/128][K/128][32 rows][4 row groups][4 blocks]:
+// the shared-memory image that tcgen05.cp copies into tensor memory.
+//
+// CTA roles (one CTA per SM, persistent over work items): warp 0 issues TMA
+// copies into a ring of stages, warp 1 issues the MMAs (one thread) and owns
+// the tensor memory, warps 2..5 run the epilogue.  Every wait is bounded;
+// on expiry the kernel sets MOEQ_ERR_TIMEOUT, every role stops, and the
+// tensor memory is released.
+#include <cuda.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "async.cuh"
+#include "internal.cuh"
+
+namespace moeq {
+namespace {
+
+constexpr int kT = 128;           // MMA M (weight rows per tile), max MMA N (routes per tile), K per slab
+constexpr int kPfThreads = 192;   // producer, MMA, 4 epilogue warps
+constexpr int kBoxA = 8192;       // bytes one A box moves from HBM (128 rows x 128 E2M1 codes)
+constexpr int kTileS = 16384;     // shared-memory bytes of one 128 x 128 operand tile (A widened, or B)
+constexpr int kAtom = 512;        // one scale-factor atom: 128 rows x 4 blocks of 32
+
+// gate/up stage: [A gate][A up][B q1][B q2][SF gate][SF up][SF x]
+constexpr int kGUStage = 4 * kTileS + 3 * kAtom + 512;   // padded to 1 KB
+constexpr int kGUStages = 3;
+// down stage: [A down][B q1][B q2][SF down][SF h]
+constexpr int kDNStage = 3 * kTileS + 2 * kAtom;
+constexpr int kDNStages = 4;
+
+// tensor-memory columns: accumulators, then a scale-factor ring (4 columns per atom)
+constexpr int kGUTmemCols = 512;   // gate 128 + up 128, SF ring 3 stages x 12
+constexpr int kDNTmemCols = 256;   // y 128, SF ring 4 stages x 8
+
+constexpr long long kWaitCycles = 2000000000LL;
+
+// ---------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major.  128B swizzle: rows of 128 bytes,
+// 8-row groups 1024 bytes apart.  None: 8 x 16-byte core matrices, groups of
+// 8 rows `sbo` bytes apart, 16-byte columns `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128(const void *p) {
+    return (uint64_t)((smem_u32(p) >> 4) & 0x3FFF) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+__device__ __forceinline__ uint64_t desc_plain(const void *p, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((smem_u32(p) >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46);
+}
+// Instruction descriptor: kind::mxf8f6f4 block-scaled, A E2M1, B E4M3, f32
+// accumulate, E8M0 scales, M 128, both operands K-major, K 32 per MMA;
+// a_sf / b_sf pick the byte (the 32-block) of each scale-factor column.
+__device__ __forceinline__ uint32_t idesc_mx(int n, int a_sf, int b_sf) {
+    return ((uint32_t)(b_sf & 3) << 4) | (5u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(kT >> 4) << 24) | ((uint32_t)(a_sf & 3) << 29);
+}
+__device__ __forceinline__ void mma_mx(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc, uint32_t sfa,
+                                       uint32_t sfb) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+__device__ __forceinline__ void tc_cp_atom(uint32_t taddr, const void *atom) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc_plain(atom, 128, 128))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_alloc(uint32_t *slot, int cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_dealloc(uint32_t taddr, int cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+// 16 consecutive f32 columns of this warp's 32 lanes
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float v[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Bounded wait that also gives up once another role has given up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// Before the CTA releases its shared and tensor memory: wait (bounded,
+// whatever happened) for the copies of the last stages issued, and for every
+// MMA this thread issued.
+__device__ __forceinline__ void drain_stages(uint64_t *full, int S, int issued) {
+    for (int c = issued > S ? issued - S : 0; c < issued; ++c)
+        mbar_wait_bounded(&full[c % S], (uint32_t)((c / S) & 1), 200000000LL);
+}
+__device__ __forceinline__ void drain_mma(uint64_t *done) {
+    tc_commit(done);
+    mbar_wait_bounded(done, 0, 200000000LL);
+}
+
+// 2^s for s in [-126, 127]
+__device__ __forceinline__ float pow2i(int s) { return __uint_as_float((uint32_t)(s + 127) << 23); }
+
+// Split v (|v| < 256 after scaling) into two E4M3 terms, v = q1 + q2 (to the
+// precision E4M3 keeps of the remainder).  Round to nearest even.
+__device__ __forceinline__ void split_e4m3(float v, uint8_t &q1, uint8_t &q2) {
+    const __nv_fp8_storage_t a = __nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+    const float av = __half2float(__half(__nv_cvt_fp8_to_halfraw(a, __NV_E4M3)));
+    const __nv_fp8_storage_t b = __nv_cvt_float_to_fp8(v - av, __NV_SATFINITE, __NV_E4M3);
+    q1 = a;
+    q2 = b;
+}
+
+// Block scale exponent for a block whose largest magnitude is m: m 2^-s in
+// [128, 256); 0 for an all-zero block.  Kept inside E8M0's range.
+__device__ __forceinline__ int block_exp(float m) {
+    if (!(m > 0.f)) return 0;
+    const int eb = (int)((__float_as_uint(m) >> 23) & 0xFF);
+    int s = (eb ? eb - 127 : -127) - 7;
+    return s < -127 ? -127 : (s > 127 ? 127 : s);
+}
+// v * 2^-s without leaving f32's range in the intermediate factor
+__device__ __forceinline__ float scale_down(float v, int s) {
+    const int a = -s / 2, b = -s - a;
+    return v * pow2i(a) * pow2i(b);
+}
+
+// Scale-factor atom byte of (row r of a 128-row tile, 32-block kb of a 4-block group)
+__device__ __forceinline__ int atom_byte(int r, int kb) { return (r & 31) * 16 + (r >> 5) * 4 + kb; }
+
+// Expert of global route tile tau: the last e with tile_base[e] <= tau.
+__device__ __forceinline__ int expert_of_tile(const int32_t *tile_base, int E, int tau) {
+    int lo = 0, hi = E;   // tile_base[lo] <= tau < tile_base[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(tile_base + mid) <= tau) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+struct Item {
+    int e, j, sub;     // expert, route tile of the expert, 128-row tile of the output
+    int row0;          // first route position of the tile
+    int cnt;           // routes in the tile (1..128)
+    int tau;           // global route tile
+};
+__device__ __forceinline__ Item decode_item(const int32_t *offsets, const int32_t *tile_base, int E, int subs,
+                                            int it) {
+    Item m;
+    m.tau = it / subs;
+    m.sub = it % subs;
+    m.e = expert_of_tile(tile_base, E, m.tau);
+    m.j = m.tau - __ldg(tile_base + m.e);
+    const int beg = __ldg(offsets + m.e), n_e = __ldg(offsets + m.e + 1) - beg;
+    m.row0 = beg + kT * m.j;
+    m.cnt = min(kT, n_e - kT * m.j);
+    return m;
+}
+
+// ---------------------------------------------------------------- small kernels
+
+// tile_base[e] = sum over e' < e of ceil(n_e' / 128); tile_base[E] = all tiles.
+__global__ void __launch_bounds__(1024) pf_tiles_kernel(const int32_t *__restrict__ offsets, int E,
+                                                        int32_t *__restrict__ tile_base) {
+    __shared__ int32_t warp_off[32];
+    __shared__ int32_t chunk_total;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += 1024) {
+        const int e = e0 + tid;
+        const int v = e < E ? (offsets[e + 1] - offsets[e] + kT - 1) / kT : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_off[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int ws = warp_off[lane];
+            int wi = ws;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += y;
+            }
+            warp_off[lane] = wi - ws;
+            if (lane == 31) chunk_total = wi;
+        }
+        __syncthreads();
+        if (e < E) tile_base[e] = carry + warp_off[warp] + incl - v;
+        carry += chunk_total;
+        __syncthreads();
+    }
+    if (tid == 0) tile_base[E] = carry;
+}
+
+// One warp per route position p: x of its token, split into two E4M3 rows
+// and a scale per 32 values, stored at row p (the gather by expert).
+__global__ void __launch_bounds__(256) pf_quant_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ perm,
+                                                         const int32_t *__restrict__ ids, const int32_t *__restrict__ offsets,
+                                                         const int32_t *__restrict__ tile_base, int E, int k, int H,
+                                                         uint8_t *__restrict__ q1, uint8_t *__restrict__ q2,
+                                                         uint8_t *__restrict__ sfx) {
+    const int n_valid = __ldg(offsets + E);
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int n_warps = (gridDim.x * blockDim.x) >> 5;
+    for (int p = warp; p < n_valid; p += n_warps) {
+        const int r = __ldg(perm + p), t = r / k, e = __ldg(ids + r);
+        const int l = p - __ldg(offsets + e), tau = __ldg(tile_base + e) + l / kT, row = l % kT;
+        const uint16_t *xr = x + (size_t)t * H;
+        // lane handles 32-blocks lane, lane+32, ...
+        for (int b = lane; b < H / 32; b += 32) {
+            float v[32];
+            const uint4 *src = reinterpret_cast<const uint4 *>(xr + b * 32);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 w = __ldg(src + c);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v[c * 8 + 2 * j] = __uint_as_float(ww[j] << 16);
+                    v[c * 8 + 2 * j + 1] = __uint_as_float(ww[j] & 0xFFFF0000u);
+                }
+            }
+            float m = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
+            const int s = block_exp(m);
+            uint32_t o1[8], o2[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                uint32_t a = 0, bb = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint8_t u1, u2;
+                    split_e4m3(scale_down(v[4 * i + j], s), u1, u2);
+                    a |= (uint32_t)u1 << (8 * j);
+                    bb |= (uint32_t)u2 << (8 * j);
+                }
+                o1[i] = a;
+                o2[i] = bb;
+            }
+            uint4 *d1 = reinterpret_cast<uint4 *>(q1 + (size_t)p * H + b * 32);
+            uint4 *d2 = reinterpret_cast<uint4 *>(q2 + (size_t)p * H + b * 32);
+            d1[0] = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+            d1[1] = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+            d2[0] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+            d2[1] = make_uint4(o2[4], o2[5], o2[6], o2[7]);
+            sfx[((size_t)tau * (H / kT) + b / 4) * kAtom + atom_byte(row, b % 4)] = (uint8_t)(s + 127);
+        }
+    }
+}
+
+// Weight scales [ne][N][K/32] -> atoms [ne][N/128][K/128][512].
+__global__ void pf_sf_atoms_kernel(const uint8_t *__restrict__ sc, int ne, int N, int K, uint8_t *__restrict__ atoms) {
+    const long long n = (long long)ne * N * (K / 32);
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const int kb = (int)(i % (K / 32));
+    const long long rowg = i / (K / 32);
+    const int row = (int)(rowg % N);
+    const long long e = rowg / N;
+    const size_t atom = ((size_t)(e * (N / kT) + row / kT) * (K / kT) + kb / 4);
+    atoms[atom * kAtom + atom_byte(row % kT, kb % 4)] = sc[i];
+}
+
+__global__ void pf_cast_kernel(const float *__restrict__ acc, __nv_bfloat16 *__restrict__ out, long long n) {
+    const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (i + 3 < n) {
+        const float4 v = *reinterpret_cast<const float4 *>(acc + i);
+        out[i] = __float2bfloat16_rn(v.x);
+        out[i + 1] = __float2bfloat16_rn(v.y);
+        out[i + 2] = __float2bfloat16_rn(v.z);
+        out[i + 3] = __float2bfloat16_rn(v.w);
+    } else {
+        for (long long j = i; j < n; ++j) out[j] = __float2bfloat16_rn(acc[j]);
+    }
+}
+
+// ---------------------------------------------------------------- gate/up
+
+struct PfArgs {
+    const int32_t *offsets, *tile_base, *perm, *ids;
+    const float *topk_w;
+    const uint8_t *sfa0, *sfa1;   // weight scale atoms: gate, up (or down in sfa0)
+    const uint8_t *sfb;           // activation scale atoms [tiles][K/128][512]
+    uint8_t *hq1, *hq2, *sfh;     // gate/up: quantised h and its scale atoms
+    float *acc;                   // down: f32 output accumulator [T][H]
+    uint32_t *status;
+    int E, H, I, k;
+};
+
+__global__ void __launch_bounds__(kPfThreads, 1)
+    pf_gateup_kernel(const __grid_constant__ CUtensorMap tWg, const __grid_constant__ CUtensorMap tWu,
+                     const __grid_constant__ CUtensorMap tX1, const __grid_constant__ CUtensorMap tX2, PfArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full[kGUStages], empty[kGUStages], tmem_full, tmem_empty, tmem_done;
+    __shared__ uint32_t tslot;
+    __shared__ volatile int abort_flag;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H, I = a.I, E = a.E;
+    const int subs = I / kT, slabs = H / kT;
+
+    if (tid == 0) {
+        for (int s = 0; s < kGUStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&tmem_full, 1);
+        mbar_init(&tmem_empty, 4);
+        mbar_init(&tmem_done, 1);
+        mbar_fence_init();
+        abort_flag = 0;
+    }
+    if (warp == 1) tc_alloc(&tslot, kGUTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tslot;
+    const uint32_t t_g = tmem, t_u = tmem + kT, t_sf = tmem + 2 * kT;
+    const int n_items = __ldg(a.tile_base + E) * subs;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int c = 0;
+            for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x) {
+                const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+                const int wrow = m.e * I + m.sub * kT;
+                const uint8_t *sg = a.sfa0 + ((size_t)(m.e * subs + m.sub) * slabs) * kAtom;
+                const uint8_t *su = a.sfa1 + ((size_t)(m.e * subs + m.sub) * slabs) * kAtom;
+                const uint8_t *sx = a.sfb + ((size_t)m.tau * slabs) * kAtom;
+                for (int sl = 0; sl < slabs; ++sl, ++c) {
+                    const int s = c % kGUStages;
+                    if (c >= kGUStages && !wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag))
+                        break;
+                    uint8_t *st = smem + (size_t)s * kGUStage;
+                    mbar_arrive_expect_tx(&full[s], 2 * kBoxA + 2 * kTileS + 3 * kAtom);
+                    tma_load_2d(st, &tWg, sl * kT, wrow, &full[s]);
+                    tma_load_2d(st + kTileS, &tWu, sl * kT, wrow, &full[s]);
+                    tma_load_2d(st + 2 * kTileS, &tX1, sl * kT, m.row0, &full[s]);
+                    tma_load_2d(st + 3 * kTileS, &tX2, sl * kT, m.row0, &full[s]);
+                    bulk_g2s(st + 4 * kTileS, sg + (size_t)sl * kAtom, kAtom, &full[s]);
+                    bulk_g2s(st + 4 * kTileS + kAtom, su + (size_t)sl * kAtom, kAtom, &full[s]);
+                    bulk_g2s(st + 4 * kTileS + 2 * kAtom, sx + (size_t)sl * kAtom, kAtom, &full[s]);
+                }
+            }
+            drain_stages(full, kGUStages, c);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int c = 0, q = 0;
+            for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
+                const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+                const int n = (m.cnt + 15) & ~15;
+                if (q > 0 && !wait_or_abort(&tmem_empty, (uint32_t)((q - 1) & 1), &abort_flag)) break;
+                tc_fence_after();
+                for (int sl = 0; sl < slabs; ++sl, ++c) {
+                    const int s = c % kGUStages;
+                    if (!wait_or_abort(&full[s], (uint32_t)((c / kGUStages) & 1), &abort_flag)) break;
+                    tc_fence_after();
+                    const uint8_t *st = smem + (size_t)s * kGUStage;
+                    const uint32_t sfg = t_sf + 12 * s, sfu = sfg + 4, sfx = sfg + 8;
+                    tc_cp_atom(sfg, st + 4 * kTileS);
+                    tc_cp_atom(sfu, st + 4 * kTileS + kAtom);
+                    tc_cp_atom(sfx, st + 4 * kTileS + 2 * kAtom);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t id = idesc_mx(n, kk, kk);
+                        const uint64_t ag = desc_sw128(st + kk * 32), au = desc_sw128(st + kTileS + kk * 32);
+                        const uint64_t b1 = desc_sw128(st + 2 * kTileS + kk * 32), b2 = desc_sw128(st + 3 * kTileS + kk * 32);
+                        const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
+                        mma_mx(t_g, ag, b1, id, acc, sfg, sfx);
+                        mma_mx(t_g, ag, b2, id, 1u, sfg, sfx);
+                        mma_mx(t_u, au, b1, id, acc, sfu, sfx);
+                        mma_mx(t_u, au, b2, id, 1u, sfu, sfx);
+                    }
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(&tmem_full);
+            }
+            drain_mma(&tmem_done);
+        }
+    } else {
+        // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 = rows of I
+        const int qd = warp & 3;
+        int q = 0;
+        for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
+            const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+            if (!wait_or_abort(&tmem_full, (uint32_t)(q & 1), &abort_flag)) break;
+            tc_fence_after();
+            const int i_row = m.sub * kT + 32 * qd + lane;   // this lane's row of I
+            const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+            for (int n0 = 0; n0 < m.cnt; n0 += 16) {
+                float g[16], u[16];
+                tc_ld16(t_g + lane_off + n0, g);
+                tc_ld16(t_u + lane_off + n0, u);
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int n = n0 + jj;
+                    if (n >= m.cnt) break;
+                    const float h = silu_f32(g[jj]) * u[jj];
+                    float mx = fabsf(h);
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    const int s = block_exp(isfinite(mx) ? mx : 3.0e38f);
+                    uint8_t b1, b2;
+                    split_e4m3(scale_down(h, s), b1, b2);
+                    const size_t p = (size_t)(m.row0 + n);
+                    a.hq1[p * I + i_row] = b1;
+                    a.hq2[p * I + i_row] = b2;
+                    if (lane == 0) a.sfh[((size_t)m.tau * subs + m.sub) * kAtom + atom_byte(n, qd)] = (uint8_t)(s + 127);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && tid == 0) atomicOr(a.status, FLAG_TIMEOUT);
+    if (warp == 1) {
+        tc_fence_after();
+        tc_dealloc(tmem, kGUTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- down
+
+__global__ void __launch_bounds__(kPfThreads, 1)
+    pf_down_kernel(const __grid_constant__ CUtensorMap tWd, const __grid_constant__ CUtensorMap tH1,
+                   const __grid_constant__ CUtensorMap tH2, PfArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full[kDNStages], empty[kDNStages], tmem_full, tmem_empty, tmem_done;
+    __shared__ uint32_t tslot;
+    __shared__ volatile int abort_flag;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H, I = a.I, E = a.E, k = a.k;
+    const int subs = H / kT, slabs = I / kT;
+
+    if (tid == 0) {
+        for (int s = 0; s < kDNStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&tmem_full, 1);
+        mbar_init(&tmem_empty, 4);
+        mbar_init(&tmem_done, 1);
+        mbar_fence_init();
+        abort_flag = 0;
+    }
+    if (warp == 1) tc_alloc(&tslot, kDNTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tslot;
+    const uint32_t t_y = tmem, t_sf = tmem + kT;
+    const int n_items = __ldg(a.tile_base + E) * subs;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int c = 0;
+            for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x) {
+                const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+                const int wrow = m.e * H + m.sub * kT;
+                const uint8_t *sw = a.sfa0 + ((size_t)(m.e * subs + m.sub) * slabs) * kAtom;
+                const uint8_t *sh = a.sfb + ((size_t)m.tau * slabs) * kAtom;
+                for (int sl = 0; sl < slabs; ++sl, ++c) {
+                    const int s = c % kDNStages;
+                    if (c >= kDNStages && !wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag))
+                        break;
+                    uint8_t *st = smem + (size_t)s * kDNStage;
+                    mbar_arrive_expect_tx(&full[s], kBoxA + 2 * kTileS + 2 * kAtom);
+                    tma_load_2d(st, &tWd, sl * kT, wrow, &full[s]);
+                    tma_load_2d(st + kTileS, &tH1, sl * kT, m.row0, &full[s]);
+                    tma_load_2d(st + 2 * kTileS, &tH2, sl * kT, m.row0, &full[s]);
+                    bulk_g2s(st + 3 * kTileS, sw + (size_t)sl * kAtom, kAtom, &full[s]);
+                    bulk_g2s(st + 3 * kTileS + kAtom, sh + (size_t)sl * kAtom, kAtom, &full[s]);
+                }
+            }
+            drain_stages(full, kDNStages, c);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int c = 0, q = 0;
+            for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
+                const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+                const int n = (m.cnt + 15) & ~15;
+                if (q > 0 && !wait_or_abort(&tmem_empty, (uint32_t)((q - 1) & 1), &abort_flag)) break;
+                tc_fence_after();
+                for (int sl = 0; sl < slabs; ++sl, ++c) {
+                    const int s = c % kDNStages;
+                    if (!wait_or_abort(&full[s], (uint32_t)((c / kDNStages) & 1), &abort_flag)) break;
+                    tc_fence_after();
+                    const uint8_t *st = smem + (size_t)s * kDNStage;
+                    const uint32_t sfw = t_sf + 8 * s, sfh = sfw + 4;
+                    tc_cp_atom(sfw, st + 3 * kTileS);
+                    tc_cp_atom(sfh, st + 3 * kTileS + kAtom);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t id = idesc_mx(n, kk, kk);
+                        const uint64_t aw = desc_sw128(st + kk * 32);
+                        const uint64_t b1 = desc_sw128(st + kTileS + kk * 32), b2 = desc_sw128(st + 2 * kTileS + kk * 32);
+                        const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
+                        mma_mx(t_y, aw, b1, id, acc, sfw, sfh);
+                        mma_mx(t_y, aw, b2, id, 1u, sfw, sfh);
+                    }
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(&tmem_full);
+            }
+            drain_mma(&tmem_done);
+        }
+    } else {
+        const int qd = warp & 3;
+        int q = 0;
+        for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
+            const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+            if (!wait_or_abort(&tmem_full, (uint32_t)(q & 1), &abort_flag)) break;
+            tc_fence_after();
+            const int h_row = m.sub * kT + 32 * qd + lane;   // this lane's output feature
+            const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+            for (int n0 = 0; n0 < m.cnt; n0 += 16) {
+                float y[16];
+                tc_ld16(t_y + lane_off + n0, y);
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int n = n0 + jj;
+                    if (n >= m.cnt) break;
+                    const int r = __ldg(a.perm + m.row0 + n);
+                    const float w = __ldg(a.topk_w + r);
+                    atomicAdd(a.acc + (size_t)(r / k) * H + h_row, w * y[jj]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && tid == 0) atomicOr(a.status, FLAG_TIMEOUT);
+    if (warp == 1) {
+        tc_fence_after();
+        tc_dealloc(tmem, kDNTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D tensor map over `rows` rows of `cols` elements, 128 x 128 boxes, 128B swizzle.
+cudaError_t make_map(CUtensorMap *map, bool e2m1, void *base, long long cols, long long rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(e2m1 ? cols / 2 : cols)};
+    const cuuint32_t box[2] = {(cuuint32_t)kT, (cuuint32_t)kT};
+    const cuuint32_t es[2] = {1, 1};
+    const CUresult r = fn(map, e2m1 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base,
+                          dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+size_t gu_smem() { return (size_t)kGUStages * kGUStage + 1024; }
+size_t dn_smem() { return (size_t)kDNStages * kDNStage + 1024; }
+
+}  // namespace
+
+bool prefill_mx_supported(const Layer &L, int T) {
+    return L.pf != nullptr && L.pf->maps_ready && T > kDecMaxTokens && L.d.fmt == MOEQ_FMT_MXFP4 &&
+           L.d.act == MOEQ_ACT_BF16;
+}
+
+cudaError_t prefill_mx_create(Layer &L) {
+    const moeq_layer_desc &d = L.d;
+    if (d.fmt != MOEQ_FMT_MXFP4 || d.act != MOEQ_ACT_BF16 || d.max_tokens <= kDecMaxTokens) return cudaSuccess;
+    if (d.hidden % kT || d.inter % kT) return cudaSuccess;
+    PrefillMx *pf = new (std::nothrow) PrefillMx();
+    if (!pf) return cudaErrorMemoryAllocation;
+    L.pf = pf;
+    const int E = d.n_experts, H = d.hidden, I = d.inter;
+    const size_t R = (size_t)d.max_tokens * d.top_k;          // route positions
+    const size_t tiles = R / kT + (size_t)E;                   // upper bound on route tiles
+    cudaError_t e = cudaSuccess;
+    auto al = [&](void **p, size_t n) {
+        if (e == cudaSuccess) e = cudaMalloc(p, n);
+    };
+    for (int p = 0; p < 3; ++p) {
+        const size_t N = p == MOEQ_DOWN ? H : I, K = p == MOEQ_DOWN ? I : H;
+        al((void **)&pf->codes[p], (size_t)E * N * K / 2);
+        al((void **)&pf->sf_atoms[p], (size_t)E * N * K / 32);
+    }
+    al((void **)&pf->tile_base, sizeof(int32_t) * (E + 1));
+    al((void **)&pf->xq[0], R * H);
+    al((void **)&pf->xq[1], R * H);
+    al((void **)&pf->sfx, tiles * (H / kT) * kAtom);
+    al((void **)&pf->hq[0], R * I);
+    al((void **)&pf->hq[1], R * I);
+    al((void **)&pf->sfh, tiles * (I / kT) * kAtom);
+    // rows and scale atoms of route positions beyond a tile's routes are read
+    // by the MMAs (their columns are discarded): keep them finite
+    if (e == cudaSuccess) e = cudaMemset(pf->xq[0], 0, R * H);
+    if (e == cudaSuccess) e = cudaMemset(pf->xq[1], 0, R * H);
+    if (e == cudaSuccess) e = cudaMemset(pf->hq[0], 0, R * I);
+    if (e == cudaSuccess) e = cudaMemset(pf->hq[1], 0, R * I);
+    if (e == cudaSuccess) e = cudaMemset(pf->sfx, 127, tiles * (H / kT) * kAtom);
+    if (e == cudaSuccess) e = cudaMemset(pf->sfh, 127, tiles * (I / kT) * kAtom);
+    if (e != cudaSuccess) return e;
+    // activation operand maps; rows past the last route position read as zeros
+    e = make_map(&pf->map_x[0], false, pf->xq[0], H, (long long)R);
+    if (e == cudaSuccess) e = make_map(&pf->map_x[1], false, pf->xq[1], H, (long long)R);
+    if (e == cudaSuccess) e = make_map(&pf->map_h[0], false, pf->hq[0], I, (long long)R);
+    if (e == cudaSuccess) e = make_map(&pf->map_h[1], false, pf->hq[1], I, (long long)R);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(pf_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu_smem());
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(pf_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn_smem());
+    // without the driver's tensor-map encoder this path stays off
+    if (e == cudaErrorNotSupported) e = cudaSuccess;
+    return e;
+}
+
+void prefill_mx_free(Layer &L) {
+    PrefillMx *pf = L.pf;
+    if (!pf) return;
+    for (int p = 0; p < 3; ++p) {
+        cudaFree(pf->codes[p]);
+        cudaFree(pf->sf_atoms[p]);
+    }
+    cudaFree(pf->tile_base);
+    cudaFree(pf->xq[0]);
+    cudaFree(pf->xq[1]);
+    cudaFree(pf->sfx);
+    cudaFree(pf->hq[0]);
+    cudaFree(pf->hq[1]);
+    cudaFree(pf->sfh);
+    delete pf;
+    L.pf = nullptr;
+}
+
+cudaError_t prefill_mx_upload(Layer &L, int p, const uint8_t *codes, const uint8_t *scales, int e0, int ne,
+                              cudaStream_t s) {
+    PrefillMx *pf = L.pf;
+    if (!pf) return cudaSuccess;
+    const int H = L.d.hidden, I = L.d.inter;
+    const int N = p == MOEQ_DOWN ? H : I, K = p == MOEQ_DOWN ? I : H;
+    cudaError_t e = cudaMemcpyAsync(pf->codes[p] + (size_t)e0 * N * (K / 2), codes, (size_t)ne * N * (K / 2),
+                                    cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return e;
+    const long long n = (long long)ne * N * (K / 32);
+    pf_sf_atoms_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(scales, ne, N, K,
+                                                                   pf->sf_atoms[p] + (size_t)e0 * N * (K / 32));
+    return cudaGetLastError();
+}
+
+cudaError_t prefill_mx_finish_upload(Layer &L) {
+    PrefillMx *pf = L.pf;
+    if (!pf) return cudaSuccess;
+    const int E = L.d.n_experts, H = L.d.hidden, I = L.d.inter;
+    cudaError_t e = make_map(&pf->map_w[MOEQ_GATE], true, pf->codes[MOEQ_GATE], H, (long long)E * I);
+    if (e == cudaSuccess) e = make_map(&pf->map_w[MOEQ_UP], true, pf->codes[MOEQ_UP], H, (long long)E * I);
+    if (e == cudaSuccess) e = make_map(&pf->map_w[MOEQ_DOWN], true, pf->codes[MOEQ_DOWN], I, (long long)E * H);
+    pf->maps_ready = e == cudaSuccess;
+    return e == cudaErrorNotSupported ? cudaSuccess : e;
+}
+
+cudaError_t launch_prefill_mx(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
+                              cudaStream_t s, const cudaEvent_t *ev) {
+    const PrefillMx *pf = L.pf;
+    const int E = L.d.n_experts, H = L.d.hidden, I = L.d.inter, k = L.d.top_k;
+    cudaError_t e = launch_route_bucket(L, ids, T * k, L.b.offsets, L.b.perm, L.b.active, s);
+    if (e != cudaSuccess) return e;
+    if (ev) record_phase(ev[1], s);
+    L.count_launches(5);
+    pf_tiles_kernel<<<1, 1024, 0, s>>>(L.b.offsets, E, pf->tile_base);
+    e = cudaMemsetAsync(L.acc, 0, sizeof(float) * (size_t)T * H, s);
+    if (e != cudaSuccess) return e;
+    {
+        const int warps = T * k < 148 * 16 ? T * k : 148 * 16;
+        pf_quant_x_kernel<<<(warps + 7) / 8, 256, 0, s>>>(reinterpret_cast<const uint16_t *>(x), L.b.perm, ids,
+                                                          L.b.offsets, pf->tile_base, E, k, H, pf->xq[0], pf->xq[1],
+                                                          pf->sfx);
+    }
+    PfArgs a{};
+    a.offsets = L.b.offsets;
+    a.tile_base = pf->tile_base;
+    a.perm = L.b.perm;
+    a.ids = ids;
+    a.topk_w = topk_w;
+    a.status = L.status;
+    a.E = E;
+    a.H = H;
+    a.I = I;
+    a.k = k;
+    a.sfa0 = pf->sf_atoms[MOEQ_GATE];
+    a.sfa1 = pf->sf_atoms[MOEQ_UP];
+    a.sfb = pf->sfx;
+    a.hq1 = pf->hq[0];
+    a.hq2 = pf->hq[1];
+    a.sfh = pf->sfh;
+    pf_gateup_kernel<<<L.sm_count, kPfThreads, gu_smem(), s>>>(pf->map_w[MOEQ_GATE], pf->map_w[MOEQ_UP], pf->map_x[0],
+                                                               pf->map_x[1], a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev) record_phase(ev[2], s);
+    PfArgs b = a;
+    b.sfa0 = pf->sf_atoms[MOEQ_DOWN];
+    b.sfa1 = nullptr;
+    b.sfb = pf->sfh;
+    b.acc = L.acc;
+    pf_down_kernel<<<L.sm_count, kPfThreads, dn_smem(), s>>>(pf->map_w[MOEQ_DOWN], pf->map_h[0], pf->map_h[1], b);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev) record_phase(ev[3], s);
+    const long long n = (long long)T * H;
+    pf_cast_kernel<<<(unsigned)((n / 4 + 255) / 256), 256, 0, s>>>(L.acc, reinterpret_cast<__nv_bfloat16 *>(out), n);
+    if (ev) record_phase(ev[4], s);
+    return cudaGetLastError();
+}
+
+}  // namespace moeq
