@@ -22,7 +22,7 @@
 // Steps of one forward (all on the stream, no host synchronisation):
 //   route/bucket (route.cu)  -> offsets[E+1], perm (route ids by expert)
 //   pf_tiles_kernel          -> tile_base[E+1]: expert e's routes form
-//                               ceil(n_e/128) tiles of up to 128 routes
+//                               ceil(n_e/64) tiles of up to 64 routes
 //   pf_quant_x_kernel        -> q1, q2 [route position][H] and their scale
 //                               atoms, one row per route (a gather of x)
 //   pf_gateup_kernel         -> per (route tile, 128 rows of I): gate and up
@@ -40,7 +40,9 @@
 //
 // CTA roles (one CTA per SM, persistent over work items): warp 0 issues TMA
 // copies into a ring of stages, warp 1 issues the MMAs (one thread) and owns
-// the tensor memory, warps 2..5 run the epilogue.  Every wait is bounded;
+// the tensor memory (two accumulator buffers, so that the epilogue of one
+// work item overlaps the MMAs of the next), warps 2..5 run the epilogue.
+// Every wait is bounded;
 // on expiry the kernel sets MOEQ_ERR_TIMEOUT, every role stops, and the
 // tensor memory is released.
 #include <cuda.h>
@@ -55,22 +57,27 @@
 namespace moeq {
 namespace {
 
-constexpr int kT = 128;           // MMA M (weight rows per tile), max MMA N (routes per tile), K per slab
+constexpr int kT = 128;           // MMA M (weight rows per tile) and K per slab
+constexpr int kRT = 64;           // routes per route tile: the largest MMA N used
 constexpr int kPfThreads = 192;   // producer, MMA, 4 epilogue warps
 constexpr int kBoxA = 8192;       // bytes one A box moves from HBM (128 rows x 128 E2M1 codes)
-constexpr int kTileS = 16384;     // shared-memory bytes of one 128 x 128 operand tile (A widened, or B)
+constexpr int kTileA = 16384;     // shared-memory bytes of one 128 x 128 A tile (codes widened)
+constexpr int kTileB = 8192;      // shared-memory bytes of one 64-route x 128 B tile (E4M3)
 constexpr int kAtom = 512;        // one scale-factor atom: 128 rows x 4 blocks of 32
 
-// gate/up stage: [A gate][A up][B q1][B q2][SF gate][SF up][SF x]
-constexpr int kGUStage = 4 * kTileS + 3 * kAtom + 512;   // padded to 1 KB
-constexpr int kGUStages = 3;
+// gate/up stage: [A gate][A up][B q1][B q2][SF gate][SF up][SF x], padded to 1 KB
+constexpr int kGUStage = 2 * kTileA + 2 * kTileB + 3 * kAtom + 512;
+constexpr int kGUStages = 4;
+constexpr int kGUFill = 2;        // stages the producer fills per step
 // down stage: [A down][B q1][B q2][SF down][SF h]
-constexpr int kDNStage = 3 * kTileS + 2 * kAtom;
-constexpr int kDNStages = 4;
+constexpr int kDNStage = kTileA + 2 * kTileB + 2 * kAtom;
+constexpr int kDNStages = 6;
+constexpr int kDNFill = 3;
 
-// tensor-memory columns: accumulators, then a scale-factor ring (4 columns per atom)
-constexpr int kGUTmemCols = 512;   // gate 128 + up 128, SF ring 3 stages x 12
-constexpr int kDNTmemCols = 256;   // y 128, SF ring 4 stages x 8
+// tensor memory: two accumulator buffers (the epilogue of one item overlaps
+// the MMAs of the next), then a scale-factor ring (4 columns per atom)
+constexpr int kGUTmemCols = 512;   // 2 x (gate 64 + up 64), SF ring 4 stages x 12
+constexpr int kDNTmemCols = 256;   // 2 x y 64, SF ring 6 stages x 8
 
 constexpr long long kWaitCycles = 2000000000LL;
 
@@ -222,14 +229,14 @@ __device__ __forceinline__ Item decode_item(const int32_t *offsets, const int32_
     m.e = expert_of_tile(tile_base, E, m.tau);
     m.j = m.tau - __ldg(tile_base + m.e);
     const int beg = __ldg(offsets + m.e), n_e = __ldg(offsets + m.e + 1) - beg;
-    m.row0 = beg + kT * m.j;
-    m.cnt = min(kT, n_e - kT * m.j);
+    m.row0 = beg + kRT * m.j;
+    m.cnt = min(kRT, n_e - kRT * m.j);
     return m;
 }
 
 // ---------------------------------------------------------------- small kernels
 
-// tile_base[e] = sum over e' < e of ceil(n_e' / 128); tile_base[E] = all tiles.
+// tile_base[e] = sum over e' < e of ceil(n_e' / 64); tile_base[E] = all tiles.
 __global__ void __launch_bounds__(1024) pf_tiles_kernel(const int32_t *__restrict__ offsets, int E,
                                                         int32_t *__restrict__ tile_base) {
     __shared__ int32_t warp_off[32];
@@ -238,7 +245,7 @@ __global__ void __launch_bounds__(1024) pf_tiles_kernel(const int32_t *__restric
     int carry = 0;
     for (int e0 = 0; e0 < E; e0 += 1024) {
         const int e = e0 + tid;
-        const int v = e < E ? (offsets[e + 1] - offsets[e] + kT - 1) / kT : 0;
+        const int v = e < E ? (offsets[e + 1] - offsets[e] + kRT - 1) / kRT : 0;
         int incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -278,7 +285,7 @@ __global__ void __launch_bounds__(256) pf_quant_x_kernel(const uint16_t *__restr
     const int n_warps = (gridDim.x * blockDim.x) >> 5;
     for (int p = warp; p < n_valid; p += n_warps) {
         const int r = __ldg(perm + p), t = r / k, e = __ldg(ids + r);
-        const int l = p - __ldg(offsets + e), tau = __ldg(tile_base + e) + l / kT, row = l % kT;
+        const int l = p - __ldg(offsets + e), tau = __ldg(tile_base + e) + l / kRT, row = l % kRT;
         const uint16_t *xr = x + (size_t)t * H;
         // lane handles 32-blocks lane, lane+32, ...
         for (int b = lane; b < H / 32; b += 32) {
@@ -367,7 +374,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                      const __grid_constant__ CUtensorMap tX1, const __grid_constant__ CUtensorMap tX2, PfArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full[kGUStages], empty[kGUStages], tmem_full, tmem_empty, tmem_done;
+    __shared__ __align__(8) uint64_t full[kGUStages], empty[kGUStages], tmem_full[2], tmem_empty[2], tmem_done;
     __shared__ uint32_t tslot;
     __shared__ volatile int abort_flag;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -379,8 +386,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(&tmem_full, 1);
-        mbar_init(&tmem_empty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tmem_full[b], 1);
+            mbar_init(&tmem_empty[b], 4);
+        }
         mbar_init(&tmem_done, 1);
         mbar_fence_init();
         abort_flag = 0;
@@ -390,57 +399,73 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
-    const uint32_t t_g = tmem, t_u = tmem + kT, t_sf = tmem + 2 * kT;
+    const uint32_t t_sf = tmem + 4 * kRT;   // buffer b: gate at b*128, up at b*128 + 64
     const int n_items = __ldg(a.tile_base + E) * subs;
 
     if (warp == 0) {
-        if (lane == 0) {
-            int c = 0;
-            for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x) {
-                const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+        // kGUFill stages per step: lanes g < kGUFill wait for and arm stage
+        // c0 + g, then lanes 7g + j issue copy j of it -- one producer step
+        // costs about the same however many copies it issues, so it issues many
+        const int my_items = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+        const int total = my_items * slabs;
+        const int g = lane / 7, j = lane % 7;
+        int c0 = 0;
+        for (; c0 < total; c0 += kGUFill) {
+            const int c = c0 + (lane < kGUFill ? lane : 0), s = c % kGUStages;
+            bool ok = true;
+            if (lane < kGUFill && c < total && c >= kGUStages)
+                ok = wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag);
+            if (__any_sync(0xffffffffu, !ok)) break;
+            if (lane < kGUFill && c < total) mbar_arrive_expect_tx(&full[s], 2 * kBoxA + 2 * kTileB + 3 * kAtom);
+            __syncwarp();
+            const int cc = c0 + g;
+            if (g < kGUFill && cc < total) {
+                const int sc = cc % kGUStages, sl = cc % slabs;
+                const Item m = decode_item(a.offsets, a.tile_base, E, subs, blockIdx.x + (cc / slabs) * gridDim.x);
+                uint8_t *st = smem + (size_t)sc * kGUStage;
+                uint8_t *sf = st + 2 * kTileA + 2 * kTileB;
                 const int wrow = m.e * I + m.sub * kT;
-                const uint8_t *sg = a.sfa0 + ((size_t)(m.e * subs + m.sub) * slabs) * kAtom;
-                const uint8_t *su = a.sfa1 + ((size_t)(m.e * subs + m.sub) * slabs) * kAtom;
-                const uint8_t *sx = a.sfb + ((size_t)m.tau * slabs) * kAtom;
-                for (int sl = 0; sl < slabs; ++sl, ++c) {
-                    const int s = c % kGUStages;
-                    if (c >= kGUStages && !wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag))
+                const size_t wsf = ((size_t)(m.e * subs + m.sub) * slabs + sl) * kAtom;
+                switch (j) {
+                    case 0: tma_load_2d(st, &tWg, sl * kT, wrow, &full[sc]); break;
+                    case 1: tma_load_2d(st + kTileA, &tWu, sl * kT, wrow, &full[sc]); break;
+                    case 2: tma_load_2d(st + 2 * kTileA, &tX1, sl * kT, m.row0, &full[sc]); break;
+                    case 3: tma_load_2d(st + 2 * kTileA + kTileB, &tX2, sl * kT, m.row0, &full[sc]); break;
+                    case 4: bulk_g2s(sf, a.sfa0 + wsf, kAtom, &full[sc]); break;
+                    case 5: bulk_g2s(sf + kAtom, a.sfa1 + wsf, kAtom, &full[sc]); break;
+                    default:
+                        bulk_g2s(sf + 2 * kAtom, a.sfb + ((size_t)m.tau * slabs + sl) * kAtom, kAtom, &full[sc]);
                         break;
-                    uint8_t *st = smem + (size_t)s * kGUStage;
-                    mbar_arrive_expect_tx(&full[s], 2 * kBoxA + 2 * kTileS + 3 * kAtom);
-                    tma_load_2d(st, &tWg, sl * kT, wrow, &full[s]);
-                    tma_load_2d(st + kTileS, &tWu, sl * kT, wrow, &full[s]);
-                    tma_load_2d(st + 2 * kTileS, &tX1, sl * kT, m.row0, &full[s]);
-                    tma_load_2d(st + 3 * kTileS, &tX2, sl * kT, m.row0, &full[s]);
-                    bulk_g2s(st + 4 * kTileS, sg + (size_t)sl * kAtom, kAtom, &full[s]);
-                    bulk_g2s(st + 4 * kTileS + kAtom, su + (size_t)sl * kAtom, kAtom, &full[s]);
-                    bulk_g2s(st + 4 * kTileS + 2 * kAtom, sx + (size_t)sl * kAtom, kAtom, &full[s]);
                 }
             }
-            drain_stages(full, kGUStages, c);
+            __syncwarp();
         }
+        if (lane == 0) drain_stages(full, kGUStages, c0 < total ? c0 : total);
     } else if (warp == 1) {
         if (lane == 0) {
             int c = 0, q = 0;
             for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
                 const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
-                const int n = (m.cnt + 15) & ~15;
-                if (q > 0 && !wait_or_abort(&tmem_empty, (uint32_t)((q - 1) & 1), &abort_flag)) break;
+                const int n = (m.cnt + 15) & ~15, b = q & 1;
+                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
                 tc_fence_after();
+                const uint32_t t_g = tmem + b * 2 * kRT, t_u = t_g + kRT;
                 for (int sl = 0; sl < slabs; ++sl, ++c) {
                     const int s = c % kGUStages;
                     if (!wait_or_abort(&full[s], (uint32_t)((c / kGUStages) & 1), &abort_flag)) break;
                     tc_fence_after();
                     const uint8_t *st = smem + (size_t)s * kGUStage;
+                    const uint8_t *sf = st + 2 * kTileA + 2 * kTileB;
                     const uint32_t sfg = t_sf + 12 * s, sfu = sfg + 4, sfx = sfg + 8;
-                    tc_cp_atom(sfg, st + 4 * kTileS);
-                    tc_cp_atom(sfu, st + 4 * kTileS + kAtom);
-                    tc_cp_atom(sfx, st + 4 * kTileS + 2 * kAtom);
+                    tc_cp_atom(sfg, sf);
+                    tc_cp_atom(sfu, sf + kAtom);
+                    tc_cp_atom(sfx, sf + 2 * kAtom);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t id = idesc_mx(n, kk, kk);
-                        const uint64_t ag = desc_sw128(st + kk * 32), au = desc_sw128(st + kTileS + kk * 32);
-                        const uint64_t b1 = desc_sw128(st + 2 * kTileS + kk * 32), b2 = desc_sw128(st + 3 * kTileS + kk * 32);
+                        const uint64_t ag = desc_sw128(st + kk * 32), au = desc_sw128(st + kTileA + kk * 32);
+                        const uint64_t b1 = desc_sw128(st + 2 * kTileA + kk * 32);
+                        const uint64_t b2 = desc_sw128(st + 2 * kTileA + kTileB + kk * 32);
                         const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
                         mma_mx(t_g, ag, b1, id, acc, sfg, sfx);
                         mma_mx(t_g, ag, b2, id, 1u, sfg, sfx);
@@ -449,7 +474,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     }
                     tc_commit(&empty[s]);
                 }
-                tc_commit(&tmem_full);
+                tc_commit(&tmem_full[b]);
             }
             drain_mma(&tmem_done);
         }
@@ -459,34 +484,36 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int q = 0;
         for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
             const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
-            if (!wait_or_abort(&tmem_full, (uint32_t)(q & 1), &abort_flag)) break;
+            const int b = q & 1;
+            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag)) break;
             tc_fence_after();
             const int i_row = m.sub * kT + 32 * qd + lane;   // this lane's row of I
-            const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+            const uint32_t t_g = tmem + b * 2 * kRT + ((uint32_t)(32 * qd) << 16), t_u = t_g + kRT;
+            uint8_t *sfh = a.sfh + ((size_t)m.tau * subs + m.sub) * kAtom;
             for (int n0 = 0; n0 < m.cnt; n0 += 16) {
                 float g[16], u[16];
-                tc_ld16(t_g + lane_off + n0, g);
-                tc_ld16(t_u + lane_off + n0, u);
+                tc_ld16(t_g + n0, g);
+                tc_ld16(t_u + n0, u);
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                     const int n = n0 + jj;
                     if (n >= m.cnt) break;
                     const float h = silu_f32(g[jj]) * u[jj];
-                    float mx = fabsf(h);
-#pragma unroll
-                    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                    const int s = block_exp(isfinite(mx) ? mx : 3.0e38f);
+                    // the 32 rows of this warp are one 32-block of the down matmul's K
+                    const float ah = fabsf(h);
+                    const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(isfinite(ah) ? ah : 3.0e38f));
+                    const int s = block_exp(__uint_as_float(mb));
                     uint8_t b1, b2;
                     split_e4m3(scale_down(h, s), b1, b2);
                     const size_t p = (size_t)(m.row0 + n);
                     a.hq1[p * I + i_row] = b1;
                     a.hq2[p * I + i_row] = b2;
-                    if (lane == 0) a.sfh[((size_t)m.tau * subs + m.sub) * kAtom + atom_byte(n, qd)] = (uint8_t)(s + 127);
+                    if (lane == 0) sfh[atom_byte(n, qd)] = (uint8_t)(s + 127);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tmem_empty);
+            if (lane == 0) mbar_arrive(&tmem_empty[b]);
         }
     }
     tc_fence_before();
@@ -505,7 +532,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                    const __grid_constant__ CUtensorMap tH2, PfArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full[kDNStages], empty[kDNStages], tmem_full, tmem_empty, tmem_done;
+    __shared__ __align__(8) uint64_t full[kDNStages], empty[kDNStages], tmem_full[2], tmem_empty[2], tmem_done;
     __shared__ uint32_t tslot;
     __shared__ volatile int abort_flag;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -517,8 +544,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(&tmem_full, 1);
-        mbar_init(&tmem_empty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tmem_full[b], 1);
+            mbar_init(&tmem_empty[b], 4);
+        }
         mbar_init(&tmem_done, 1);
         mbar_fence_init();
         abort_flag = 0;
@@ -528,60 +557,72 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
-    const uint32_t t_y = tmem, t_sf = tmem + kT;
+    const uint32_t t_sf = tmem + 2 * kRT;   // buffer b at b*64
     const int n_items = __ldg(a.tile_base + E) * subs;
 
     if (warp == 0) {
-        if (lane == 0) {
-            int c = 0;
-            for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x) {
-                const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
-                const int wrow = m.e * H + m.sub * kT;
-                const uint8_t *sw = a.sfa0 + ((size_t)(m.e * subs + m.sub) * slabs) * kAtom;
-                const uint8_t *sh = a.sfb + ((size_t)m.tau * slabs) * kAtom;
-                for (int sl = 0; sl < slabs; ++sl, ++c) {
-                    const int s = c % kDNStages;
-                    if (c >= kDNStages && !wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag))
-                        break;
-                    uint8_t *st = smem + (size_t)s * kDNStage;
-                    mbar_arrive_expect_tx(&full[s], kBoxA + 2 * kTileS + 2 * kAtom);
-                    tma_load_2d(st, &tWd, sl * kT, wrow, &full[s]);
-                    tma_load_2d(st + kTileS, &tH1, sl * kT, m.row0, &full[s]);
-                    tma_load_2d(st + 2 * kTileS, &tH2, sl * kT, m.row0, &full[s]);
-                    bulk_g2s(st + 3 * kTileS, sw + (size_t)sl * kAtom, kAtom, &full[s]);
-                    bulk_g2s(st + 3 * kTileS + kAtom, sh + (size_t)sl * kAtom, kAtom, &full[s]);
+        // kDNFill stages per step (see the gate/up kernel): lanes 5g + j issue
+        // copy j of stage c0 + g
+        const int my_items = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+        const int total = my_items * slabs;
+        const int g = lane / 5, j = lane % 5;
+        int c0 = 0;
+        for (; c0 < total; c0 += kDNFill) {
+            const int c = c0 + (lane < kDNFill ? lane : 0), s = c % kDNStages;
+            bool ok = true;
+            if (lane < kDNFill && c < total && c >= kDNStages)
+                ok = wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag);
+            if (__any_sync(0xffffffffu, !ok)) break;
+            if (lane < kDNFill && c < total) mbar_arrive_expect_tx(&full[s], kBoxA + 2 * kTileB + 2 * kAtom);
+            __syncwarp();
+            const int cc = c0 + g;
+            if (g < kDNFill && cc < total) {
+                const int sc = cc % kDNStages, sl = cc % slabs;
+                const Item m = decode_item(a.offsets, a.tile_base, E, subs, blockIdx.x + (cc / slabs) * gridDim.x);
+                uint8_t *st = smem + (size_t)sc * kDNStage;
+                uint8_t *sf = st + kTileA + 2 * kTileB;
+                switch (j) {
+                    case 0: tma_load_2d(st, &tWd, sl * kT, m.e * H + m.sub * kT, &full[sc]); break;
+                    case 1: tma_load_2d(st + kTileA, &tH1, sl * kT, m.row0, &full[sc]); break;
+                    case 2: tma_load_2d(st + kTileA + kTileB, &tH2, sl * kT, m.row0, &full[sc]); break;
+                    case 3: bulk_g2s(sf, a.sfa0 + ((size_t)(m.e * subs + m.sub) * slabs + sl) * kAtom, kAtom, &full[sc]); break;
+                    default: bulk_g2s(sf + kAtom, a.sfb + ((size_t)m.tau * slabs + sl) * kAtom, kAtom, &full[sc]); break;
                 }
             }
-            drain_stages(full, kDNStages, c);
+            __syncwarp();
         }
+        if (lane == 0) drain_stages(full, kDNStages, c0 < total ? c0 : total);
     } else if (warp == 1) {
         if (lane == 0) {
             int c = 0, q = 0;
             for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
                 const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
-                const int n = (m.cnt + 15) & ~15;
-                if (q > 0 && !wait_or_abort(&tmem_empty, (uint32_t)((q - 1) & 1), &abort_flag)) break;
+                const int n = (m.cnt + 15) & ~15, b = q & 1;
+                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
                 tc_fence_after();
+                const uint32_t t_y = tmem + b * kRT;
                 for (int sl = 0; sl < slabs; ++sl, ++c) {
                     const int s = c % kDNStages;
                     if (!wait_or_abort(&full[s], (uint32_t)((c / kDNStages) & 1), &abort_flag)) break;
                     tc_fence_after();
                     const uint8_t *st = smem + (size_t)s * kDNStage;
+                    const uint8_t *sf = st + kTileA + 2 * kTileB;
                     const uint32_t sfw = t_sf + 8 * s, sfh = sfw + 4;
-                    tc_cp_atom(sfw, st + 3 * kTileS);
-                    tc_cp_atom(sfh, st + 3 * kTileS + kAtom);
+                    tc_cp_atom(sfw, sf);
+                    tc_cp_atom(sfh, sf + kAtom);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t id = idesc_mx(n, kk, kk);
                         const uint64_t aw = desc_sw128(st + kk * 32);
-                        const uint64_t b1 = desc_sw128(st + kTileS + kk * 32), b2 = desc_sw128(st + 2 * kTileS + kk * 32);
+                        const uint64_t b1 = desc_sw128(st + kTileA + kk * 32);
+                        const uint64_t b2 = desc_sw128(st + kTileA + kTileB + kk * 32);
                         const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
                         mma_mx(t_y, aw, b1, id, acc, sfw, sfh);
                         mma_mx(t_y, aw, b2, id, 1u, sfw, sfh);
                     }
                     tc_commit(&empty[s]);
                 }
-                tc_commit(&tmem_full);
+                tc_commit(&tmem_full[b]);
             }
             drain_mma(&tmem_done);
         }
@@ -590,25 +631,39 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int q = 0;
         for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
             const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
-            if (!wait_or_abort(&tmem_full, (uint32_t)(q & 1), &abort_flag)) break;
+            const int b = q & 1;
+            // the tile's routes: token and weight, two per lane, shared by shuffles
+            int tk0 = 0, tk1 = 0;
+            float w0 = 0.f, w1 = 0.f;
+            if (lane < m.cnt) {
+                const int r = __ldg(a.perm + m.row0 + lane);
+                tk0 = r / k;
+                w0 = __ldg(a.topk_w + r);
+            }
+            if (lane + 32 < m.cnt) {
+                const int r = __ldg(a.perm + m.row0 + 32 + lane);
+                tk1 = r / k;
+                w1 = __ldg(a.topk_w + r);
+            }
+            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag)) break;
             tc_fence_after();
             const int h_row = m.sub * kT + 32 * qd + lane;   // this lane's output feature
-            const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+            const uint32_t t_y = tmem + b * kRT + ((uint32_t)(32 * qd) << 16);
             for (int n0 = 0; n0 < m.cnt; n0 += 16) {
                 float y[16];
-                tc_ld16(t_y + lane_off + n0, y);
+                tc_ld16(t_y + n0, y);
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                     const int n = n0 + jj;
                     if (n >= m.cnt) break;
-                    const int r = __ldg(a.perm + m.row0 + n);
-                    const float w = __ldg(a.topk_w + r);
-                    atomicAdd(a.acc + (size_t)(r / k) * H + h_row, w * y[jj]);
+                    const int tk = __shfl_sync(0xffffffffu, n < 32 ? tk0 : tk1, n & 31);
+                    const float w = __shfl_sync(0xffffffffu, n < 32 ? w0 : w1, n & 31);
+                    atomicAdd(a.acc + (size_t)tk * H + h_row, w * y[jj]);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tmem_empty);
+            if (lane == 0) mbar_arrive(&tmem_empty[b]);
         }
     }
     tc_fence_before();
@@ -639,13 +694,14 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D tensor map over `rows` rows of `cols` elements, 128 x 128 boxes, 128B swizzle.
-cudaError_t make_map(CUtensorMap *map, bool e2m1, void *base, long long cols, long long rows) {
+// 2-D tensor map over `rows` rows of `cols` elements, boxes of 128 elements x
+// `box_rows` rows, 128B swizzle.
+cudaError_t make_map(CUtensorMap *map, bool e2m1, void *base, long long cols, long long rows, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)(e2m1 ? cols / 2 : cols)};
-    const cuuint32_t box[2] = {(cuuint32_t)kT, (cuuint32_t)kT};
+    const cuuint32_t box[2] = {(cuuint32_t)kT, (cuuint32_t)box_rows};
     const cuuint32_t es[2] = {1, 1};
     const CUresult r = fn(map, e2m1 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base,
                           dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -672,7 +728,7 @@ cudaError_t prefill_mx_create(Layer &L) {
     L.pf = pf;
     const int E = d.n_experts, H = d.hidden, I = d.inter;
     const size_t R = (size_t)d.max_tokens * d.top_k;          // route positions
-    const size_t tiles = R / kT + (size_t)E;                   // upper bound on route tiles
+    const size_t tiles = R / kRT + (size_t)E;                  // upper bound on route tiles
     cudaError_t e = cudaSuccess;
     auto al = [&](void **p, size_t n) {
         if (e == cudaSuccess) e = cudaMalloc(p, n);
@@ -699,10 +755,10 @@ cudaError_t prefill_mx_create(Layer &L) {
     if (e == cudaSuccess) e = cudaMemset(pf->sfh, 127, tiles * (I / kT) * kAtom);
     if (e != cudaSuccess) return e;
     // activation operand maps; rows past the last route position read as zeros
-    e = make_map(&pf->map_x[0], false, pf->xq[0], H, (long long)R);
-    if (e == cudaSuccess) e = make_map(&pf->map_x[1], false, pf->xq[1], H, (long long)R);
-    if (e == cudaSuccess) e = make_map(&pf->map_h[0], false, pf->hq[0], I, (long long)R);
-    if (e == cudaSuccess) e = make_map(&pf->map_h[1], false, pf->hq[1], I, (long long)R);
+    e = make_map(&pf->map_x[0], false, pf->xq[0], H, (long long)R, kRT);
+    if (e == cudaSuccess) e = make_map(&pf->map_x[1], false, pf->xq[1], H, (long long)R, kRT);
+    if (e == cudaSuccess) e = make_map(&pf->map_h[0], false, pf->hq[0], I, (long long)R, kRT);
+    if (e == cudaSuccess) e = make_map(&pf->map_h[1], false, pf->hq[1], I, (long long)R, kRT);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(pf_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu_smem());
     if (e == cudaSuccess) e = cudaFuncSetAttribute(pf_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn_smem());
     // without the driver's tensor-map encoder this path stays off
@@ -747,9 +803,9 @@ cudaError_t prefill_mx_finish_upload(Layer &L) {
     PrefillMx *pf = L.pf;
     if (!pf) return cudaSuccess;
     const int E = L.d.n_experts, H = L.d.hidden, I = L.d.inter;
-    cudaError_t e = make_map(&pf->map_w[MOEQ_GATE], true, pf->codes[MOEQ_GATE], H, (long long)E * I);
-    if (e == cudaSuccess) e = make_map(&pf->map_w[MOEQ_UP], true, pf->codes[MOEQ_UP], H, (long long)E * I);
-    if (e == cudaSuccess) e = make_map(&pf->map_w[MOEQ_DOWN], true, pf->codes[MOEQ_DOWN], I, (long long)E * H);
+    cudaError_t e = make_map(&pf->map_w[MOEQ_GATE], true, pf->codes[MOEQ_GATE], H, (long long)E * I, kT);
+    if (e == cudaSuccess) e = make_map(&pf->map_w[MOEQ_UP], true, pf->codes[MOEQ_UP], H, (long long)E * I, kT);
+    if (e == cudaSuccess) e = make_map(&pf->map_w[MOEQ_DOWN], true, pf->codes[MOEQ_DOWN], I, (long long)E * H, kT);
     pf->maps_ready = e == cudaSuccess;
     return e == cudaErrorNotSupported ? cudaSuccess : e;
 }

@@ -183,7 +183,9 @@ def test_forward_host_and_profiled_match_forward():
     assert_close(out_to_f64(out), oracle_ref(L, x, ids, w), "bf16")
     times = [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
     assert all(t >= 0 for t in times)
-    np.testing.assert_allclose(out_to_f64(out), ref, rtol=0, atol=np.abs(ref).max() * 1e-6)
+    # the same result as moeq_forward up to the order of the f32 additions of a
+    # token's routes, which the prefill-sized paths do not fix (atomics)
+    assert_close(out_to_f64(out), ref, "bf16")
 
 
 def test_zero_tokens_is_a_noop_and_bad_sizes_fail():
