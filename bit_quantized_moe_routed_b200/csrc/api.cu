@@ -83,6 +83,7 @@ void free_layer(moeq_layer *L) {
     cudaFree(L->ids_stage);
     cudaFree(L->w_stage);
     prefill_mx_free(*L);
+    prefill_vq_free(*L);
     delete L;
 }
 
@@ -114,6 +115,8 @@ moeq_status launch_forward(moeq_layer *L, const void *x, const int32_t *ids, con
     // the prefill kernels read x rows as 16-byte vectors
     if (prefill_mx_supported(*L, T) && ((uintptr_t)x & 15u) == 0)
         return from_cuda(launch_prefill_mx(*L, x, ids, w, T, out, s, ev));
+    if (prefill_vq_supported(*L, T) && ((uintptr_t)x & 15u) == 0)
+        return from_cuda(launch_prefill_vq(*L, x, ids, w, T, out, s, ev));
     cudaError_t e = launch_route_bucket(*L, ids, T * L->d.top_k, L->b.offsets, L->b.perm, L->b.active, s);
     if (e != cudaSuccess) return from_cuda(e);
     if (ev) record_phase(ev[1], s);
@@ -192,6 +195,7 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     ALLOC(L->w_stage, sizeof(float) * M * k);
 #undef ALLOC
     if (e == cudaSuccess) e = prefill_mx_create(*L);
+    if (e == cudaSuccess) e = prefill_vq_create(*L);
     if (e == cudaSuccess) e = cudaMemset(L->status, 0, sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMemset(L->dec_counters, 0, sizeof(int) * (H / 32 + 1));
     if (e != cudaSuccess) {

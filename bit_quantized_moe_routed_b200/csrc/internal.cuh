@@ -74,9 +74,21 @@ struct PrefillMx {
     bool maps_ready = false;
 };
 
+// Tensor-core path for VQ layers with bf16 activations (prefill_vq.cu):
+// activations gathered by route, bf16 intermediates, tensor maps over them.
+struct PrefillVq {
+    CUtensorMap map_x;             // gathered activations [route position][H] bf16
+    CUtensorMap map_h;             // intermediates [route position][I] bf16
+    int32_t *tile_base = nullptr;  // [E+1]
+    uint16_t *xg = nullptr;
+    uint16_t *hg = nullptr;
+    bool ready = false;
+};
+
 struct Layer {
     moeq_layer_desc d{};
     PrefillMx *pf = nullptr;
+    PrefillVq *pv = nullptr;
     DevWeights w;
     Buckets b;
     float *h = nullptr;        // [max_tokens*k][I] SwiGLU intermediates, route-sorted order
@@ -130,6 +142,13 @@ cudaError_t prefill_mx_upload(Layer &L, int p, const uint8_t *codes, const uint8
                               cudaStream_t s);
 cudaError_t prefill_mx_finish_upload(Layer &L);
 cudaError_t launch_prefill_mx(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
+                              cudaStream_t s, const cudaEvent_t *ev);
+// tile_base[e] = sum over e' < e of ceil(n_e' / 64) (the route tiles of the tensor-core paths)
+cudaError_t launch_route_tiles(const int32_t *offsets, int E, int32_t *tile_base, cudaStream_t s);
+bool prefill_vq_supported(const Layer &L, int T);
+cudaError_t prefill_vq_create(Layer &L);
+void prefill_vq_free(Layer &L);
+cudaError_t launch_prefill_vq(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
                               cudaStream_t s, const cudaEvent_t *ev);
 cudaError_t launch_ffn_simt(const Layer &L, const void *x, const float *topk_w, int32_t n_tokens,
                             void *out, cudaStream_t s, const cudaEvent_t *ev);

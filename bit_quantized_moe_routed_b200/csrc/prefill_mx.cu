@@ -53,12 +53,12 @@
 
 #include "async.cuh"
 #include "internal.cuh"
+#include "umma.cuh"
 
 namespace moeq {
 namespace {
 
-constexpr int kT = 128;           // MMA M (weight rows per tile) and K per slab
-constexpr int kRT = 64;           // routes per route tile: the largest MMA N used
+using namespace umma;
 constexpr int kPfThreads = 192;   // producer, MMA, 4 epilogue warps
 constexpr int kBoxA = 8192;       // bytes one A box moves from HBM (128 rows x 128 E2M1 codes)
 constexpr int kTileA = 16384;     // shared-memory bytes of one 128 x 128 A tile (codes widened)
@@ -79,100 +79,6 @@ constexpr int kDNFill = 3;
 constexpr int kGUTmemCols = 512;   // 2 x (gate 64 + up 64), SF ring 4 stages x 12
 constexpr int kDNTmemCols = 256;   // 2 x y 64, SF ring 6 stages x 8
 
-constexpr long long kWaitCycles = 2000000000LL;
-
-// ---------------------------------------------------------------- PTX helpers
-
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Shared-memory matrix descriptor, K-major.  128B swizzle: rows of 128 bytes,
-// 8-row groups 1024 bytes apart.  None: 8 x 16-byte core matrices, groups of
-// 8 rows `sbo` bytes apart, 16-byte columns `lbo` bytes apart.
-__device__ __forceinline__ uint64_t desc_sw128(const void *p) {
-    return (uint64_t)((smem_u32(p) >> 4) & 0x3FFF) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
-           (2ull << 61);
-}
-__device__ __forceinline__ uint64_t desc_plain(const void *p, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((smem_u32(p) >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46);
-}
-// Instruction descriptor: kind::mxf8f6f4 block-scaled, A E2M1, B E4M3, f32
-// accumulate, E8M0 scales, M 128, both operands K-major, K 32 per MMA;
-// a_sf / b_sf pick the byte (the 32-block) of each scale-factor column.
-__device__ __forceinline__ uint32_t idesc_mx(int n, int a_sf, int b_sf) {
-    return ((uint32_t)(b_sf & 3) << 4) | (5u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
-           ((uint32_t)(kT >> 4) << 24) | ((uint32_t)(a_sf & 3) << 29);
-}
-__device__ __forceinline__ void mma_mx(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc, uint32_t sfa,
-                                       uint32_t sfb) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
-        : "memory");
-}
-__device__ __forceinline__ void tc_cp_atom(uint32_t taddr, const void *atom) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc_plain(atom, 128, 128))
-                 : "memory");
-}
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_alloc(uint32_t *slot, int cols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(cols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tc_dealloc(uint32_t taddr, int cols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
-}
-// 16 consecutive f32 columns of this warp's 32 lanes
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, float v[16]) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Bounded wait that also gives up once another role has given up.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitCycles) {
-            *abort_flag = 1;
-            return false;
-        }
-    }
-    return true;
-}
-
-// Before the CTA releases its shared and tensor memory: wait (bounded,
-// whatever happened) for the copies of the last stages issued, and for every
-// MMA this thread issued.
-__device__ __forceinline__ void drain_stages(uint64_t *full, int S, int issued) {
-    for (int c = issued > S ? issued - S : 0; c < issued; ++c)
-        mbar_wait_bounded(&full[c % S], (uint32_t)((c / S) & 1), 200000000LL);
-}
-__device__ __forceinline__ void drain_mma(uint64_t *done) {
-    tc_commit(done);
-    mbar_wait_bounded(done, 0, 200000000LL);
-}
 
 // 2^s for s in [-126, 127]
 __device__ __forceinline__ float pow2i(int s) { return __uint_as_float((uint32_t)(s + 127) << 23); }
@@ -199,39 +105,6 @@ __device__ __forceinline__ int block_exp(float m) {
 __device__ __forceinline__ float scale_down(float v, int s) {
     const int a = -s / 2, b = -s - a;
     return v * pow2i(a) * pow2i(b);
-}
-
-// Scale-factor atom byte of (row r of a 128-row tile, 32-block kb of a 4-block group)
-__device__ __forceinline__ int atom_byte(int r, int kb) { return (r & 31) * 16 + (r >> 5) * 4 + kb; }
-
-// Expert of global route tile tau: the last e with tile_base[e] <= tau.
-__device__ __forceinline__ int expert_of_tile(const int32_t *tile_base, int E, int tau) {
-    int lo = 0, hi = E;   // tile_base[lo] <= tau < tile_base[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(tile_base + mid) <= tau) lo = mid;
-        else hi = mid;
-    }
-    return lo;
-}
-
-struct Item {
-    int e, j, sub;     // expert, route tile of the expert, 128-row tile of the output
-    int row0;          // first route position of the tile
-    int cnt;           // routes in the tile (1..128)
-    int tau;           // global route tile
-};
-__device__ __forceinline__ Item decode_item(const int32_t *offsets, const int32_t *tile_base, int E, int subs,
-                                            int it) {
-    Item m;
-    m.tau = it / subs;
-    m.sub = it % subs;
-    m.e = expert_of_tile(tile_base, E, m.tau);
-    m.j = m.tau - __ldg(tile_base + m.e);
-    const int beg = __ldg(offsets + m.e), n_e = __ldg(offsets + m.e + 1) - beg;
-    m.row0 = beg + kRT * m.j;
-    m.cnt = min(kRT, n_e - kRT * m.j);
-    return m;
 }
 
 // ---------------------------------------------------------------- small kernels
@@ -377,6 +250,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     __shared__ __align__(8) uint64_t full[kGUStages], empty[kGUStages], tmem_full[2], tmem_empty[2], tmem_done;
     __shared__ uint32_t tslot;
     __shared__ volatile int abort_flag;
+    __shared__ RouteTables rt;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H, I = a.I, E = a.E;
     const int subs = I / kT, slabs = H / kT;
@@ -394,13 +268,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_fence_init();
         abort_flag = 0;
     }
+    load_route_tables(rt, a.offsets, a.tile_base, a.E);
     if (warp == 1) tc_alloc(&tslot, kGUTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
     const uint32_t t_sf = tmem + 4 * kRT;   // buffer b: gate at b*128, up at b*128 + 64
-    const int n_items = __ldg(a.tile_base + E) * subs;
+    const int n_items = rt.tb[E] * subs;
 
     if (warp == 0) {
         // kGUFill stages per step: lanes g < kGUFill wait for and arm stage
@@ -421,7 +296,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int cc = c0 + g;
             if (g < kGUFill && cc < total) {
                 const int sc = cc % kGUStages, sl = cc % slabs;
-                const Item m = decode_item(a.offsets, a.tile_base, E, subs, blockIdx.x + (cc / slabs) * gridDim.x);
+                const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (cc / slabs) * gridDim.x);
                 uint8_t *st = smem + (size_t)sc * kGUStage;
                 uint8_t *sf = st + 2 * kTileA + 2 * kTileB;
                 const int wrow = m.e * I + m.sub * kT;
@@ -445,7 +320,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (lane == 0) {
             int c = 0, q = 0;
             for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
-                const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+                const Item m = decode_item(rt.off, rt.tb, E, subs, it);
                 const int n = (m.cnt + 15) & ~15, b = q & 1;
                 if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
                 tc_fence_after();
@@ -483,7 +358,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int qd = warp & 3;
         int q = 0;
         for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
-            const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+            const Item m = decode_item(rt.off, rt.tb, E, subs, it);
             const int b = q & 1;
             if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag)) break;
             tc_fence_after();
@@ -535,6 +410,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     __shared__ __align__(8) uint64_t full[kDNStages], empty[kDNStages], tmem_full[2], tmem_empty[2], tmem_done;
     __shared__ uint32_t tslot;
     __shared__ volatile int abort_flag;
+    __shared__ RouteTables rt;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H, I = a.I, E = a.E, k = a.k;
     const int subs = H / kT, slabs = I / kT;
@@ -552,13 +428,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_fence_init();
         abort_flag = 0;
     }
+    load_route_tables(rt, a.offsets, a.tile_base, a.E);
     if (warp == 1) tc_alloc(&tslot, kDNTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tslot;
     const uint32_t t_sf = tmem + 2 * kRT;   // buffer b at b*64
-    const int n_items = __ldg(a.tile_base + E) * subs;
+    const int n_items = rt.tb[E] * subs;
 
     if (warp == 0) {
         // kDNFill stages per step (see the gate/up kernel): lanes 5g + j issue
@@ -578,7 +455,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int cc = c0 + g;
             if (g < kDNFill && cc < total) {
                 const int sc = cc % kDNStages, sl = cc % slabs;
-                const Item m = decode_item(a.offsets, a.tile_base, E, subs, blockIdx.x + (cc / slabs) * gridDim.x);
+                const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (cc / slabs) * gridDim.x);
                 uint8_t *st = smem + (size_t)sc * kDNStage;
                 uint8_t *sf = st + kTileA + 2 * kTileB;
                 switch (j) {
@@ -596,7 +473,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (lane == 0) {
             int c = 0, q = 0;
             for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
-                const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+                const Item m = decode_item(rt.off, rt.tb, E, subs, it);
                 const int n = (m.cnt + 15) & ~15, b = q & 1;
                 if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
                 tc_fence_after();
@@ -630,7 +507,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int qd = warp & 3;
         int q = 0;
         for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
-            const Item m = decode_item(a.offsets, a.tile_base, E, subs, it);
+            const Item m = decode_item(rt.off, rt.tb, E, subs, it);
             const int b = q & 1;
             // the tile's routes: token and weight, two per lane, shared by shuffles
             int tk0 = 0, tk1 = 0;
@@ -713,6 +590,11 @@ size_t gu_smem() { return (size_t)kGUStages * kGUStage + 1024; }
 size_t dn_smem() { return (size_t)kDNStages * kDNStage + 1024; }
 
 }  // namespace
+
+cudaError_t launch_route_tiles(const int32_t *offsets, int E, int32_t *tile_base, cudaStream_t s) {
+    pf_tiles_kernel<<<1, 1024, 0, s>>>(offsets, E, tile_base);
+    return cudaGetLastError();
+}
 
 bool prefill_mx_supported(const Layer &L, int T) {
     return L.pf != nullptr && L.pf->maps_ready && T > kDecMaxTokens && L.d.fmt == MOEQ_FMT_MXFP4 &&

@@ -1,0 +1,593 @@
+// prefill_vq.cu -- VQ13(+R8) routed-expert FFN on the 5th-generation tensor
+// cores (bf16 activations, any token count).
+//
+// Format ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): every 8
+// consecutive weights of an expert row are one 13-bit index into the layer's
+// 8192 x 8 codebook (optionally plus an 8-bit index into a 256 x 8 residual
+// book), times an f16 row gain; one codebook pair serves every expert and
+// gate/up/down ("Why 13 bits": the books stay in shared memory while every
+// selected expert is decoded).  Weight = ((base + residual) * gain) in f32,
+// rounded once to bf16 for the tensor cores; activations are bf16 already,
+// so the MMAs are tcgen05.mma kind::f16 (bf16 x bf16 -> f32).
+//
+// Steps of one forward:
+//   route/bucket, route tiles (as for MXFP4: tiles of up to 64 routes)
+//   vq_gather_x_kernel  -> x rows in route order (bf16)
+//   vq_gateup_kernel    -> per (route tile, 128 rows of I): decoder warps
+//                          expand gate and up codes into bf16 tiles in shared
+//                          memory, the MMA thread multiplies them with the
+//                          route tile, the epilogue writes h = silu(g) u (bf16)
+//   vq_down_kernel      -> per (route tile, 128 rows of H): y, weighted and
+//                          added into acc[T][H] (f32 atomics)
+//   cast                -> out = bf16(acc)
+//
+// CTA roles (one CTA per SM): warp 0 loads the codebooks once, then the
+// activation tiles by TMA; warp 1 issues the MMAs; warps 2..9 decode weight
+// tiles (16-byte codeword gathers from shared memory: the step that bounds
+// this path); warps 10..13 run the epilogue.  Every wait is bounded.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <new>
+
+#include "async.cuh"
+#include "internal.cuh"
+#include "umma.cuh"
+
+namespace moeq {
+namespace {
+
+using namespace umma;
+
+constexpr int kDecWarps = 8;
+constexpr int kVqThreads = 32 * (2 + kDecWarps + 4);
+constexpr int kKS = 64;                        // K per slab: 64 bf16 = one 128-byte row
+constexpr int kTileA = kT * kKS * 2;           // 16 KB
+constexpr int kTileB = kRT * kKS * 2;          // 8 KB
+constexpr int kBook13 = 8192 * 16, kBook8 = 256 * 16;
+constexpr int kGUStage = 2 * kTileA + kTileB;  // [A gate][A up][B]
+constexpr int kGUStages = 2;
+constexpr int kDNStage = kTileA + kTileB;      // [A down][B]
+constexpr int kDNStages = 3;
+
+// kind::f16 instruction descriptor: bf16 A and B (K-major), f32 accumulate, M 128
+__device__ __forceinline__ uint32_t idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kT >> 4) << 24);
+}
+__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+struct VqProj {
+    const uint8_t *idx13;   // [E*N][K*13/64]
+    const uint8_t *idx8;    // [E*N][K/8] or null
+    const uint16_t *gain;   // [E*N] f16 or null
+};
+
+// The index data of vector j (K offset 8j within slab sl) of global row
+// `grow`, fetched ahead of its decode so that the global loads overlap the
+// gathers of earlier slabs: the bytes holding its 13-bit index, its residual
+// index and its row gain.
+struct VecRaw {
+    uint32_t win;   // bytes of the 13-bit field, little-endian
+    uint32_t i8;
+    uint32_t gain;  // f16 bits, 0x3C00 (1.0) when the layer has no gains
+};
+__device__ __forceinline__ VecRaw fetch_vec(const VqProj &pj, int K, size_t grow, int sl, int j) {
+    VecRaw v;
+    const uint8_t *irow = pj.idx13 + grow * (size_t)(K * 13 / 64);
+    const uint32_t bit = (uint32_t)sl * (kKS / 8 * 13) + 13u * (uint32_t)j;
+    const uint8_t *pb = irow + (bit >> 3);
+    v.win = (uint32_t)__ldg(pb) | ((uint32_t)__ldg(pb + 1) << 8);
+    // the third byte only when the field reaches it (never past the row)
+    if ((bit & 7u) > 3u) v.win |= (uint32_t)__ldg(pb + 2) << 16;
+    v.i8 = pj.idx8 ? (uint32_t)__ldg(pj.idx8 + grow * (size_t)(K / 8) + (size_t)sl * (kKS / 8) + j) : 0u;
+    v.gain = pj.gain ? (uint32_t)__ldg(pj.gain + grow) : 0x3C00u;
+    return v;
+}
+
+// Expand a fetched vector into 8 bf16 weights at the 128B-swizzled K-major
+// position (tile row r, 16-byte chunk j) of a shared-memory A tile.
+__device__ __forceinline__ void expand_vec(const VecRaw &v, bool r8, int sl, int j, const uint8_t *book13,
+                                           const uint8_t *book8, uint8_t *tile, int r) {
+    const uint32_t bit = (uint32_t)sl * (kKS / 8 * 13) + 13u * (uint32_t)j;
+    const uint32_t idx = (v.win >> (bit & 7u)) & 0x1FFFu;
+    const uint4 c = lds128(book13 + (size_t)idx * 16);
+    float w[8] = {bf16lo(c.x), bf16hi(c.x), bf16lo(c.y), bf16hi(c.y), bf16lo(c.z), bf16hi(c.z), bf16lo(c.w), bf16hi(c.w)};
+    if (r8) {
+        const uint4 rr = lds128(book8 + (size_t)v.i8 * 16);
+        w[0] += bf16lo(rr.x); w[1] += bf16hi(rr.x); w[2] += bf16lo(rr.y); w[3] += bf16hi(rr.y);
+        w[4] += bf16lo(rr.z); w[5] += bf16hi(rr.z); w[6] += bf16lo(rr.w); w[7] += bf16hi(rr.w);
+    }
+    if (v.gain != 0x3C00u) {
+        const float gn = __half2float(__ushort_as_half((unsigned short)v.gain));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] *= gn;
+    }
+    const uint4 o = make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
+    *reinterpret_cast<uint4 *>(tile + (r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4)) = o;
+}
+
+// One warp per route position: its token's x row, in route order.
+__global__ void __launch_bounds__(256) vq_gather_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ perm,
+                                                          const int32_t *__restrict__ offsets, int E, int k, int H,
+                                                          uint16_t *__restrict__ xg) {
+    const int n_valid = __ldg(offsets + E);
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int n_warps = (gridDim.x * blockDim.x) >> 5;
+    for (int p = warp; p < n_valid; p += n_warps) {
+        const int t = __ldg(perm + p) / k;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)p * H);
+        for (int i = lane; i < H / 8; i += 32) dst[i] = __ldg(src + i);
+    }
+}
+
+struct VqArgs {
+    const int32_t *offsets, *tile_base, *perm;
+    const float *topk_w;
+    VqProj w0, w1;            // gate/up: gate, up; down: down in w0
+    const uint8_t *book13, *book8;
+    uint16_t *hg;             // gate/up output [route position][I] bf16
+    float *acc;               // down output [T][H]
+    uint32_t *status;
+    int E, H, I, k;
+};
+
+// Shared pieces of both kernels: the codebooks into shared memory (warp 0,
+// before its TMA loop), on `bar`.
+__device__ __forceinline__ void load_books(uint8_t *b13, uint8_t *b8, const VqArgs &a, uint64_t *bar, int lane) {
+    const uint32_t bytes = kBook13 + (a.book8 ? kBook8 : 0);
+    if (lane == 0) mbar_arrive_expect_tx(bar, bytes);
+    __syncwarp();
+    if (lane < 8) bulk_g2s(b13 + lane * (kBook13 / 8), a.book13 + lane * (kBook13 / 8), kBook13 / 8, bar);
+    if (lane == 8 && a.book8) bulk_g2s(b8, a.book8, kBook8, bar);
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------- gate/up
+
+__global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_constant__ CUtensorMap tX, VqArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *b13 = smem + kGUStages * kGUStage, *b8 = b13 + kBook13;
+    __shared__ __align__(8) uint64_t a_full[kGUStages], b_full[kGUStages], empty[kGUStages], tmem_full[2],
+        tmem_empty[2], tmem_done, book_bar;
+    __shared__ uint32_t tslot;
+    __shared__ volatile int abort_flag;
+    __shared__ RouteTables rt;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H, I = a.I, E = a.E;
+    const int subs = I / kT, slabs = H / kKS;
+
+    if (tid == 0) {
+        for (int s = 0; s < kGUStages; ++s) {
+            mbar_init(&a_full[s], kDecWarps);
+            mbar_init(&b_full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tmem_full[b], 1);
+            mbar_init(&tmem_empty[b], 4);
+        }
+        mbar_init(&tmem_done, 1);
+        mbar_init(&book_bar, 1);
+        mbar_fence_init();
+        abort_flag = 0;
+    }
+    load_route_tables(rt, a.offsets, a.tile_base, a.E);
+    if (warp == 1) tc_alloc(&tslot, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tslot;   // buffer b: gate at 128 b, up at 128 b + 64
+    const int n_items = rt.tb[E] * subs;
+    const int my_items = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    const int total = my_items * slabs;
+
+    if (warp == 0) {
+        load_books(b13, b8, a, &book_bar, lane);
+        if (lane == 0) {
+            int c = 0;
+            for (; c < total; ++c) {
+                const int s = c % kGUStages;
+                if (c >= kGUStages && !wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag)) break;
+                const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
+                mbar_arrive_expect_tx(&b_full[s], kTileB);
+                tma_load_2d(smem + (size_t)s * kGUStage + 2 * kTileA, &tX, (c % slabs) * kKS, m.row0, &b_full[s]);
+            }
+            drain_stages(b_full, kGUStages, c);
+            mbar_wait_bounded(&book_bar, 0, 200000000LL);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int c = 0;
+            for (int q = 0; q < my_items && !abort_flag; ++q) {
+                const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + q * gridDim.x);
+                const int n = (m.cnt + 15) & ~15, b = q & 1;
+                const uint32_t id = idesc_bf16(n);
+                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
+                tc_fence_after();
+                const uint32_t t_g = tmem + b * 2 * kRT, t_u = t_g + kRT;
+                for (int sl = 0; sl < slabs; ++sl, ++c) {
+                    const int s = c % kGUStages;
+                    const uint32_t par = (uint32_t)((c / kGUStages) & 1);
+                    if (!wait_or_abort(&a_full[s], par, &abort_flag) || !wait_or_abort(&b_full[s], par, &abort_flag)) break;
+                    tc_fence_after();
+                    const uint8_t *st = smem + (size_t)s * kGUStage;
+#pragma unroll
+                    for (int kk = 0; kk < kKS / 16; ++kk) {
+                        const uint64_t ag = desc_sw128(st + kk * 32), au = desc_sw128(st + kTileA + kk * 32);
+                        const uint64_t bx = desc_sw128(st + 2 * kTileA + kk * 32);
+                        const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
+                        mma_bf16(t_g, ag, bx, id, acc);
+                        mma_bf16(t_u, au, bx, id, acc);
+                    }
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(&tmem_full[b]);
+            }
+            drain_mma(&tmem_done);
+        }
+    } else if (warp < 2 + kDecWarps) {
+        // decoders: per slab 2 matrices x 128 rows x 8 vectors; this thread
+        // always takes vector j of rows r0 + 32 i (i < 4) of both matrices, and
+        // fetches their index data two slabs ahead
+        const int dt = tid - 64, j = dt & 7, r0 = dt >> 3;
+        const bool r8 = a.book8 != nullptr;
+        VecRaw pa[8], pb[8];   // index data of slabs c and c + 1
+        auto fetch = [&](int c, VecRaw *dst) {
+            if (c >= total) return;
+            const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
+            const size_t row0 = (size_t)m.e * I + m.sub * kT + r0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = fetch_vec(i < 4 ? a.w0 : a.w1, H, row0 + 32 * (i & 3), c % slabs, j);
+        };
+        fetch(0, pa);
+        fetch(1, pb);
+        bool ok = wait_or_abort(&book_bar, 0, &abort_flag);
+        for (int c = 0; c < total && ok; ++c) {
+            const int s = c % kGUStages, sl = c % slabs;
+            if (c >= kGUStages) ok = wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            uint8_t *st = smem + (size_t)s * kGUStage;
+            VecRaw cur[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                cur[i] = pa[i];
+                pa[i] = pb[i];
+            }
+            fetch(c + 2, pb);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) expand_vec(cur[i], r8, sl, j, b13, b8, st + (i >> 2) * kTileA, r0 + 32 * (i & 3));
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[s]);
+        }
+    } else {
+        // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 = rows of I
+        const int qd = warp & 3;
+        for (int q = 0; q < my_items && !abort_flag; ++q) {
+            const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + q * gridDim.x);
+            const int b = q & 1;
+            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag)) break;
+            tc_fence_after();
+            const int i_row = m.sub * kT + 32 * qd + lane;
+            const uint32_t t_g = tmem + b * 2 * kRT + ((uint32_t)(32 * qd) << 16), t_u = t_g + kRT;
+            for (int n0 = 0; n0 < m.cnt; n0 += 16) {
+                float g[16], u[16];
+                tc_ld16(t_g + n0, g);
+                tc_ld16(t_u + n0, u);
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int n = n0 + jj;
+                    if (n >= m.cnt) break;
+                    const __nv_bfloat16 h = __float2bfloat16_rn(silu_f32(g[jj]) * u[jj]);
+                    a.hg[(size_t)(m.row0 + n) * I + i_row] = *reinterpret_cast<const uint16_t *>(&h);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[b]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && tid == 0) atomicOr(a.status, FLAG_TIMEOUT);
+    if (warp == 1) {
+        tc_fence_after();
+        tc_dealloc(tmem, 256);
+    }
+}
+
+// ---------------------------------------------------------------- down
+
+__global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_constant__ CUtensorMap tH, VqArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *b13 = smem + kDNStages * kDNStage, *b8 = b13 + kBook13;
+    __shared__ __align__(8) uint64_t a_full[kDNStages], b_full[kDNStages], empty[kDNStages], tmem_full[2],
+        tmem_empty[2], tmem_done, book_bar;
+    __shared__ uint32_t tslot;
+    __shared__ volatile int abort_flag;
+    __shared__ RouteTables rt;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H, I = a.I, E = a.E, k = a.k;
+    const int subs = H / kT, slabs = I / kKS;
+
+    if (tid == 0) {
+        for (int s = 0; s < kDNStages; ++s) {
+            mbar_init(&a_full[s], kDecWarps);
+            mbar_init(&b_full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tmem_full[b], 1);
+            mbar_init(&tmem_empty[b], 4);
+        }
+        mbar_init(&tmem_done, 1);
+        mbar_init(&book_bar, 1);
+        mbar_fence_init();
+        abort_flag = 0;
+    }
+    load_route_tables(rt, a.offsets, a.tile_base, a.E);
+    if (warp == 1) tc_alloc(&tslot, 128);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tslot;   // buffer b at 64 b
+    const int n_items = rt.tb[E] * subs;
+    const int my_items = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    const int total = my_items * slabs;
+
+    if (warp == 0) {
+        load_books(b13, b8, a, &book_bar, lane);
+        if (lane == 0) {
+            int c = 0;
+            for (; c < total; ++c) {
+                const int s = c % kDNStages;
+                if (c >= kDNStages && !wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag)) break;
+                const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
+                mbar_arrive_expect_tx(&b_full[s], kTileB);
+                tma_load_2d(smem + (size_t)s * kDNStage + kTileA, &tH, (c % slabs) * kKS, m.row0, &b_full[s]);
+            }
+            drain_stages(b_full, kDNStages, c);
+            mbar_wait_bounded(&book_bar, 0, 200000000LL);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int c = 0;
+            for (int q = 0; q < my_items && !abort_flag; ++q) {
+                const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + q * gridDim.x);
+                const int n = (m.cnt + 15) & ~15, b = q & 1;
+                const uint32_t id = idesc_bf16(n);
+                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
+                tc_fence_after();
+                const uint32_t t_y = tmem + b * kRT;
+                for (int sl = 0; sl < slabs; ++sl, ++c) {
+                    const int s = c % kDNStages;
+                    const uint32_t par = (uint32_t)((c / kDNStages) & 1);
+                    if (!wait_or_abort(&a_full[s], par, &abort_flag) || !wait_or_abort(&b_full[s], par, &abort_flag)) break;
+                    tc_fence_after();
+                    const uint8_t *st = smem + (size_t)s * kDNStage;
+#pragma unroll
+                    for (int kk = 0; kk < kKS / 16; ++kk)
+                        mma_bf16(t_y, desc_sw128(st + kk * 32), desc_sw128(st + kTileA + kk * 32), id,
+                                 (sl > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(&tmem_full[b]);
+            }
+            drain_mma(&tmem_done);
+        }
+    } else if (warp < 2 + kDecWarps) {
+        // decoders: per slab 128 rows x 8 vectors; this thread takes vector j
+        // of rows r0 + 32 i (i < 4), index data fetched two slabs ahead
+        const int dt = tid - 64, j = dt & 7, r0 = dt >> 3;
+        const bool r8 = a.book8 != nullptr;
+        VecRaw pa[4], pb[4];   // index data of slabs c and c + 1
+        auto fetch = [&](int c, VecRaw *dst) {
+            if (c >= total) return;
+            const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
+            const size_t row0 = (size_t)m.e * H + m.sub * kT + r0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = fetch_vec(a.w0, I, row0 + 32 * i, c % slabs, j);
+        };
+        fetch(0, pa);
+        fetch(1, pb);
+        bool ok = wait_or_abort(&book_bar, 0, &abort_flag);
+        for (int c = 0; c < total && ok; ++c) {
+            const int s = c % kDNStages, sl = c % slabs;
+            if (c >= kDNStages) ok = wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            uint8_t *st = smem + (size_t)s * kDNStage;
+            VecRaw cur[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                cur[i] = pa[i];
+                pa[i] = pb[i];
+            }
+            fetch(c + 2, pb);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) expand_vec(cur[i], r8, sl, j, b13, b8, st, r0 + 32 * i);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[s]);
+        }
+    } else {
+        const int qd = warp & 3;
+        for (int q = 0; q < my_items && !abort_flag; ++q) {
+            const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + q * gridDim.x);
+            const int b = q & 1;
+            int tk0 = 0, tk1 = 0;
+            float w0 = 0.f, w1 = 0.f;
+            if (lane < m.cnt) {
+                const int r = __ldg(a.perm + m.row0 + lane);
+                tk0 = r / k;
+                w0 = __ldg(a.topk_w + r);
+            }
+            if (lane + 32 < m.cnt) {
+                const int r = __ldg(a.perm + m.row0 + 32 + lane);
+                tk1 = r / k;
+                w1 = __ldg(a.topk_w + r);
+            }
+            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag)) break;
+            tc_fence_after();
+            const int h_row = m.sub * kT + 32 * qd + lane;
+            const uint32_t t_y = tmem + b * kRT + ((uint32_t)(32 * qd) << 16);
+            for (int n0 = 0; n0 < m.cnt; n0 += 16) {
+                float y[16];
+                tc_ld16(t_y + n0, y);
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int n = n0 + jj;
+                    if (n >= m.cnt) break;
+                    const int tk = __shfl_sync(0xffffffffu, n < 32 ? tk0 : tk1, n & 31);
+                    const float w = __shfl_sync(0xffffffffu, n < 32 ? w0 : w1, n & 31);
+                    atomicAdd(a.acc + (size_t)tk * H + h_row, w * y[jj]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[b]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && tid == 0) atomicOr(a.status, FLAG_TIMEOUT);
+    if (warp == 1) {
+        tc_fence_after();
+        tc_dealloc(tmem, 128);
+    }
+}
+
+__global__ void vq_cast_kernel(const float *__restrict__ acc, __nv_bfloat16 *__restrict__ out, long long n) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) out[i] = __float2bfloat16_rn(acc[i]);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// bf16 [rows][cols] with 64 x 64 boxes, 128B swizzle
+cudaError_t make_bf16_map(CUtensorMap *map, void *base, long long cols, long long rows) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+        return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kKS, (cuuint32_t)kRT};
+    const cuuint32_t es[2] = {1, 1};
+    const CUresult r = reinterpret_cast<EncodeTiledFn>(p)(
+        map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+size_t gu_smem() { return (size_t)kGUStages * kGUStage + kBook13 + kBook8 + 1024; }
+size_t dn_smem() { return (size_t)kDNStages * kDNStage + kBook13 + kBook8 + 1024; }
+
+}  // namespace
+
+bool prefill_vq_supported(const Layer &L, int T) {
+    return L.pv != nullptr && L.pv->ready && T >= 1 && L.d.fmt != MOEQ_FMT_MXFP4 && L.d.act == MOEQ_ACT_BF16;
+}
+
+cudaError_t prefill_vq_create(Layer &L) {
+    const moeq_layer_desc &d = L.d;
+    if (d.fmt == MOEQ_FMT_MXFP4 || d.act != MOEQ_ACT_BF16) return cudaSuccess;
+    if (d.hidden % kT || d.inter % kT) return cudaSuccess;
+    PrefillVq *pv = new (std::nothrow) PrefillVq();
+    if (!pv) return cudaErrorMemoryAllocation;
+    L.pv = pv;
+    const size_t R = (size_t)d.max_tokens * d.top_k;
+    cudaError_t e = cudaMalloc((void **)&pv->tile_base, sizeof(int32_t) * (d.n_experts + 1));
+    if (e == cudaSuccess) e = cudaMalloc((void **)&pv->xg, R * d.hidden * 2);
+    if (e == cudaSuccess) e = cudaMalloc((void **)&pv->hg, R * d.inter * 2);
+    // route positions past a tile's routes feed discarded MMA columns: keep them finite
+    if (e == cudaSuccess) e = cudaMemset(pv->xg, 0, R * d.hidden * 2);
+    if (e == cudaSuccess) e = cudaMemset(pv->hg, 0, R * d.inter * 2);
+    if (e != cudaSuccess) return e;
+    e = make_bf16_map(&pv->map_x, pv->xg, d.hidden, (long long)R);
+    if (e == cudaSuccess) e = make_bf16_map(&pv->map_h, pv->hg, d.inter, (long long)R);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(vq_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu_smem());
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(vq_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn_smem());
+    if (e == cudaSuccess) pv->ready = true;
+    return e == cudaErrorNotSupported ? cudaSuccess : e;
+}
+
+void prefill_vq_free(Layer &L) {
+    PrefillVq *pv = L.pv;
+    if (!pv) return;
+    cudaFree(pv->tile_base);
+    cudaFree(pv->xg);
+    cudaFree(pv->hg);
+    delete pv;
+    L.pv = nullptr;
+}
+
+cudaError_t launch_prefill_vq(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
+                              cudaStream_t s, const cudaEvent_t *ev) {
+    const PrefillVq *pv = L.pv;
+    const int E = L.d.n_experts, H = L.d.hidden, I = L.d.inter, k = L.d.top_k;
+    cudaError_t e = launch_route_bucket(L, ids, T * k, L.b.offsets, L.b.perm, L.b.active, s);
+    if (e != cudaSuccess) return e;
+    if (ev) record_phase(ev[1], s);
+    L.count_launches(5);
+    if ((e = launch_route_tiles(L.b.offsets, E, pv->tile_base, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(L.acc, 0, sizeof(float) * (size_t)T * H, s)) != cudaSuccess) return e;
+    {
+        const int warps = T * k < 148 * 16 ? T * k : 148 * 16;
+        vq_gather_x_kernel<<<(warps + 7) / 8, 256, 0, s>>>(reinterpret_cast<const uint16_t *>(x), L.b.perm, L.b.offsets,
+                                                            E, k, H, pv->xg);
+    }
+    VqArgs a{};
+    a.offsets = L.b.offsets;
+    a.tile_base = pv->tile_base;
+    a.perm = L.b.perm;
+    a.topk_w = topk_w;
+    a.book13 = reinterpret_cast<const uint8_t *>(L.w.book13);
+    a.book8 = L.d.fmt == MOEQ_FMT_VQ13_R8 ? reinterpret_cast<const uint8_t *>(L.w.book8) : nullptr;
+    a.hg = pv->hg;
+    a.acc = L.acc;
+    a.status = L.status;
+    a.E = E;
+    a.H = H;
+    a.I = I;
+    a.k = k;
+    auto proj = [&](int p) {
+        const ProjView v = L.view(p);
+        return VqProj{v.idx13, v.idx8, v.gain};
+    };
+    a.w0 = proj(MOEQ_GATE);
+    a.w1 = proj(MOEQ_UP);
+    vq_gateup_kernel<<<L.sm_count, kVqThreads, gu_smem(), s>>>(pv->map_x, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev) record_phase(ev[2], s);
+    VqArgs b = a;
+    b.w0 = proj(MOEQ_DOWN);
+    b.w1 = VqProj{nullptr, nullptr, nullptr};
+    vq_down_kernel<<<L.sm_count, kVqThreads, dn_smem(), s>>>(pv->map_h, b);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev) record_phase(ev[3], s);
+    const long long n = (long long)T * H;
+    vq_cast_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(L.acc, reinterpret_cast<__nv_bfloat16 *>(out), n);
+    if (ev) record_phase(ev[4], s);
+    return cudaGetLastError();
+}
+
+}  // namespace moeq
