@@ -171,7 +171,9 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
             ALLOC(L->w.codes[p], (size_t)E * MxGeom(N, K).expert_bytes());
             (void)rows;
         } else {
-            ALLOC(L->w.idx13[p], rows * row_bytes(fmt, 0, K));
+            // 16 bytes of slack: the tensor-core path reads each row's 13-byte
+            // index chunk of a 64-column slab as four aligned 32-bit words
+            ALLOC(L->w.idx13[p], rows * row_bytes(fmt, 0, K) + 16);
             if (fmt == MOEQ_FMT_VQ13_R8) ALLOC(L->w.idx8[p], rows * row_bytes(fmt, 1, K));
             ALLOC(L->w.gain[p], rows * sizeof(uint16_t));
         }

@@ -6,9 +6,10 @@
 // 8192 x 8 codebook (optionally plus an 8-bit index into a 256 x 8 residual
 // book), times an f16 row gain; one codebook pair serves every expert and
 // gate/up/down ("Why 13 bits": the books stay in shared memory while every
-// selected expert is decoded).  Weight = ((base + residual) * gain) in f32,
-// rounded once to bf16 for the tensor cores; activations are bf16 already,
-// so the MMAs are tcgen05.mma kind::f16 (bf16 x bf16 -> f32).
+// selected expert is decoded).  Weight = (base + residual) * gain, in bf16
+// for the tensor cores; activations are bf16 already,
+// so the MMAs are tcgen05.mma kind::f16 (bf16 x bf16 -> f32).  The expansion
+// adds base and residual codewords and applies the gain in bf16 pairs.
 //
 // Steps of one forward:
 //   route/bucket, route tiles (as for MXFP4: tiles of up to 64 routes)
@@ -49,6 +50,7 @@ constexpr int kGUStage = 2 * kTileA + kTileB;  // [A gate][A up][B]
 constexpr int kGUStages = 2;
 constexpr int kDNStage = kTileA + kTileB;      // [A down][B]
 constexpr int kDNStages = 3;
+constexpr int kPrefetch = 6;                   // slabs ahead the activation boxes are pulled into L2
 
 // kind::f16 instruction descriptor: bf16 A and B (K-major), f32 accumulate, M 128
 __device__ __forceinline__ uint32_t idesc_bf16(int n) {
@@ -62,61 +64,99 @@ __device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uin
         : "memory");
 }
 
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
 struct VqProj {
     const uint8_t *idx13;   // [E*N][K*13/64]
     const uint8_t *idx8;    // [E*N][K/8] or null
     const uint16_t *gain;   // [E*N] f16 or null
 };
 
-// The index data of vector j (K offset 8j within slab sl) of global row
-// `grow`, fetched ahead of its decode so that the global loads overlap the
-// gathers of earlier slabs: the bytes holding its 13-bit index, its residual
-// index and its row gain.
-struct VecRaw {
-    uint32_t win;   // bytes of the 13-bit field, little-endian
-    uint32_t i8;
-    uint32_t gain;  // f16 bits, 0x3C00 (1.0) when the layer has no gains
+// The index data of one row for one 64-column slab, fetched ahead of its
+// decode so that the global loads overlap the gathers of earlier slabs: the
+// 13-byte chunk of 13-bit indices as four aligned words (the allocation has
+// slack for the last row), the eight residual indices and the row gain.
+struct RowRaw {
+    uint32_t w[4];
+    uint32_t shift;   // bit offset of the chunk inside w
+    uint32_t i8lo, i8hi;
+    uint32_t gain;    // f16 bits, 0x3C00 (1.0) when the layer has no gains
 };
-__device__ __forceinline__ VecRaw fetch_vec(const VqProj &pj, int K, size_t grow, int sl, int j) {
-    VecRaw v;
-    const uint8_t *irow = pj.idx13 + grow * (size_t)(K * 13 / 64);
-    const uint32_t bit = (uint32_t)sl * (kKS / 8 * 13) + 13u * (uint32_t)j;
-    const uint8_t *pb = irow + (bit >> 3);
-    v.win = (uint32_t)__ldg(pb) | ((uint32_t)__ldg(pb + 1) << 8);
-    // the third byte only when the field reaches it (never past the row)
-    if ((bit & 7u) > 3u) v.win |= (uint32_t)__ldg(pb + 2) << 16;
-    v.i8 = pj.idx8 ? (uint32_t)__ldg(pj.idx8 + grow * (size_t)(K / 8) + (size_t)sl * (kKS / 8) + j) : 0u;
+__device__ __forceinline__ RowRaw fetch_row(const VqProj &pj, int K, size_t grow, int sl) {
+    RowRaw v;
+    const uint8_t *chunk = pj.idx13 + grow * (size_t)(K * 13 / 64) + (size_t)sl * (kKS / 8 * 13 / 8);
+    const uintptr_t ad = reinterpret_cast<uintptr_t>(chunk);
+    const uint32_t *wp = reinterpret_cast<const uint32_t *>(ad & ~uintptr_t(3));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v.w[i] = __ldg(wp + i);
+    v.shift = (uint32_t)(ad & 3) * 8;
+    if (pj.idx8) {
+        const uint2 q = __ldg(reinterpret_cast<const uint2 *>(pj.idx8 + grow * (size_t)(K / 8) + (size_t)sl * (kKS / 8)));
+        v.i8lo = q.x;
+        v.i8hi = q.y;
+    } else {
+        v.i8lo = v.i8hi = 0;
+    }
     v.gain = pj.gain ? (uint32_t)__ldg(pj.gain + grow) : 0x3C00u;
     return v;
 }
+// The eight 13-bit indices of a fetched row chunk (index j at bits 13j..).
+__device__ __forceinline__ void row_indices(const RowRaw &v, uint32_t idx[8]) {
+    const uint32_t x0 = __funnelshift_r(v.w[0], v.w[1], v.shift), x1 = __funnelshift_r(v.w[1], v.w[2], v.shift);
+    const uint32_t x2 = __funnelshift_r(v.w[2], v.w[3], v.shift), x3 = v.w[3] >> v.shift;
+    idx[0] = x0 & 0x1FFFu;
+    idx[1] = (x0 >> 13) & 0x1FFFu;
+    idx[2] = __funnelshift_r(x0, x1, 26) & 0x1FFFu;
+    idx[3] = (x1 >> 7) & 0x1FFFu;
+    idx[4] = __funnelshift_r(x1, x2, 20) & 0x1FFFu;
+    idx[5] = (x2 >> 1) & 0x1FFFu;
+    idx[6] = (x2 >> 14) & 0x1FFFu;
+    idx[7] = __funnelshift_r(x2, x3, 27) & 0x1FFFu;
+}
 
-// Expand a fetched vector into 8 bf16 weights at the 128B-swizzled K-major
-// position (tile row r, 16-byte chunk j) of a shared-memory A tile.
-__device__ __forceinline__ void expand_vec(const VecRaw &v, bool r8, int sl, int j, const uint8_t *book13,
-                                           const uint8_t *book8, uint8_t *tile, int r) {
-    const uint32_t bit = (uint32_t)sl * (kKS / 8 * 13) + 13u * (uint32_t)j;
-    const uint32_t idx = (v.win >> (bit & 7u)) & 0x1FFFu;
-    const uint4 c = lds128(book13 + (size_t)idx * 16);
-    float w[8] = {bf16lo(c.x), bf16hi(c.x), bf16lo(c.y), bf16hi(c.y), bf16lo(c.z), bf16hi(c.z), bf16lo(c.w), bf16hi(c.w)};
+__device__ __forceinline__ uint32_t bf16x2_add(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Expand vector j of a row (13-bit index idx, residual index i8, gain bits)
+// into 8 bf16 weights at the 128B-swizzled K-major position (tile row r,
+// 16-byte chunk j) of a shared-memory A tile.  The base and residual
+// codewords are added as bf16 pairs (one rounding of the exact sum) and
+// scaled by the row gain as bf16 pairs: the tensor cores take bf16 operands,
+// and two roundings to bf16 stay far inside the output tolerance
+// (moeq_dequant keeps the exact f32 weights).
+__device__ __forceinline__ void expand_vec(uint32_t idx, uint32_t i8, uint32_t gain, bool r8, int j,
+                                           const uint8_t *book13, const uint8_t *book8, uint8_t *tile, int r) {
+    uint4 o = lds128(book13 + (size_t)idx * 16);
     if (r8) {
-        const uint4 rr = lds128(book8 + (size_t)v.i8 * 16);
-        w[0] += bf16lo(rr.x); w[1] += bf16hi(rr.x); w[2] += bf16lo(rr.y); w[3] += bf16hi(rr.y);
-        w[4] += bf16lo(rr.z); w[5] += bf16hi(rr.z); w[6] += bf16lo(rr.w); w[7] += bf16hi(rr.w);
+        const uint4 rr = lds128(book8 + (size_t)i8 * 16);
+        o = make_uint4(bf16x2_add(o.x, rr.x), bf16x2_add(o.y, rr.y), bf16x2_add(o.z, rr.z), bf16x2_add(o.w, rr.w));
     }
-    if (v.gain != 0x3C00u) {
-        const float gn = __half2float(__ushort_as_half((unsigned short)v.gain));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] *= gn;
+    if (gain != 0x3C00u) {
+        const __nv_bfloat16 gb = __float2bfloat16_rn(__half2float(__ushort_as_half((unsigned short)gain)));
+        const uint32_t g2 = (uint32_t)*reinterpret_cast<const uint16_t *>(&gb) * 0x10001u;
+        o = make_uint4(bf16x2_mul(o.x, g2), bf16x2_mul(o.y, g2), bf16x2_mul(o.z, g2), bf16x2_mul(o.w, g2));
     }
-    const uint4 o = make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
     *reinterpret_cast<uint4 *>(tile + (r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4)) = o;
+}
+
+// Decode vectors [J0, J0 + NV) of one fetched row into tile row r.
+template <int J0, int NV>
+__device__ __forceinline__ void expand_row(const RowRaw &v, bool r8, const uint8_t *book13, const uint8_t *book8,
+                                           uint8_t *tile, int r) {
+    uint32_t idx[8];
+    row_indices(v, idx);
+#pragma unroll
+    for (int jj = 0; jj < NV; ++jj) {
+        const int j = J0 + jj;
+        const uint32_t i8 = ((j < 4 ? v.i8lo : v.i8hi) >> (8 * (j & 3))) & 0xFFu;
+        expand_vec(idx[j], i8, v.gain, r8, j, book13, book8, tile, r);
+    }
 }
 
 // One warp per route position: its token's x row, in route order.
@@ -206,6 +246,11 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
                 const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
                 mbar_arrive_expect_tx(&b_full[s], kTileB);
                 tma_load_2d(smem + (size_t)s * kGUStage + 2 * kTileA, &tX, (c % slabs) * kKS, m.row0, &b_full[s]);
+                // the ring is short: start the activation box of a later slab towards L2
+                if (c + kPrefetch < total) {
+                    const Item mp = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + ((c + kPrefetch) / slabs) * gridDim.x);
+                    tma_prefetch_2d(&tX, ((c + kPrefetch) % slabs) * kKS, mp.row0);
+                }
             }
             drain_stages(b_full, kGUStages, c);
             mbar_wait_bounded(&book_bar, 0, 200000000LL);
@@ -241,39 +286,42 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
             drain_mma(&tmem_done);
         }
     } else if (warp < 2 + kDecWarps) {
-        // decoders: per slab 2 matrices x 128 rows x 8 vectors; this thread
-        // always takes vector j of rows r0 + 32 i (i < 4) of both matrices, and
-        // fetches their index data two slabs ahead
-        const int dt = tid - 64, j = dt & 7, r0 = dt >> 3;
+        // decoders: per slab 2 matrices x 128 rows x 8 vectors; thread t
+        // takes all 8 vectors of row t % 128 of matrix t / 128.  Its index
+        // data comes from HBM four slabs ahead, into a ring of four register
+        // sets indexed at compile time (moving a register whose load is still
+        // in flight would wait for it)
+        const int dt = tid - 64, mat = dt >> 7, r = dt & 127;
         const bool r8 = a.book8 != nullptr;
-        VecRaw pa[8], pb[8];   // index data of slabs c and c + 1
-        auto fetch = [&](int c, VecRaw *dst) {
+        const VqProj &pj = mat ? a.w1 : a.w0;
+        auto fetch = [&](int c, RowRaw &dst) {
             if (c >= total) return;
             const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
-            const size_t row0 = (size_t)m.e * I + m.sub * kT + r0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = fetch_vec(i < 4 ? a.w0 : a.w1, H, row0 + 32 * (i & 3), c % slabs, j);
+            dst = fetch_row(pj, H, (size_t)m.e * I + m.sub * kT + r, c % slabs);
         };
-        fetch(0, pa);
-        fetch(1, pb);
+        RowRaw q0, q1, q2, q3;
+        fetch(0, q0);
+        fetch(1, q1);
+        fetch(2, q2);
+        fetch(3, q3);
         bool ok = wait_or_abort(&book_bar, 0, &abort_flag);
-        for (int c = 0; c < total && ok; ++c) {
-            const int s = c % kGUStages, sl = c % slabs;
+        auto step = [&](int c, RowRaw &q) {
+            if (c >= total || !ok) return;
+            const int s = c % kGUStages;
             if (c >= kGUStages) ok = wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            uint8_t *st = smem + (size_t)s * kGUStage;
-            VecRaw cur[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                cur[i] = pa[i];
-                pa[i] = pb[i];
-            }
-            fetch(c + 2, pb);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) expand_vec(cur[i], r8, sl, j, b13, b8, st + (i >> 2) * kTileA, r0 + 32 * (i & 3));
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) return;
+            expand_row<0, 8>(q, r8, b13, b8, smem + (size_t)s * kGUStage + mat * kTileA, r);
+            fetch(c + 4, q);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[s]);
+        };
+        for (int c = 0; c < total && ok; c += 4) {
+            step(c, q0);
+            step(c + 1, q1);
+            step(c + 2, q2);
+            step(c + 3, q3);
         }
     } else {
         // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 = rows of I
@@ -361,6 +409,10 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_con
                 const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
                 mbar_arrive_expect_tx(&b_full[s], kTileB);
                 tma_load_2d(smem + (size_t)s * kDNStage + kTileA, &tH, (c % slabs) * kKS, m.row0, &b_full[s]);
+                if (c + kPrefetch < total) {
+                    const Item mp = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + ((c + kPrefetch) / slabs) * gridDim.x);
+                    tma_prefetch_2d(&tH, ((c + kPrefetch) % slabs) * kKS, mp.row0);
+                }
             }
             drain_stages(b_full, kDNStages, c);
             mbar_wait_bounded(&book_bar, 0, 200000000LL);
@@ -392,38 +444,40 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_con
             drain_mma(&tmem_done);
         }
     } else if (warp < 2 + kDecWarps) {
-        // decoders: per slab 128 rows x 8 vectors; this thread takes vector j
-        // of rows r0 + 32 i (i < 4), index data fetched two slabs ahead
-        const int dt = tid - 64, j = dt & 7, r0 = dt >> 3;
+        // decoders: per slab 128 rows x 8 vectors; thread t takes vectors
+        // 4 (t % 2) .. + 3 of row t / 2, index data fetched two slabs ahead
+        const int dt = tid - 64, r = dt >> 1, j0 = (dt & 1) * 4;
         const bool r8 = a.book8 != nullptr;
-        VecRaw pa[4], pb[4];   // index data of slabs c and c + 1
-        auto fetch = [&](int c, VecRaw *dst) {
+        auto fetch = [&](int c, RowRaw &dst) {
             if (c >= total) return;
             const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
-            const size_t row0 = (size_t)m.e * H + m.sub * kT + r0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = fetch_vec(a.w0, I, row0 + 32 * i, c % slabs, j);
+            dst = fetch_row(a.w0, I, (size_t)m.e * H + m.sub * kT + r, c % slabs);
         };
-        fetch(0, pa);
-        fetch(1, pb);
+        RowRaw q0, q1, q2, q3;   // four slabs ahead, as in the gate/up kernel
+        fetch(0, q0);
+        fetch(1, q1);
+        fetch(2, q2);
+        fetch(3, q3);
         bool ok = wait_or_abort(&book_bar, 0, &abort_flag);
-        for (int c = 0; c < total && ok; ++c) {
-            const int s = c % kDNStages, sl = c % slabs;
+        auto step = [&](int c, RowRaw &q) {
+            if (c >= total || !ok) return;
+            const int s = c % kDNStages;
             if (c >= kDNStages) ok = wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            uint8_t *st = smem + (size_t)s * kDNStage;
-            VecRaw cur[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                cur[i] = pa[i];
-                pa[i] = pb[i];
-            }
-            fetch(c + 2, pb);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) expand_vec(cur[i], r8, sl, j, b13, b8, st, r0 + 32 * i);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) return;
+            uint8_t *tile = smem + (size_t)s * kDNStage;
+            if (j0 == 0) expand_row<0, 4>(q, r8, b13, b8, tile, r);
+            else expand_row<4, 4>(q, r8, b13, b8, tile, r);
+            fetch(c + 4, q);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[s]);
+        };
+        for (int c = 0; c < total && ok; c += 4) {
+            step(c, q0);
+            step(c + 1, q1);
+            step(c + 2, q2);
+            step(c + 3, q3);
         }
     } else {
         const int qd = warp & 3;

@@ -24,6 +24,13 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// Pull a future box of a tensor map into L2 (no shared memory involved).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
 // Shared-memory matrix descriptor, K-major.  128B swizzle: rows of 128 bytes,
 // 8-row groups 1024 bytes apart.  None: 8 x 16-byte core matrices, groups of
 // 8 rows `sbo` bytes apart, 16-byte columns `lbo` bytes apart.
