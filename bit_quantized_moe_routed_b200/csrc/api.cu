@@ -74,7 +74,6 @@ void free_layer(moeq_layer *L) {
     cudaFree(L->b.active);
     cudaFree(L->h);
     cudaFree(L->acc);
-    cudaFree(L->dec_gmax);
     cudaFree(L->dec_ybuf);
     cudaFree(L->dec_counters);
     cudaFree(L->status);
@@ -187,7 +186,6 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     ALLOC(L->b.perm, sizeof(int32_t) * M * k);
     ALLOC(L->h, sizeof(float) * M * k * I);
     ALLOC(L->acc, sizeof(float) * M * H);
-    ALLOC(L->dec_gmax, sizeof(float) * kDecMaxGrid * kDecMaxTokens);
     ALLOC(L->dec_ybuf, sizeof(float) * kDecMaxRoutes * kDecMaxTokens * H);
     ALLOC(L->dec_counters, sizeof(int) * (H / 32 + 1));
     ALLOC(L->status, sizeof(uint32_t));

@@ -13,8 +13,11 @@
 // per 1024-column chunk of K, so every chunk of a unit is in compute at
 // once; inside a group each warp takes a share of the chunk's 32-weight
 // block columns for both halves (gate and up, or the two 16-row down tiles),
-// i.e. two independent accumulator chains.  Once per unit, after one
-// barrier, threads spread over all warps sum the partial fragments.
+// i.e. two independent accumulator chains.  A warp reads the fragments of
+// its next group while it computes the current one.  Per unit the warps
+// hand their partial fragments to two epilogue warps through a two-slot
+// ring (full/empty mbarriers), which sum them (SwiGLU and h for gate/up),
+// so the consumers never wait for one another.
 //
 // Memory: the device layout (MxGeom) keeps each (16-row tile, 1024-column
 // chunk) block contiguous, so a producer warp streams a chunk of a unit as
@@ -22,7 +25,9 @@
 // full/empty mbarriers, unit by unit and chunk by chunk; the activations
 // arrive first, one bulk copy per token.  Bulk copies of several KB are what
 // keep HBM busy; the layout also makes the fragment and scale reads
-// bank-conflict free.
+// bank-conflict free.  The gate/up kernel lets the down kernel launch as its
+// CTAs finish (programmatic dependent launch): the down weights stream in
+// while gate/up drains, and only the down consumers wait for h.
 //
 // Math: warp-level mma.sync.m16n8k16 (f16 in, f32 accumulate).  Each thread
 // reads its A-fragment slice of four 32-weight blocks (bytes 4t..4t+3 of
@@ -30,15 +35,15 @@
 // cvt.rn.f16x2.e2m1x2 (exact).  Per block the two MMAs accumulate into a
 // fresh fragment that is folded into the running f32 sum times the block's
 // E8M0 scale (one packed f32x2 FMA per row pair), so the scale is applied
-// exactly.  The B operand (activations, or w * h for the down projection) is
-// f16 after a per-token power-of-two prescale that puts the largest
-// magnitude in [2^14, 2^15): f16 cannot overflow, and the scale is undone in
-// f32.
+// exactly.  The B operand is f16 after a power-of-two prescale that puts the
+// largest magnitude in [2^14, 2^15): per token for the activations, per
+// (expert, token) column of w * h for the down projection.  f16 cannot
+// overflow, and the scale is undone in f32.
 //
-// Combine: the down kernel writes each expert's contribution to its own
-// slice of a scratch buffer; the last unit to finish a 32-row tile
-// (per-tile arrival counter) sums the experts in a fixed order, undoes the
-// prescale and writes bf16 out, so the result does not depend on timing.
+// Combine: the down kernel writes each expert's contribution, prescale
+// undone, to its own slice of a scratch buffer; the last unit to finish a
+// 32-row tile (per-tile arrival counter) sums the experts in a fixed order
+// and writes bf16 out, so the result does not depend on timing.
 #include "async.cuh"
 #include "internal.cuh"
 
@@ -56,17 +61,27 @@ struct RouteTable {
     int col_beg[kMaxR + 1];  // routes of expert slot d: route[col_beg[d] .. col_beg[d+1])
     int route[kMaxR];        // valid route ids sorted by (expert, route id)
     int sid[kMaxR];          // copy of topk_ids
+    float w[kMaxR];          // copy of topk_w (kept on chip: a global load per unit stalls the warps)
+    uint8_t tok[kMaxR];      // token of route id r (r / k)
 };
 
 // Warp 0 builds the table (R = T*k <= 64 routes).
-__device__ void build_route_table(RouteTable &tb, const int32_t *__restrict__ ids, int R, int E,
-                                  uint32_t *status, bool report) {
+__device__ void build_route_table(RouteTable &tb, const int32_t *__restrict__ ids, const float *__restrict__ topk_w,
+                                  int R, int k, int E, uint32_t *status, bool report) {
     const unsigned full = 0xffffffffu;
     const int lane = threadIdx.x & 31;
     const int r0 = lane, r1 = lane + 32;
     const int id0 = r0 < R ? ids[r0] : -1, id1 = r1 < R ? ids[r1] : -1;
-    if (r0 < R) tb.sid[r0] = id0;
-    if (r1 < R) tb.sid[r1] = id1;
+    if (r0 < R) {
+        tb.sid[r0] = id0;
+        tb.w[r0] = topk_w[r0];
+        tb.tok[r0] = (uint8_t)(r0 / k);
+    }
+    if (r1 < R) {
+        tb.sid[r1] = id1;
+        tb.w[r1] = topk_w[r1];
+        tb.tok[r1] = (uint8_t)(r1 / k);
+    }
     const bool v0 = id0 >= 0 && id0 < E, v1 = id1 >= 0 && id1 < E;
     const bool bad = (r0 < R && !v0 && id0 != -1) || (r1 < R && !v1 && id1 != -1);
     if (report && __any_sync(full, bad) && lane == 0) atomicOr(status, FLAG_ROUTE_RANGE);
@@ -197,9 +212,9 @@ __device__ __forceinline__ void named_sync_consumers() {
 
 // ---------------------------------------------------------------- staging
 
-// Warp roles: kCW consumer warps plus one producer warp that streams
-// (tile, chunk) blocks into a ring of shared-memory stages.
-constexpr int kWSThreads = 32 * (kCW + 1);
+// Warp roles: kCW consumer warps, one producer warp that streams (tile,
+// chunk) blocks into a ring of shared-memory stages, and epilogue warps
+// that reduce the consumers' partial sums.
 constexpr int kProducerWarp = kCW;
 constexpr int kKC = 1024;                       // weights of K per chunk (the layout's chunk)
 constexpr int kBlk = 16 * (kKC / 2 + kKC / 32); // one (16-row tile, chunk) block of the device layout
@@ -208,7 +223,7 @@ constexpr int kBlk = 16 * (kKC / 2 + kKC / 32); // one (16-row tile, chunk) bloc
 // cps blocks], each half one contiguous run of the device layout.
 __host__ __device__ inline size_t piece_bytes(int cps) { return 2 * (size_t)cps * kBlk; }
 constexpr int kMaxStages = 12;
-constexpr int kMaxDynSmem = 232448 - 4096;      // leave room for static shared memory
+constexpr int kMaxDynSmem = 232448 - 5120;      // leave room for static shared memory (4.3 KB in the down kernel)
 
 // Shared-memory address of this thread's fragment word (bytes 4t..4t+3 of
 // the four blocks of K-group grp) of staged row r (0..15) of a block.
@@ -237,17 +252,28 @@ __device__ __forceinline__ void my_range(int n, int &beg, int &end) {
 // the stage's barrier is in the phase of piece p; this keeps a warp that
 // runs ahead of the others from matching the parity of a phase two rounds
 // old.
+// n / d and n % d for 0 <= n < 2^16 and 2 <= d < 2^16 with one
+// multiply-high, m = ceil(2^32 / d) (the error n (m d - 2^32) / 2^32 stays
+// below one part in d): integer division by a runtime value would take
+// the conversion pipe, which the weight decode keeps busy.
+struct FastDiv {
+    uint32_t d, m;
+    __device__ __forceinline__ uint32_t div(uint32_t n) const { return __umulhi(n, m); }
+};
+inline FastDiv make_fastdiv(uint32_t d) { return {d, (uint32_t)((0x100000000ull + d - 1) / d)}; }
+
 template <typename BlockOf>
-__device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_t *empty, int S, int cps,
+__device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_t *empty, FastDiv S, int cps,
                                         int n_pieces, uint32_t *status, volatile int *issued, BlockOf block_of) {
     const int lane = threadIdx.x & 31, i = lane >> 1, half = lane & 1;
-    const int G = min(S, max(1, 4 / cps));
+    const int G = min((int)S.d, max(1, 4 / cps));
     const uint32_t half_bytes = (uint32_t)cps * kBlk;
     for (int p0 = 0; p0 < n_pieces; p0 += G) {
         const int p = p0 + i;
         const bool mine = i < G && p < n_pieces;
-        const int s = mine ? p % S : 0;
-        if (mine && half == 0 && p >= S && !mbar_wait_bounded(&empty[s], (uint32_t)((p / S - 1) & 1)))
+        const uint32_t rnd = S.div((uint32_t)p);
+        const int s = mine ? p - (int)(rnd * S.d) : 0;
+        if (mine && half == 0 && rnd > 0 && !mbar_wait_bounded(&empty[s], (rnd - 1) & 1u))
             atomicOr(status, FLAG_TIMEOUT);
         __syncwarp();
         if (mine && half == 0) mbar_arrive_expect_tx(&full[s], 2u * half_bytes);
@@ -263,10 +289,18 @@ __device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_
             *issued = min(p0 + G, n_pieces);
         }
     }
+    // wait for the last copy of every stage to land, so that no copy is in
+    // flight when the CTA exits (consumers that gave up on a wait exit early)
+    if (lane == 0)
+        for (int p = max(0, n_pieces - (int)S.d); p < n_pieces; ++p) {
+            const uint32_t rnd = S.div((uint32_t)p);
+            if (!mbar_wait_bounded(&full[p - (int)(rnd * S.d)], rnd & 1u)) atomicOr(status, FLAG_TIMEOUT);
+        }
+    __syncwarp();
 }
 
 // Consumer: wait until piece p is issued, then for its data.  False on timeout.
-__device__ __forceinline__ bool wait_piece(uint64_t *full, int S, int p, volatile int *issued) {
+__device__ __forceinline__ bool wait_piece(uint64_t *full, FastDiv S, int p, volatile int *issued) {
     if (*issued <= p) {
         const long long t0 = clock64();
         while (*issued <= p) {
@@ -274,7 +308,8 @@ __device__ __forceinline__ bool wait_piece(uint64_t *full, int S, int p, volatil
             __nanosleep(32);
         }
     }
-    return mbar_wait_bounded(&full[p % S], (uint32_t)((p / S) & 1));
+    const uint32_t rnd = S.div((uint32_t)p);
+    return mbar_wait_bounded(&full[p - (int)(rnd * S.d)], rnd & 1u);
 }
 
 // Chunk q of every unit is computed by the 16/NCH warps [q*16/NCH, ...): a
@@ -356,10 +391,16 @@ struct GateUpArgs {
     const int32_t *ids;                 // [T][k]
     const float *topk_w;                // [T][k]
     float *h;                           // [T*k][I] f32, by route id
-    float *gmax;                        // [gridDim.x][kMaxT]: per-CTA max |w h| per token
     uint32_t *status;
-    int T, k, E, H, I, n_stages, cps;
+    FastDiv S;                          // stages
+    int T, k, E, H, I, cps;
 };
+
+// Partial-sum slots between the consumer warps and the epilogue warps.
+constexpr int kRedSlots = 2;
+constexpr int kEpiWarps = 2;
+constexpr int kGUThreads = 32 * (kCW + 1 + kEpiWarps);
+constexpr int kEpiWarp0 = kCW + 1;
 
 __host__ __device__ inline size_t gu_xs_off(int n_stages, int cps) { return (size_t)n_stages * piece_bytes(cps); }
 __host__ __device__ inline size_t gu_red_off(int n_stages, int cps, int T, int H) {
@@ -370,22 +411,30 @@ __host__ __device__ inline size_t gu_bytes(int n_stages, int cps, int T, int H) 
 }
 
 // Unit i -> (expert slot d, column chunk, 16-row tile): experts with more
-// than 8 routes take one pass per 8 columns.
+// than 8 routes take one pass per 8 columns.  A CTA keeps its own range of
+// units as packed words: d | tile << 6 | first column << 15 | columns << 22.
 struct GUItems {
     int n;
     int beg[kMaxR + 1];
 };
+constexpr int kMaxUnits = 128;   // units of one CTA (checked on the host)
+__device__ __forceinline__ int unit_d(uint32_t u) { return (int)(u & 63u); }
+__device__ __forceinline__ int unit_tile(uint32_t u) { return (int)((u >> 6) & 511u); }
+__device__ __forceinline__ int unit_cb(uint32_t u) { return (int)((u >> 15) & 127u); }
+__device__ __forceinline__ int unit_ncol(uint32_t u) { return (int)(u >> 22); }
 
 template <int NCH>   // K chunks per unit = H / kKC
-__global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs a) {
+__global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ RouteTable tb;
     __shared__ GUItems items;
-    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], xbar;
+    __shared__ uint32_t units[kMaxUnits];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], xbar, red_full[kRedSlots],
+        red_empty[kRedSlots];
     __shared__ int issued;   // chunks issued by the producer (see produce)
+    __shared__ int n_units, unit0;
     __shared__ float xinv[kMaxT];
-    __shared__ unsigned cta_max[kMaxT];
-    const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages, cps = a.cps, Tc = red_cols(a.T);
+    const int H = a.H, I = a.I, T = a.T, k = a.k, S = (int)a.S.d, cps = a.cps, Tc = red_cols(a.T);
     uint8_t *stages = smem_raw;
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw + gu_xs_off(S, cps));
     float *red = reinterpret_cast<float *>(smem_raw + gu_red_off(S, cps, T, H));
@@ -395,19 +444,26 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     const int tiles = I / 16;
     const MxGeom geo(I, H);
     constexpr int WPC = kCW / NCH;   // warps per chunk
+    const int lcps = cps == 4 ? 2 : (cps == 2 ? 1 : 0);
 
+    // the down kernel may take SMs as this grid's CTAs finish: it streams
+    // its weights at once and reads h only after this grid completes
+    pdl_launch_dependents();
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], WPC * cps);
         }
         mbar_init(&xbar, 1);
+        for (int r = 0; r < kRedSlots; ++r) {
+            mbar_init(&red_full[r], kCW);
+            mbar_init(&red_empty[r], kEpiWarps);
+        }
         mbar_fence_init();
         issued = 0;
     }
-    if (tid < kMaxT) cta_max[tid] = 0u;
     if (warp == 0) {
-        build_route_table(tb, a.ids, T * k, a.E, a.status, blockIdx.x == 0);
+        build_route_table(tb, a.ids, a.topk_w, T * k, k, a.E, a.status, blockIdx.x == 0);
         __syncwarp();
         if (lane == 0) {
             int n = 0;
@@ -417,32 +473,66 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
             }
             items.beg[tb.D] = n;
             items.n = n;
+            int i0, i1;
+            my_range(n, i0, i1);
+            unit0 = i0;
+            n_units = min(i1 - i0, kMaxUnits);
+        }
+        __syncwarp();
+        // this CTA's units, one per lane
+        for (int j = lane; j < n_units; j += 32) {
+            const int i = unit0 + j;
+            int d = 0;
+            while (items.beg[d + 1] <= i) ++d;
+            const int rel = i - items.beg[d], pass = rel / tiles, tile = rel - pass * tiles;
+            const int cb = tb.col_beg[d] + pass * 8, ncol = min(8, tb.col_beg[d + 1] - cb);
+            units[j] = (uint32_t)d | ((uint32_t)tile << 6) | ((uint32_t)cb << 15) | ((uint32_t)ncol << 22);
         }
     }
     __syncthreads();
-    int i0, i1;
-    my_range(items.n, i0, i1);
-    const int n_mine = i1 - i0;
-    auto decode_item = [&](int i, int &d, int &rel) {
-        d = 0;
-        while (items.beg[d + 1] <= i) ++d;
-        rel = i - items.beg[d];
-    };
+    const int n_mine = n_units;
 
     if (warp == kProducerWarp) {
         // the activations first (one bulk copy per token row, into padded rows)
         if (lane == 0) mbar_arrive_expect_tx(&xbar, (uint32_t)(T * H * 2));
         __syncwarp();
         if (lane < T) bulk_g2s(xs + (size_t)lane * xs_stride, a.x + (size_t)lane * H, H * 2, &xbar);
-        produce(stages, full, empty, S, cps, n_mine * NCH / cps, a.status, &issued,
+        produce(stages, full, empty, a.S, cps, n_mine * NCH / cps, a.status, &issued,
                 [&](int p, const uint8_t *&b0, const uint8_t *&b1) {
                     const int c = p * cps;
-                    int d, rel;
-                    decode_item(i0 + c / NCH, d, rel);
-                    const size_t off = (size_t)tb.expert[d] * geo.expert_bytes() + geo.block_off(rel % tiles, c % NCH);
+                    const uint32_t u = units[c / NCH];
+                    const size_t off = (size_t)tb.expert[unit_d(u)] * geo.expert_bytes() +
+                                       geo.block_off(unit_tile(u), c % NCH);
                     b0 = a.codes_g + off;
                     b1 = a.codes_u + off;
                 });
+        return;
+    }
+
+    if (warp >= kEpiWarp0) {
+        // epilogue: sum the 16 warps' partial fragments of a unit, SwiGLU, h
+        const int e = warp - kEpiWarp0;
+        bool to = false;
+        for (int j = 0; j < n_mine && !to; ++j) {
+            const int slot = j % kRedSlots;
+            if (!mbar_wait_bounded(&red_full[slot], (uint32_t)((j / kRedSlots) & 1))) {
+                to = true;
+                break;
+            }
+            const uint32_t u = units[j];
+            const int cb = unit_cb(u), ncol = unit_ncol(u), n0 = unit_tile(u) * 16;
+            const float *rb = red + (size_t)slot * kCW * 2 * 16 * Tc;
+            for (int idx = lane + 32 * e; idx < 16 * ncol; idx += 32 * kEpiWarps) {
+                const int row = idx & 15, col = idx >> 4;
+                const float gs = sum_partials(rb, Tc, 0, row, col), us = sum_partials(rb, Tc, 1, row, col);
+                const int route = tb.route[cb + col];
+                const float inv = xinv[tb.tok[route]];
+                a.h[(size_t)route * I + n0 + row] = silu_f32(gs * inv) * (us * inv);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_empty[slot]);
+        }
+        if (to && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
         return;
     }
 
@@ -479,57 +569,73 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     }
     named_sync_consumers();
 
+    // Each warp walks its groups of every unit one ahead: the fragments of
+    // the next group (the next unit's first group at the end of a unit) are
+    // read from shared memory while the current group is computed.  A unit's
+    // stage is released once its last group is in registers, before the
+    // warp waits for the next unit's piece.
     const int q = warp / WPC, wi = warp % WPC;   // this warp's chunk of every unit and its place in it
-    for (int j = 0; j < n_mine; ++j) {
-        int d, rel;
-        decode_item(i0 + j, d, rel);
-        const int cb = tb.col_beg[d] + (rel / tiles) * 8, n0 = (rel % tiles) * 16;
-        const int ncol = min(8, tb.col_beg[d + 1] - cb);
+    constexpr int NG = NCH / 2;                  // groups of this warp per unit
+    const uint8_t *st0 = stages, *st1 = stages;
+    int s_cur = 0;
+    auto open_unit = [&](int j, const uint8_t *&b0, const uint8_t *&b1, int &s) {
+        const int c = j * NCH + q, pc = c >> lcps;
+        if (!wait_piece(full, a.S, pc, &issued)) timed_out = true;
+        s = pc - (int)(a.S.div((uint32_t)pc) * a.S.d);
+        // [gate blocks of the piece][up blocks of the piece]
+        b0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c & (cps - 1)) * kBlk;
+        b1 = b0 + (size_t)cps * kBlk;
+    };
+    GroupFrags cur;
+    if (n_mine > 0) {
+        open_unit(0, st0, st1, s_cur);
+        load_group(st0, st1, g, t, wi * NG, cur);
+    }
+    for (int j = 0; j < n_mine && !timed_out; ++j) {
+        const uint32_t u = units[j];
+        const int cb = unit_cb(u), ncol = unit_ncol(u);
         const bool live = g < ncol;
-        const int tok = live ? tb.route[cb + g] / k : 0;
+        const int tok = live ? tb.tok[tb.route[cb + g]] : 0;
         const uint16_t *xrow = xs + (size_t)tok * xs_stride + 8 * t;
         float aG[4] = {0.f, 0.f, 0.f, 0.f}, aU[4] = {0.f, 0.f, 0.f, 0.f};
-        {
-            const int c = j * NCH + q, pc = c / cps, s = pc % S;
-            if (!wait_piece(full, S, pc, &issued)) timed_out = true;
-            // [gate blocks of the piece][up blocks of the piece]
-            const uint8_t *st0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c % cps) * kBlk;
-            const uint8_t *st1 = st0 + (size_t)cps * kBlk;
-            GroupFrags fr[NCH / 2];
 #pragma unroll
-            for (int p = 0; p < NCH / 2; ++p) load_group(st0, st1, g, t, wi * (NCH / 2) + p, fr[p]);
-            // the stage is free again once every warp holds its share
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-#pragma unroll
-            for (int p = 0; p < NCH / 2; ++p) {
-                const int gp = wi * (NCH / 2) + p;
-                const uint16_t *xq = xrow + (size_t)(q * (kKC / 32) + gp * 4) * 32;
-                uint4 xb[4];
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) xb[jj] = live ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
-                compute_group(fr[p], xb, aG, aU);
+        for (int p = 0; p < NG; ++p) {
+            const int gp = wi * NG + p;
+            const uint8_t *n0 = st0, *n1 = st1;
+            int ns = s_cur;
+            GroupFrags nxt;
+            if (p + 1 < NG) {
+                load_group(st0, st1, g, t, gp + 1, nxt);
+            } else {
+                // every group of this unit was read before the compute that
+                // precedes this step: release the stage before waiting for
+                // the next unit's piece (holding it could wait on itself)
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s_cur]);
+                if (j + 1 < n_mine) {
+                    open_unit(j + 1, n0, n1, ns);
+                    load_group(n0, n1, g, t, wi * NG, nxt);
+                }
             }
+            const uint16_t *xq = xrow + (size_t)(q * (kKC / 32) + gp * 4) * 32;
+            uint4 xb[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) xb[jj] = live ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
+            compute_group(cur, xb, aG, aU);
+            cur = nxt;
+            st0 = n0;
+            st1 = n1;
+            s_cur = ns;
         }
-        float *rb = red + (size_t)(j & 1) * kCW * 2 * 16 * Tc;
-        put_partials(rb, Tc, warp, g, t, aG, aU);
-        named_sync_consumers();
-        if ((lane & 3) == 0) {   // readers spread over the warps: (row, column) = r % 16, r / 16
-            const int r = warp + kCW * (lane >> 2), row = r & 15, col = r >> 4;
-            if (col < ncol) {
-                const float gs = sum_partials(rb, Tc, 0, row, col), us = sum_partials(rb, Tc, 1, row, col);
-                const int route = tb.route[cb + col];
-                const float inv = xinv[route / k];
-                const float hv = silu_f32(gs * inv) * (us * inv);
-                a.h[(size_t)route * I + n0 + row] = hv;
-                const float wh = fabsf(a.topk_w[route] * hv);
-                if (wh > 0.f) atomicMax(&cta_max[route / k], __float_as_uint(isfinite(wh) ? wh : 3.0e38f));
-            }
-        }
+        // hand the partial fragments to the epilogue warps
+        const int slot = j % kRedSlots;
+        if (j >= kRedSlots && !mbar_wait_bounded(&red_empty[slot], (uint32_t)((j / kRedSlots - 1) & 1)))
+            timed_out = true;
+        put_partials(red + (size_t)slot * kCW * 2 * 16 * Tc, Tc, warp, g, t, aG, aU);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_full[slot]);
     }
     if (timed_out && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
-    named_sync_consumers();
-    if (tid < kMaxT) a.gmax[(size_t)blockIdx.x * kMaxT + tid] = __uint_as_float(cta_max[tid]);
 }
 
 // ---------------------------------------------------------------- down
@@ -537,22 +643,23 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_gateup_mx_kernel(GateUpArgs
 struct DownArgs {
     const uint8_t *codes;           // down projection in the device layout (MxGeom)
     const float *h;                 // [T*k][I]
-    const float *gmax;              // [n_gmax][kMaxT]
-    int n_gmax;
     const int32_t *ids;
     const float *topk_w;
     float *ybuf;                    // [kMaxR expert slots][kMaxT][H]
     int *counters;                  // [H/32], zero between calls
     uint16_t *out;                  // bf16 [T][H]
     uint32_t *status;
-    int T, k, E, H, I, n_stages, cps;
+    FastDiv S;                      // stages
+    int T, k, E, H, I, cps;
 };
 
 // Staged (expert, token) B columns per CTA.  A CTA's contiguous range of
-// units is shorter than one expert's tiles, so it touches at most two
-// experts: 2T columns (capped; beyond the cap B is built from h in L2).
+// units is no longer than one expert's tiles when the grid has at least as
+// many CTAs as there are routed experts, so it touches at most two experts:
+// at most 2T columns.
 constexpr int kMaxBSlots = 16;
 constexpr int kMaxTiles = 128;   // H / 32 for H <= 4096
+constexpr int kDNThreads = kGUThreads;
 __host__ __device__ inline int dn_slots(int T) { return 2 * T < kMaxBSlots ? 2 * T : kMaxBSlots; }
 __host__ __device__ inline size_t dn_red_off(int n_stages, int cps, int T, int I) {
     return (size_t)n_stages * piece_bytes(cps) + sizeof(uint16_t) * (size_t)dn_slots(T) * (I + kXPad);
@@ -562,18 +669,18 @@ __host__ __device__ inline size_t dn_bytes(int n_stages, int cps, int T, int I) 
 }
 
 template <int NCH>   // K chunks per unit = I / kKC
-__global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) {
+__global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ RouteTable tb;
-    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], red_full[kRedSlots], red_empty[kRedSlots];
     __shared__ int issued;   // chunks issued by the producer (see produce)
-    __shared__ float tok_scale[kMaxT], tok_inv[kMaxT];
-    __shared__ int slot_of[kMaxR][kMaxT];   // (expert slot - d_lo, token) -> staged B column, -1 none
+    __shared__ int slot_of[2][kMaxT];    // (expert slot - d_lo, token) -> staged B column, -1 none
     __shared__ int slot_d[kMaxBSlots], slot_t[kMaxBSlots];
+    __shared__ unsigned slot_max[kMaxBSlots];
+    __shared__ float slot_scale[kMaxBSlots], slot_inv[kMaxBSlots];
     __shared__ int n_slots, n_last;
     __shared__ int last_tiles[kMaxTiles];
-    const int H = a.H, I = a.I, T = a.T, k = a.k, S = a.n_stages, cps = a.cps, Tc = red_cols(a.T);
-    const int cap = dn_slots(T);
+    const int H = a.H, I = a.I, T = a.T, k = a.k, S = (int)a.S.d, cps = a.cps, Tc = red_cols(a.T);
     uint8_t *stages = smem_raw;
     uint16_t *bs = reinterpret_cast<uint16_t *>(smem_raw + (size_t)S * piece_bytes(cps));   // [slot][I+pad] f16
     float *red = reinterpret_cast<float *>(smem_raw + dn_red_off(S, cps, T, I));
@@ -583,33 +690,42 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
     const int tiles = H / 32;
     const MxGeom geo(H, I);
     constexpr int WPC = kCW / NCH;   // warps per chunk
+    const int lcps = cps == 4 ? 2 : (cps == 2 ? 1 : 0);
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], WPC * cps);
         }
+        for (int r = 0; r < kRedSlots; ++r) {
+            mbar_init(&red_full[r], kCW);
+            mbar_init(&red_empty[r], kEpiWarps);
+        }
         mbar_fence_init();
         issued = 0;
         n_last = 0;
     }
-    if (warp == 0) build_route_table(tb, a.ids, T * k, a.E, nullptr, false);
+    if (tid < kMaxBSlots) slot_max[tid] = 0u;
+    if (warp == 0) build_route_table(tb, a.ids, a.topk_w, T * k, k, a.E, nullptr, false);
     __syncthreads();
     const int n_units = tb.D * tiles;
     if (tb.D == 0) {   // no valid route at all: every output is zero
-        for (int i = blockIdx.x * kWSThreads + tid; i < T * H; i += gridDim.x * kWSThreads) a.out[i] = 0;
+        for (int i = blockIdx.x * kDNThreads + tid; i < T * H; i += gridDim.x * kDNThreads) a.out[i] = 0;
         return;
     }
     int u0, u1;
     my_range(n_units, u0, u1);
     const int n_mine = u1 - u0;
+    // unit u -> expert slot u / tiles, 32-row tile u % tiles (tiles is a power of two)
+    const int ltiles = 31 - __clz(tiles);
+    const int d_lo = n_mine > 0 ? u0 >> ltiles : 0;
 
     if (warp == kProducerWarp) {
         // the weights do not depend on the gate/up kernel: stream them at once
-        produce(stages, full, empty, S, cps, n_mine * NCH / cps, a.status, &issued,
+        produce(stages, full, empty, a.S, cps, n_mine * NCH / cps, a.status, &issued,
                 [&](int p, const uint8_t *&b0, const uint8_t *&b1) {
                     const int c = p * cps;
-                    const int u = u0 + c / NCH, d = u / tiles, t32 = u % tiles, q = c % NCH;
+                    const int u = u0 + c / NCH, d = u >> ltiles, t32 = u & (tiles - 1), q = c % NCH;
                     const uint8_t *eb = a.codes + (size_t)tb.expert[d] * geo.expert_bytes();
                     b0 = eb + geo.block_off(2 * t32, q);
                     b1 = eb + geo.block_off(2 * t32 + 1, q);
@@ -617,149 +733,179 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
         return;
     }
 
-    // the experts this CTA's units touch, and their (expert, token) columns
-    const int d_lo = n_mine > 0 ? u0 / tiles : 0, d_hi = n_mine > 0 ? (u1 - 1) / tiles : -1;
+    if (warp >= kEpiWarp0) {
+        // epilogue: sum the 16 warps' partial fragments of a unit, undo the
+        // column's prescale and store the expert's f32 slice for the combine
+        const int e = warp - kEpiWarp0;
+        bool to = false;
+        for (int j = 0; j < n_mine && !to; ++j) {
+            const int slot = j % kRedSlots;
+            if (!mbar_wait_bounded(&red_full[slot], (uint32_t)((j / kRedSlots) & 1))) {
+                to = true;
+                break;
+            }
+            const int u = u0 + j, d = u >> ltiles, m0 = (u & (tiles - 1)) * 32;
+            const float *rb = red + (size_t)slot * kCW * 2 * 16 * Tc;
+            for (int idx = lane + 32 * e; idx < 32 * T; idx += 32 * kEpiWarps) {
+                const int row = idx & 31, col = idx >> 5;
+                const int sl = slot_of[d - d_lo][col];
+                const float v = sl >= 0 ? sum_partials(rb, Tc, row >> 4, row & 15, col) * slot_inv[sl] : 0.f;
+                __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row, v);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_empty[slot]);
+        }
+        if (to && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
+        __threadfence();
+        asm volatile("bar.sync 3, %0;" ::"r"(32 * (kCW + kEpiWarps)) : "memory");
+        return;
+    }
+
+    // ---- consumers.  The (expert, token) columns of this CTA's experts
     if (tid == 0) {
         int ns = 0;
-        for (int d = d_lo; d <= d_hi; ++d)
-            for (int tk = 0; tk < T; ++tk) {
-                bool used = false;
-                for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) used |= (tb.route[cc] / k == tk);
-                int sl = -1;
-                if (used) {
-                    if (ns < cap) {
-                        slot_d[ns] = d;
-                        slot_t[ns] = tk;
-                    }
-                    sl = ns++;
+        const int d_hi = n_mine > 0 ? (u1 - 1) >> ltiles : -1;
+        for (int dd = 0; dd < 2; ++dd)
+            for (int tk = 0; tk < kMaxT; ++tk) slot_of[dd][tk] = -1;
+        for (int d = d_lo; d <= d_hi && d < d_lo + 2; ++d)
+            for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) {
+                const int tk = tb.tok[tb.route[cc]];
+                if (ns < kMaxBSlots && slot_of[d - d_lo][tk] < 0) {
+                    slot_of[d - d_lo][tk] = ns;
+                    slot_d[ns] = d;
+                    slot_t[ns++] = tk;
                 }
-                slot_of[d - d_lo][tk] = sl;
             }
         n_slots = ns;
     }
-    // h and gmax come from the gate/up kernel
+    // h comes from the gate/up kernel
     pdl_wait_primary();
-    if (warp < kMaxT) {
-        // eight independent loads per lane cover 256 CTAs in one round trip
-        float v[8];
+    named_sync_consumers();
+    // B column sl = (sum of w_r h_r over the token's routes to the expert,
+    // in f32) * 2^s_sl in f16, the power of two putting the column's largest
+    // magnitude in [2^14, 2^15): f16 cannot overflow and the epilogue undoes
+    // the scale exactly.  Pass 1 finds the maxima with the values kept in
+    // registers (two 8-value pieces per thread; larger layers build them
+    // again in pass 2).
+    const int n_idx = n_slots * (I / 8);
+    auto col8 = [&](int idx, float *vv) {   // 8 values of B column idx / (I/8) from k = 8 (idx % (I/8))
+        const int sl = idx / (I / 8), k8 = (idx % (I / 8)) * 8, d = slot_d[sl], tk = slot_t[sl];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int i = lane + 32 * q;
-            v[q] = i < a.n_gmax ? __ldcg(a.gmax + (size_t)i * kMaxT + warp) : 0.f;
+        for (int i = 0; i < 8; ++i) vv[i] = 0.f;
+        for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) {
+            const int r = tb.route[cc];
+            if (tb.tok[r] != tk) continue;
+            const float w = tb.w[r];
+            const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(a.h + (size_t)r * I + k8));
+            const float4 h1 = __ldcg(reinterpret_cast<const float4 *>(a.h + (size_t)r * I + k8 + 4));
+            vv[0] = fmaf(w, h0.x, vv[0]); vv[1] = fmaf(w, h0.y, vv[1]); vv[2] = fmaf(w, h0.z, vv[2]);
+            vv[3] = fmaf(w, h0.w, vv[3]); vv[4] = fmaf(w, h1.x, vv[4]); vv[5] = fmaf(w, h1.y, vv[5]);
+            vv[6] = fmaf(w, h1.z, vv[6]); vv[7] = fmaf(w, h1.w, vv[7]);
         }
-        float m = fmaxf(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])), fmaxf(fmaxf(v[4], v[5]), fmaxf(v[6], v[7])));
-        for (int i = lane + 256; i < a.n_gmax; i += 32) m = fmaxf(m, __ldcg(a.gmax + (size_t)i * kMaxT + warp));
+        float m = 0.f;
 #pragma unroll
-        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) {
-            const int s = prescale_exp(m);
-            tok_scale[warp] = exp2i(s);
-            tok_inv[warp] = exp2i(-s);
-        }
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(vv[i]));
+        if (m > 0.f) atomicMax(&slot_max[sl], __float_as_uint(isfinite(m) ? m : 3.0e38f));
+    };
+    float v[2][8];
+#pragma unroll
+    for (int it = 0; it < 2; ++it)
+        if (tid + it * 32 * kCW < n_idx) col8(tid + it * 32 * kCW, v[it]);
+    for (int idx = tid + 2 * 32 * kCW; idx < n_idx; idx += 32 * kCW) {
+        float vv[8];
+        col8(idx, vv);
     }
     named_sync_consumers();
-    const bool staged = n_slots <= cap;
-    if (staged) {
-        // B column (d, token) = sum over the token's routes to expert d of
-        // w * prescale * h, as f16 (summed in f32 first)
-        for (int idx = tid; idx < n_slots * (I / 8); idx += 32 * kCW) {
-            const int sl = idx / (I / 8), k8 = (idx % (I / 8)) * 8;
-            const int d = slot_d[sl], tk = slot_t[sl];
-            float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) {
-                const int r = tb.route[cc];
-                if (r / k != tk) continue;
-                const float rs = a.topk_w[r] * tok_scale[tk];
-                const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(a.h + (size_t)r * I + k8));
-                const float4 h1 = __ldcg(reinterpret_cast<const float4 *>(a.h + (size_t)r * I + k8 + 4));
-                v[0] = fmaf(rs, h0.x, v[0]); v[1] = fmaf(rs, h0.y, v[1]); v[2] = fmaf(rs, h0.z, v[2]);
-                v[3] = fmaf(rs, h0.w, v[3]); v[4] = fmaf(rs, h1.x, v[4]); v[5] = fmaf(rs, h1.y, v[5]);
-                v[6] = fmaf(rs, h1.z, v[6]); v[7] = fmaf(rs, h1.w, v[7]);
-            }
-            __half2 p0 = __floats2half2_rn(v[0], v[1]), p1 = __floats2half2_rn(v[2], v[3]);
-            __half2 p2 = __floats2half2_rn(v[4], v[5]), p3 = __floats2half2_rn(v[6], v[7]);
-            *reinterpret_cast<uint4 *>(bs + (size_t)sl * bs_stride + k8) =
-                make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
-                           *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
-        }
-        named_sync_consumers();
+    if (tid < n_slots) {
+        const int sc = prescale_exp(__uint_as_float(slot_max[tid]));
+        slot_scale[tid] = exp2i(sc);
+        slot_inv[tid] = exp2i(-sc);
     }
+    named_sync_consumers();
+    auto put_b = [&](int idx, const float *vv) {
+        const int sl = idx / (I / 8), k8 = (idx % (I / 8)) * 8;
+        const float rs = slot_scale[sl];
+        __half2 p0 = __floats2half2_rn(rs * vv[0], rs * vv[1]), p1 = __floats2half2_rn(rs * vv[2], rs * vv[3]);
+        __half2 p2 = __floats2half2_rn(rs * vv[4], rs * vv[5]), p3 = __floats2half2_rn(rs * vv[6], rs * vv[7]);
+        *reinterpret_cast<uint4 *>(bs + (size_t)sl * bs_stride + k8) =
+            make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
+                       *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
+    };
+#pragma unroll
+    for (int it = 0; it < 2; ++it)
+        if (tid + it * 32 * kCW < n_idx) put_b(tid + it * 32 * kCW, v[it]);
+    for (int idx = tid + 2 * 32 * kCW; idx < n_idx; idx += 32 * kCW) {
+        float vv[8];
+        col8(idx, vv);
+        put_b(idx, vv);
+    }
+    named_sync_consumers();
 
+    // the units, one group ahead as in the gate/up kernel
     const int q = warp / WPC, wi = warp % WPC;   // this warp's chunk of every unit and its place in it
+    constexpr int NG = NCH / 2;
     bool timed_out = false;
-    for (int j = 0; j < n_mine; ++j) {
-        const int u = u0 + j;
-        const int d = u / tiles, tile = u % tiles, m0 = tile * 32;
+    const uint8_t *st0 = stages, *st1 = stages;
+    int s_cur = 0;
+    auto open_unit = [&](int j, const uint8_t *&b0, const uint8_t *&b1, int &s) {
+        const int c = j * NCH + q, pc = c >> lcps;
+        if (!wait_piece(full, a.S, pc, &issued)) timed_out = true;
+        s = pc - (int)(a.S.div((uint32_t)pc) * a.S.d);
+        // [rows m0..+15: blocks of the piece][rows m0+16..+31: blocks of the piece]
+        b0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c & (cps - 1)) * kBlk;
+        b1 = b0 + (size_t)cps * kBlk;
+    };
+    GroupFrags cur;
+    if (n_mine > 0) {
+        open_unit(0, st0, st1, s_cur);
+        load_group(st0, st1, g, t, wi * NG, cur);
+    }
+    for (int j = 0; j < n_mine && !timed_out; ++j) {
+        const int d = (u0 + j) >> ltiles;
         const int my_slot = (g < T) ? slot_of[d - d_lo][g] : -1;   // B column g = token g
+        const uint16_t *brow = bs + (size_t)(my_slot < 0 ? 0 : my_slot) * bs_stride + 8 * t;
         float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-        {
-            uint4 xb[NCH / 2][4];
 #pragma unroll
-            for (int p = 0; p < NCH / 2; ++p) {
-                const int gp = wi * (NCH / 2) + p;
-                const int kbase = q * kKC + gp * 128 + 8 * t;   // this thread's first K of the group's block 0
-                if (staged) {
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        xb[p][jj] = my_slot >= 0 ? lds128(bs + (size_t)my_slot * bs_stride + kbase + jj * 32)
-                                                 : make_uint4(0u, 0u, 0u, 0u);
-                } else {
-                    // more columns than staged slots: build B from h in L2
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        if (g < T)
-                            for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) {
-                                const int r = tb.route[cc];
-                                if (r / k != g) continue;
-                                const float rs = a.topk_w[r] * tok_scale[g];
-                                const float *hp = a.h + (size_t)r * I + kbase + jj * 32;
-                                const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(hp));
-                                const float4 h1 = __ldcg(reinterpret_cast<const float4 *>(hp + 4));
-                                v[0] = fmaf(rs, h0.x, v[0]); v[1] = fmaf(rs, h0.y, v[1]);
-                                v[2] = fmaf(rs, h0.z, v[2]); v[3] = fmaf(rs, h0.w, v[3]);
-                                v[4] = fmaf(rs, h1.x, v[4]); v[5] = fmaf(rs, h1.y, v[5]);
-                                v[6] = fmaf(rs, h1.z, v[6]); v[7] = fmaf(rs, h1.w, v[7]);
-                            }
-                        __half2 p0 = __floats2half2_rn(v[0], v[1]), p1 = __floats2half2_rn(v[2], v[3]);
-                        __half2 p2 = __floats2half2_rn(v[4], v[5]), p3 = __floats2half2_rn(v[6], v[7]);
-                        xb[p][jj] = make_uint4(*reinterpret_cast<uint32_t *>(&p0), *reinterpret_cast<uint32_t *>(&p1),
-                                               *reinterpret_cast<uint32_t *>(&p2), *reinterpret_cast<uint32_t *>(&p3));
-                    }
+        for (int p = 0; p < NG; ++p) {
+            const int gp = wi * NG + p;
+            const uint8_t *n0 = st0, *n1 = st1;
+            int ns = s_cur;
+            GroupFrags nxt;
+            if (p + 1 < NG) {
+                load_group(st0, st1, g, t, gp + 1, nxt);
+            } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s_cur]);
+                if (j + 1 < n_mine) {
+                    open_unit(j + 1, n0, n1, ns);
+                    load_group(n0, n1, g, t, wi * NG, nxt);
                 }
             }
-            const int c = j * NCH + q, pc = c / cps, s = pc % S;
-            if (!wait_piece(full, S, pc, &issued)) timed_out = true;
-            // [rows m0..+15: blocks of the piece][rows m0+16..+31: blocks of the piece]
-            const uint8_t *st0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c % cps) * kBlk;
-            const uint8_t *st1 = st0 + (size_t)cps * kBlk;
-            GroupFrags fr[NCH / 2];
+            const uint16_t *xq = brow + q * kKC + gp * 128;
+            uint4 xb[4];
 #pragma unroll
-            for (int p = 0; p < NCH / 2; ++p) load_group(st0, st1, g, t, wi * (NCH / 2) + p, fr[p]);
-            // the stage is free again once every warp holds its share
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-#pragma unroll
-            for (int p = 0; p < NCH / 2; ++p) compute_group(fr[p], xb[p], acc0, acc1);
+            for (int jj = 0; jj < 4; ++jj) xb[jj] = my_slot >= 0 ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
+            compute_group(cur, xb, acc0, acc1);
+            cur = nxt;
+            st0 = n0;
+            st1 = n1;
+            s_cur = ns;
         }
-        float *rb = red + (size_t)(j & 1) * kCW * 2 * 16 * Tc;
-        put_partials(rb, Tc, warp, g, t, acc0, acc1);
-        named_sync_consumers();
-        if ((lane & 1) == 0) {   // readers spread over the warps: (row, token) = r % 32, r / 32
-            const int r = warp + kCW * (lane >> 1), row = r & 31, col = r >> 5;
-            if (col < T)
-                __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row,
-                       sum_partials(rb, Tc, row >> 4, row & 15, col));
-        }
+        const int slot = j % kRedSlots;
+        if (j >= kRedSlots && !mbar_wait_bounded(&red_empty[slot], (uint32_t)((j / kRedSlots - 1) & 1)))
+            timed_out = true;
+        put_partials(red + (size_t)slot * kCW * 2 * 16 * Tc, Tc, warp, g, t, acc0, acc1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_full[slot]);
     }
+    if (timed_out && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
     // Combine: once every expert's slice of a 32-row tile is in, the CTA
-    // whose unit completed it sums the slices in expert order, undoes the
-    // prescale and writes bf16; the order of the sum does not depend on
-    // timing.
-    __threadfence();
-    named_sync_consumers();
+    // whose unit completed it sums the slices in expert order and writes
+    // bf16; the order of the sum does not depend on timing.  The epilogue
+    // warps fenced their slices before this barrier.
+    asm volatile("bar.sync 3, %0;" ::"r"(32 * (kCW + kEpiWarps)) : "memory");
     for (int j = tid; j < n_mine; j += 32 * kCW) {
-        const int tile = (u0 + j) % tiles;
+        const int tile = (u0 + j) & (tiles - 1);
         if (atomicAdd(a.counters + tile, 1) == tb.D - 1) last_tiles[atomicAdd(&n_last, 1)] = tile;
     }
     named_sync_consumers();
@@ -769,12 +915,11 @@ __global__ void __launch_bounds__(kWSThreads, 1) dec_down_mx_kernel(DownArgs a) 
             const int row = idx & 31, col = (idx >> 5) % T, m0 = last_tiles[(idx >> 5) / T] * 32;
             float sum = 0.f;
             for (int dd = 0; dd < tb.D; ++dd) sum += __ldcg(a.ybuf + ((size_t)dd * kMaxT + col) * H + m0 + row);
-            __nv_bfloat16 o = __float2bfloat16_rn(sum * tok_inv[col]);
+            __nv_bfloat16 o = __float2bfloat16_rn(sum);
             a.out[(size_t)col * H + m0 + row] = *reinterpret_cast<uint16_t *>(&o);
         }
         for (int li = tid; li < n_last; li += 32 * kCW) a.counters[last_tiles[li]] = 0;
     }
-    if (timed_out && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
 }
 
 template <typename K, typename A>
@@ -832,7 +977,6 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     ga.ids = ids;
     ga.topk_w = topk_w;
     ga.h = L.h;
-    ga.gmax = L.dec_gmax;
     ga.status = L.status;
     ga.T = T;
     ga.k = L.d.top_k;
@@ -840,19 +984,17 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     ga.H = H;
     ga.I = I;
     const StagePlan gp = gu_plan(T, H);
-    ga.n_stages = gp.S;
+    ga.S = make_fastdiv((uint32_t)gp.S);
     ga.cps = gp.cps;
     L.count_launches(2);
     if (ev) record_phase(ev[1], s);   // routing is fused into both kernels' prologues
-    cudaError_t e = launch_ex(dec_gateup_mx_kernel<NCU>, dim3(grid), dim3(kWSThreads),
-                              gu_bytes(ga.n_stages, ga.cps, T, H), s, false, ga);
+    cudaError_t e = launch_ex(dec_gateup_mx_kernel<NCU>, dim3(grid), dim3(kGUThreads),
+                              gu_bytes(gp.S, ga.cps, T, H), s, false, ga);
     if (e != cudaSuccess) return e;
     if (ev) record_phase(ev[2], s);
     DownArgs da;
     da.codes = L.w.codes[MOEQ_DOWN];
     da.h = L.h;
-    da.gmax = L.dec_gmax;
-    da.n_gmax = grid;
     da.ids = ids;
     da.topk_w = topk_w;
     da.ybuf = L.dec_ybuf;
@@ -865,12 +1007,12 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     da.H = H;
     da.I = I;
     const StagePlan dp = dn_plan(T, I);
-    da.n_stages = dp.S;
+    da.S = make_fastdiv((uint32_t)dp.S);
     da.cps = dp.cps;
     // programmatic dependent launch: the down kernel's producer streams
     // weights while the gate/up kernel drains; its consumers wait for that
     // grid before reading h.  Not with phase events between the launches.
-    e = launch_ex(dec_down_mx_kernel<NCD>, dim3(grid), dim3(kWSThreads), dn_bytes(da.n_stages, da.cps, T, I), s, ev == nullptr,
+    e = launch_ex(dec_down_mx_kernel<NCD>, dim3(grid), dim3(kDNThreads), dn_bytes(dp.S, da.cps, T, I), s, ev == nullptr,
                   da);
     if (e != cudaSuccess) return e;
     if (ev) {
@@ -889,6 +1031,12 @@ bool decode_mx_supported(const Layer &L, int T) {
     if (!((d.hidden == 2048 || d.hidden == 4096) && (d.inter == 2048 || d.inter == 4096))) return false;
     for (int tt = 1; tt <= kMaxT; ++tt)
         if (gu_plan(tt, d.hidden).S < 2 || dn_plan(tt, d.inter).S < 2) return false;
+    // a CTA's gate/up units fit its unit table
+    const long long max_units = (long long)std::min(kMaxR, d.n_experts) * (d.inter / 16);
+    if (L.sm_count <= 0 || (max_units + L.sm_count - 1) / L.sm_count > kMaxUnits) return false;
+    // a down CTA's units span at most two experts: one CTA per routed expert at least
+    if (L.sm_count < std::min(kMaxR, d.n_experts)) return false;
+    if (d.hidden / 32 > kMaxTiles) return false;
     return L.sm_count > 0 && L.sm_count <= kDecMaxGrid;
 }
 

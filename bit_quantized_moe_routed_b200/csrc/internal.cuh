@@ -94,7 +94,6 @@ struct Layer {
     float *h = nullptr;        // [max_tokens*k][I] SwiGLU intermediates, route-sorted order
     float *acc = nullptr;      // [max_tokens][H] f32 combine accumulator
     // decode fast path scratch
-    float *dec_gmax = nullptr;     // [kDecMaxGrid][kDecMaxTokens] per-CTA max |w h| per token
     float *dec_ybuf = nullptr;     // [kDecMaxRoutes][kDecMaxTokens][H] per-expert partial outputs
     int *dec_counters = nullptr;   // [H/32] per-tile arrival counters, zero between calls
     uint32_t *status = nullptr;
