@@ -71,15 +71,17 @@ __device__ void build_route_table(RouteTable &tb, const int32_t *__restrict__ id
     const unsigned full = 0xffffffffu;
     const int lane = threadIdx.x & 31;
     const int r0 = lane, r1 = lane + 32;
-    const int id0 = r0 < R ? ids[r0] : -1, id1 = r1 < R ? ids[r1] : -1;
+    // all four loads in flight before the first use: one memory round trip
+    const int id0 = r0 < R ? __ldg(ids + r0) : -1, id1 = r1 < R ? __ldg(ids + r1) : -1;
+    const float w0 = r0 < R ? __ldg(topk_w + r0) : 0.f, w1 = r1 < R ? __ldg(topk_w + r1) : 0.f;
     if (r0 < R) {
         tb.sid[r0] = id0;
-        tb.w[r0] = topk_w[r0];
+        tb.w[r0] = w0;
         tb.tok[r0] = (uint8_t)(r0 / k);
     }
     if (r1 < R) {
         tb.sid[r1] = id1;
-        tb.w[r1] = topk_w[r1];
+        tb.w[r1] = w1;
         tb.tok[r1] = (uint8_t)(r1 / k);
     }
     const bool v0 = id0 >= 0 && id0 < E, v1 = id1 >= 0 && id1 < E;
@@ -235,10 +237,10 @@ __device__ __forceinline__ const uint8_t *scale_ptr(const uint8_t *blk, int r, i
     return blk + 16 * (kKC / 2) + grp * 64 + r * 4;
 }
 
-// This CTA's contiguous share [beg, end) of n units.
+// This CTA's contiguous share [beg, end) of n units (n * gridDim.x < 2^32).
 __device__ __forceinline__ void my_range(int n, int &beg, int &end) {
-    beg = (int)(((long long)n * blockIdx.x) / gridDim.x);
-    end = (int)(((long long)n * (blockIdx.x + 1)) / gridDim.x);
+    beg = (int)(((unsigned)n * blockIdx.x) / gridDim.x);
+    end = (int)(((unsigned)n * (blockIdx.x + 1)) / gridDim.x);
 }
 
 // Chunk c of this CTA is chunk c % nch of unit c / nch (units in order),
@@ -446,9 +448,6 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     constexpr int WPC = kCW / NCH;   // warps per chunk
     const int lcps = cps == 4 ? 2 : (cps == 2 ? 1 : 0);
 
-    // the down kernel may take SMs as this grid's CTAs finish: it streams
-    // its weights at once and reads h only after this grid completes
-    pdl_launch_dependents();
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
@@ -479,17 +478,26 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
             n_units = min(i1 - i0, kMaxUnits);
         }
         __syncwarp();
-        // this CTA's units, one per lane
+        // this CTA's units, one per lane (tiles is a power of two; binary
+        // search for the expert slot: beg[d] <= i < beg[d + 1])
+        const int ltiles = 31 - __clz(tiles), D = tb.D;
         for (int j = lane; j < n_units; j += 32) {
             const int i = unit0 + j;
-            int d = 0;
-            while (items.beg[d + 1] <= i) ++d;
-            const int rel = i - items.beg[d], pass = rel / tiles, tile = rel - pass * tiles;
+            int lo = 0, hi = D - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (items.beg[mid] <= i) lo = mid;
+                else hi = mid - 1;
+            }
+            const int d = lo, rel = i - items.beg[d], pass = rel >> ltiles, tile = rel & (tiles - 1);
             const int cb = tb.col_beg[d] + pass * 8, ncol = min(8, tb.col_beg[d + 1] - cb);
             units[j] = (uint32_t)d | ((uint32_t)tile << 6) | ((uint32_t)cb << 15) | ((uint32_t)ncol << 22);
         }
     }
     __syncthreads();
+    // the down kernel may take SMs as this grid's CTAs finish: it streams
+    // its weights at once and reads h only after this grid completes
+    pdl_launch_dependents();
     const int n_mine = n_units;
 
     if (warp == kProducerWarp) {
