@@ -34,6 +34,30 @@ import synth  # noqa: E402
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernel per launch, from one ncu capture of the named source (summary under
+# profiles/); reported only while that source is byte-identical, else null.
+NCU_TRAFFIC = {
+    "decode_mxfp4": ("bit_quantized_moe_routed_b200/csrc/decode_mx.cu",
+                     "9dc1c3cf39cf9142a48095b63126a6b4610db41122e78a902ff63157e2a54b5e",
+                     71354368.0 + 1934848.0, "profiles/dec_gateup_mx_decode_mxfp4.md"),
+}
+
+
+def ncu_traffic(workload):
+    import hashlib
+    ent = NCU_TRAFFIC.get(workload)
+    if ent is None:
+        return None, None
+    src, sha, traffic, summary = ent
+    try:
+        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), src), "rb") as f:
+            ok = hashlib.sha256(f.read()).hexdigest() == sha
+    except OSError:
+        ok = False
+    return (traffic, summary) if ok else (None, None)
+
+
 # workload -> (config name, overrides)
 WORKLOADS = {
     "decode_mxfp4": ("decode_mxfp4", {}),
@@ -377,10 +401,13 @@ def main():
             bytes_gu = d_mean * (proj_bytes(cfg, 0) + proj_bytes(cfg, 1)) + book_bytes(cfg)
             achieved = bytes_gu / (phase_ms[1] / 1e3) / 1e9
             peak = float(peaks["hbm_gbs"])
+            traffic, traffic_src = ncu_traffic(args.workload)
             roof = {"kernel": "gate/up + SwiGLU", "bound": "hbm", "achieved": achieved, "peak": peak,
-                    "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                    "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                     "peak_source": f"{peak_src} hbm_gbs",
                     "per_launch_bytes": bytes_gu, "launch_ms": phase_ms[1], "timing": phase_how}
+            if traffic_src:
+                roof["traffic_source"] = traffic_src
             d_all = float(np.mean([len(np.unique(ids_h[i])) for i in range(args.warmup, n_total)]))
             step_bytes = d_all * sum(proj_bytes(cfg, p) for p in range(3)) + book_bytes(cfg)
             extra = {"step_weight_gbs": step_bytes / (ms_step / 1e3) / 1e9,
