@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/); reported only while that source is byte-identical, else null.
 NCU_TRAFFIC = {
     "decode_mxfp4": ("bit_quantized_moe_routed_b200/csrc/decode_mx.cu",
-                     "9dc1c3cf39cf9142a48095b63126a6b4610db41122e78a902ff63157e2a54b5e",
-                     71354368.0 + 1934848.0, "profiles/dec_gateup_mx_decode_mxfp4.md"),
+                     "80d729b2dfb3c66eba4ba9591ceb0320940fee7bdb965691a42bfea2bf85ec80",
+                     71356416.0 + 1291520.0, "profiles/dec_gateup_mx_decode_mxfp4.md"),
 }
 
 

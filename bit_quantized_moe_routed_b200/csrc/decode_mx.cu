@@ -270,6 +270,8 @@ __device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_
     const int lane = threadIdx.x & 31, i = lane >> 1, half = lane & 1;
     const int G = min((int)S.d, max(1, 4 / cps));
     const uint32_t half_bytes = (uint32_t)cps * kBlk;
+    // every weight byte is read once per call
+    const uint64_t policy = l2_evict_first_policy();
     for (int p0 = 0; p0 < n_pieces; p0 += G) {
         const int p = p0 + i;
         const bool mine = i < G && p < n_pieces;
@@ -283,7 +285,8 @@ __device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_
         if (mine) {
             const uint8_t *b0, *b1;
             block_of(p, b0, b1);
-            bulk_g2s(stages + (size_t)s * piece_bytes(cps) + half * half_bytes, half ? b1 : b0, half_bytes, &full[s]);
+            bulk_g2s_hint(stages + (size_t)s * piece_bytes(cps) + half * half_bytes, half ? b1 : b0, half_bytes, &full[s],
+                          policy);
         }
         __syncwarp();
         if (lane == 0) {
@@ -946,18 +949,26 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 }
 
 // Stages and chunks per stage (cps, a divisor of the unit's nch chunks) for
-// a kernel whose other shared memory takes `fixed` bytes: the largest pieces
-// that still leave three stages, else one chunk per stage.
+// a kernel whose other shared memory takes `fixed` bytes: of the choices
+// with at least three stages, the one with the most bytes in flight (larger
+// pieces on a tie), else one chunk per stage.
 struct StagePlan {
     int S, cps;
 };
 StagePlan plan_stages(int nch, size_t fixed) {
+    StagePlan best{0, 1};
+    long long best_bytes = -1;
     for (int cps = nch; cps >= 1; cps /= 2) {
         long long s = ((long long)kMaxDynSmem - (long long)fixed) / (long long)piece_bytes(cps);
         if (s > kMaxStages) s = kMaxStages;
-        if (s >= 3 || cps == 1) return {(int)(s < 0 ? 0 : s), cps};
+        if (s < 3 && cps != 1) continue;
+        const long long bytes = s * (long long)piece_bytes(cps);
+        if (bytes > best_bytes) {
+            best = {(int)(s < 0 ? 0 : s), cps};
+            best_bytes = bytes;
+        }
     }
-    return {0, 1};
+    return best;
 }
 StagePlan gu_plan(int T, int H) { return plan_stages(H / kKC, gu_bytes(0, 1, T, H)); }
 StagePlan dn_plan(int T, int I) { return plan_stages(I / kKC, dn_bytes(0, 1, T, I)); }
