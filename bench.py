@@ -229,6 +229,23 @@ def run_reference(args, cfg):
     return 0
 
 
+def reduce_times(ms, e2e_s, world, dev):
+    """The timed regions' durations, maximised over the ranks (every rank ran
+    the same steps on its own GPU: replicas, no collective in the data path)."""
+    if world <= 1:
+        return ms, e2e_s
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([ms, e2e_s], device=dev, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt[0]), float(tt[1])
+
+
+def job_tokens_per_s(world, tokens_per_step, steps, ms):
+    """Whole-job throughput: the tokens all ranks processed over the slowest rank's time."""
+    return world * tokens_per_step * steps / (ms / 1e3)
+
+
 def config_obj(args, cfg, how):
     return {"workload": args.workload, "hidden": cfg.H, "inter": cfg.I, "experts": cfg.E, "top_k": cfg.k,
             "tokens_per_step": cfg.T, "format": cfg.fmt, "act": cfg.act, "routing": cfg.routing,
@@ -379,11 +396,7 @@ def main():
         lay.forward_host_ptr(xh.data_ptr(), ih.data_ptr(), wh.data_ptr(), cfg.T, oh.data_ptr())
     e2e_s = time.perf_counter() - t0
 
-    # max over ranks
-    if world > 1:
-        tt = torch.tensor([ms, e2e_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, e2e_s = float(tt[0]), float(tt[1])
+    ms, e2e_s = reduce_times(ms, e2e_s, world, dev)
 
     if rank == 0:
         peaks = FALLBACK_PEAKS
@@ -392,7 +405,7 @@ def main():
             peaks = json.load(open(PEAKS_FILE))
             peak_src = "measured"
         ms_step = ms / args.steps
-        value = world * cfg.T * args.steps / (ms / 1e3)
+        value = job_tokens_per_s(world, cfg.T, args.steps, ms)
         n_routes = int(((ids_h[args.warmup:] >= 0) & (ids_h[args.warmup:] < cfg.E)).sum()) / args.steps
         if is_decode(cfg):
             # dominant kernel: gate/up + SwiGLU; algorithmic bytes = distinct
@@ -429,7 +442,7 @@ def main():
             "data": "synthetic", "config": config_obj(args, cfg, how),
             "roofline": roof, "phase_ms": dict(zip(["route", "gateup", "down_combine", "cast"], phase_ms)),
             "step": extra,
-            "e2e": {"value": world * cfg.T * e2e_steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h_bytes,
+            "e2e": {"value": job_tokens_per_s(world, cfg.T, e2e_steps, e2e_s * 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h_bytes,
                     "d2h_bytes_per_step": d_bytes, "steps": e2e_steps,
                     "how": "moeq_forward_host per step: pinned H2D of x/ids/w, forward, D2H of out, sync"},
             "gpu_launches": int(launches_per_step * args.steps),
