@@ -322,9 +322,9 @@ __device__ __forceinline__ bool wait_piece(uint64_t *full, FastDiv S, int p, vol
 // down tiles) and each of those warps takes NCH of them, K-groups
 // (i*NCH/2 ...) of both halves, so NCH chunks are in compute at once and
 // each warp runs two independent accumulator chains.  The partial
-// fragments go to red[unit parity][warp][half][row][column] and are summed
-// in warp order after one barrier per unit.  A unit has at most Tc = min(T,
-// 8) columns, so only those are kept.
+// fragments go to red[slot][warp][half][row][column] (two slots, handed to
+// the epilogue warps) and are summed in warp order.  A unit has at most
+// Tc = min(T, 8) columns, so only those are kept.
 __host__ __device__ inline int red_cols(int T) { return T < kMaxT ? T : kMaxT; }
 __host__ __device__ inline size_t red_bytes(int T) {
     return 2 * (size_t)kCW * 2 * 16 * red_cols(T) * sizeof(float);
@@ -415,8 +415,9 @@ __host__ __device__ inline size_t gu_bytes(int n_stages, int cps, int T, int H) 
     return gu_red_off(n_stages, cps, T, H) + red_bytes(T);
 }
 
-// Unit i -> (expert slot d, column chunk, 16-row tile): experts with more
-// than 8 routes take one pass per 8 columns.  A CTA keeps its own range of
+// Unit i -> (expert slot d, column chunk, 16-row tile): an expert's routes
+// are taken Tc = min(T, 8) columns per pass (the width of the partial-sum
+// slots; more routes than tokens only when a token lists an expert twice).  A CTA keeps its own range of
 // units as packed words: d | tile << 6 | first column << 15 | columns << 22.
 struct GUItems {
     int n;
@@ -471,7 +472,7 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
             int n = 0;
             for (int d = 0; d < tb.D; ++d) {
                 items.beg[d] = n;
-                n += ((tb.col_beg[d + 1] - tb.col_beg[d] + 7) / 8) * tiles;
+                n += ((tb.col_beg[d + 1] - tb.col_beg[d] + Tc - 1) / Tc) * tiles;
             }
             items.beg[tb.D] = n;
             items.n = n;
@@ -493,7 +494,7 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
                 else hi = mid - 1;
             }
             const int d = lo, rel = i - items.beg[d], pass = rel >> ltiles, tile = rel & (tiles - 1);
-            const int cb = tb.col_beg[d] + pass * 8, ncol = min(8, tb.col_beg[d + 1] - cb);
+            const int cb = tb.col_beg[d] + pass * Tc, ncol = min(Tc, tb.col_beg[d + 1] - cb);
             units[j] = (uint32_t)d | ((uint32_t)tile << 6) | ((uint32_t)cb << 15) | ((uint32_t)ncol << 22);
         }
     }
@@ -1051,7 +1052,7 @@ bool decode_mx_supported(const Layer &L, int T) {
     for (int tt = 1; tt <= kMaxT; ++tt)
         if (gu_plan(tt, d.hidden).S < 2 || dn_plan(tt, d.inter).S < 2) return false;
     // a CTA's gate/up units fit its unit table
-    const long long max_units = (long long)std::min(kMaxR, d.n_experts) * (d.inter / 16);
+    const long long max_units = (long long)kMaxR * (d.inter / 16);   // passes <= routes
     if (L.sm_count <= 0 || (max_units + L.sm_count - 1) / L.sm_count > kMaxUnits) return false;
     // a down CTA's units span at most two experts: one CTA per routed expert at least
     if (L.sm_count < std::min(kMaxR, d.n_experts)) return false;

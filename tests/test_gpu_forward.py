@@ -203,3 +203,21 @@ def test_zero_tokens_is_a_noop_and_bad_sizes_fail():
     with pytest.raises(moeq.MoeqError) as ei:
         lay.forward(x, ids, w)
     assert ei.value.code == moeq.INVALID_ARGUMENT
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T", [1, 3])
+def test_decode_mxfp4_token_lists_an_expert_twice(T):
+    # fewer tokens than routes to one expert: the gate/up passes are as wide
+    # as the partial-sum slots (T columns), so every route is kept
+    cfg = synth.get_cfg("decode_mxfp4", H=2048, I=2048, E=16, k=8, T=T)
+    L = synth.gen_layer(cfg, seed=41)
+    x = synth.gen_activations(cfg, seed=41)
+    ids, w = synth.gen_routing(cfg, seed=41)
+    ids[:, 1] = ids[:, 0]          # slot 1 repeats slot 0's expert
+    ids[0, 5] = ids[0, 0]          # and a third route to it for token 0
+    lay = dev_layer(L)
+    n0 = lay.kernel_launches()
+    out = run(lay, cfg, x, ids, w)
+    assert lay.kernel_launches() - n0 == 2        # the decode kernels
+    assert_close(out, oracle_ref(L, x, ids, w), "bf16", f"repeated experts, T={T}")
