@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/); reported only while that source is byte-identical, else null.
 NCU_TRAFFIC = {
     "decode_mxfp4": ("bit_quantized_moe_routed_b200/csrc/decode_mx.cu",
-                     "80d729b2dfb3c66eba4ba9591ceb0320940fee7bdb965691a42bfea2bf85ec80",
-                     71356416.0 + 1291520.0, "profiles/dec_gateup_mx_decode_mxfp4.md"),
+                     "249e3588b7a0e1f97cddb2e8c8848f1a84d35aab4e66a57ce0b95be515b62a89",
+                     71356160.0 + 1307392.0, "profiles/dec_gateup_mx_decode_mxfp4.md"),
 }
 
 
