@@ -21,6 +21,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -146,8 +147,9 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") \
-            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/moeq_clocks_{os.getpid()}.csv"
+        # the raw samples go to MOEQ_CLOCKS_DIR when set, else the temp directory
+        out_dir = os.environ.get("MOEQ_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"moeq_clocks_rank{gpu_index}_{os.getpid()}.csv")
 
     def start(self):
         try:
