@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/); reported only while that source is byte-identical, else null.
 NCU_TRAFFIC = {
     "decode_mxfp4": ("bit_quantized_moe_routed_b200/csrc/decode_mx.cu",
-                     "249e3588b7a0e1f97cddb2e8c8848f1a84d35aab4e66a57ce0b95be515b62a89",
-                     71356160.0 + 1307392.0, "profiles/dec_gateup_mx_decode_mxfp4.md"),
+                     "cb4d53ad3f7f4874d349a354b20ab88a4c324dfbc93c35ff65c831140f9a4c20",
+                     71364352.0 + 997376.0, "profiles/dec_gateup_mx_decode_mxfp4.md"),
 }
 
 

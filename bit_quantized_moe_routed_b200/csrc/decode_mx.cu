@@ -27,7 +27,9 @@
 // keep HBM busy; the layout also makes the fragment and scale reads
 // bank-conflict free.  The gate/up kernel lets the down kernel launch as its
 // CTAs finish (programmatic dependent launch): the down weights stream in
-// while gate/up drains, and only the down consumers wait for h.
+// while gate/up drains, and only the down consumers wait for h.  The down
+// kernel does the same for the next gate/up launch, which waits for it
+// before reading anything.
 //
 // Math: warp-level mma.sync.m16n8k16 (f16 in, f32 accumulate).  Each thread
 // reads its A-fragment slice of four 32-weight blocks (bytes 4t..4t+3 of
@@ -465,6 +467,11 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
         mbar_fence_init();
         issued = 0;
     }
+    // launched as a programmatic dependent of the previous kernel in the
+    // stream: its outputs (these inputs, or h that kernel still reads) are
+    // ready and free only after this wait; the dependents this kernel lets
+    // launch below therefore see finished inputs as well
+    pdl_wait_primary();
     if (warp == 0) {
         build_route_table(tb, a.ids, a.topk_w, T * k, k, a.E, a.status, blockIdx.x == 0);
         __syncwarp();
@@ -720,6 +727,9 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
     if (tid < kMaxBSlots) slot_max[tid] = 0u;
     if (warp == 0) build_route_table(tb, a.ids, a.topk_w, T * k, k, a.E, nullptr, false);
     __syncthreads();
+    // the next kernel may take SMs as this grid's CTAs finish (it waits for
+    // this grid's completion before touching memory this kernel uses)
+    pdl_launch_dependents();
     const int n_units = tb.D * tiles;
     if (tb.D == 0) {   // no valid route at all: every output is zero
         for (int i = blockIdx.x * kDNThreads + tid; i < T * H; i += gridDim.x * kDNThreads) a.out[i] = 0;
@@ -1009,7 +1019,7 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     L.count_launches(2);
     if (ev) record_phase(ev[1], s);   // routing is fused into both kernels' prologues
     cudaError_t e = launch_ex(dec_gateup_mx_kernel<NCU>, dim3(grid), dim3(kGUThreads),
-                              gu_bytes(gp.S, ga.cps, T, H), s, false, ga);
+                              gu_bytes(gp.S, ga.cps, T, H), s, ev == nullptr, ga);
     if (e != cudaSuccess) return e;
     if (ev) record_phase(ev[2], s);
     DownArgs da;
