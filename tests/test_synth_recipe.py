@@ -9,12 +9,6 @@ import synth
 from synth.gen import BOOK13_ROWS, BOOK8_ROWS, idx13_row_bytes
 
 
-def _softmax64(z):
-    z = np.asarray(z, np.float64)
-    e = np.exp(z - z.max())
-    return e / e.sum()
-
-
 def test_uniform_routing_top_k_of_normal_logits():
     cfg = synth.get_cfg("decode_mxfp4", T=256)
     ids, w = synth.gen_routing(cfg, seed=3)
