@@ -144,9 +144,12 @@ MOEQ_API moeq_status moeq_upload_weights(moeq_layer_t layer, const moeq_weights 
  *   topk_w    device f32 [n_tokens][top_k]; any values (need not sum to 1)
  *   out       device, act dtype, [n_tokens][hidden]; overwritten
  * Asynchronous on `stream`: all pointers must stay valid until the stream
- * reaches the end of the call.  The sum over routes is accumulated in f32
- * and rounded once (RNE) to the output dtype; the order in which routes are
- * added is not specified.  n_tokens == 0 is a no-op.
+ * reaches the end of the call.  Stream order holds as usual; at decode sizes
+ * the first kernel may be scheduled while the previous kernel on the stream
+ * drains (programmatic dependent launch) but waits for it to complete before
+ * it reads any argument or workspace.  The sum over routes is accumulated in
+ * f32 and rounded once (RNE) to the output dtype; the order in which routes
+ * are added is not specified.  n_tokens == 0 is a no-op.
  * Errors (synchronous): INVALID_ARGUMENT (NULL pointer, n_tokens < 0 or >
  * max_tokens), NOT_UPLOADED, CUDA (launch). */
 MOEQ_API moeq_status moeq_forward(moeq_layer_t layer, const void *x, const int32_t *topk_ids,
