@@ -39,24 +39,30 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel per launch, from one ncu capture of the named source (summary under
 # profiles/); reported only while that source is byte-identical, else null.
 NCU_TRAFFIC = {
-    "decode_mxfp4": ("bit_quantized_moe_routed_b200/csrc/decode_mx.cu",
-                     "cb4d53ad3f7f4874d349a354b20ab88a4c324dfbc93c35ff65c831140f9a4c20",
+    "decode_mxfp4": (("bit_quantized_moe_routed_b200/csrc/decode_mx.cu",
+                      "bit_quantized_moe_routed_b200/csrc/async.cuh",
+                      "bit_quantized_moe_routed_b200/csrc/internal.cuh"),
+                     "da02a205cbb6dd722b2c28527a5684af27b376e3b21fcaf2b688e9d4968283fd",
                      71364352.0 + 997376.0, "profiles/dec_gateup_mx_decode_mxfp4.md"),
 }
 
 
 def ncu_traffic(workload):
+    """(bytes per launch, summary file) while the kernel's sources (its file and
+    the headers it includes, hashed in order) are those that were profiled."""
     import hashlib
     ent = NCU_TRAFFIC.get(workload)
     if ent is None:
         return None, None
-    src, sha, traffic, summary = ent
+    srcs, sha, traffic, summary = ent
+    h = hashlib.sha256()
     try:
-        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), src), "rb") as f:
-            ok = hashlib.sha256(f.read()).hexdigest() == sha
+        for src in srcs:
+            with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), src), "rb") as f:
+                h.update(f.read())
     except OSError:
-        ok = False
-    return (traffic, summary) if ok else (None, None)
+        return None, None
+    return (traffic, summary) if h.hexdigest() == sha else (None, None)
 
 
 # workload -> (config name, overrides)
