@@ -75,6 +75,10 @@ WORKLOADS = {
     "decode_vq_t8_r0": ("decode_vq", dict(T=8, fmt="vq13")),
     "prefill_mxfp4_zipf": ("prefill_mxfp4_zipf", {}),
     "prefill_vq_overflow": ("prefill_vq_overflow", {}),
+    # reduced layers (64 experts, 512 tokens; under 2 GB on the device) for
+    # counter captures of the tensor-core kernels; not bench lines
+    "prefill_mxfp4_zipf_e64_t512": ("prefill_mxfp4_zipf", dict(E=64, T=512)),
+    "prefill_vq_overflow_e64_t512": ("prefill_vq_overflow", dict(E=64, T=512)),
 }
 
 
@@ -280,41 +284,74 @@ def cpu_baseline(cfg, L, xs, ids, w, seconds=12.0):
 
 # ------------------------------------------------------------------ our arm
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="decode_mxfp4", choices=sorted(WORKLOADS))
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
-    assert args.warmup >= 3, "at least 3 warm-up steps"
-    cfg = workload_cfg(args.workload)
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    if args.impl == "reference":
-        return run_reference(args, cfg)
+# Workloads the default run times after the headline one, one layer at a
+# time (each layer is freed before the next is built): the prefill
+# micro-batches and the VQ decode batch sizes.
+EXTRA_WORKLOADS = ("prefill_mxfp4_zipf", "prefill_vq_overflow", "decode_vq_t1", "decode_vq_t4", "decode_vq_t8")
 
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        return json.load(open(PEAKS_FILE)), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def roofline(cfg, workload, ids_h, warmup, n_total, launch_ms, ms_step, peaks, peak_src, phase_how):
+    """The dominant kernel's roofline (gate/up + SwiGLU) and whole-step figures.
+
+    Decode: algorithmic bytes = distinct experts per step x compressed
+    gate+up bytes per expert (+ codebooks), against the measured HBM copy
+    bandwidth.  Prefill: 2 x routes x 2 x H x I flop, against the measured
+    burst bf16 GEMM rate (the kernel runs for milliseconds inside a
+    sub-second graph, not under a seconds-long power-capped load)."""
+    n_steps = n_total - warmup
+    if is_decode(cfg):
+        d_mean = float(np.mean([len(np.unique(ids_h[i][(ids_h[i] >= 0) & (ids_h[i] < cfg.E)]))
+                                for i in range(warmup, n_total)]))
+        bytes_gu = d_mean * (proj_bytes(cfg, 0) + proj_bytes(cfg, 1)) + book_bytes(cfg)
+        achieved = bytes_gu / (launch_ms / 1e3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        traffic, traffic_src = ncu_traffic(workload)
+        roof = {"kernel": "gate/up + SwiGLU", "bound": "hbm", "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} hbm_gbs", "per_launch_bytes": bytes_gu,
+                "per_unit": "compressed gate+up bytes of one expert (+ codebooks once per launch)",
+                "units_per_launch": d_mean, "launch_ms": launch_ms, "timing": phase_how}
+        if traffic_src:
+            roof["traffic_source"] = traffic_src
+        step_bytes = d_mean * sum(proj_bytes(cfg, p) for p in range(3)) + book_bytes(cfg)
+        extra = {"step_weight_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                 "step_hbm_frac": step_bytes / (ms_step / 1e3) / 1e9 / peak}
+    else:
+        n_routes = int(((ids_h[warmup:] >= 0) & (ids_h[warmup:] < cfg.E)).sum()) / n_steps
+        fl_gu = 2 * n_routes * 2 * cfg.H * cfg.I
+        achieved = fl_gu / (launch_ms / 1e3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        traffic, traffic_src = ncu_traffic(workload)
+        roof = {"kernel": "gate/up + SwiGLU", "bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} bf16_tflops (burst)", "per_launch_flops": fl_gu,
+                "per_unit": "2 x 2 x H x I flop per route", "units_per_launch": n_routes,
+                "launch_ms": launch_ms, "timing": phase_how}
+        if traffic_src:
+            roof["traffic_source"] = traffic_src
+        extra = {"step_tflops": flops(cfg, n_routes) / (ms_step / 1e3) / 1e12,
+                 "step_tensor_frac": flops(cfg, n_routes) / (ms_step / 1e3) / 1e12 / peak}
+    return roof, extra
+
+
+def measure(workload, steps, warmup, world, rank, local, barrier, cpu_seconds, with_cpu):
+    """Time `steps` forwards of one workload (after `warmup` eager ones) as one
+    replayed CUDA graph, then the per-phase durations, then the host-buffer
+    entry point.  Returns this rank's figures; the caller reduces over ranks."""
     import torch
-    import torch.distributed as dist
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
     from bit_quantized_moe_routed_b200 import moeq
 
+    cfg = workload_cfg(workload)
     L = synth.gen_layer(cfg)
     lay = moeq.Layer(cfg.H, cfg.I, cfg.E, cfg.k, cfg.T, cfg.fmt, cfg.act, device=local)
     lay.upload(L)
-    n_total = args.warmup + args.steps
+    n_total = warmup + steps
     xs_h, ids_h, w_h, how = step_inputs(cfg, n_total, seed=rank)
     dev = torch.device("cuda", local)
     to_x = (lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)) \
@@ -325,22 +362,22 @@ def main():
     ws = torch.from_numpy(np.ascontiguousarray(w_h[:uniq])).to(dev)
     outs = torch.empty((uniq, cfg.T, cfg.H), dtype=xs.dtype, device=dev)
 
-    def step(i, out=None):
+    def step(i):
         j = i % uniq
-        lay.forward(xs[j], ids[j], ws[j], out=outs[j] if out is None else out)
+        lay.forward(xs[j], ids[j], ws[j], out=outs[j])
 
     # warm-up: W eager steps
     l0 = lay.kernel_launches()
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
-    launches_per_step = (lay.kernel_launches() - l0) // args.warmup
+    launches_per_step = (lay.kernel_launches() - l0) // warmup
 
     # capture the K timed steps as one CUDA graph
     cap = torch.cuda.Stream(device=dev)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=cap):
-        for i in range(args.warmup, n_total):
+        for i in range(warmup, n_total):
             step(i)
     g.replay()                      # untimed: graph upload
     torch.cuda.synchronize()
@@ -369,23 +406,22 @@ def main():
     clocks = sampler.stop()
 
     # per-phase kernel durations over the same K steps (a second graph with
-    # phase events between the kernels)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # event-record nodes between the kernels, on the launching stream)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     for row in ev:              # torch creates the CUDA event at its first record
         for e in row:
             e.record()
     torch.cuda.synchronize()
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g2, stream=cap):
-        for n, i in enumerate(range(args.warmup, n_total)):
+        for n, i in enumerate(range(warmup, n_total)):
             j = i % uniq
             lay.forward_profiled(xs[j], ids[j], ws[j], outs[j], ev[n])
     g2.replay()
     torch.cuda.synchronize()
     g2.replay()
     torch.cuda.synchronize()
-    phase_ms = [sum(ev[n][p].elapsed_time(ev[n][p + 1]) for n in range(args.steps)) / args.steps
-                for p in range(4)]
+    phase_ms = [sum(ev[n][p].elapsed_time(ev[n][p + 1]) for n in range(steps)) / steps for p in range(4)]
     phase_how = "event-record nodes between the kernels of a replayed graph of the same K steps"
 
     # end to end through the host-buffer entry point (pinned host memory)
@@ -395,7 +431,7 @@ def main():
     oh = torch.empty_like(xh).pin_memory()
     h_bytes = xh.numel() * xh.element_size() + ih.numel() * 4 + wh.numel() * 4
     d_bytes = oh.numel() * oh.element_size()
-    e2e_steps = min(args.steps, 200)
+    e2e_steps = min(steps, 200)
     for _ in range(3):
         lay.forward_host_ptr(xh.data_ptr(), ih.data_ptr(), wh.data_ptr(), cfg.T, oh.data_ptr())
     barrier()
@@ -403,67 +439,103 @@ def main():
     for _ in range(e2e_steps):
         lay.forward_host_ptr(xh.data_ptr(), ih.data_ptr(), wh.data_ptr(), cfg.T, oh.data_ptr())
     e2e_s = time.perf_counter() - t0
+    status = lay.status()
+    del g, g2
+    lay.close()
+    res = {"cfg": cfg, "how": how, "ms": ms, "e2e_s": e2e_s, "e2e_steps": e2e_steps, "phase_ms": phase_ms,
+           "phase_how": phase_how, "launches_per_step": launches_per_step, "clocks": clocks,
+           "h_bytes": h_bytes, "d_bytes": d_bytes, "ids_h": ids_h, "status": status}
+    if with_cpu and rank == 0:
+        res["cpu_baseline"] = cpu_baseline(cfg, L, xs_h, ids_h, w_h, seconds=cpu_seconds)
+    return res
 
-    ms, e2e_s = reduce_times(ms, e2e_s, world, dev)
+
+def summarize(args, workload, r, world, steps, warmup, peaks, peak_src):
+    """The contract's fields for one measured workload (times already reduced over ranks)."""
+    cfg = r["cfg"]
+    ms_step = r["ms"] / steps
+    roof, extra = roofline(cfg, workload, r["ids_h"], warmup, warmup + steps, r["phase_ms"][1], ms_step,
+                           peaks, peak_src, r["phase_how"])
+    a = argparse.Namespace(**vars(args))
+    a.workload = workload
+    line = {
+        "metric": "MoE-layer tokens/s", "value": job_tokens_per_s(world, cfg.T, steps, r["ms"]),
+        "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.act == "bf16" else "f32", "data": "synthetic",
+        "config": config_obj(a, cfg, r["how"]),
+        "roofline": roof, "phase_ms": dict(zip(["route", "gateup", "down_combine", "cast"], r["phase_ms"])),
+        "step": extra,
+        "e2e": {"value": job_tokens_per_s(world, cfg.T, r["e2e_steps"], r["e2e_s"] * 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": r["h_bytes"], "d2h_bytes_per_step": r["d_bytes"], "steps": r["e2e_steps"],
+                "how": "moeq_forward_host per step: pinned H2D of x/ids/w, forward, D2H of out, sync"},
+        "gpu_launches": int(r["launches_per_step"] * steps),
+        "clocks": r["clocks"],
+        "device_status": r["status"],
+    }
+    if "cpu_baseline" in r:
+        line["cpu_baseline"] = r["cpu_baseline"]
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="decode_mxfp4", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only --workload (by default the prefill and VQ workloads follow the headline one)")
+    ap.add_argument("--extra-steps", type=int, default=30, help="timed steps of each extra workload")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    cfg = workload_cfg(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import torch
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    peaks, peak_src = load_peaks()
+    with_cpu = not args.no_cpu_baseline and world == 1
+    r = measure(args.workload, args.steps, args.warmup, world, rank, local, barrier, 12.0, with_cpu)
+    r["ms"], r["e2e_s"] = reduce_times(r["ms"], r["e2e_s"], world, dev)
+    line = summarize(args, args.workload, r, world, args.steps, args.warmup, peaks, peak_src) if rank == 0 else None
+
+    extra = {}
+    extra_names = () if (args.no_extra or args.workload != "decode_mxfp4") else EXTRA_WORKLOADS
+    for name in extra_names:
+        rx = measure(name, args.extra_steps, args.warmup, world, rank, local, barrier, 6.0, with_cpu)
+        rx["ms"], rx["e2e_s"] = reduce_times(rx["ms"], rx["e2e_s"], world, dev)
+        if rank == 0:
+            lx = summarize(args, name, rx, world, args.extra_steps, args.warmup, peaks, peak_src)
+            for key in ("metric", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "data"):
+                lx.pop(key, None)
+            extra[name] = lx
+        torch.cuda.empty_cache()
 
     if rank == 0:
-        peaks = FALLBACK_PEAKS
-        peak_src = "fallback"
-        if os.path.exists(PEAKS_FILE):
-            peaks = json.load(open(PEAKS_FILE))
-            peak_src = "measured"
-        ms_step = ms / args.steps
-        value = job_tokens_per_s(world, cfg.T, args.steps, ms)
-        n_routes = int(((ids_h[args.warmup:] >= 0) & (ids_h[args.warmup:] < cfg.E)).sum()) / args.steps
-        if is_decode(cfg):
-            # dominant kernel: gate/up + SwiGLU; algorithmic bytes = distinct
-            # experts per step x compressed gate+up bytes per expert (+ books)
-            d_mean = float(np.mean([len(np.unique(ids_h[i])) for i in range(args.warmup, n_total)]))
-            bytes_gu = d_mean * (proj_bytes(cfg, 0) + proj_bytes(cfg, 1)) + book_bytes(cfg)
-            achieved = bytes_gu / (phase_ms[1] / 1e3) / 1e9
-            peak = float(peaks["hbm_gbs"])
-            traffic, traffic_src = ncu_traffic(args.workload)
-            roof = {"kernel": "gate/up + SwiGLU", "bound": "hbm", "achieved": achieved, "peak": peak,
-                    "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                    "peak_source": f"{peak_src} hbm_gbs",
-                    "per_launch_bytes": bytes_gu, "launch_ms": phase_ms[1], "timing": phase_how}
-            if traffic_src:
-                roof["traffic_source"] = traffic_src
-            d_all = float(np.mean([len(np.unique(ids_h[i])) for i in range(args.warmup, n_total)]))
-            step_bytes = d_all * sum(proj_bytes(cfg, p) for p in range(3)) + book_bytes(cfg)
-            extra = {"step_weight_gbs": step_bytes / (ms_step / 1e3) / 1e9,
-                     "step_hbm_frac": step_bytes / (ms_step / 1e3) / 1e9 / peak}
-        else:
-            fl_gu = 2 * n_routes * 2 * cfg.H * cfg.I
-            achieved = fl_gu / (phase_ms[1] / 1e3) / 1e12
-            peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-            roof = {"kernel": "gate/up + SwiGLU", "bound": "tensor", "achieved": achieved, "peak": peak,
-                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                    "peak_source": f"{peak_src} bf16_tflops_sustained",
-                    "per_launch_flops": fl_gu, "launch_ms": phase_ms[1], "timing": phase_how}
-            extra = {"step_tflops": flops(cfg, n_routes) / (ms_step / 1e3) / 1e12,
-                     "step_tensor_frac": flops(cfg, n_routes) / (ms_step / 1e3) / 1e12 / peak}
-        line = {
-            "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.act == "bf16" else "f32",
-            "data": "synthetic", "config": config_obj(args, cfg, how),
-            "roofline": roof, "phase_ms": dict(zip(["route", "gateup", "down_combine", "cast"], phase_ms)),
-            "step": extra,
-            "e2e": {"value": job_tokens_per_s(world, cfg.T, e2e_steps, e2e_s * 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h_bytes,
-                    "d2h_bytes_per_step": d_bytes, "steps": e2e_steps,
-                    "how": "moeq_forward_host per step: pinned H2D of x/ids/w, forward, D2H of out, sync"},
-            "gpu_launches": int(launches_per_step * args.steps),
-            "clocks": clocks,
-        }
-        if not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(cfg, L, xs_h, ids_h, w_h)
+        if extra:
+            line["workloads"] = extra
         print(json.dumps(line), flush=True)
-    del g, g2
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-    lay.close()
     return 0
 
 

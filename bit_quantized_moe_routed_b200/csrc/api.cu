@@ -1,6 +1,7 @@
 // api.cu -- the extern "C" entry points of libmoeq (declared in moeq.h):
 // argument validation, device memory ownership and kernel dispatch.
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -9,6 +10,29 @@
 #include "internal.cuh"
 
 using namespace moeq;
+
+namespace moeq {
+
+// Host-side fault injection for tests: MOEQ_TEST_FAIL_ALLOC=n makes the
+// n-th device allocation of this process (1-based, counted over every
+// allocation the library makes) report out-of-memory.
+namespace {
+std::atomic<long> g_alloc_count{0};
+}
+cudaError_t dev_alloc(void **p, size_t bytes) {
+    static const long fail_at = [] {
+        const char *s = std::getenv("MOEQ_TEST_FAIL_ALLOC");
+        return s ? std::atol(s) : 0L;
+    }();
+    const long n = ++g_alloc_count;
+    if (fail_at > 0 && n == fail_at) {
+        *p = nullptr;
+        return cudaErrorMemoryAllocation;
+    }
+    return cudaMalloc(p, bytes ? bytes : 16);
+}
+
+}  // namespace moeq
 
 // The opaque handle of moeq.h is the library's layer object.
 struct moeq_layer : moeq::Layer {};
@@ -34,22 +58,6 @@ moeq_status from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return MOEQ_OK;
     if (e == cudaErrorMemoryAllocation) return MOEQ_ERR_OUT_OF_MEMORY;
     return MOEQ_ERR_CUDA;
-}
-
-// Host-side fault injection for tests: MOEQ_TEST_FAIL_ALLOC=n makes the
-// n-th device allocation of this process (1-based) report out-of-memory.
-long g_alloc_count = 0;
-cudaError_t dev_alloc(void **p, size_t bytes) {
-    static long fail_at = [] {
-        const char *s = std::getenv("MOEQ_TEST_FAIL_ALLOC");
-        return s ? std::atol(s) : 0L;
-    }();
-    ++g_alloc_count;
-    if (fail_at > 0 && g_alloc_count == fail_at) {
-        *p = nullptr;
-        return cudaErrorMemoryAllocation;
-    }
-    return cudaMalloc(p, bytes ? bytes : 16);
 }
 
 size_t row_bytes(int fmt, int plane, int K) {
@@ -154,6 +162,10 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     if (!L) return MOEQ_ERR_OUT_OF_MEMORY;
     L->d = *desc;
     cudaDeviceGetAttribute(&L->sm_count, cudaDevAttrMultiProcessorCount, desc->device);
+    if (const char *wc = std::getenv("MOEQ_TEST_WAIT_CYCLES")) {
+        const long long v = std::atoll(wc);
+        if (v > 0) L->wait_cycles = v;
+    }
     const int E = desc->n_experts, H = desc->hidden, I = desc->inter, k = desc->top_k;
     const size_t M = (size_t)desc->max_tokens;
     const int fmt = desc->fmt;
@@ -371,6 +383,10 @@ moeq_status moeq_layer_status(moeq_layer_t L, int32_t clear) {
     uint32_t v = 0;
     cudaError_t e = cudaMemcpy(&v, L->status, sizeof(v), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && clear) e = cudaMemset(L->status, 0, sizeof(uint32_t));
+    // a kernel that gave up on a wait may have left the decode combine's
+    // per-tile arrival counters part-way: clearing the status resets them
+    if (e == cudaSuccess && clear && (v & FLAG_TIMEOUT))
+        e = cudaMemset(L->dec_counters, 0, sizeof(int) * (L->d.hidden / 32 + 1));
     if (e != cudaSuccess) return from_cuda(e);
     if (v & FLAG_ROUTE_RANGE) return MOEQ_ERR_ROUTE_OUT_OF_RANGE;
     if (v & FLAG_TIMEOUT) return MOEQ_ERR_TIMEOUT;

@@ -67,6 +67,31 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     return true;
 }
 
+// Wait for phase `parity` of `bar` unless another role of the CTA has given
+// up (*abort != 0), for at most `max_cycles` SM clocks; on expiry this
+// thread raises *abort itself.  Returns false when it did not see the phase
+// complete.  The first probe is the fast path; the loop re-reads the flag
+// between suspended probes.
+__device__ __forceinline__ bool mbar_wait_abort(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                long long max_cycles) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort) return false;
+        if (clock64() - t0 > max_cycles) {
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+// The limit of the drains that run before a CTA exits (its own copies in
+// flight, its own tensor-core operations): fixed and long, so that no
+// asynchronous operation outlives the CTA whatever limit the other waits
+// were given (about 0.1 s).
+constexpr long long kDrainCycles = 200000000LL;
+
 // Global -> shared bulk copy (no tensor map).  dst and src 16-byte aligned,
 // bytes a multiple of 16; completion is signalled on `bar` as tx bytes.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

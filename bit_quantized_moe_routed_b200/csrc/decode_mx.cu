@@ -46,6 +46,8 @@
 // undone, to its own slice of a scratch buffer; the last unit to finish a
 // 32-row tile (per-tile arrival counter) sums the experts in a fixed order
 // and writes bf16 out, so the result does not depend on timing.
+#include <mutex>
+
 #include "async.cuh"
 #include "internal.cuh"
 
@@ -268,20 +270,23 @@ inline FastDiv make_fastdiv(uint32_t d) { return {d, (uint32_t)((0x100000000ull 
 
 template <typename BlockOf>
 __device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_t *empty, FastDiv S, int cps,
-                                        int n_pieces, uint32_t *status, volatile int *issued, BlockOf block_of) {
+                                        int n_pieces, volatile int *abort, long long limit, volatile int *issued,
+                                        BlockOf block_of) {
     const int lane = threadIdx.x & 31, i = lane >> 1, half = lane & 1;
     const int G = min((int)S.d, max(1, 4 / cps));
     const uint32_t half_bytes = (uint32_t)cps * kBlk;
     // every weight byte is read once per call
     const uint64_t policy = l2_evict_first_policy();
+    int n_issued = 0;
     for (int p0 = 0; p0 < n_pieces; p0 += G) {
         const int p = p0 + i;
         const bool mine = i < G && p < n_pieces;
         const uint32_t rnd = S.div((uint32_t)p);
         const int s = mine ? p - (int)(rnd * S.d) : 0;
-        if (mine && half == 0 && rnd > 0 && !mbar_wait_bounded(&empty[s], (rnd - 1) & 1u))
-            atomicOr(status, FLAG_TIMEOUT);
-        __syncwarp();
+        bool ok = true;
+        if (mine && half == 0 && rnd > 0) ok = mbar_wait_abort(&empty[s], (rnd - 1) & 1u, abort, limit);
+        // once any role of the CTA has given up, issue nothing more
+        if (__any_sync(0xffffffffu, !ok || *abort)) break;
         if (mine && half == 0) mbar_arrive_expect_tx(&full[s], 2u * half_bytes);
         __syncwarp();
         if (mine) {
@@ -291,32 +296,41 @@ __device__ __forceinline__ void produce(uint8_t *stages, uint64_t *full, uint64_
                           policy);
         }
         __syncwarp();
+        n_issued = min(p0 + G, n_pieces);
         if (lane == 0) {
             __threadfence_block();
-            *issued = min(p0 + G, n_pieces);
+            *issued = n_issued;
         }
     }
-    // wait for the last copy of every stage to land, so that no copy is in
-    // flight when the CTA exits (consumers that gave up on a wait exit early)
+    // Before the CTA exits, wait for the copies this warp issued and that may
+    // still be in flight: the last S pieces (piece p - S was consumed, so
+    // landed, before piece p reused its stage).  The limit is the fixed drain
+    // limit, whatever happened to the other waits.
     if (lane == 0)
-        for (int p = max(0, n_pieces - (int)S.d); p < n_pieces; ++p) {
+        for (int p = max(0, n_issued - (int)S.d); p < n_issued; ++p) {
             const uint32_t rnd = S.div((uint32_t)p);
-            if (!mbar_wait_bounded(&full[p - (int)(rnd * S.d)], rnd & 1u)) atomicOr(status, FLAG_TIMEOUT);
+            if (!mbar_wait_bounded(&full[p - (int)(rnd * S.d)], rnd & 1u, kDrainCycles)) *abort = 1;
         }
     __syncwarp();
 }
 
-// Consumer: wait until piece p is issued, then for its data.  False on timeout.
-__device__ __forceinline__ bool wait_piece(uint64_t *full, FastDiv S, int p, volatile int *issued) {
+// Consumer: wait until piece p is issued, then for its data.  False when it
+// gave up (limit reached, or another role gave up first).
+__device__ __forceinline__ bool wait_piece(uint64_t *full, FastDiv S, int p, volatile int *issued,
+                                           volatile int *abort, long long limit) {
     if (*issued <= p) {
         const long long t0 = clock64();
         while (*issued <= p) {
-            if (clock64() - t0 > 2000000000LL) return false;
+            if (*abort) return false;
+            if (clock64() - t0 > limit) {
+                *abort = 1;
+                return false;
+            }
             __nanosleep(32);
         }
     }
     const uint32_t rnd = S.div((uint32_t)p);
-    return mbar_wait_bounded(&full[p - (int)(rnd * S.d)], rnd & 1u);
+    return mbar_wait_abort(&full[p - (int)(rnd * S.d)], rnd & 1u, abort, limit);
 }
 
 // Chunk q of every unit is computed by the 16/NCH warps [q*16/NCH, ...): a
@@ -399,6 +413,7 @@ struct GateUpArgs {
     const float *topk_w;                // [T][k]
     float *h;                           // [T*k][I] f32, by route id
     uint32_t *status;
+    long long wait_cycles;              // limit of every wait but the final drains
     FastDiv S;                          // stages
     int T, k, E, H, I, cps;
 };
@@ -440,6 +455,7 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], xbar, red_full[kRedSlots],
         red_empty[kRedSlots];
     __shared__ int issued;   // chunks issued by the producer (see produce)
+    __shared__ volatile int abort_flag;   // set by the first role that gives up on a wait
     __shared__ int n_units, unit0;
     __shared__ float xinv[kMaxT];
     const int H = a.H, I = a.I, T = a.T, k = a.k, S = (int)a.S.d, cps = a.cps, Tc = red_cols(a.T);
@@ -466,7 +482,9 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
         }
         mbar_fence_init();
         issued = 0;
+        abort_flag = 0;
     }
+    const long long lim = a.wait_cycles;
     // launched as a programmatic dependent of the previous kernel in the
     // stream: its outputs (these inputs, or h that kernel still reads) are
     // ready and free only after this wait; the dependents this kernel lets
@@ -516,7 +534,7 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
         if (lane == 0) mbar_arrive_expect_tx(&xbar, (uint32_t)(T * H * 2));
         __syncwarp();
         if (lane < T) bulk_g2s(xs + (size_t)lane * xs_stride, a.x + (size_t)lane * H, H * 2, &xbar);
-        produce(stages, full, empty, a.S, cps, n_mine * NCH / cps, a.status, &issued,
+        produce(stages, full, empty, a.S, cps, n_mine * NCH / cps, &abort_flag, lim, &issued,
                 [&](int p, const uint8_t *&b0, const uint8_t *&b1) {
                     const int c = p * cps;
                     const uint32_t u = units[c / NCH];
@@ -531,13 +549,9 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     if (warp >= kEpiWarp0) {
         // epilogue: sum the 16 warps' partial fragments of a unit, SwiGLU, h
         const int e = warp - kEpiWarp0;
-        bool to = false;
-        for (int j = 0; j < n_mine && !to; ++j) {
+        for (int j = 0; j < n_mine; ++j) {
             const int slot = j % kRedSlots;
-            if (!mbar_wait_bounded(&red_full[slot], (uint32_t)((j / kRedSlots) & 1))) {
-                to = true;
-                break;
-            }
+            if (!mbar_wait_abort(&red_full[slot], (uint32_t)((j / kRedSlots) & 1), &abort_flag, lim)) break;
             const uint32_t u = units[j];
             const int cb = unit_cb(u), ncol = unit_ncol(u), n0 = unit_tile(u) * 16;
             const float *rb = red + (size_t)slot * kCW * 2 * 16 * Tc;
@@ -551,13 +565,14 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
             __syncwarp();
             if (lane == 0) mbar_arrive(&red_empty[slot]);
         }
-        if (to && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
+        __syncwarp();
+        if (abort_flag && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
         return;
     }
 
     // ---- consumers: x -> f16 in place, with a per-token power-of-two
     // prescale (warp w <-> token w)
-    bool timed_out = !mbar_wait_bounded(&xbar, 0);
+    bool timed_out = !mbar_wait_abort(&xbar, 0, &abort_flag, lim);
     if (warp < T) {
         uint4 *row = reinterpret_cast<uint4 *>(xs + (size_t)warp * xs_stride);
         float m = 0.f;
@@ -599,7 +614,7 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     int s_cur = 0;
     auto open_unit = [&](int j, const uint8_t *&b0, const uint8_t *&b1, int &s) {
         const int c = j * NCH + q, pc = c >> lcps;
-        if (!wait_piece(full, a.S, pc, &issued)) timed_out = true;
+        if (!wait_piece(full, a.S, pc, &issued, &abort_flag, lim)) timed_out = true;
         s = pc - (int)(a.S.div((uint32_t)pc) * a.S.d);
         // [gate blocks of the piece][up blocks of the piece]
         b0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c & (cps - 1)) * kBlk;
@@ -648,13 +663,13 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
         }
         // hand the partial fragments to the epilogue warps
         const int slot = j % kRedSlots;
-        if (j >= kRedSlots && !mbar_wait_bounded(&red_empty[slot], (uint32_t)((j / kRedSlots - 1) & 1)))
+        if (j >= kRedSlots && !mbar_wait_abort(&red_empty[slot], (uint32_t)((j / kRedSlots - 1) & 1), &abort_flag, lim))
             timed_out = true;
         put_partials(red + (size_t)slot * kCW * 2 * 16 * Tc, Tc, warp, g, t, aG, aU);
         __syncwarp();
         if (lane == 0) mbar_arrive(&red_full[slot]);
     }
-    if (timed_out && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
+    if ((timed_out || abort_flag) && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
 }
 
 // ---------------------------------------------------------------- down
@@ -668,6 +683,7 @@ struct DownArgs {
     int *counters;                  // [H/32], zero between calls
     uint16_t *out;                  // bf16 [T][H]
     uint32_t *status;
+    long long wait_cycles;          // limit of every wait but the final drains
     FastDiv S;                      // stages
     int T, k, E, H, I, cps;
 };
@@ -693,6 +709,7 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
     __shared__ RouteTable tb;
     __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], red_full[kRedSlots], red_empty[kRedSlots];
     __shared__ int issued;   // chunks issued by the producer (see produce)
+    __shared__ volatile int abort_flag;   // set by the first role that gives up on a wait
     __shared__ int slot_of[2][kMaxT];    // (expert slot - d_lo, token) -> staged B column, -1 none
     __shared__ int slot_d[kMaxBSlots], slot_t[kMaxBSlots];
     __shared__ unsigned slot_max[kMaxBSlots];
@@ -722,8 +739,10 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
         }
         mbar_fence_init();
         issued = 0;
+        abort_flag = 0;
         n_last = 0;
     }
+    const long long lim = a.wait_cycles;
     if (tid < kMaxBSlots) slot_max[tid] = 0u;
     if (warp == 0) build_route_table(tb, a.ids, a.topk_w, T * k, k, a.E, nullptr, false);
     __syncthreads();
@@ -744,7 +763,7 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
 
     if (warp == kProducerWarp) {
         // the weights do not depend on the gate/up kernel: stream them at once
-        produce(stages, full, empty, a.S, cps, n_mine * NCH / cps, a.status, &issued,
+        produce(stages, full, empty, a.S, cps, n_mine * NCH / cps, &abort_flag, lim, &issued,
                 [&](int p, const uint8_t *&b0, const uint8_t *&b1) {
                     const int c = p * cps;
                     const int u = u0 + c / NCH, d = u >> ltiles, t32 = u & (tiles - 1), q = c % NCH;
@@ -759,13 +778,9 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
         // epilogue: sum the 16 warps' partial fragments of a unit, undo the
         // column's prescale and store the expert's f32 slice for the combine
         const int e = warp - kEpiWarp0;
-        bool to = false;
-        for (int j = 0; j < n_mine && !to; ++j) {
+        for (int j = 0; j < n_mine; ++j) {
             const int slot = j % kRedSlots;
-            if (!mbar_wait_bounded(&red_full[slot], (uint32_t)((j / kRedSlots) & 1))) {
-                to = true;
-                break;
-            }
+            if (!mbar_wait_abort(&red_full[slot], (uint32_t)((j / kRedSlots) & 1), &abort_flag, lim)) break;
             const int u = u0 + j, d = u >> ltiles, m0 = (u & (tiles - 1)) * 32;
             const float *rb = red + (size_t)slot * kCW * 2 * 16 * Tc;
             for (int idx = lane + 32 * e; idx < 32 * T; idx += 32 * kEpiWarps) {
@@ -777,7 +792,8 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
             __syncwarp();
             if (lane == 0) mbar_arrive(&red_empty[slot]);
         }
-        if (to && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
+        __syncwarp();
+        if (abort_flag && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
         __threadfence();
         asm volatile("bar.sync 3, %0;" ::"r"(32 * (kCW + kEpiWarps)) : "memory");
         return;
@@ -871,7 +887,7 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
     int s_cur = 0;
     auto open_unit = [&](int j, const uint8_t *&b0, const uint8_t *&b1, int &s) {
         const int c = j * NCH + q, pc = c >> lcps;
-        if (!wait_piece(full, a.S, pc, &issued)) timed_out = true;
+        if (!wait_piece(full, a.S, pc, &issued, &abort_flag, lim)) timed_out = true;
         s = pc - (int)(a.S.div((uint32_t)pc) * a.S.d);
         // [rows m0..+15: blocks of the piece][rows m0+16..+31: blocks of the piece]
         b0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c & (cps - 1)) * kBlk;
@@ -914,13 +930,13 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
             s_cur = ns;
         }
         const int slot = j % kRedSlots;
-        if (j >= kRedSlots && !mbar_wait_bounded(&red_empty[slot], (uint32_t)((j / kRedSlots - 1) & 1)))
+        if (j >= kRedSlots && !mbar_wait_abort(&red_empty[slot], (uint32_t)((j / kRedSlots - 1) & 1), &abort_flag, lim))
             timed_out = true;
         put_partials(red + (size_t)slot * kCW * 2 * 16 * Tc, Tc, warp, g, t, acc0, acc1);
         __syncwarp();
         if (lane == 0) mbar_arrive(&red_full[slot]);
     }
-    if (timed_out && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
+    if ((timed_out || abort_flag) && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
     // Combine: once every expert's slice of a 32-row tile is in, the CTA
     // whose unit completed it sums the slices in expert order and writes
     // bf16; the order of the sum does not depend on timing.  The epilogue
@@ -989,17 +1005,21 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
                        cudaStream_t s, const cudaEvent_t *ev) {
     const int H = L.d.hidden, I = L.d.inter;
     const int grid = L.sm_count;
-    static bool attr_done[64] = {};
+    // the kernels' shared-memory limit, once per device (the caller made the
+    // layer's device current); concurrent first calls from several host
+    // threads run it once
+    static std::once_flag attr_once[64];
+    static cudaError_t attr_err[64];
     const int dev = L.d.device;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
+    std::call_once(attr_once[dev], [&] {
         cudaError_t e = cudaFuncSetAttribute(dec_gateup_mx_kernel<NCU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kMaxDynSmem);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(dec_down_mx_kernel<NCD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
+        attr_err[dev] = e;
+    });
+    if (attr_err[dev] != cudaSuccess) return attr_err[dev];
     GateUpArgs ga;
     ga.codes_g = L.w.codes[MOEQ_GATE];
     ga.codes_u = L.w.codes[MOEQ_UP];
@@ -1008,6 +1028,7 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     ga.topk_w = topk_w;
     ga.h = L.h;
     ga.status = L.status;
+    ga.wait_cycles = L.wait_cycles;
     ga.T = T;
     ga.k = L.d.top_k;
     ga.E = L.d.n_experts;
@@ -1031,6 +1052,7 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     da.counters = L.dec_counters;
     da.out = reinterpret_cast<uint16_t *>(out);
     da.status = L.status;
+    da.wait_cycles = L.wait_cycles;
     da.T = T;
     da.k = L.d.top_k;
     da.E = L.d.n_experts;

@@ -104,6 +104,11 @@ struct Layer {
     float *w_stage = nullptr;
     bool uploaded = false;
     int sm_count = 0;
+    // limit, in SM clocks, of the kernels' waits on one another (mbarriers,
+    // issue counters); on expiry a kernel raises FLAG_TIMEOUT and unwinds.
+    // About a second at the default; a test may shorten it at create
+    // (MOEQ_TEST_WAIT_CYCLES) to make a wait run out on purpose.
+    long long wait_cycles = 2000000000LL;
     // kernels launched (or captured into a graph) by this layer so far
     mutable long long launches = 0;
     void count_launches(int n) const { launches += n; }
@@ -123,6 +128,10 @@ struct Layer {
     }
     int elem_bytes() const { return d.act == MOEQ_ACT_F32 ? 4 : 2; }
 };
+
+// Every device allocation of the library goes through here (cudaMalloc, plus
+// the MOEQ_TEST_FAIL_ALLOC fault injection of the tests).
+cudaError_t dev_alloc(void **p, size_t bytes);
 
 // ---- launchers (each returns cudaGetLastError() of its launch) ----
 cudaError_t launch_route_bucket(const Layer &L, const int32_t *topk_ids, int32_t n_routes,

@@ -239,6 +239,7 @@ struct PfArgs {
     uint8_t *hq1, *hq2, *sfh;     // gate/up: quantised h and its scale atoms
     float *acc;                   // down: f32 output accumulator [T][H]
     uint32_t *status;
+    long long wait_cycles;        // limit of every wait but the final drains
     int E, H, I, k;
 };
 
@@ -289,7 +290,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int c = c0 + (lane < kGUFill ? lane : 0), s = c % kGUStages;
             bool ok = true;
             if (lane < kGUFill && c < total && c >= kGUStages)
-                ok = wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag);
+                ok = wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag, a.wait_cycles);
             if (__any_sync(0xffffffffu, !ok)) break;
             if (lane < kGUFill && c < total) mbar_arrive_expect_tx(&full[s], 2 * kBoxA + 2 * kTileB + 3 * kAtom);
             __syncwarp();
@@ -322,12 +323,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
                 const Item m = decode_item(rt.off, rt.tb, E, subs, it);
                 const int n = (m.cnt + 15) & ~15, b = q & 1;
-                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
+                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag, a.wait_cycles)) break;
                 tc_fence_after();
                 const uint32_t t_g = tmem + b * 2 * kRT, t_u = t_g + kRT;
                 for (int sl = 0; sl < slabs; ++sl, ++c) {
                     const int s = c % kGUStages;
-                    if (!wait_or_abort(&full[s], (uint32_t)((c / kGUStages) & 1), &abort_flag)) break;
+                    if (!wait_or_abort(&full[s], (uint32_t)((c / kGUStages) & 1), &abort_flag, a.wait_cycles)) break;
                     tc_fence_after();
                     const uint8_t *st = smem + (size_t)s * kGUStage;
                     const uint8_t *sf = st + 2 * kTileA + 2 * kTileB;
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
             const Item m = decode_item(rt.off, rt.tb, E, subs, it);
             const int b = q & 1;
-            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag)) break;
+            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag, a.wait_cycles)) break;
             tc_fence_after();
             const int i_row = m.sub * kT + 32 * qd + lane;   // this lane's row of I
             const uint32_t t_g = tmem + b * 2 * kRT + ((uint32_t)(32 * qd) << 16), t_u = t_g + kRT;
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int c = c0 + (lane < kDNFill ? lane : 0), s = c % kDNStages;
             bool ok = true;
             if (lane < kDNFill && c < total && c >= kDNStages)
-                ok = wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag);
+                ok = wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag, a.wait_cycles);
             if (__any_sync(0xffffffffu, !ok)) break;
             if (lane < kDNFill && c < total) mbar_arrive_expect_tx(&full[s], kBoxA + 2 * kTileB + 2 * kAtom);
             __syncwarp();
@@ -475,12 +476,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int it = blockIdx.x; it < n_items && !abort_flag; it += gridDim.x, ++q) {
                 const Item m = decode_item(rt.off, rt.tb, E, subs, it);
                 const int n = (m.cnt + 15) & ~15, b = q & 1;
-                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
+                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag, a.wait_cycles)) break;
                 tc_fence_after();
                 const uint32_t t_y = tmem + b * kRT;
                 for (int sl = 0; sl < slabs; ++sl, ++c) {
                     const int s = c % kDNStages;
-                    if (!wait_or_abort(&full[s], (uint32_t)((c / kDNStages) & 1), &abort_flag)) break;
+                    if (!wait_or_abort(&full[s], (uint32_t)((c / kDNStages) & 1), &abort_flag, a.wait_cycles)) break;
                     tc_fence_after();
                     const uint8_t *st = smem + (size_t)s * kDNStage;
                     const uint8_t *sf = st + kTileA + 2 * kTileB;
@@ -522,7 +523,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 tk1 = r / k;
                 w1 = __ldg(a.topk_w + r);
             }
-            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag)) break;
+            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag, a.wait_cycles)) break;
             tc_fence_after();
             const int h_row = m.sub * kT + 32 * qd + lane;   // this lane's output feature
             const uint32_t t_y = tmem + b * kRT + ((uint32_t)(32 * qd) << 16);
@@ -613,7 +614,7 @@ cudaError_t prefill_mx_create(Layer &L) {
     const size_t tiles = R / kRT + (size_t)E;                  // upper bound on route tiles
     cudaError_t e = cudaSuccess;
     auto al = [&](void **p, size_t n) {
-        if (e == cudaSuccess) e = cudaMalloc(p, n);
+        if (e == cudaSuccess) e = dev_alloc(p, n);
     };
     for (int p = 0; p < 3; ++p) {
         const size_t N = p == MOEQ_DOWN ? H : I, K = p == MOEQ_DOWN ? I : H;
@@ -716,6 +717,7 @@ cudaError_t launch_prefill_mx(const Layer &L, const void *x, const int32_t *ids,
     a.ids = ids;
     a.topk_w = topk_w;
     a.status = L.status;
+    a.wait_cycles = L.wait_cycles;
     a.E = E;
     a.H = H;
     a.I = I;

@@ -182,6 +182,7 @@ struct VqArgs {
     uint16_t *hg;             // gate/up output [route position][I] bf16
     float *acc;               // down output [T][H]
     uint32_t *status;
+    long long wait_cycles;        // limit of every wait but the final drains
     int E, H, I, k;
 };
 
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
             int c = 0;
             for (; c < total; ++c) {
                 const int s = c % kGUStages;
-                if (c >= kGUStages && !wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag)) break;
+                if (c >= kGUStages && !wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag, a.wait_cycles)) break;
                 const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
                 mbar_arrive_expect_tx(&b_full[s], kTileB);
                 tma_load_2d(smem + (size_t)s * kGUStage + 2 * kTileA, &tX, (c % slabs) * kKS, m.row0, &b_full[s]);
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
                 }
             }
             drain_stages(b_full, kGUStages, c);
-            mbar_wait_bounded(&book_bar, 0, 200000000LL);
+            mbar_wait_bounded(&book_bar, 0, kDrainCycles);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -262,13 +263,13 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
                 const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + q * gridDim.x);
                 const int n = (m.cnt + 15) & ~15, b = q & 1;
                 const uint32_t id = idesc_bf16(n);
-                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
+                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag, a.wait_cycles)) break;
                 tc_fence_after();
                 const uint32_t t_g = tmem + b * 2 * kRT, t_u = t_g + kRT;
                 for (int sl = 0; sl < slabs; ++sl, ++c) {
                     const int s = c % kGUStages;
                     const uint32_t par = (uint32_t)((c / kGUStages) & 1);
-                    if (!wait_or_abort(&a_full[s], par, &abort_flag) || !wait_or_abort(&b_full[s], par, &abort_flag)) break;
+                    if (!wait_or_abort(&a_full[s], par, &abort_flag, a.wait_cycles) || !wait_or_abort(&b_full[s], par, &abort_flag, a.wait_cycles)) break;
                     tc_fence_after();
                     const uint8_t *st = smem + (size_t)s * kGUStage;
 #pragma unroll
@@ -304,11 +305,11 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
         fetch(1, q1);
         fetch(2, q2);
         fetch(3, q3);
-        bool ok = wait_or_abort(&book_bar, 0, &abort_flag);
+        bool ok = wait_or_abort(&book_bar, 0, &abort_flag, a.wait_cycles);
         auto step = [&](int c, RowRaw &q) {
             if (c >= total || !ok) return;
             const int s = c % kGUStages;
-            if (c >= kGUStages) ok = wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag);
+            if (c >= kGUStages) ok = wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag, a.wait_cycles);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) return;
             expand_row<0, 8>(q, r8, b13, b8, smem + (size_t)s * kGUStage + mat * kTileA, r);
@@ -329,7 +330,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
         for (int q = 0; q < my_items && !abort_flag; ++q) {
             const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + q * gridDim.x);
             const int b = q & 1;
-            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag)) break;
+            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag, a.wait_cycles)) break;
             tc_fence_after();
             const int i_row = m.sub * kT + 32 * qd + lane;
             const uint32_t t_g = tmem + b * 2 * kRT + ((uint32_t)(32 * qd) << 16), t_u = t_g + kRT;
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_con
             int c = 0;
             for (; c < total; ++c) {
                 const int s = c % kDNStages;
-                if (c >= kDNStages && !wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag)) break;
+                if (c >= kDNStages && !wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag, a.wait_cycles)) break;
                 const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
                 mbar_arrive_expect_tx(&b_full[s], kTileB);
                 tma_load_2d(smem + (size_t)s * kDNStage + kTileA, &tH, (c % slabs) * kKS, m.row0, &b_full[s]);
@@ -415,7 +416,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_con
                 }
             }
             drain_stages(b_full, kDNStages, c);
-            mbar_wait_bounded(&book_bar, 0, 200000000LL);
+            mbar_wait_bounded(&book_bar, 0, kDrainCycles);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -424,13 +425,13 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_con
                 const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + q * gridDim.x);
                 const int n = (m.cnt + 15) & ~15, b = q & 1;
                 const uint32_t id = idesc_bf16(n);
-                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag)) break;
+                if (q >= 2 && !wait_or_abort(&tmem_empty[b], (uint32_t)(((q >> 1) - 1) & 1), &abort_flag, a.wait_cycles)) break;
                 tc_fence_after();
                 const uint32_t t_y = tmem + b * kRT;
                 for (int sl = 0; sl < slabs; ++sl, ++c) {
                     const int s = c % kDNStages;
                     const uint32_t par = (uint32_t)((c / kDNStages) & 1);
-                    if (!wait_or_abort(&a_full[s], par, &abort_flag) || !wait_or_abort(&b_full[s], par, &abort_flag)) break;
+                    if (!wait_or_abort(&a_full[s], par, &abort_flag, a.wait_cycles) || !wait_or_abort(&b_full[s], par, &abort_flag, a.wait_cycles)) break;
                     tc_fence_after();
                     const uint8_t *st = smem + (size_t)s * kDNStage;
 #pragma unroll
@@ -458,11 +459,11 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_con
         fetch(1, q1);
         fetch(2, q2);
         fetch(3, q3);
-        bool ok = wait_or_abort(&book_bar, 0, &abort_flag);
+        bool ok = wait_or_abort(&book_bar, 0, &abort_flag, a.wait_cycles);
         auto step = [&](int c, RowRaw &q) {
             if (c >= total || !ok) return;
             const int s = c % kDNStages;
-            if (c >= kDNStages) ok = wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag);
+            if (c >= kDNStages) ok = wait_or_abort(&empty[s], (uint32_t)((c / kDNStages - 1) & 1), &abort_flag, a.wait_cycles);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) return;
             uint8_t *tile = smem + (size_t)s * kDNStage;
@@ -496,7 +497,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_con
                 tk1 = r / k;
                 w1 = __ldg(a.topk_w + r);
             }
-            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag)) break;
+            if (!wait_or_abort(&tmem_full[b], (uint32_t)((q >> 1) & 1), &abort_flag, a.wait_cycles)) break;
             tc_fence_after();
             const int h_row = m.sub * kT + 32 * qd + lane;
             const uint32_t t_y = tmem + b * kRT + ((uint32_t)(32 * qd) << 16);
@@ -569,9 +570,9 @@ cudaError_t prefill_vq_create(Layer &L) {
     if (!pv) return cudaErrorMemoryAllocation;
     L.pv = pv;
     const size_t R = (size_t)d.max_tokens * d.top_k;
-    cudaError_t e = cudaMalloc((void **)&pv->tile_base, sizeof(int32_t) * (d.n_experts + 1));
-    if (e == cudaSuccess) e = cudaMalloc((void **)&pv->xg, R * d.hidden * 2);
-    if (e == cudaSuccess) e = cudaMalloc((void **)&pv->hg, R * d.inter * 2);
+    cudaError_t e = dev_alloc((void **)&pv->tile_base, sizeof(int32_t) * (d.n_experts + 1));
+    if (e == cudaSuccess) e = dev_alloc((void **)&pv->xg, R * d.hidden * 2);
+    if (e == cudaSuccess) e = dev_alloc((void **)&pv->hg, R * d.inter * 2);
     // route positions past a tile's routes feed discarded MMA columns: keep them finite
     if (e == cudaSuccess) e = cudaMemset(pv->xg, 0, R * d.hidden * 2);
     if (e == cudaSuccess) e = cudaMemset(pv->hg, 0, R * d.inter * 2);
@@ -619,6 +620,7 @@ cudaError_t launch_prefill_vq(const Layer &L, const void *x, const int32_t *ids,
     a.hg = pv->hg;
     a.acc = L.acc;
     a.status = L.status;
+    a.wait_cycles = L.wait_cycles;
     a.E = E;
     a.H = H;
     a.I = I;

@@ -106,21 +106,32 @@ route_bucket_kernel(const int32_t *__restrict__ ids, int32_t n_routes, int32_t E
     (void)s_total;
 }
 
+constexpr int kMaxDevices = 64;
+std::mutex g_route_mu;   // guards the per-device set-up of both entry points
+bool g_route_attr[kMaxDevices] = {};
+
+// The kernel's dynamic shared-memory limit on device `dev` (current), set
+// once per device under g_route_mu.
+cudaError_t route_smem_limit(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_route_mu);
+    if (!g_route_attr[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(route_bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(sizeof(int32_t) * kMaxExperts * (2 + kWarps)));
+        if (e != cudaSuccess) return e;
+        g_route_attr[dev] = true;
+    }
+    return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_route_bucket(const Layer &L, const int32_t *topk_ids, int32_t n_routes,
                                 int32_t *offsets, int32_t *perm, int32_t *active, cudaStream_t s) {
     const int E = L.d.n_experts;
     size_t smem = sizeof(int32_t) * (size_t)E * (2 + kWarps);
-    static bool attr_set[64] = {};
-    int dev = L.d.device;
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        cudaError_t err = cudaFuncSetAttribute(route_bucket_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)(sizeof(int32_t) * kMaxExperts * (2 + kWarps)));
-        if (err != cudaSuccess) return err;
-        attr_set[dev] = true;
-    }
+    const cudaError_t err = route_smem_limit(L.d.device);
+    if (err != cudaSuccess) return err;
     L.count_launches(1);
     route_bucket_kernel<<<1, kThreads, smem, s>>>(topk_ids, n_routes, E, offsets, perm, active,
                                                   L.status);
@@ -142,20 +153,19 @@ constexpr int kNoAllocWords = kMaxExperts + 2;        // 4104 bytes
 // from cudaGetSymbolAddress, once per device.
 static __device__ __align__(256) int32_t g_route_scratch[kNoAllocWords];
 
-constexpr int kNoAllocMaxDevices = 64;
+constexpr int kNoAllocMaxDevices = kMaxDevices;
 std::mutex g_noalloc_mu;
 int32_t *g_noalloc_scratch[kNoAllocMaxDevices] = {};
 
 // Set-up for the current device `dev` (once): the scratch's device address
 // and the kernel's dynamic shared-memory limit.
 cudaError_t noalloc_scratch(int dev, int32_t **out) {
+    cudaError_t e = route_smem_limit(dev);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
     if (!g_noalloc_scratch[dev]) {
         int32_t *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_route_scratch);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(route_bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(sizeof(int32_t) * kMaxExperts * (2 + kWarps)));
+        e = cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_route_scratch);
         if (e != cudaSuccess) return e;
         g_noalloc_scratch[dev] = p;
     }

@@ -13,7 +13,6 @@ namespace umma {
 
 constexpr int kT = 128;           // MMA M (weight rows per tile)
 constexpr int kRT = 64;           // routes per route tile: the largest MMA N used
-constexpr long long kWaitCycles = 2000000000LL;
 
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
@@ -91,13 +90,14 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float v[16]) {
 // Bounded wait that also gives up once another role has given up.  It polls
 // with test_wait: a thread suspended in try_wait can resume well after the
 // phase completed, and every hand-off between the roles is on the critical
-// path.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+// path.  `limit` is the layer's wait limit in SM clocks.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                              long long limit) {
     if (mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_test_wait(bar, parity)) {
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             return false;
         }
@@ -110,11 +110,11 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
 // MMA this thread issued.
 __device__ __forceinline__ void drain_stages(uint64_t *full, int S, int issued) {
     for (int c = issued > S ? issued - S : 0; c < issued; ++c)
-        mbar_wait_bounded(&full[c % S], (uint32_t)((c / S) & 1), 200000000LL);
+        mbar_wait_bounded(&full[c % S], (uint32_t)((c / S) & 1), kDrainCycles);
 }
 __device__ __forceinline__ void drain_mma(uint64_t *done) {
     tc_commit(done);
-    mbar_wait_bounded(done, 0, 200000000LL);
+    mbar_wait_bounded(done, 0, kDrainCycles);
 }
 
 // Scale-factor atom byte of (row r of a 128-row tile, 32-block kb of a 4-block group)

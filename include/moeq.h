@@ -208,7 +208,12 @@ MOEQ_API moeq_status moeq_route(moeq_layer_t layer, const int32_t *topk_ids, int
  * threads, race on it and must be ordered by the caller.  The first call on
  * each device sets up (looks up the array's device address and sets the
  * kernel's shared-memory limit); make that first call before any stream
- * capture on that device.
+ * capture on that device.  The library itself makes no allocating call
+ * here, but under the CUDA runtime's lazy module loading the first call on
+ * a device may be what makes the runtime load this module, which places
+ * the module's code and the scratch array in device memory: one more
+ * reason to make the first call early, before the device's memory is
+ * handed to another pool.
  * Errors: INVALID_ARGUMENT (NULL pointer, n_tokens < 1, top_k outside
  * [1, 64], n_experts < 1, n_tokens*top_k > 2^30), UNSUPPORTED (n_experts >
  * 1024), CUDA. */
@@ -238,8 +243,15 @@ MOEQ_API moeq_status moeq_dequant(moeq_layer_t layer, int32_t expert, int32_t pr
 
 /* The layer's device status word, read after synchronizing the device:
  * MOEQ_OK, or the first-raised device flag (MOEQ_ERR_ROUTE_OUT_OF_RANGE,
- * MOEQ_ERR_TIMEOUT).  clear != 0 resets it.  Errors: INVALID_ARGUMENT,
- * CUDA. */
+ * MOEQ_ERR_TIMEOUT).  clear != 0 resets it.
+ * MOEQ_ERR_TIMEOUT means that a kernel's bounded wait on another part of
+ * the same kernel (about a second; never expected in normal operation)
+ * gave up: the kernel stopped issuing work, waited for its own copies and
+ * tensor-core operations in flight, released its on-chip memory and
+ * returned, so the device stays usable, but that forward's output is
+ * undefined.  Clearing the status after a timeout also resets the decode
+ * path's workspace counters (per-tile arrival counts that a forward which
+ * gave up part-way can leave behind).  Errors: INVALID_ARGUMENT, CUDA. */
 MOEQ_API moeq_status moeq_layer_status(moeq_layer_t layer, int32_t clear);
 
 /* Number of kernels the layer has launched so far (a launch captured into

@@ -13,6 +13,7 @@ from .oracle import (  # noqa: F401
     f16_to_f64,
     dequant,
     forward,
+    forward_by_expert,
     num_threads,
     route_bucket,
 )

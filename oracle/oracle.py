@@ -181,3 +181,57 @@ def forward(layer, x, topk_ids, topk_w, tokens=None, want_h=False, want_counts=F
         res.append(counts)
     res.append(int(invalid))
     return tuple(res)
+
+
+def _silu64(z):
+    # silu(z) = z / (1 + e^-z); for very negative z, e^-z overflows to +inf
+    # and the quotient is -0 (as in the C restatement), never NaN
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def forward_by_expert(layer, x, topk_ids, topk_w, tokens=None):
+    """The layer output of ``forward`` computed expert by expert, for
+    micro-batches the per-route C loop takes minutes on (a 2048-token layer).
+
+    Same definition ("MiMo-V2.6-Flash-RL GGUF for a single DGX Spark",
+    "Architecture notes": k routed experts per token, gate/up/down experts;
+    "MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe": the weight formats):
+    for every expert e with routes, its three matrices are dequantised once
+    to their exact f32 values by ``dequant`` (the C restatement), widened to
+    f64, and applied to all of e's routed tokens with numpy f64 matrix
+    products (the library matmul is the step; nothing is fused):
+        G = X_e W_gate,e^T,  U = X_e W_up,e^T,  Hh = silu(G) * U,
+        Y = Hh W_down,e^T,   out[t] += w[t][s] * Y[route (t, s)].
+    Routes are added slot by slot in slot order.  Ids of -1 are no route;
+    other ids outside [0, E) are skipped and counted (among the requested
+    tokens).
+
+    Returns (out [n][H] float64, number of invalid ids)."""
+    cfg = layer.cfg
+    xf = _x_f64(layer, x)
+    ids = np.ascontiguousarray(topk_ids, dtype=np.int32)
+    w = np.ascontiguousarray(topk_w, dtype=np.float32).astype(np.float64)
+    T, k = ids.shape
+    assert k == cfg.k and w.shape == ids.shape and xf.shape == (T, cfg.H)
+    if tokens is None:
+        tok = np.arange(T)
+    else:
+        tok = np.asarray(tokens, dtype=np.int64)
+    row_of = np.full(T, -1, np.int64)          # output row of each requested token
+    row_of[tok] = np.arange(len(tok))
+    out = np.zeros((len(tok), cfg.H), np.float64)
+    invalid = int(((ids[tok] != -1) & ((ids[tok] < 0) | (ids[tok] >= cfg.E))).sum())
+    sel = (ids >= 0) & (ids < cfg.E) & (row_of[:, None] >= 0)
+    for e in np.unique(ids[sel]):
+        t_idx, s_idx = np.nonzero(sel & (ids == e))
+        Wg = dequant(layer, int(e), 0).astype(np.float64)
+        Wu = dequant(layer, int(e), 1).astype(np.float64)
+        Wd = dequant(layer, int(e), 2).astype(np.float64)
+        X = xf[t_idx]
+        Hh = _silu64(X @ Wg.T) * (X @ Wu.T)
+        Y = Hh @ Wd.T
+        for s in np.unique(s_idx):
+            m = s_idx == s           # one route per token in a slot: rows are distinct
+            out[row_of[t_idx[m]]] += w[t_idx[m], s][:, None] * Y[m]
+    return out, invalid

@@ -41,6 +41,62 @@ def test_medium_layers(shape, fmt, act, gains):
     assert_close(out, oracle_ref(L, x, ids, w), act, f"{fmt}/{act}/{shape}")
 
 
+# A layer whose tensor-core work lists wrap the persistent grid several
+# times: 1024 tokens x 8 routes over 64 experts is about 128 routes per
+# expert, i.e. two 64-route tiles x 8 row tiles per expert, about 1000 work
+# items per projection for 148 CTAs.  Every row is compared, so a fault in
+# a late item (the accumulator double buffer, the scheduler's wrap-around)
+# cannot hide.
+WRAP = dict(H=1024, I=1024, E=64, k=8, T=1024)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "vq13", "vq13r8"])
+def test_wrapping_work_lists_every_row(fmt):
+    cfg = synth.get_cfg("tiny_mxfp4", fmt=fmt, act="bf16", gains=(fmt == "vq13r8"), scale_exp=(-9, -5), **WRAP)
+    L = synth.gen_layer(cfg, seed=51)
+    x = synth.gen_activations(cfg, seed=51)
+    ids, w = synth.gen_routing(cfg, seed=51)
+    lay = dev_layer(L)
+    out = run(lay, cfg, x, ids, w)
+    ref, invalid = oracle.forward_by_expert(L, x, ids, w)
+    assert invalid == 0
+    assert_close(out, ref, "bf16", f"wrap {fmt}")
+    # a second routing through the same layer (work lists rebuilt, nothing
+    # carried over from the first call)
+    ids2, w2 = synth.gen_routing(cfg.replace(routing="zipf", unrouted=(3,)), seed=52)
+    out2 = run(lay, cfg, x, ids2, w2)
+    ref2, _ = oracle.forward_by_expert(L, x, ids2, w2)
+    assert_close(out2, ref2, "bf16", f"wrap {fmt} second call")
+
+
+def _wide_range_x(cfg, seed):
+    """bf16 activations whose every 32-value block holds one element of
+    magnitude about 1e3 and 31 of about 1e-3: the widest spread the
+    per-block scaling of the tensor-core MXFP4 path (and the per-token
+    prescale of the decode path) has to carry."""
+    rng = np.random.default_rng(seed)
+    xf = rng.normal(0.0, 1e-3, size=(cfg.T, cfg.H)).astype(np.float32)
+    big = rng.integers(0, 32, size=(cfg.T, cfg.H // 32))
+    sign = rng.choice([-1.0, 1.0], size=big.shape)
+    rows = np.arange(cfg.T)[:, None]
+    xf[rows, np.arange(cfg.H // 32)[None, :] * 32 + big] = sign * rng.uniform(500.0, 2000.0, size=big.shape)
+    return synth.bf16_bits_from_f32(xf)
+
+
+@pytest.mark.parametrize("shape", [dict(H=1024, I=512, E=16, k=4, T=200),     # tensor-core MXFP4
+                                   dict(H=2048, I=2048, E=16, k=8, T=4)],     # decode kernels
+                         ids=["prefill", "decode"])
+@pytest.mark.parametrize("fmt", ["mxfp4", "vq13r8"])
+def test_wide_dynamic_range_inside_a_block(shape, fmt):
+    cfg = synth.get_cfg("tiny_mxfp4", fmt=fmt, act="bf16", scale_exp=(-9, -5), **shape)
+    L = synth.gen_layer(cfg, seed=61)
+    x = _wide_range_x(cfg, 61)
+    ids, w = synth.gen_routing(cfg, seed=61)
+    lay = dev_layer(L)
+    out = run(lay, cfg, x, ids, w)
+    assert_close(out, oracle_ref(L, x, ids, w), "bf16", f"wide range {fmt} {shape}")
+
+
 # decode-sized MXFP4 layers (1..8 tokens, bf16): the grouped-GEMV path
 DECODE = [
     dict(H=2048, I=2048, E=16, k=2, T=1),

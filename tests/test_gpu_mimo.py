@@ -1,10 +1,11 @@
 """The MiMo-shaped workloads (hidden 4096, inter 2048, 256 experts, top-8)
-against the oracle: every decode output, and sampled tokens of the two
-2048-token prefill micro-batches (the oracle computes them one by one)."""
+against the oracle: every output row of every workload, the two 2048-token
+prefill micro-batches included (the oracle's expert-by-expert leg computes
+all 2048 rows in about a minute of host time)."""
 import numpy as np
 import pytest
 
-from _gpu_util import assert_close, oracle_ref, run, sample_tokens, synth
+from _gpu_util import assert_close, oracle, oracle_ref, run, synth
 
 pytestmark = pytest.mark.gpu
 
@@ -29,29 +30,25 @@ def test_decode_vq(mimo_layers, T, residual):
     assert_close(out, oracle_ref(L, x, ids, w), "bf16", f"decode_vq T={T} r={residual}")
 
 
-def test_prefill_mxfp4_zipf_sampled(mimo_layers):
+def test_prefill_mxfp4_zipf_all_rows(mimo_layers):
     L, lay = mimo_layers["decode_mxfp4"]
     cfg = synth.get_cfg("prefill_mxfp4_zipf")
     x = synth.gen_activations(cfg)
     ids, w = synth.gen_routing(cfg)
     out = run(lay, cfg, x, ids, w)
     assert np.isfinite(out).all()
-    # the hottest expert's first and last tokens, a never-routed expert's
-    # absence, and a spread of others
-    hot = np.bincount(ids.ravel(), minlength=cfg.E).argmax()
-    hot_tok = np.nonzero((ids == hot).any(1))[0]
-    tok = np.unique(np.concatenate([sample_tokens(cfg.T, 10), hot_tok[[0, -1]]])).astype(np.int32)
-    ref = oracle_ref(L, x, ids, w, tokens=tok)
-    assert_close(out[tok], ref, "bf16", "prefill_mxfp4_zipf")
+    ref, invalid = oracle.forward_by_expert(L, x, ids, w)
+    assert invalid == 0
+    assert_close(out, ref, "bf16", "prefill_mxfp4_zipf")
 
 
-def test_prefill_vq_overflow_sampled(mimo_layers):
+def test_prefill_vq_overflow_all_rows(mimo_layers):
     L, lay = mimo_layers["prefill_vq_overflow"]
     cfg = synth.get_cfg("prefill_vq_overflow")
     x = synth.gen_activations(cfg)
     ids, w = synth.gen_routing(cfg)
     out = run(lay, cfg, x, ids, w)
     assert np.isfinite(out).all()
-    tok = sample_tokens(cfg.T, 12, seed=1)
-    ref = oracle_ref(L, x, ids, w, tokens=tok)
-    assert_close(out[tok], ref, "bf16", "prefill_vq_overflow")
+    ref, invalid = oracle.forward_by_expert(L, x, ids, w)
+    assert invalid == 0
+    assert_close(out, ref, "bf16", "prefill_vq_overflow")

@@ -191,7 +191,13 @@ def _silu(z):
     return z / (1.0 + math.exp(-z)) if z > -700 else -0.0
 
 
-def test_forward_constant_weights_closed_form():
+# the per-route C loop and the expert-by-expert leg (numpy f64 products of
+# the same exact weights) must both satisfy every forward pin
+FORWARDS = {"per_route": oracle.forward, "by_expert": oracle.forward_by_expert}
+
+
+@pytest.mark.parametrize("impl", sorted(FORWARDS))
+def test_forward_constant_weights_closed_form(impl):
     # every weight 1.0: g = u = S = sum(x), h = silu(S) S, y_m = I h,
     # out_t = sum_s w_s I silu(S_t) S_t
     cfg = _tiny_cfg()
@@ -200,14 +206,15 @@ def test_forward_constant_weights_closed_form():
         L.codes[p][:] = 0x22
     x = synth.gen_activations(cfg, seed=1)
     ids, w = synth.gen_routing(cfg, seed=1)
-    out, _ = oracle.forward(L, x, ids, w)
+    out, _ = FORWARDS[impl](L, x, ids, w)
     for t in range(cfg.T):
         S = float(np.sum(x[t].astype(np.float64)))
         want = float(np.sum(w[t].astype(np.float64))) * cfg.I * _silu(S) * S
         np.testing.assert_allclose(out[t], want, rtol=1e-12)
 
 
-def test_forward_orientation_one_hot():
+@pytest.mark.parametrize("impl", sorted(FORWARDS))
+def test_forward_orientation_one_hot(impl):
     # W_gate[n][k] = [k == n], W_up[n][k] = 2 [k == n+1], W_down[m][n] =
     # [n == m mod I] * (1 if m < I else -0.5): g_n = x_n, u_n = 2 x_{n+1},
     # h_n = silu(x_n) 2 x_{n+1}, y_m = c_m h_{m mod I}.  A transposed matrix,
@@ -230,8 +237,12 @@ def test_forward_orientation_one_hot():
     ids = np.full((cfg.T, cfg.k), -1, np.int32)
     ids[:, 1] = e
     w = np.full((cfg.T, cfg.k), 0.75, np.float32)
-    out, counts, invalid = oracle.forward(L, x, ids, w, want_counts=True)
-    assert invalid == 0 and list(counts) == [cfg.T] * 3
+    if impl == "per_route":
+        out, counts, invalid = oracle.forward(L, x, ids, w, want_counts=True)
+        assert invalid == 0 and list(counts) == [cfg.T] * 3
+    else:
+        out, invalid = oracle.forward_by_expert(L, x, ids, w)
+        assert invalid == 0
     for t in range(cfg.T):
         xt = x[t].astype(np.float64)
         h = np.array([_silu(xt[n]) * 2.0 * xt[n + 1] for n in range(I)])
@@ -272,6 +283,32 @@ def test_forward_matches_dense_brute_force(fmt):
     ref = _dense_reference(L, x, ids, w)
     np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-11 * np.abs(ref).max())
     assert invalid == 0 and list(counts) == [cfg.T * cfg.k] * 3
+    out2, invalid2 = oracle.forward_by_expert(L, x, ids, w)
+    np.testing.assert_allclose(out2, ref, rtol=1e-11, atol=1e-11 * np.abs(ref).max())
+    assert invalid2 == 0
+
+
+@pytest.mark.parametrize("fmt,act", [("mxfp4", "bf16"), ("mxfp4", "f32"), ("vq13", "bf16"), ("vq13r8", "bf16")])
+def test_forward_by_expert_matches_per_route(fmt, act):
+    # a medium layer with repeated experts inside a token, no-route and
+    # out-of-range ids, and a token subset in a scrambled order: the
+    # expert-by-expert leg agrees with the per-route C loop to f64 rounding
+    cfg = synth.get_cfg("tiny_mxfp4", H=256, I=192, E=12, k=4, T=40, fmt=fmt, act=act,
+                        gains=(fmt == "vq13r8"), scale_exp=(-9, -5))
+    L = synth.gen_layer(cfg, seed=12)
+    x = synth.gen_activations(cfg, seed=12)
+    ids, w = synth.gen_routing(cfg, seed=12)
+    ids[3, 1] = ids[3, 0]
+    ids[7, :] = -1
+    ids[9, 2] = cfg.E + 3
+    ids[11, 0] = -9
+    w[5] *= -3.0
+    for tokens in (None, np.array([39, 3, 7, 0, 9, 22], np.int32)):
+        ref, inv = oracle.forward(L, x, ids, w, tokens=tokens)
+        got, inv2 = oracle.forward_by_expert(L, x, ids, w, tokens=tokens)
+        assert inv == inv2 == (2 if tokens is None else 1)
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13 * np.abs(ref).max())
+    assert not got[2].any()     # token 7 has no route
 
 
 def test_routes_per_token_and_invalid_ids():

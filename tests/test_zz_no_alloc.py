@@ -1,13 +1,15 @@
 """moeq_route_noalloc, the route/bucket step with its scratch in a fixed
-in-library array (no device allocation), gives exactly the buckets of
-moeq_route, call after call.  Collected last so that it also runs after
-every other test has used the device."""
+in-library array (no device allocation), for callers that cannot allocate
+device memory.  It must give exactly the oracle's buckets, and exactly those
+of moeq_route (the entry point that uses a layer's workspace), call after
+call.  Collected last so that it also runs after every other test has used
+the device."""
 import ctypes as C
 
 import numpy as np
 import pytest
 
-from _gpu_util import torch_mod
+from _gpu_util import oracle, torch_mod
 
 pytestmark = pytest.mark.gpu
 
@@ -33,16 +35,22 @@ def test_route_noalloc_matches_route_on_consecutive_calls():
         ids[u < 0.04] = -1
         ids[(u >= 0.04) & (u < 0.04 + p_bad)] = E + 5
         ids_dev = torch.from_numpy(ids).cuda()
+        orc_off, orc_perm, orc_bad = oracle.route_bucket(ids, E)
         want_off, want_perm = lay.route(ids_dev)
         offs = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
         perm = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
         assert _noalloc(lib, ids_dev, T, k, E, offs, perm, stream) == moeq.OK
         torch.cuda.synchronize()
-        assert torch.equal(offs, want_off)
-        n = int(want_off[E])
+        n = int(orc_off[E])
         assert n == int(((ids >= 0) & (ids < E)).sum())
-        assert torch.equal(perm[:n], want_perm[:n])
+        assert orc_bad == int(((ids != -1) & ((ids < 0) | (ids >= E))).sum())
+        # against the oracle, bit for bit
+        assert np.array_equal(offs.cpu().numpy(), orc_off)
+        assert np.array_equal(perm[:n].cpu().numpy(), orc_perm)
         assert bool((perm[n:] == -7).all())   # nothing written past the valid routes
+        # and against moeq_route
+        assert torch.equal(offs, want_off)
+        assert torch.equal(perm[:n], want_perm[:n])
         lay.status(clear=True)
 
 
