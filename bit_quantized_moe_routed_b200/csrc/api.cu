@@ -2,6 +2,7 @@
 // argument validation, device memory ownership and kernel dispatch.
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -91,6 +92,7 @@ void free_layer(moeq_layer *L) {
     cudaFree(L->w_stage);
     prefill_mx_free(*L);
     prefill_vq_free(*L);
+    router_free(*L);
     delete L;
 }
 
@@ -363,6 +365,41 @@ moeq_status moeq_forward_host(moeq_layer_t L, const void *x, const int32_t *ids,
     e = cudaMemcpyAsync(out, L->out_stage, xb, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     return from_cuda(e);
+}
+
+moeq_status moeq_router_upload(moeq_layer_t L, const float *wr, int32_t score, void *stream) {
+    if (!L || !wr || (score != MOEQ_SCORE_SIGMOID && score != MOEQ_SCORE_SOFTMAX)) return MOEQ_ERR_INVALID_ARGUMENT;
+    const size_t n = (size_t)L->d.n_experts * L->d.hidden;
+    for (size_t i = 0; i < n; ++i)   // finite and within bf16's range (the terms of the bf16 path)
+        if (!(std::fabs(wr[i]) <= 3.38e38f)) return MOEQ_ERR_INVALID_ARGUMENT;
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    return from_cuda(router_upload(*L, wr, score, (cudaStream_t)stream));
+}
+
+moeq_status moeq_router(moeq_layer_t L, const void *x, int32_t T, int32_t *topk_ids, float *topk_w, float *logits,
+                        void *stream) {
+    if (!L || !x || !topk_ids || !topk_w || T < 1 || T > L->d.max_tokens) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (((uintptr_t)x & 3u) != 0) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (!L->router || !L->router->ready) return MOEQ_ERR_NOT_UPLOADED;
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    return from_cuda(launch_router(*L, x, T, topk_ids, topk_w, logits, (cudaStream_t)stream));
+}
+
+moeq_status moeq_forward_routed(moeq_layer_t L, const void *x, int32_t T, int32_t *topk_ids, float *topk_w,
+                                void *out, void *stream) {
+    if (!L || T < 0 || T > L->d.max_tokens) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (T == 0) return MOEQ_OK;
+    if (!x || !topk_ids || !topk_w || !out || ((uintptr_t)x & 3u) != 0) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (!L->uploaded) return MOEQ_ERR_NOT_UPLOADED;
+    if (!L->router || !L->router->ready) return MOEQ_ERR_NOT_UPLOADED;
+    DeviceGuard g(L->d.device);
+    if (g.err != cudaSuccess) return MOEQ_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = launch_router(*L, x, T, topk_ids, topk_w, nullptr, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    return launch_forward(L, x, topk_ids, topk_w, T, out, s);
 }
 
 moeq_status moeq_dequant(moeq_layer_t L, int32_t expert, int32_t proj, float *out, void *stream) {

@@ -85,8 +85,20 @@ struct PrefillVq {
     bool ready = false;
 };
 
+// Router of a layer (router.cu): the router matrix in the kernels' layout,
+// the partial logits of the K slices and the token tiles' arrival counters.
+struct RouterState {
+    uint4 *wfrag = nullptr;    // bf16 activations: three bf16 terms of Wr in tensor-core fragment order
+    float *wt = nullptr;       // f32 activations: Wr transposed, [H][E]
+    float *part = nullptr;     // [K slices][T][E] partial logits
+    int *counters = nullptr;   // [token tiles], zero between calls
+    int score = 0;             // moeq_score
+    bool ready = false;
+};
+
 struct Layer {
     moeq_layer_desc d{};
+    RouterState *router = nullptr;
     PrefillMx *pf = nullptr;
     PrefillVq *pv = nullptr;
     DevWeights w;
@@ -158,6 +170,10 @@ cudaError_t prefill_vq_create(Layer &L);
 void prefill_vq_free(Layer &L);
 cudaError_t launch_prefill_vq(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
                               cudaStream_t s, const cudaEvent_t *ev);
+cudaError_t router_upload(Layer &L, const float *wr, int score, cudaStream_t s);
+void router_free(Layer &L);
+cudaError_t launch_router(const Layer &L, const void *x, int T, int32_t *topk_ids, float *topk_w, float *logits,
+                          cudaStream_t s);
 cudaError_t launch_ffn_simt(const Layer &L, const void *x, const float *topk_w, int32_t n_tokens,
                             void *out, cudaStream_t s, const cudaEvent_t *ev);
 

@@ -30,7 +30,9 @@ GATE, UP, DOWN = 0, 1, 2
 # every symbol the header declares
 EXPORTS = ("moeq_layer_create", "moeq_upload_weights", "moeq_forward", "moeq_forward_host",
            "moeq_forward_profiled", "moeq_route", "moeq_dequant", "moeq_layer_status",
-           "moeq_status_string", "moeq_layer_destroy", "moeq_kernel_launches", "moeq_route_noalloc")
+           "moeq_status_string", "moeq_layer_destroy", "moeq_kernel_launches", "moeq_route_noalloc",
+           "moeq_router_upload", "moeq_router", "moeq_forward_routed")
+SCORE = {"sigmoid": 0, "softmax": 1}
 
 
 class LayerDesc(C.Structure):
@@ -55,6 +57,10 @@ _lib.moeq_forward_profiled.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_v
 _lib.moeq_route.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]
 _lib.moeq_route_noalloc.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p]
 _lib.moeq_dequant.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p]
+_lib.moeq_router_upload.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p]
+_lib.moeq_router.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
+_lib.moeq_forward_routed.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_void_p]
 _lib.moeq_layer_status.argtypes = [C.c_void_p, C.c_int32]
 _lib.moeq_status_string.argtypes = [C.c_int]
 _lib.moeq_status_string.restype = C.c_char_p
@@ -63,7 +69,8 @@ _lib.moeq_layer_destroy.restype = None
 _lib.moeq_kernel_launches.argtypes = [C.c_void_p]
 _lib.moeq_kernel_launches.restype = C.c_int64
 for _f in ("moeq_layer_create", "moeq_upload_weights", "moeq_forward", "moeq_forward_host", "moeq_dequant",
-           "moeq_layer_status", "moeq_forward_profiled", "moeq_route", "moeq_route_noalloc"):
+           "moeq_layer_status", "moeq_forward_profiled", "moeq_route", "moeq_route_noalloc",
+           "moeq_router_upload", "moeq_router", "moeq_forward_routed"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -219,6 +226,40 @@ class Layer:
         _check(_lib.moeq_dequant(self._h, expert, proj, C.c_void_p(out.data_ptr()), _stream_ptr(stream)),
                "moeq_dequant")
         return out
+
+    def router_upload(self, wr, score="sigmoid", stream=None):
+        """Router matrix ``wr``: host float32 [E][H]; ``score``: "sigmoid" or "softmax"."""
+        wr = np.ascontiguousarray(wr, dtype=np.float32)
+        assert wr.shape == (self.E, self.H)
+        _check(_lib.moeq_router_upload(self._h, wr.ctypes.data, SCORE[score], _stream_ptr(stream)),
+               "moeq_router_upload")
+
+    def router(self, x, want_logits=False, stream=None):
+        """(topk_ids int32 [T][k], topk_w float32 [T][k], logits float32 [T][E] or None), cuda tensors."""
+        import torch
+        assert x.is_cuda and x.is_contiguous()
+        T = x.shape[0]
+        ids = torch.empty((T, self.k), dtype=torch.int32, device=x.device)
+        w = torch.empty((T, self.k), dtype=torch.float32, device=x.device)
+        z = torch.empty((T, self.E), dtype=torch.float32, device=x.device) if want_logits else None
+        _check(_lib.moeq_router(self._h, C.c_void_p(x.data_ptr()), T, C.c_void_p(ids.data_ptr()),
+                                C.c_void_p(w.data_ptr()), C.c_void_p(z.data_ptr() if z is not None else 0),
+                                _stream_ptr(stream)), "moeq_router")
+        return ids, w, z
+
+    def forward_routed(self, x, out=None, stream=None):
+        """Router + forward: (out [T][H], topk_ids [T][k], topk_w [T][k]), cuda tensors."""
+        import torch
+        assert x.is_cuda and x.is_contiguous()
+        T = x.shape[0]
+        ids = torch.empty((T, self.k), dtype=torch.int32, device=x.device)
+        w = torch.empty((T, self.k), dtype=torch.float32, device=x.device)
+        if out is None:
+            out = torch.empty_like(x)
+        _check(_lib.moeq_forward_routed(self._h, C.c_void_p(x.data_ptr()), T, C.c_void_p(ids.data_ptr()),
+                                        C.c_void_p(w.data_ptr()), C.c_void_p(out.data_ptr()), _stream_ptr(stream)),
+               "moeq_forward_routed")
+        return out, ids, w
 
     def kernel_launches(self) -> int:
         return int(_lib.moeq_kernel_launches(self._h))

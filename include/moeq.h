@@ -68,6 +68,8 @@ typedef enum {
 typedef enum { MOEQ_FMT_MXFP4 = 0, MOEQ_FMT_VQ13 = 1, MOEQ_FMT_VQ13_R8 = 2 } moeq_format;
 typedef enum { MOEQ_ACT_F32 = 0, MOEQ_ACT_BF16 = 1 } moeq_dtype;
 typedef enum { MOEQ_GATE = 0, MOEQ_UP = 1, MOEQ_DOWN = 2 } moeq_proj;
+/* Routing weights of the router (moeq_router_upload). */
+typedef enum { MOEQ_SCORE_SIGMOID = 0, MOEQ_SCORE_SOFTMAX = 1 } moeq_score;
 
 typedef struct {
     int32_t hidden;      /* H: model width (K of gate/up, N of down)              */
@@ -220,6 +222,53 @@ MOEQ_API moeq_status moeq_route(moeq_layer_t layer, const int32_t *topk_ids, int
 MOEQ_API moeq_status moeq_route_noalloc(const int32_t *topk_ids, int32_t n_tokens, int32_t top_k,
                                         int32_t n_experts, int32_t *offsets_out, int32_t *perm_out,
                                         void *stream);
+
+/* The router that produces a forward's routing ("MiMo-V2.6-Flash-RL GGUF for
+ * a single DGX Spark", "Architecture notes": sigmoid routing, 8 of 256
+ * routed experts per token, no shared expert).  For token t:
+ *   z[t][e] = sum_h x[t][h] wr[e][h]                        (the logits)
+ *   topk_ids[t] = the top_k experts of largest z, in descending z, equal z
+ *                 to the lower expert id first
+ *   topk_w[t][j] = s_j / sum_i s_i over the selected experts, where
+ *                 s = 1 / (1 + e^-z) (MOEQ_SCORE_SIGMOID, the pages' router)
+ *                 or s = e^(z - z_max) (MOEQ_SCORE_SOFTMAX, a softmax over
+ *                 the selected logits)
+ * The pages give no more: the matrix shape, the selection on z (the sigmoid
+ * is increasing) and the normalisation over the selected experts are this
+ * library's readings.
+ *
+ * moeq_router_upload: copies the router matrix, host f32 [n_experts][hidden]
+ * row-major (every value finite and of magnitude <= 3.38e38), into the
+ * layer and fixes the weighting `score` (moeq_score).  The library stores it
+ * in its own layout and allocates, on first upload, the router's workspace
+ * (sized by max_tokens); the caller may free wr when the call returns (it
+ * synchronizes `stream`).  May be called again to replace the matrix.
+ * Errors: INVALID_ARGUMENT (NULL, unknown score, a non-finite or too large
+ * value), OUT_OF_MEMORY, CUDA. */
+MOEQ_API moeq_status moeq_router_upload(moeq_layer_t layer, const float *wr, int32_t score, void *stream);
+
+/* Run the router on x (device, the layer's act dtype, [n_tokens][hidden],
+ * 4-byte aligned) into topk_ids (device int32 [n_tokens][top_k]) and topk_w
+ * (device f32 [n_tokens][top_k]), and, when `logits` is not NULL, the logits
+ * themselves (device f32 [n_tokens][n_experts]).  The logits are accumulated
+ * in f32 from the exact f32 products of x and wr (for bf16 x the router
+ * matrix is held as three bf16 terms whose sum is wr to 24 bits); the sum
+ * over a row is split into K slices added in a fixed order, so results do
+ * not depend on timing.  The selection is taken on those f32 logits, the
+ * weights are computed in f32.  Asynchronous on `stream`; uses the router's
+ * workspace (calls on one layer must be ordered).
+ * Errors: INVALID_ARGUMENT (NULL, n_tokens outside [1, max_tokens],
+ * misaligned x), NOT_UPLOADED (no router matrix), CUDA. */
+MOEQ_API moeq_status moeq_router(moeq_layer_t layer, const void *x, int32_t n_tokens, int32_t *topk_ids,
+                                 float *topk_w, float *logits, void *stream);
+
+/* moeq_router followed by moeq_forward on the routing it produced: out =
+ * the layer output of x (both device, act dtype, [n_tokens][hidden]);
+ * topk_ids / topk_w are caller-owned device buffers that receive the
+ * routing.  n_tokens == 0 is a no-op.  Errors: as moeq_router and
+ * moeq_forward. */
+MOEQ_API moeq_status moeq_forward_routed(moeq_layer_t layer, const void *x, int32_t n_tokens, int32_t *topk_ids,
+                                         float *topk_w, void *out, void *stream);
 
 /* moeq_forward that also records five caller-created CUDA events (passed
  * as cudaEvent_t cast to void*) on `stream` at its phase boundaries:

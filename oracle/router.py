@@ -1,4 +1,4 @@
-"""Sigmoid router with top-k selection: the step that produces the routing the
+"""Router with top-k selection: the step that produces the routing the
 routed-expert path takes as input.
 
 TEST INFRASTRUCTURE ONLY, like the rest of this package: a plain float64
@@ -15,10 +15,16 @@ routing.  The pages say no more about the router; the readings taken here:
     keeps experts apart where their scores round to the same float64 value,
     and equal z go to the lower expert id first;
   - the routing weights are the selected scores divided by their sum.
+The synthetic workloads of the expert path draw their routing weights as a
+softmax over the k selected logits instead; ``score="softmax"`` gives that
+reading (weights exp(z_i) / sum over the selected j of exp(z_j)), with the
+same selection.
 """
 from __future__ import annotations
 
 import numpy as np
+
+SCORES = ("sigmoid", "softmax")
 
 
 def router_logits(x, Wr):
@@ -35,18 +41,33 @@ def router_logits(x, Wr):
     return z
 
 
-def router_topk(x, Wr, k: int):
-    """(topk_ids int32 [T][k], topk_w float32 [T][k], scores float64 [T][E])."""
-    z = router_logits(x, Wr)
+def topk_from_logits(z, k: int, score: str = "sigmoid"):
+    """The selection and weighting steps alone, on given logits z [T][E]
+    (any float type, compared as given): (ids int32 [T][k], w float64 [T][k]).
+    Descending z, equal z by ascending expert id; weights as in the module
+    docstring, computed in float64."""
+    assert score in SCORES
+    z = np.asarray(z)
     T, E = z.shape
     assert 1 <= k <= E
-    s = 1.0 / (1.0 + np.exp(-z))
     ids = np.empty((T, k), np.int32)
-    w = np.empty((T, k), np.float32)
+    w = np.empty((T, k), np.float64)
     for t in range(T):
-        # descending z, equal z by ascending expert id
         order = sorted(range(E), key=lambda e: (-z[t, e], e))[:k]
-        sel = s[t, order]
+        zs = np.array([float(z[t, e]) for e in order], np.float64)
+        if score == "sigmoid":
+            sel = 1.0 / (1.0 + np.exp(-zs))
+        else:
+            sel = np.exp(zs - zs[0])          # zs[0] is the largest selected logit
         ids[t] = order
-        w[t] = (sel / sel.sum()).astype(np.float32)
-    return ids, w, s
+        w[t] = sel / sel.sum()
+    return ids, w
+
+
+def router_topk(x, Wr, k: int, score: str = "sigmoid"):
+    """(topk_ids int32 [T][k], topk_w float32 [T][k], scores float64 [T][E]);
+    scores are the sigmoid of the logits for either weighting."""
+    z = router_logits(x, Wr)
+    s = 1.0 / (1.0 + np.exp(-z))
+    ids, w = topk_from_logits(z, k, score)
+    return ids, w.astype(np.float32), s

@@ -14,6 +14,7 @@ from .gen import (  # noqa: F401
     gen_layer,
     gen_routing,
     gen_activations,
+    gen_router,
     gen_disjoint_routing_schedule,
     bf16_bits_from_f32,
     f32_from_bf16_bits,

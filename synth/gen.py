@@ -25,6 +25,8 @@ component number alone, whatever else is drawn):
   uniform random bytes.
 * component 30+p -- projection p's optional f16 row gains, uniform in
   [0.5, 2) rounded to f16.
+* component 40  -- router matrix Wr [E][H] float32 ~ N(0, 1/H), so that with
+  N(0,1) activations the router logits are about N(0,1).
 
 Projections are p = 0 gate [I][H], 1 up [I][H], 2 down [H][I]; rows are
 output features and K (the reduction axis) is contiguous.
@@ -254,6 +256,11 @@ def gen_disjoint_routing_schedule(cfg: LayerCfg, n_steps: int, seed: int = 0):
         ids[i, 0] = sets[i % n_sets]
         w[i, 0] = _softmax64(top)
     return ids, w
+
+
+def gen_router(cfg: LayerCfg, seed: int = 0) -> np.ndarray:
+    """Router matrix Wr float32 [E][H] (component 40)."""
+    return _rng(seed, 40).normal(0.0, 1.0 / np.sqrt(cfg.H), size=(cfg.E, cfg.H)).astype(np.float32)
 
 
 def gen_activations(cfg: LayerCfg, seed: int = 0, T: Optional[int] = None) -> np.ndarray:

@@ -4,7 +4,7 @@ import math
 
 import numpy as np
 
-from oracle.router import router_topk
+from oracle.router import router_topk, topk_from_logits
 
 
 def test_zero_activations_tie_every_expert():
@@ -79,3 +79,37 @@ def test_weights_normalised_distinct_and_descending():
     np.testing.assert_allclose(w.sum(axis=1), 1.0, atol=1e-6)
     assert (np.diff(w, axis=1) <= 0).all()
     assert all(len(set(r)) == 8 for r in ids.tolist())
+
+
+def test_softmax_weighting_hand_example():
+    # z = (ln 3, 0, -ln 3), k = 2: softmax over the selected (ln 3, 0) gives
+    # (3/4, 1/4); the sigmoid reading gives (3/4, 1/2) / (5/4) = (0.6, 0.4)
+    Wr = np.array([[1.0], [0.0], [-1.0]])
+    x = np.array([[math.log(3.0)]])
+    ids, w, _ = router_topk(x, Wr, 2, score="softmax")
+    assert ids.tolist() == [[0, 1]]
+    np.testing.assert_allclose(w[0], [0.75, 0.25], rtol=1e-7)
+    ids2, w2, _ = router_topk(x, Wr, 2, score="sigmoid")
+    assert ids2.tolist() == [[0, 1]]
+    np.testing.assert_allclose(w2[0], [0.6, 0.4], rtol=1e-7)
+
+
+def test_softmax_weighting_matches_the_workload_generator():
+    # the expert path's synthetic routing (uniform) draws N(0,1) logits over E,
+    # keeps the k largest and softmaxes them: the oracle's softmax reading on
+    # those logits must give the same ids and weights
+    import synth
+    cfg = synth.get_cfg("decode_mxfp4", T=6)
+    ids_g, w_g = synth.gen_routing(cfg, seed=9)
+    logits = synth.gen._rng(9, 0).normal(0.0, 1.0, size=(cfg.T, cfg.E))
+    ids, w = topk_from_logits(logits, cfg.k, "softmax")
+    assert np.array_equal(ids, ids_g)
+    np.testing.assert_allclose(w, w_g, rtol=1e-6)
+
+
+def test_selection_uses_the_given_logits_exactly():
+    # two logits one float32 ulp apart are ordered as given, ties by id
+    z = np.array([[1.0, np.nextafter(np.float32(1.0), np.float32(2.0)), 1.0, -3.0]], np.float32)
+    ids, w = topk_from_logits(z, 3)
+    assert ids.tolist() == [[1, 0, 2]]
+    assert abs(w.sum() - 1.0) < 1e-15
