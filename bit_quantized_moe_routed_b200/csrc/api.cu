@@ -85,6 +85,8 @@ void free_layer(moeq_layer *L) {
     cudaFree(L->acc);
     cudaFree(L->dec_ybuf);
     cudaFree(L->dec_counters);
+    cudaFree(L->vq_acc);
+    cudaFree(L->vq_done);
     cudaFree(L->status);
     cudaFree(L->x_stage);
     cudaFree(L->out_stage);
@@ -124,6 +126,9 @@ moeq_status launch_forward(moeq_layer *L, const void *x, const int32_t *ids, con
     // the prefill kernels read x rows as 16-byte vectors
     if (prefill_mx_supported(*L, T) && ((uintptr_t)x & 15u) == 0)
         return from_cuda(launch_prefill_mx(*L, x, ids, w, T, out, s, ev));
+    // the VQ decode kernels also store out as 8-byte vectors
+    if (decode_vq_supported(*L, T) && ((uintptr_t)x & 15u) == 0 && ((uintptr_t)out & 7u) == 0)
+        return from_cuda(launch_decode_vq(*L, x, ids, w, T, out, s, ev));
     if (prefill_vq_supported(*L, T) && ((uintptr_t)x & 15u) == 0)
         return from_cuda(launch_prefill_vq(*L, x, ids, w, T, out, s, ev));
     cudaError_t e = launch_route_bucket(*L, ids, T * L->d.top_k, L->b.offsets, L->b.perm, L->b.active, s);
@@ -194,6 +199,8 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     if (fmt != MOEQ_FMT_MXFP4) {
         ALLOC(L->w.book13, sizeof(uint16_t) * kBook13Rows * 8);
         if (fmt == MOEQ_FMT_VQ13_R8) ALLOC(L->w.book8, sizeof(uint16_t) * kBook8Rows * 8);
+        ALLOC(L->vq_acc, sizeof(float) * kDecMaxTokens * H);
+        ALLOC(L->vq_done, sizeof(int));
     }
     ALLOC(L->b.offsets, sizeof(int32_t) * (E + 1));
     ALLOC(L->b.active, sizeof(int32_t) * (E + 1));
@@ -212,6 +219,8 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     if (e == cudaSuccess) e = prefill_vq_create(*L);
     if (e == cudaSuccess) e = cudaMemset(L->status, 0, sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMemset(L->dec_counters, 0, sizeof(int) * (H / 32 + 1));
+    if (e == cudaSuccess && L->vq_acc) e = cudaMemset(L->vq_acc, 0, sizeof(float) * kDecMaxTokens * H);
+    if (e == cudaSuccess && L->vq_done) e = cudaMemset(L->vq_done, 0, sizeof(int));
     if (e != cudaSuccess) {
         free_layer(L);
         cudaGetLastError();  // clear a sticky allocation error

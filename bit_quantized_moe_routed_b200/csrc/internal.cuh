@@ -108,6 +108,8 @@ struct Layer {
     // decode fast path scratch
     float *dec_ybuf = nullptr;     // [kDecMaxRoutes][kDecMaxTokens][H] per-expert partial outputs
     int *dec_counters = nullptr;   // [H/32] per-tile arrival counters, zero between calls
+    float *vq_acc = nullptr;       // VQ decode: [kDecMaxTokens][H] f32 combine accumulator, zero between calls
+    int *vq_done = nullptr;        // VQ decode: CTA arrival counter of the down kernel, zero between calls
     uint32_t *status = nullptr;
     // staging for moeq_forward_host
     void *x_stage = nullptr;
@@ -165,6 +167,9 @@ cudaError_t launch_prefill_mx(const Layer &L, const void *x, const int32_t *ids,
                               cudaStream_t s, const cudaEvent_t *ev);
 // tile_base[e] = sum over e' < e of ceil(n_e' / 64) (the route tiles of the tensor-core paths)
 cudaError_t launch_route_tiles(const int32_t *offsets, int E, int32_t *tile_base, cudaStream_t s);
+bool decode_vq_supported(const Layer &L, int T);
+cudaError_t launch_decode_vq(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
+                             cudaStream_t s, const cudaEvent_t *ev);
 bool prefill_vq_supported(const Layer &L, int T);
 cudaError_t prefill_vq_create(Layer &L);
 void prefill_vq_free(Layer &L);

@@ -27,11 +27,12 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 # one layer per kernel family: decode MXFP4 (grouped GEMV), tensor-core
-# MXFP4, tensor-core VQ13+R8, f32 (SIMT, no device waits)
+# MXFP4, tensor-core VQ13+R8, decode VQ13+R8 (grouped GEMV)
 FAMILIES = {
     "decode_mxfp4": dict(fmt="mxfp4", act="bf16", H=2048, I=2048, E=16, k=8, T=4),
     "prefill_mxfp4": dict(fmt="mxfp4", act="bf16", H=1024, I=512, E=16, k=4, T=300),
     "vq13r8": dict(fmt="vq13r8", act="bf16", H=1024, I=512, E=16, k=4, T=300),
+    "decode_vq13r8": dict(fmt="vq13r8", act="bf16", H=2048, I=2048, E=16, k=8, T=4),
 }
 
 
@@ -72,8 +73,10 @@ _ALLOC_CHILD = textwrap.dedent("""
     torch.cuda.set_device(0)
     from bit_quantized_moe_routed_b200 import moeq
     free0 = torch.cuda.mem_get_info()[0]
+    created = False
     try:
         lay = moeq.Layer(1024, 1024, 64, 8, {max_tokens}, {fmt!r}, "bf16")
+        created = True
         print("CREATED")
         lay.close()
     except moeq.MoeqError as e:
@@ -81,8 +84,10 @@ _ALLOC_CHILD = textwrap.dedent("""
     torch.cuda.synchronize()
     free1 = torch.cuda.mem_get_info()[0]
     print("LEAK", free0 - free1)
-    lay = moeq.Layer(1024, 1024, 64, 8, {max_tokens}, {fmt!r}, "bf16")   # the next create succeeds
-    lay.close()
+    if not created:
+        # the injected failure was used up: the next create succeeds
+        lay = moeq.Layer(1024, 1024, 64, 8, {max_tokens}, {fmt!r}, "bf16")
+        lay.close()
     print("DONE")
 """)
 

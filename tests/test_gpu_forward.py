@@ -277,3 +277,61 @@ def test_decode_mxfp4_token_lists_an_expert_twice(T):
     out = run(lay, cfg, x, ids, w)
     assert lay.kernel_launches() - n0 == 2        # the decode kernels
     assert_close(out, oracle_ref(L, x, ids, w), "bf16", f"repeated experts, T={T}")
+
+
+# decode-sized VQ layers (1..8 tokens, bf16): the VQ grouped-GEMV kernels
+VQ_DECODE = [
+    dict(H=2048, I=2048, E=16, k=2, T=1),
+    dict(H=2048, I=2048, E=8, k=8, T=8),      # every expert gets 8 routes
+    dict(H=2048, I=4096, E=32, k=8, T=3),
+    dict(H=4096, I=2048, E=64, k=8, T=8),
+    dict(H=4096, I=4096, E=16, k=4, T=2),
+]
+
+
+@pytest.mark.parametrize("fmt,gains", [("vq13", False), ("vq13r8", True)])
+@pytest.mark.parametrize("shape", VQ_DECODE, ids=[f"H{s['H']}I{s['I']}E{s['E']}k{s['k']}T{s['T']}" for s in VQ_DECODE])
+def test_decode_vq_shapes(shape, fmt, gains):
+    cfg = synth.get_cfg("decode_vq", fmt=fmt, gains=gains, **shape)
+    L = synth.gen_layer(cfg, seed=35)
+    x = synth.gen_activations(cfg, seed=35)
+    ids, w = synth.gen_routing(cfg, seed=35)
+    lay = dev_layer(L)
+    n0 = lay.kernel_launches()
+    out = run(lay, cfg, x, ids, w)
+    assert lay.kernel_launches() - n0 == 2        # the two VQ decode kernels
+    assert_close(out, oracle_ref(L, x, ids, w), "bf16", f"{fmt} {shape}")
+    # a second call with another routing: the accumulator and the arrival
+    # counter must have been cleared by the first
+    ids2, w2 = synth.gen_routing(cfg, seed=36)
+    out2 = run(lay, cfg, x, ids2, w2)
+    assert_close(out2, oracle_ref(L, x, ids2, w2), "bf16", f"{fmt} {shape} second call")
+
+
+def test_decode_vq_duplicates_no_routes_and_extremes():
+    from bit_quantized_moe_routed_b200 import moeq
+    cfg = synth.get_cfg("decode_vq", H=2048, I=2048, E=4, k=4, T=8, gains=True)
+    L = synth.gen_layer(cfg, seed=37)
+    x = synth.gen_activations(cfg, seed=37)
+    rng = np.random.default_rng(37)
+    ids = rng.integers(0, 2, size=(cfg.T, cfg.k)).astype(np.int32)   # repeats within tokens
+    ids[3, :] = -1
+    ids[5, 2] = -1
+    ids[6, 1] = cfg.E + 2                                             # out of range: skipped, reported
+    w = rng.normal(size=(cfg.T, cfg.k)).astype(np.float32)
+    xf = synth.f32_from_bf16_bits(x)
+    xf[1] = 0.0
+    xf[4] *= 2.0 ** 30
+    xf[7] *= 2.0 ** -50
+    x = synth.bf16_bits_from_f32(xf)
+    lay = dev_layer(L)
+    out = run(lay, cfg, x, ids, w)
+    assert lay.status(clear=True) == moeq.ROUTE_OUT_OF_RANGE
+    w_ref = w.copy()
+    w_ref[6, 1] = 0.0
+    ref = oracle_ref(L, x, np.where(ids < cfg.E, ids, -1), w_ref)
+    assert not out[1].any() and not out[3].any()
+    assert_close(out, ref, "bf16", "vq duplicates/extremes")
+    out0 = run(lay, cfg, x, np.full_like(ids, -1), w)
+    assert not out0.any()
+    assert lay.status() == moeq.OK
