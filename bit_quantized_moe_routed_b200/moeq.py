@@ -31,7 +31,7 @@ GATE, UP, DOWN = 0, 1, 2
 EXPORTS = ("moeq_layer_create", "moeq_upload_weights", "moeq_forward", "moeq_forward_host",
            "moeq_forward_profiled", "moeq_route", "moeq_dequant", "moeq_layer_status",
            "moeq_status_string", "moeq_layer_destroy", "moeq_kernel_launches", "moeq_route_noalloc",
-           "moeq_router_upload", "moeq_router", "moeq_forward_routed")
+           "moeq_router_upload", "moeq_router", "moeq_forward_routed", "moeq_vq_encode")
 SCORE = {"sigmoid": 0, "softmax": 1}
 
 
@@ -61,6 +61,8 @@ _lib.moeq_router_upload.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_
 _lib.moeq_router.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
 _lib.moeq_forward_routed.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p,
                                      C.c_void_p]
+_lib.moeq_vq_encode.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                C.c_void_p, C.c_void_p, C.c_void_p]
 _lib.moeq_layer_status.argtypes = [C.c_void_p, C.c_int32]
 _lib.moeq_status_string.argtypes = [C.c_int]
 _lib.moeq_status_string.restype = C.c_char_p
@@ -70,7 +72,7 @@ _lib.moeq_kernel_launches.argtypes = [C.c_void_p]
 _lib.moeq_kernel_launches.restype = C.c_int64
 for _f in ("moeq_layer_create", "moeq_upload_weights", "moeq_forward", "moeq_forward_host", "moeq_dequant",
            "moeq_layer_status", "moeq_forward_profiled", "moeq_route", "moeq_route_noalloc",
-           "moeq_router_upload", "moeq_router", "moeq_forward_routed"):
+           "moeq_router_upload", "moeq_router", "moeq_forward_routed", "moeq_vq_encode"):
     getattr(_lib, _f).restype = C.c_int
 
 
@@ -116,6 +118,23 @@ def route_noalloc(topk_ids, n_experts, offsets_out, perm_out, stream=None):
     _check(_lib.moeq_route_noalloc(C.c_void_p(topk_ids.data_ptr()), T, k, n_experts,
                                    C.c_void_p(offsets_out.data_ptr()), C.c_void_p(perm_out.data_ptr()),
                                    _stream_ptr(stream)), "moeq_route_noalloc")
+
+
+def vq_encode(w, book13, book8=None, gain=None, col_weight=None, stream=None):
+    """moeq_vq_encode on cuda tensors: w float32 [N][K]; book13 / book8
+    bf16 bit patterns (int16 or uint16 tensors) [8192][8] / [256][8]; gain
+    f16 bit patterns [N] or None; col_weight float32 [K] or None.  Returns
+    (idx13 uint8 [N][K*13/64], idx8 uint8 [N][K/8] or None)."""
+    import torch
+    N, K = w.shape
+    idx13 = torch.empty((N, K * 13 // 64), dtype=torch.uint8, device=w.device)
+    idx8 = torch.empty((N, K // 8), dtype=torch.uint8, device=w.device) if book8 is not None else None
+
+    def p(t):
+        return C.c_void_p(t.data_ptr() if t is not None else 0)
+    _check(_lib.moeq_vq_encode(p(w), N, K, p(gain), p(col_weight), p(book13), p(book8), p(idx13), p(idx8),
+                               _stream_ptr(stream)), "moeq_vq_encode")
+    return idx13, idx8
 
 
 class Layer:

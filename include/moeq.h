@@ -270,6 +270,39 @@ MOEQ_API moeq_status moeq_router(moeq_layer_t layer, const void *x, int32_t n_to
 MOEQ_API moeq_status moeq_forward_routed(moeq_layer_t layer, const void *x, int32_t n_tokens, int32_t *topk_ids,
                                          float *topk_w, void *out, void *stream);
 
+/* VQ encoder: the indices that store a matrix in the VQ13 / VQ13_R8 format
+ * ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe": every 8 consecutive
+ * weights of an expert row become one index into the layer's codebook,
+ * times one f16 row gain; a 256-entry residual book codes what the first
+ * stage left, and the 13-bit stage is byte-identical with and without it;
+ * assignment minimises an importance-weighted error with per-column
+ * weights).  The codebooks, gains and column weights are given; training
+ * them is not part of this library.
+ *   w           device f32 [n_rows][n_cols], row-major, 16-byte aligned;
+ *               n_cols a multiple of 64
+ *   gain        device f16 [n_rows] row gains, or NULL (gain 1)
+ *   col_weight  device f32 [n_cols] importance of each column (>= 0), or
+ *               NULL (all 1)
+ *   book13      device bf16 [8192][8], 16-byte aligned
+ *   book8       device bf16 [256][8], 16-byte aligned, or NULL (no residual
+ *               stage; then idx8_out must be NULL too)
+ *   idx13_out   device uint8 [n_rows][n_cols*13/64]: per row, the 13-bit
+ *               indices as the little-endian bitstream of moeq_weights
+ *   idx8_out    device uint8 [n_rows][n_cols/8], 8-byte aligned: residual
+ *               indices, or NULL
+ * For vector j of row n (columns 8j..8j+7) the base index c minimises
+ * sum_i col_weight_i (w_i - g book13[c][i])^2 (g the row's gain); then, for
+ * that c, the residual index r minimises sum_i col_weight_i
+ * (w_i - g (book13[c][i] + book8[r][i]))^2.  The errors are evaluated in f32
+ * in the expanded form g^2 sum cw b^2 - 2 g sum (cw w) b; ties go to the
+ * lowest index; the base index does not depend on the residual stage.
+ * Every output byte of the rows is written; the call allocates nothing and
+ * is asynchronous on `stream` (current device).  Errors: INVALID_ARGUMENT
+ * (NULL, sizes, alignment, book8 without idx8_out or the reverse), CUDA. */
+MOEQ_API moeq_status moeq_vq_encode(const float *w, int32_t n_rows, int32_t n_cols, const uint16_t *gain,
+                                    const float *col_weight, const uint16_t *book13, const uint16_t *book8,
+                                    uint8_t *idx13_out, uint8_t *idx8_out, void *stream);
+
 /* moeq_forward that also records five caller-created CUDA events (passed
  * as cudaEvent_t cast to void*) on `stream` at its phase boundaries:
  * events[0] before the first launch, [1] after route/bucket, [2] after the
