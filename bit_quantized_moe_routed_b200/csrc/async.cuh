@@ -86,6 +86,24 @@ __device__ __forceinline__ bool mbar_wait_abort(uint64_t *bar, uint32_t parity, 
     return true;
 }
 
+// mbar_wait_abort with non-suspending probes (test_wait): for a wait that
+// the whole CTA makes once, where a suspended thread would only add
+// latency; with a short limit it gives up as soon as the phase is not
+// complete.
+__device__ __forceinline__ bool mbar_poll_abort(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                long long max_cycles) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_test_wait(bar, parity)) {
+        if (*abort) return false;
+        if (clock64() - t0 > max_cycles) {
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
 // The limit of the drains that run before a CTA exits (its own copies in
 // flight, its own tensor-core operations): fixed and long, so that no
 // asynchronous operation outlives the CTA whatever limit the other waits

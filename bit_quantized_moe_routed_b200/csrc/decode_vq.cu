@@ -88,18 +88,6 @@ __device__ void build_cols(ColTable &ct, const RouteTable &tb) {
     }
 }
 
-// Both books into shared memory with bulk copies (warp 0), on `bar`.
-__device__ void load_books(uint8_t *b13, uint8_t *b8, const VqdArgs &a, uint64_t *bar) {
-    const int lane = threadIdx.x & 31;
-    if (lane == 0) mbar_arrive_expect_tx(bar, kB13Bytes + (a.book8 ? kB8Bytes : 0));
-    __syncwarp();
-    if (lane < 4)
-        bulk_g2s(b13 + lane * (kB13Bytes / 4), reinterpret_cast<const uint8_t *>(a.book13) + lane * (kB13Bytes / 4),
-                 kB13Bytes / 4, bar);
-    if (lane == 4 && a.book8) bulk_g2s(b8, a.book8, kB8Bytes, bar);
-    __syncwarp();
-}
-
 // Skewed staging of a row of K values split into 32 lane chunks of 8 VPL:
 // element c at c + 8 (c / (8 VPL)), so chunk l starts at 8 l (VPL + 1).
 template <int VPL>
@@ -158,20 +146,6 @@ __device__ __forceinline__ uint32_t hadd2_bf16(uint32_t a, uint32_t b) {
     asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
-// The 8 weights of a vector: base (+ residual) as bf16 pairs.
-template <bool R8>
-__device__ __forceinline__ uint4 codeword(const uint8_t *b13, const uint8_t *b8, uint32_t c, uint32_t r) {
-    uint4 v = lds128(b13 + 16u * c);
-    if constexpr (R8) {
-        const uint4 q = lds128(b8 + 16u * r);
-        v.x = hadd2_bf16(v.x, q.x);
-        v.y = hadd2_bf16(v.y, q.y);
-        v.z = hadd2_bf16(v.z, q.z);
-        v.w = hadd2_bf16(v.w, q.w);
-    }
-    return v;
-}
-
 // (acc0, acc1) += (a.lo, a.hi) * (b.lo, b.hi) for bf16 pairs a, b, in f32.
 __device__ __forceinline__ void dot2(float &acc0, float &acc1, uint32_t a, uint32_t b) {
     asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
@@ -200,6 +174,59 @@ __device__ __forceinline__ void warp_range(int n, int &i0, int &i1) {
     i1 = (int)(n * (gw + 1) / nw);
 }
 
+// ---------------------------------------------------------------- books
+
+// Shared-memory bytes of the books; with RI the residual book is stored 8
+// times, copy q in 16-byte bank group q only (entry r of copy q at
+// (8 r + q) * 16), and lane l reads copy l % 8: the 8 lanes of a quarter
+// warp then never share a bank group, however random their indices.
+template <bool R8, bool RI>
+constexpr int books_bytes() { return kB13Bytes + (R8 ? (RI ? 8 * kB8Bytes : kB8Bytes) : 0); }
+// Staged-operand bytes of each kernel for K = 256 VPL.
+constexpr int gu_stage_bytes(int TB, int VPL) { return TB * (256 * VPL + 256) * 2; }
+constexpr int dn_stage_bytes(int TB, int VPL) { return 2 * TB * (256 * VPL + 256) * 2; }
+// The residual book interleaved when it and the staged operands fit.
+template <int VPL, bool R8, int TB, bool DOWN>
+constexpr bool use_ri() {
+    return R8 && books_bytes<true, true>() + (DOWN ? dn_stage_bytes(TB, VPL) : gu_stage_bytes(TB, VPL)) <= kVMaxSmem;
+}
+
+// Both books into shared memory (warp 0): the base book by bulk copies on
+// `bar`; the residual book by the same copy, or, interleaved (RI), by the
+// whole CTA with plain loads (call fill_ri after the barrier's init).
+template <bool RI>
+__device__ void load_books(uint8_t *b13, uint8_t *b8, const VqdArgs &a, uint64_t *bar) {
+    const int lane = threadIdx.x & 31;
+    const bool copy8 = a.book8 && !RI;
+    if (lane == 0) mbar_arrive_expect_tx(bar, kB13Bytes + (copy8 ? kB8Bytes : 0));
+    __syncwarp();
+    if (lane < 4)
+        bulk_g2s(b13 + lane * (kB13Bytes / 4), reinterpret_cast<const uint8_t *>(a.book13) + lane * (kB13Bytes / 4),
+                 kB13Bytes / 4, bar);
+    if (lane == 4 && copy8) bulk_g2s(b8, a.book8, kB8Bytes, bar);
+    __syncwarp();
+}
+__device__ void fill_ri(uint8_t *b8, const uint16_t *book8) {
+    for (int i = threadIdx.x; i < kBook8Rows * 8; i += kVThreads) {
+        const int r = i >> 3, q = i & 7;
+        reinterpret_cast<uint4 *>(b8)[8 * r + q] = __ldg(reinterpret_cast<const uint4 *>(book8) + r);
+    }
+}
+
+// The 8 weights of a vector: base (+ residual) as bf16 pairs.
+template <bool R8, bool RI>
+__device__ __forceinline__ uint4 codeword2(const uint8_t *b13, const uint8_t *b8, uint32_t c, uint32_t r, int q8) {
+    uint4 v = lds128(b13 + 16u * c);
+    if constexpr (R8) {
+        const uint4 q = lds128(b8 + 16u * (RI ? 8u * r + (uint32_t)q8 : r));
+        v.x = hadd2_bf16(v.x, q.x);
+        v.y = hadd2_bf16(v.y, q.y);
+        v.z = hadd2_bf16(v.z, q.z);
+        v.w = hadd2_bf16(v.w, q.w);
+    }
+    return v;
+}
+
 // ---------------------------------------------------------------- gate/up
 
 template <int VPL, bool R8>
@@ -208,13 +235,69 @@ struct GURow {
     Idx8<VPL> g8, u8;
 };
 
+// Shared state of a CTA that the per-row work reads.
+struct VqdShared {
+    RouteTable tb;
+    ColTable ct;
+};
+
+// One gate/up row pair for an expert with NC token columns: the dot
+// products over the lane's stretch, the warp sums, SwiGLU, h.
+// Columns j0 .. j0 + NC - 1 (at most four per pass: more would not fit the
+// registers; a fifth to eighth column takes a second pass over the row).
+// The index words must be aligned (Idx13::align) before the first pass.
+template <int VPL, bool R8, bool RI, int NC>
+__device__ __forceinline__ void gu_row(const VqdArgs &a, const VqdShared &s, const uint8_t *b13, const uint8_t *b8,
+                                       const uint16_t *xs, int xstride, int chunk, int d, int n, int j0,
+                                       const GURow<VPL, R8> &r) {
+    const int lane = threadIdx.x & 31, q8 = lane & 7, I = a.I;
+    float ag[NC][2], au[NC][2];
+    const uint16_t *xr[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+        ag[j][0] = ag[j][1] = au[j][0] = au[j][1] = 0.f;
+        xr[j] = xs + (size_t)s.ct.tok[d][j0 + j] * xstride + chunk;
+    }
+#pragma unroll
+    for (int m = 0; m < VPL; ++m) {
+        uint32_t rg = 0, ru = 0;
+        if constexpr (R8) {
+            rg = r.g8.get(m);
+            ru = r.u8.get(m);
+        }
+        const uint4 wg = codeword2<R8, RI>(b13, b8, r.g13.get(m), rg, q8);
+        const uint4 wu = codeword2<R8, RI>(b13, b8, r.u13.get(m), ru, q8);
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+            const uint4 xv = lds128(xr[j] + 8 * m);
+            dot8(ag[j], wg, xv);
+            dot8(au[j], wu, xv);
+        }
+    }
+    const size_t row = (size_t)s.tb.expert[d] * I + n;
+    const float gg = a.gain[0] ? f16_bits_to_f32(__ldg(a.gain[0] + row)) : 1.f;
+    const float gu = a.gain[1] ? f16_bits_to_f32(__ldg(a.gain[1] + row)) : 1.f;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+        const float g = warp_sum(ag[j][0] + ag[j][1]) * gg;
+        const float u = warp_sum(au[j][0] + au[j][1]) * gu;
+        const float hv = silu_f32(g) * u;
+        // every route of (expert d, token of column j0 + j)
+        const int tk = s.ct.tok[d][j0 + j];
+        for (int c = s.tb.col_beg[d] + lane; c < s.tb.col_beg[d + 1]; c += 32) {
+            const int rt = s.tb.route[c];
+            if (s.tb.tok[rt] == tk) a.h[(size_t)rt * I + n] = hv;
+        }
+    }
+}
+
 template <int VPL, bool R8, int TB>   // VPL = H / 256; TB >= tokens
 __global__ void __launch_bounds__(kVThreads, 1) vqd_gateup_kernel(VqdArgs a) {
+    constexpr bool RI = use_ri<VPL, R8, TB, false>();
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *b13 = smem, *b8 = smem + kB13Bytes;
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem + kB13Bytes + kB8Bytes);
-    __shared__ RouteTable tb;
-    __shared__ ColTable ct;
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem + books_bytes<R8, RI>());
+    __shared__ VqdShared s;
     __shared__ __align__(8) uint64_t bar;
     const int H = a.H, I = a.I, T = a.T;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -224,13 +307,14 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_gateup_kernel(VqdArgs a) {
         mbar_fence_init();
     }
     __syncthreads();
-    // the books are weights: stream them before waiting for the previous kernel
-    if (warp == 0) load_books(b13, b8, a, &bar);
+    // the books are weights: fetch them before waiting for the previous kernel
+    if (warp == 0) load_books<RI>(b13, b8, a, &bar);
+    if constexpr (RI) fill_ri(b8, a.book8);
     pdl_wait_primary();
     if (warp == 0) {
-        build_route_table(tb, a.ids, a.topk_w, T * a.k, a.k, a.E, a.status, blockIdx.x == 0);
+        build_route_table(s.tb, a.ids, a.topk_w, T * a.k, a.k, a.E, a.status, blockIdx.x == 0);
         __syncwarp();
-        build_cols(ct, tb);
+        build_cols(s.ct, s.tb);
     }
     // activations, bf16, skewed rows
     for (int i = threadIdx.x; i < T * (H / 8); i += kVThreads) {
@@ -240,21 +324,20 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_gateup_kernel(VqdArgs a) {
     }
     volatile int abort_flag = 0;
     // block-uniform: the warps' shuffles below need every lane
-    const bool books_ok = __syncthreads_and(mbar_wait_abort(&bar, 0, &abort_flag, a.wait_cycles));
+    const bool books_ok = __syncthreads_and(mbar_poll_abort(&bar, 0, &abort_flag, a.wait_cycles));
     pdl_launch_dependents();
     if (!books_ok) {
-        if (lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
+        if (threadIdx.x == 0) atomicOr(a.status, FLAG_TIMEOUT);
         return;
     }
 
     const int RB13 = H * 13 / 64, RB8 = H / 8;
     const int lI = 31 - __clz(I);
     int i0, i1;
-    warp_range(tb.D * I, i0, i1);
+    warp_range(s.tb.D * I, i0, i1);
     const int chunk = skew_pos<VPL>(lane * 8 * VPL);   // this lane's columns in a staged row
     auto load = [&](int i, GURow<VPL, R8> &r) {
-        const int d = i >> lI, n = i & (I - 1);
-        const size_t row = (size_t)tb.expert[d] * I + n;
+        const size_t row = (size_t)s.tb.expert[i >> lI] * I + (i & (I - 1));
         r.g13.load(a.idx13[0] + row * RB13, lane);
         r.u13.load(a.idx13[1] + row * RB13, lane);
         if constexpr (R8) {
@@ -264,48 +347,20 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_gateup_kernel(VqdArgs a) {
     };
     auto compute = [&](int i, GURow<VPL, R8> &r) {
         const int d = i >> lI, n = i & (I - 1);
-        const int ncol = ct.ncol[d];
         r.g13.align();
         r.u13.align();
-        float ag[TB][2], au[TB][2];
-#pragma unroll
-        for (int j = 0; j < TB; ++j) ag[j][0] = ag[j][1] = au[j][0] = au[j][1] = 0.f;
-        const uint16_t *xr[TB];
-#pragma unroll
-        for (int j = 0; j < TB; ++j) xr[j] = xs + (size_t)(j < ncol ? ct.tok[d][j] : 0) * xstride + chunk;
-#pragma unroll
-        for (int m = 0; m < VPL; ++m) {
-            uint32_t rg = 0, ru = 0;
-            if constexpr (R8) {
-                rg = r.g8.get(m);
-                ru = r.u8.get(m);
-            }
-            const uint4 wg = codeword<R8>(b13, b8, r.g13.get(m), rg);
-            const uint4 wu = codeword<R8>(b13, b8, r.u13.get(m), ru);
-#pragma unroll
-            for (int j = 0; j < TB; ++j) {
-                if (j < ncol) {
-                    const uint4 xv = lds128(xr[j] + 8 * m);
-                    dot8(ag[j], wg, xv);
-                    dot8(au[j], wu, xv);
-                }
-            }
+        // the expert's column count, a compile-time constant inside
+        const int nc = s.ct.ncol[d];
+        if (nc > 4) {
+            if constexpr (TB >= 8) gu_row<VPL, R8, RI, 4>(a, s, b13, b8, xs, xstride, chunk, d, n, 0, r);
         }
-        const size_t row = (size_t)tb.expert[d] * I + n;
-        const float gg = a.gain[0] ? f16_bits_to_f32(__ldg(a.gain[0] + row)) : 1.f;
-        const float gu = a.gain[1] ? f16_bits_to_f32(__ldg(a.gain[1] + row)) : 1.f;
-#pragma unroll
-        for (int j = 0; j < TB; ++j) {
-            if (j >= ncol) break;
-            const float g = warp_sum(ag[j][0] + ag[j][1]) * gg;
-            const float u = warp_sum(au[j][0] + au[j][1]) * gu;
-            const float hv = silu_f32(g) * u;
-            // every route of (expert d, token of column j)
-            const int tk = ct.tok[d][j];
-            for (int c = tb.col_beg[d] + lane; c < tb.col_beg[d + 1]; c += 32) {
-                const int rt = tb.route[c];
-                if (tb.tok[rt] == tk) a.h[(size_t)rt * I + n] = hv;
-            }
+        const int j0 = nc > 4 ? 4 : 0;
+        switch (nc - j0) {
+            case 1: gu_row<VPL, R8, RI, 1>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
+            case 2: if constexpr (TB >= 2) gu_row<VPL, R8, RI, 2>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
+            case 3: if constexpr (TB >= 4) gu_row<VPL, R8, RI, 3>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
+            case 4: if constexpr (TB >= 4) gu_row<VPL, R8, RI, 4>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
+            default: break;
         }
     };
     GURow<VPL, R8> ra, rb;
@@ -327,13 +382,40 @@ struct DNRow {
     Idx8<VPL> c8;
 };
 
+// One output row m of expert slot d (staged columns at vr) for NC columns:
+// the dot products, the warp sums, one atomic per (row, token).
+template <int VPL, bool R8, bool RI, int NC>
+__device__ __forceinline__ void dn_row(const VqdArgs &a, const VqdShared &s, const uint8_t *b13, const uint8_t *b8,
+                                       const uint16_t *vr, int vstride, int d, int m, int j0, const DNRow<VPL, R8> &r) {
+    const int lane = threadIdx.x & 31, q8 = lane & 7, H = a.H;
+    vr += (size_t)j0 * vstride;
+    float ay[NC][2];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) ay[j][0] = ay[j][1] = 0.f;
+#pragma unroll
+    for (int mm = 0; mm < VPL; ++mm) {
+        uint32_t rr = 0;
+        if constexpr (R8) rr = r.c8.get(mm);
+        const uint4 wv = codeword2<R8, RI>(b13, b8, r.c13.get(mm), rr, q8);
+#pragma unroll
+        for (int j = 0; j < NC; ++j) dot8(ay[j], wv, lds128(vr + (size_t)j * vstride + 8 * mm));
+    }
+    const size_t row = (size_t)s.tb.expert[d] * H + m;
+    const float gd = a.gain[2] ? f16_bits_to_f32(__ldg(a.gain[2] + row)) : 1.f;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+        const float y = warp_sum(ay[j][0] + ay[j][1]) * gd;
+        if (lane == 0) atomicAdd(a.acc + (size_t)s.ct.tok[d][j0 + j] * H + m, y);
+    }
+}
+
 template <int VPL, bool R8, int TB>   // VPL = I / 256
 __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
+    constexpr bool RI = use_ri<VPL, R8, TB, true>();
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *b13 = smem, *b8 = smem + kB13Bytes;
-    uint16_t *vs = reinterpret_cast<uint16_t *>(smem + kB13Bytes + kB8Bytes);   // [2][TB][skewed I] bf16
-    __shared__ RouteTable tb;
-    __shared__ ColTable ct;
+    uint16_t *vs = reinterpret_cast<uint16_t *>(smem + books_bytes<R8, RI>());   // [2][TB][skewed I] bf16
+    __shared__ VqdShared s;
     __shared__ __align__(8) uint64_t bar;
     __shared__ int is_last;
     const int H = a.H, I = a.I, T = a.T;
@@ -345,16 +427,17 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
     }
     __syncthreads();
     if (warp == 0) {
-        load_books(b13, b8, a, &bar);
-        build_route_table(tb, a.ids, a.topk_w, T * a.k, a.k, a.E, nullptr, false);
+        load_books<RI>(b13, b8, a, &bar);
+        build_route_table(s.tb, a.ids, a.topk_w, T * a.k, a.k, a.E, nullptr, false);
         __syncwarp();
-        build_cols(ct, tb);
+        build_cols(s.ct, s.tb);
     }
+    if constexpr (RI) fill_ri(b8, a.book8);
     __syncthreads();
     // this CTA's items (expert slot, output row) span at most two experts
     // (the grid has at least as many CTAs as there are experts)
     const int lH = 31 - __clz(H);
-    const int n_items = tb.D * H;
+    const int n_items = s.tb.D * H;
     const int c0 = (int)((long long)n_items * blockIdx.x / gridDim.x);
     const int c1 = (int)((long long)n_items * (blockIdx.x + 1) / gridDim.x);
     const int d_lo = c0 >> lH;
@@ -365,14 +448,14 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
     // tk), v[k] = sum over the routes r of (d, tk) of w_r h_r[k], as bf16
     for (int dd = 0; dd < 2 && d_lo + dd <= d_hi; ++dd) {
         const int d = d_lo + dd;
-        const int nc = ct.ncol[d];
+        const int nc = s.ct.ncol[d];
         for (int idx = threadIdx.x; idx < nc * (I / 8); idx += kVThreads) {
-            const int j = idx / (I / 8), k8 = (idx % (I / 8)) * 8, tk = ct.tok[d][j];
+            const int j = idx / (I / 8), k8 = (idx % (I / 8)) * 8, tk = s.ct.tok[d][j];
             float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (int c = tb.col_beg[d]; c < tb.col_beg[d + 1]; ++c) {
-                const int rt = tb.route[c];
-                if (tb.tok[rt] != tk) continue;
-                const float w = tb.w[rt];
+            for (int c = s.tb.col_beg[d]; c < s.tb.col_beg[d + 1]; ++c) {
+                const int rt = s.tb.route[c];
+                if (s.tb.tok[rt] != tk) continue;
+                const float w = s.tb.w[rt];
                 const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(a.h + (size_t)rt * I + k8));
                 const float4 h1 = __ldcg(reinterpret_cast<const float4 *>(a.h + (size_t)rt * I + k8 + 4));
                 v[0] = fmaf(w, h0.x, v[0]); v[1] = fmaf(w, h0.y, v[1]); v[2] = fmaf(w, h0.z, v[2]);
@@ -387,7 +470,7 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
         }
     }
     volatile int abort_flag = 0;
-    const bool books_ok = __syncthreads_and(mbar_wait_abort(&bar, 0, &abort_flag, a.wait_cycles));
+    const bool books_ok = __syncthreads_and(mbar_poll_abort(&bar, 0, &abort_flag, a.wait_cycles));
     pdl_launch_dependents();
 
     if (books_ok) {
@@ -397,34 +480,25 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
         const int w1 = c0 + (int)((long long)(c1 - c0) * (warp + 1) / kVWarps);
         const int chunk = skew_pos<VPL>(lane * 8 * VPL);
         auto load = [&](int i, DNRow<VPL, R8> &r) {
-            const size_t row = (size_t)tb.expert[i >> lH] * H + (i & (H - 1));
+            const size_t row = (size_t)s.tb.expert[i >> lH] * H + (i & (H - 1));
             r.c13.load(a.idx13[2] + row * RB13, lane);
             if constexpr (R8) r.c8.load(a.idx8[2] + row * RB8, lane);
         };
         auto compute = [&](int i, DNRow<VPL, R8> &r) {
-            const int d = i >> lH, m = i & (H - 1), dd = d - d_lo;
-            const int ncol = ct.ncol[d];
+            const int d = i >> lH, m = i & (H - 1);
+            const uint16_t *vr = vs + (size_t)(d - d_lo) * TB * vstride + chunk;
             r.c13.align();
-            float ay[TB][2];
-#pragma unroll
-            for (int j = 0; j < TB; ++j) ay[j][0] = ay[j][1] = 0.f;
-            const uint16_t *vr = vs + (size_t)dd * TB * vstride + chunk;
-#pragma unroll
-            for (int m = 0; m < VPL; ++m) {
-                uint32_t rr = 0;
-                if constexpr (R8) rr = r.c8.get(m);
-                const uint4 wv = codeword<R8>(b13, b8, r.c13.get(m), rr);
-#pragma unroll
-                for (int j = 0; j < TB; ++j)
-                    if (j < ncol) dot8(ay[j], wv, lds128(vr + (size_t)j * vstride + 8 * m));
+            const int nc = s.ct.ncol[d];
+            if (nc > 4) {
+                if constexpr (TB >= 8) dn_row<VPL, R8, RI, 4>(a, s, b13, b8, vr, vstride, d, m, 0, r);
             }
-            const size_t row = (size_t)tb.expert[d] * H + m;
-            const float gd = a.gain[2] ? f16_bits_to_f32(__ldg(a.gain[2] + row)) : 1.f;
-#pragma unroll
-            for (int j = 0; j < TB; ++j) {
-                if (j >= ncol) break;
-                const float y = warp_sum(ay[j][0] + ay[j][1]) * gd;
-                if (lane == 0) atomicAdd(a.acc + (size_t)ct.tok[d][j] * H + m, y);
+            const int j0 = nc > 4 ? 4 : 0;
+            switch (nc - j0) {
+                case 1: dn_row<VPL, R8, RI, 1>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
+                case 2: if constexpr (TB >= 2) dn_row<VPL, R8, RI, 2>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
+                case 3: if constexpr (TB >= 4) dn_row<VPL, R8, RI, 3>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
+                case 4: if constexpr (TB >= 4) dn_row<VPL, R8, RI, 4>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
+                default: break;
             }
         };
         DNRow<VPL, R8> ra, rb;
@@ -461,8 +535,10 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
 
 // ---------------------------------------------------------------- host
 
-size_t gu_smem(int TB, int H, int VPL) { return kB13Bytes + kB8Bytes + (size_t)TB * (H + H / VPL) * 2; }
-size_t dn_smem(int TB, int I, int VPL) { return kB13Bytes + kB8Bytes + (size_t)2 * TB * (I + I / VPL) * 2; }
+template <int VPL, bool R8, int TB>
+size_t gu_smem() { return books_bytes<R8, use_ri<VPL, R8, TB, false>()>() + gu_stage_bytes(TB, VPL); }
+template <int VPL, bool R8, int TB>
+size_t dn_smem() { return books_bytes<R8, use_ri<VPL, R8, TB, true>()>() + dn_stage_bytes(TB, VPL); }
 
 int tokens_bound(int T) { return T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8)); }
 
@@ -498,10 +574,10 @@ cudaError_t run(const Layer &L, const VqdArgs &a, cudaStream_t s, const cudaEven
     if (err[dev] != cudaSuccess) return err[dev];
     L.count_launches(2);
     if (ev) record_phase(ev[1], s);
-    cudaError_t e = launch_pdl(vqd_gateup_kernel<VPLG, R8, TB>, L.sm_count, gu_smem(TB, a.H, VPLG), s, ev == nullptr, a);
+    cudaError_t e = launch_pdl(vqd_gateup_kernel<VPLG, R8, TB>, L.sm_count, gu_smem<VPLG, R8, TB>(), s, ev == nullptr, a);
     if (e != cudaSuccess) return e;
     if (ev) record_phase(ev[2], s);
-    e = launch_pdl(vqd_down_kernel<VPLD, R8, TB>, L.sm_count, dn_smem(TB, a.I, VPLD), s, ev == nullptr, a);
+    e = launch_pdl(vqd_down_kernel<VPLD, R8, TB>, L.sm_count, dn_smem<VPLD, R8, TB>(), s, ev == nullptr, a);
     if (e != cudaSuccess) return e;
     if (ev) {
         record_phase(ev[3], s);
@@ -537,9 +613,10 @@ bool decode_vq_supported(const Layer &L, int T) {
     if (!L.vq_acc || !L.vq_done) return false;
     if (T < 1 || T > kVMaxT || T * d.top_k > dec::kMaxR) return false;
     if (!((d.hidden == 2048 || d.hidden == 4096) && (d.inter == 2048 || d.inter == 4096))) return false;
+    // the staged operands fit beside the books (without the interleaved residual copies)
     const int TB = tokens_bound(T);
-    if (gu_smem(TB, d.hidden, d.hidden / 256) > (size_t)kVMaxSmem) return false;
-    if (dn_smem(TB, d.inter, d.inter / 256) > (size_t)kVMaxSmem) return false;
+    if (books_bytes<true, false>() + gu_stage_bytes(TB, d.hidden / 256) > kVMaxSmem) return false;
+    if (books_bytes<true, false>() + dn_stage_bytes(TB, d.inter / 256) > kVMaxSmem) return false;
     // a down CTA's items span at most two experts: at least one CTA per routed expert
     return L.sm_count >= std::min(dec::kMaxR, d.n_experts) && L.sm_count <= 4096;
 }

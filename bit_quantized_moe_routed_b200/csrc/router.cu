@@ -87,9 +87,10 @@ __device__ void select_topk(float (&v)[kMaxPerLane], int E, int k, int score, in
     __syncwarp();
     if (lane == 0) {
         // k <= 64 selected values; the first is the largest
+        const float zmax = sel_z[0];
         float sum = 0.f;
         for (int j = 0; j < k; ++j) {
-            const float s = score == 0 ? 1.0f / (1.0f + expf(-sel_z[j])) : expf(sel_z[j] - sel_z[0]);
+            const float s = score == 0 ? 1.0f / (1.0f + expf(-sel_z[j])) : expf(sel_z[j] - zmax);
             sel_z[j] = s;
             sum += s;
         }
