@@ -9,6 +9,8 @@ from .oracle import (  # noqa: F401
     e2m1,
     e8m0,
     idx13,
+    e4m3,
+    gvq1_idx,
     bf16_to_f32,
     f16_to_f64,
     dequant,

@@ -151,10 +151,69 @@ void orc_row_vq(const uint8_t *idx13_row, const uint8_t *idx8_row,
 }
 
 /* ------------------------------------------------------------------ */
+/* GVQ1-style rows: 12-bit stream + 1-bit plane, 1-byte book entries   */
+/* ------------------------------------------------------------------ */
+
+/* E4M3 (the OCP 8-bit float without infinities): bit 7 sign, bits 6..3 the
+ * exponent e (bias 7), bits 2..0 the mantissa m.  e = 0: m/8 * 2^-6
+ * (subnormal); otherwise (1 + m/8) * 2^(e-7); e = 15 with m = 7 is NaN.
+ * Largest magnitude 448.  [Reading: the VQ page gives the books 1-byte
+ * entries ("Why 13 bits plus an 8-bit residual": 64 KiB + 2 KiB) without a
+ * number format.] */
+double orc_e4m3(uint32_t b)
+{
+    int s = (int)((b >> 7) & 1u);
+    int e = (int)((b >> 3) & 15u);
+    int m = (int)(b & 7u);
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Index j of a GVQ1 row [VQ "Recipe": "the 12-bit code stream plus a 1-bit
+ * plane"]: the low 12 bits are bits 12j..12j+11 of the row's little-endian
+ * 12-bit stream, bit 12 is bit j of the row's bit plane (bit q of a stream
+ * is bit q%8 of byte q/8, as for the 13-bit stream). */
+uint32_t orc_gvq1_idx(const uint8_t *code12_row, const uint8_t *hi_row, int64_t j)
+{
+    uint32_t idx = 0;
+    for (int q = 0; q < 12; ++q) {
+        int64_t p = 12 * j + q;
+        idx |= ((uint32_t)(code12_row[p >> 3] >> (p & 7)) & 1u) << q;
+    }
+    idx |= ((uint32_t)(hi_row[j >> 3] >> (j & 7)) & 1u) << 12;
+    return idx;
+}
+
+/* GVQ1 row: w[8j+i] = (e4m3(B13q[c][i]) * s13 + e4m3(B8q[r][i]) * s8) * gain,
+ * every operation an IEEE f32 one in that order (the E4M3 value is exact in
+ * f32); idx8_row / book8q NULL: no residual term; gain_bits NULL: gain 1. */
+void orc_row_gvq1(const uint8_t *code12_row, const uint8_t *hi_row, const uint8_t *idx8_row,
+                  const uint8_t *book13q, const uint8_t *book8q, float s13, float s8,
+                  const uint16_t *gain_bits, int K, float *w)
+{
+    float gain = gain_bits ? (float)orc_f16_to_f64(*gain_bits) : 1.0f;
+    for (int j = 0; j < K / 8; ++j) {
+        uint32_t c = orc_gvq1_idx(code12_row, hi_row, j);
+        for (int i = 0; i < 8; ++i) {
+            float v = (float)orc_e4m3(book13q[c * 8 + i]) * s13;
+            if (idx8_row && book8q) {
+                float r = (float)orc_e4m3(book8q[(uint32_t)idx8_row[j] * 8 + i]) * s8;
+                v = v + r;
+            }
+            if (gain_bits) v = v * gain;
+            w[8 * j + i] = v;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* Layer description                                                   */
 /* ------------------------------------------------------------------ */
 
-enum { ORC_MXFP4 = 0, ORC_VQ13 = 1, ORC_VQ13_R8 = 2 };
+enum { ORC_MXFP4 = 0, ORC_VQ13 = 1, ORC_VQ13_R8 = 2, ORC_GVQ1 = 3, ORC_GVQ1_R8 = 4 };
 
 typedef struct {
     int32_t H, I, E, k, fmt;
@@ -166,6 +225,12 @@ typedef struct {
     const uint16_t *gain[3];   /* f16 row gains   [E][N] or NULL   */
     const uint16_t *book13;    /* bf16 [8192][8]                   */
     const uint16_t *book8;     /* bf16 [256][8] or NULL            */
+    /* GVQ1 / GVQ1_R8 (idx8 and gain as above) */
+    const uint8_t *code12[3];  /* 12-bit stream   [E][N][K*3/16]   */
+    const uint8_t *hi1[3];     /* bit-12 plane    [E][N][K/64]     */
+    const uint8_t *gbook13;    /* e4m3 [8192][8]                   */
+    const uint8_t *gbook8;     /* e4m3 [256][8] or NULL            */
+    float gscale13, gscale8;
 } orc_layer;
 
 static void proj_shape(const orc_layer *L, int p, int *N, int *K)
@@ -182,6 +247,11 @@ void orc_dequant_row(const orc_layer *L, int e, int p, int n, float *w)
     int64_t row = (int64_t)e * N + n;
     if (L->fmt == ORC_MXFP4) {
         orc_row_mxfp4(L->codes[p] + row * (K / 2), L->scales[p] + row * (K / 32), K, w);
+    } else if (L->fmt == ORC_GVQ1 || L->fmt == ORC_GVQ1_R8) {
+        const int r8 = L->fmt == ORC_GVQ1_R8;
+        orc_row_gvq1(L->code12[p] + row * ((int64_t)K * 3 / 16), L->hi1[p] + row * (K / 64),
+                     r8 ? L->idx8[p] + row * (K / 8) : NULL, L->gbook13, r8 ? L->gbook8 : NULL,
+                     L->gscale13, L->gscale8, L->gain[p] ? L->gain[p] + row : NULL, K, w);
     } else {
         int64_t sb = (int64_t)K * 13 / 64;
         const uint8_t *i8 = (L->fmt == ORC_VQ13_R8) ? L->idx8[p] + row * (K / 8) : NULL;

@@ -18,7 +18,7 @@ _SO = os.path.join(_HERE, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-_FMT = {"mxfp4": 0, "vq13": 1, "vq13r8": 2}
+_FMT = {"mxfp4": 0, "vq13": 1, "vq13r8": 2, "gvq1": 3, "gvq1r8": 4}
 
 
 class _Layer(C.Structure):
@@ -27,6 +27,8 @@ class _Layer(C.Structure):
         ("codes", C.c_void_p * 3), ("scales", C.c_void_p * 3), ("idx13", C.c_void_p * 3),
         ("idx8", C.c_void_p * 3), ("gain", C.c_void_p * 3),
         ("book13", C.c_void_p), ("book8", C.c_void_p),
+        ("code12", C.c_void_p * 3), ("hi1", C.c_void_p * 3), ("gbook13", C.c_void_p), ("gbook8", C.c_void_p),
+        ("gscale13", C.c_float), ("gscale8", C.c_float),
     ]
 
 
@@ -59,6 +61,10 @@ def lib():
         L.orc_f16_to_f64.argtypes = [C.c_uint16]
         L.orc_idx13.restype = C.c_uint32
         L.orc_idx13.argtypes = [C.c_void_p, C.c_int64]
+        L.orc_e4m3.restype = C.c_double
+        L.orc_e4m3.argtypes = [C.c_uint32]
+        L.orc_gvq1_idx.restype = C.c_uint32
+        L.orc_gvq1_idx.argtypes = [C.c_void_p, C.c_void_p, C.c_int64]
         L.orc_dequant.restype = None
         L.orc_dequant.argtypes = [C.POINTER(_Layer), C.c_int, C.c_int, C.c_void_p]
         L.orc_forward.restype = C.c_int64
@@ -77,6 +83,16 @@ def e2m1(code: int) -> float:
 
 def e8m0(b: int) -> float:
     return lib().orc_e8m0(b)
+
+
+def e4m3(b: int) -> float:
+    return lib().orc_e4m3(b)
+
+
+def gvq1_idx(code12_row: np.ndarray, hi_row: np.ndarray, j: int) -> int:
+    c = np.ascontiguousarray(code12_row, dtype=np.uint8)
+    h = np.ascontiguousarray(hi_row, dtype=np.uint8)
+    return int(lib().orc_gvq1_idx(c.ctypes.data, h.ctypes.data, j))
 
 
 def bf16_to_f32(bits: int) -> float:
@@ -131,6 +147,13 @@ def _layer_struct(layer):
         s.gain[p] = c(layer.gain[p], np.uint16)
     s.book13 = c(layer.book13, np.uint16)
     s.book8 = c(layer.book8, np.uint16)
+    for p in range(3):
+        s.code12[p] = c(layer.code12[p], np.uint8)
+        s.hi1[p] = c(layer.hi1[p], np.uint8)
+    s.gbook13 = c(layer.gbook13, np.uint8)
+    s.gbook8 = c(layer.gbook8, np.uint8)
+    s.gscale13 = float(layer.gscale[0]) if layer.gscale is not None else 0.0
+    s.gscale8 = float(layer.gscale[1]) if layer.gscale is not None else 0.0
     return s, keep
 
 

@@ -19,4 +19,6 @@ from .gen import (  # noqa: F401
     bf16_bits_from_f32,
     f32_from_bf16_bits,
     idx13_row_bytes,
+    gvq1_code_row_bytes,
+    e4m3_bytes_from_f32,
 )

@@ -27,6 +27,11 @@ component number alone, whatever else is drawn):
   [0.5, 2) rounded to f16.
 * component 40  -- router matrix Wr [E][H] float32 ~ N(0, 1/H), so that with
   N(0,1) activations the router logits are about N(0,1).
+* GVQ1 layers ("gvq1" / "gvq1r8"): the base and residual books are N(0,1)
+  draws (components 2 and 3) rounded to E4M3 bytes (by torch), with book
+  scales book13_sigma * book13_mult and book8_sigma; component 10+p gives
+  the 12-bit code stream as uniform random bytes, component 50+p the bit-12
+  plane, component 20+p the residual indices.
 
 Projections are p = 0 gate [I][H], 1 up [I][H], 2 down [H][I]; rows are
 output features and K (the reduction axis) is contiguous.
@@ -128,6 +133,19 @@ def _f16_bits_from_f32(a: np.ndarray) -> np.ndarray:
     return np.asarray(a, dtype=np.float32).astype(np.float16).view(np.uint16)
 
 
+def e4m3_bytes_from_f32(a: np.ndarray) -> np.ndarray:
+    """float -> E4M3 bytes (uint8), round-to-nearest-even via torch's float8_e4m3fn."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.float8_e4m3fn)
+    return t.view(torch.uint8).numpy().copy()
+
+
+def gvq1_code_row_bytes(K: int) -> int:
+    """Bytes of one row's GVQ1 12-bit code stream: K/8 codes of 12 bits."""
+    assert K % 64 == 0
+    return (K // VEC) * 12 // 8
+
+
 def idx13_row_bytes(K: int) -> int:
     """Bytes of one row's 13-bit index stream: K/8 indices of 13 bits."""
     assert K % 64 == 0, "K must be a multiple of 64 for whole bytes per row"
@@ -145,6 +163,11 @@ class Layer:
     book13: Optional[np.ndarray] = None                          # uint16 [8192][8]
     book8: Optional[np.ndarray] = None                           # uint16 [256][8]
     gain: list = field(default_factory=lambda: [None] * 3)     # uint16 f16 [E][N]
+    code12: list = field(default_factory=lambda: [None] * 3)   # GVQ1 12-bit streams [E][N][K*3/16]
+    hi1: list = field(default_factory=lambda: [None] * 3)      # GVQ1 bit-12 planes [E][N][K/64]
+    gbook13: Optional[np.ndarray] = None                         # uint8 e4m3 [8192][8]
+    gbook8: Optional[np.ndarray] = None                          # uint8 e4m3 [256][8]
+    gscale: Optional[tuple] = None                               # (scale of gbook13, scale of gbook8) f32
 
     @property
     def fmt(self) -> str:
@@ -153,13 +176,17 @@ class Layer:
     def without_residual(self) -> "Layer":
         """The same layer with the residual stage switched off (the base
         stage arrays are shared, byte for byte)."""
+        if self.cfg.fmt.startswith("gvq1"):
+            return Layer(cfg=self.cfg.replace(fmt="gvq1"), code12=list(self.code12), hi1=list(self.hi1),
+                         gbook13=self.gbook13, gscale=self.gscale, gain=list(self.gain))
         return Layer(cfg=self.cfg.replace(fmt="vq13"), idx13=list(self.idx13),
                      book13=self.book13, gain=list(self.gain))
 
     def weight_bytes_per_expert(self) -> int:
         tot = 0
         for p in range(3):
-            for arr in (self.codes[p], self.scales[p], self.idx13[p], self.idx8[p], self.gain[p]):
+            for arr in (self.codes[p], self.scales[p], self.idx13[p], self.idx8[p], self.gain[p], self.code12[p],
+                        self.hi1[p]):
                 if arr is not None:
                     tot += arr[0].nbytes
         return tot
@@ -192,6 +219,20 @@ def gen_layer(cfg: LayerCfg, seed: int = 0, experts: Optional[range] = None) -> 
             for p in range(3):
                 N, K = cfg.shape(p)
                 L.idx8[p] = _random_bytes(_rng(seed, 20 + p), (E, N, K // VEC))
+    elif cfg.fmt in ("gvq1", "gvq1r8"):
+        L.gbook13 = e4m3_bytes_from_f32(_rng(seed, 2).normal(0.0, 1.0, size=(BOOK13_ROWS, VEC)))
+        s8 = 0.0
+        for p in range(3):
+            N, K = cfg.shape(p)
+            L.code12[p] = _random_bytes(_rng(seed, 10 + p), (E, N, gvq1_code_row_bytes(K)))
+            L.hi1[p] = _random_bytes(_rng(seed, 50 + p), (E, N, K // 64))
+        if cfg.fmt == "gvq1r8":
+            L.gbook8 = e4m3_bytes_from_f32(_rng(seed, 3).normal(0.0, 1.0, size=(BOOK8_ROWS, VEC)))
+            s8 = cfg.book8_sigma
+            for p in range(3):
+                N, K = cfg.shape(p)
+                L.idx8[p] = _random_bytes(_rng(seed, 20 + p), (E, N, K // VEC))
+        L.gscale = (float(np.float32(cfg.book13_sigma * cfg.book13_mult)), float(np.float32(s8)))
     else:
         raise ValueError(cfg.fmt)
     if cfg.gains:
