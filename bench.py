@@ -68,6 +68,7 @@ def ncu_traffic(workload):
 # workload -> (config name, overrides)
 WORKLOADS = {
     "decode_mxfp4": ("decode_mxfp4", {}),
+    "decode_mxfp4_t8": ("decode_mxfp4", dict(T=8)),
     "decode_vq_t1": ("decode_vq", dict(T=1)),
     "decode_vq_t4": ("decode_vq", dict(T=4)),
     "decode_vq_t8": ("decode_vq", dict(T=8)),

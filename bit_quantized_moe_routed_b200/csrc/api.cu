@@ -75,7 +75,11 @@ void free_layer(moeq_layer *L) {
         cudaFree(L->w.idx13[p]);
         cudaFree(L->w.idx8[p]);
         cudaFree(L->w.gain[p]);
+        cudaFree(L->w.code12[p]);
+        cudaFree(L->w.hi1[p]);
     }
+    cudaFree(L->w.gbook13);
+    cudaFree(L->w.gbook8);
     cudaFree(L->w.book13);
     cudaFree(L->w.book8);
     cudaFree(L->b.offsets);
@@ -108,7 +112,7 @@ bool desc_valid(const moeq_layer_desc *d) {
         // 1024-weight chunks (the device layout, MxGeom)
         if (d->hidden % 128 || d->inter % 128) return false;
         if ((d->hidden > 1024 && d->hidden % 1024) || (d->inter > 1024 && d->inter % 1024)) return false;
-    } else if (d->fmt == MOEQ_FMT_VQ13 || d->fmt == MOEQ_FMT_VQ13_R8) {
+    } else if (is_vq13(d->fmt) || is_gvq1(d->fmt)) {
         if (d->hidden % 64 || d->inter % 64) return false;
     } else {
         return false;
@@ -188,6 +192,11 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
             // codes and scales share one plane in the device layout (MxGeom)
             ALLOC(L->w.codes[p], (size_t)E * MxGeom(N, K).expert_bytes());
             (void)rows;
+        } else if (is_gvq1(fmt)) {
+            ALLOC(L->w.code12[p], rows * K * 3 / 16);
+            ALLOC(L->w.hi1[p], rows * K / 64);
+            if (has_r8(fmt)) ALLOC(L->w.idx8[p], rows * (K / 8));
+            ALLOC(L->w.gain[p], rows * sizeof(uint16_t));
         } else {
             // 16 bytes of slack: the tensor-core path reads each row's 13-byte
             // index chunk of a 64-column slab as four aligned 32-bit words
@@ -196,9 +205,15 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
             ALLOC(L->w.gain[p], rows * sizeof(uint16_t));
         }
     }
-    if (fmt != MOEQ_FMT_MXFP4) {
+    if (is_vq13(fmt)) {
         ALLOC(L->w.book13, sizeof(uint16_t) * kBook13Rows * 8);
         if (fmt == MOEQ_FMT_VQ13_R8) ALLOC(L->w.book8, sizeof(uint16_t) * kBook8Rows * 8);
+    }
+    if (is_gvq1(fmt)) {
+        ALLOC(L->w.gbook13, (size_t)kBook13Rows * 8);
+        if (has_r8(fmt)) ALLOC(L->w.gbook8, (size_t)kBook8Rows * 8);
+    }
+    if (fmt != MOEQ_FMT_MXFP4) {
         ALLOC(L->vq_acc, sizeof(float) * kDecMaxTokens * H);
         ALLOC(L->vq_done, sizeof(int));
     }
@@ -240,12 +255,13 @@ void moeq_layer_destroy(moeq_layer_t layer) {
 moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *stream) {
     if (!L || !w) return MOEQ_ERR_INVALID_ARGUMENT;
     const int fmt = L->d.fmt, E = L->d.n_experts, H = L->d.hidden, I = L->d.inter;
-    const bool mx = fmt == MOEQ_FMT_MXFP4, r8 = fmt == MOEQ_FMT_VQ13_R8;
+    const bool mx = fmt == MOEQ_FMT_MXFP4, vq = is_vq13(fmt), gq = is_gvq1(fmt), r8 = has_r8(fmt);
     // presence / absence of every plane
     int n_gain = 0;
     for (int p = 0; p < 3; ++p) {
         if (mx != (w->codes[p] != nullptr) || mx != (w->scales[p] != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
-        if (mx == (w->idx13[p] != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
+        if (vq != (w->idx13[p] != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
+        if (gq != (w->code12[p] != nullptr) || gq != (w->hi1[p] != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
         if (r8 != (w->idx8[p] != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
         if (w->gain[p]) {
             if (mx) return MOEQ_ERR_INVALID_ARGUMENT;
@@ -253,7 +269,17 @@ moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *str
         }
     }
     if (n_gain != 0 && n_gain != 3) return MOEQ_ERR_INVALID_ARGUMENT;
-    if (mx == (w->book13 != nullptr) || r8 != (w->book8 != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (vq != (w->book13 != nullptr) || (vq && r8) != (w->book8 != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (gq != (w->gbook13 != nullptr) || (gq && r8) != (w->gbook8 != nullptr)) return MOEQ_ERR_INVALID_ARGUMENT;
+    if (gq) {
+        // E4M3 NaN entries and non-finite scales are not valid
+        for (size_t i = 0; i < (size_t)kBook13Rows * 8; ++i)
+            if ((w->gbook13[i] & 0x7F) == 0x7F) return MOEQ_ERR_INVALID_ARGUMENT;
+        if (r8)
+            for (size_t i = 0; i < (size_t)kBook8Rows * 8; ++i)
+                if ((w->gbook8[i] & 0x7F) == 0x7F) return MOEQ_ERR_INVALID_ARGUMENT;
+        if (!std::isfinite(w->gscale[0]) || (r8 && !std::isfinite(w->gscale[1]))) return MOEQ_ERR_INVALID_ARGUMENT;
+    }
     // E8M0 255 is NaN and not a valid scale
     if (mx) {
         for (int p = 0; p < 3; ++p) {
@@ -293,6 +319,13 @@ moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *str
                     e = launch_mx_pack(tmp_c, tmp_s, L->w.codes[p] + (size_t)e0 * geo.expert_bytes(), geo, ne, s);
                 if (e == cudaSuccess) e = prefill_mx_upload(*L, p, tmp_c, tmp_s, e0, ne, s);
             }
+        } else if (gq) {
+            e = cudaMemcpyAsync(L->w.code12[p], w->code12[p], rows * K * 3 / 16, cudaMemcpyHostToDevice, s);
+            if (e == cudaSuccess) e = cudaMemcpyAsync(L->w.hi1[p], w->hi1[p], rows * K / 64, cudaMemcpyHostToDevice, s);
+            if (e == cudaSuccess && r8)
+                e = cudaMemcpyAsync(L->w.idx8[p], w->idx8[p], rows * (K / 8), cudaMemcpyHostToDevice, s);
+            if (e == cudaSuccess && n_gain)
+                e = cudaMemcpyAsync(L->w.gain[p], w->gain[p], rows * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
         } else {
             e = cudaMemcpyAsync(L->w.idx13[p], w->idx13[p], rows * row_bytes(fmt, 0, K), cudaMemcpyHostToDevice, s);
             if (e == cudaSuccess && r8)
@@ -301,16 +334,24 @@ moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *str
                 e = cudaMemcpyAsync(L->w.gain[p], w->gain[p], rows * sizeof(uint16_t), cudaMemcpyHostToDevice, s);
         }
     }
-    if (e == cudaSuccess && !mx)
+    if (e == cudaSuccess && vq)
         e = cudaMemcpyAsync(L->w.book13, w->book13, sizeof(uint16_t) * kBook13Rows * 8, cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && r8)
+    if (e == cudaSuccess && vq && r8)
         e = cudaMemcpyAsync(L->w.book8, w->book8, sizeof(uint16_t) * kBook8Rows * 8, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && gq)
+        e = cudaMemcpyAsync(L->w.gbook13, w->gbook13, (size_t)kBook13Rows * 8, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && gq && r8)
+        e = cudaMemcpyAsync(L->w.gbook8, w->gbook8, (size_t)kBook8Rows * 8, cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e == cudaSuccess && mx) e = prefill_mx_finish_upload(*L);
     cudaFree(tmp_c);
     cudaFree(tmp_s);
     if (e != cudaSuccess) return from_cuda(e);
     L->w.has_gain = n_gain == 3;
+    if (gq) {
+        L->w.gscale[0] = w->gscale[0];
+        L->w.gscale[1] = r8 ? w->gscale[1] : 0.f;
+    }
     L->uploaded = true;
     return MOEQ_OK;
 }

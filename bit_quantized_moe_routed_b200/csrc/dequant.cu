@@ -58,6 +58,31 @@ __global__ void dequant_vq_kernel(const uint8_t *__restrict__ idx13, const uint8
     }
 }
 
+// GVQ1 ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe": 12-bit code
+// stream plus a 1-bit plane): w[8j+i] = (e4m3(B13q[c][i]) * s13 +
+// e4m3(B8q[r][i]) * s8) * gain, each step one f32 operation in that order.
+__global__ void dequant_gvq1_kernel(const uint8_t *__restrict__ code12, const uint8_t *__restrict__ hi1,
+                                    const uint8_t *__restrict__ idx8, const uint8_t *__restrict__ b13q,
+                                    const uint8_t *__restrict__ b8q, float s13, float s8,
+                                    const uint16_t *__restrict__ gain, int N, int K, float *__restrict__ out) {
+    const int groups = K / 8;
+    long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= (long long)N * groups) return;
+    int n = (int)(u / groups), j = (int)(u % groups);
+    const uint32_t c = gvq1_idx_at(code12 + (size_t)n * K * 3 / 16, hi1 + (size_t)n * K / 64, j);
+    const uint8_t *b = b13q + (size_t)c * 8;
+    const uint8_t *r = idx8 ? b8q + (size_t)idx8[(size_t)n * groups + j] * 8 : nullptr;
+    float g = gain ? f16_bits_to_f32(gain[n]) : 1.0f;
+    float *o = out + (size_t)n * K + (size_t)j * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float v = __fmul_rn(e4m3_to_f32(b[i]), s13);
+        if (r) v = __fadd_rn(v, __fmul_rn(e4m3_to_f32(r[i]), s8));
+        if (gain) v = __fmul_rn(v, g);
+        o[i] = v;
+    }
+}
+
 // Logical planes (codes [ne][N][K/2], scales [ne][N][K/32]) -> device
 // layout (MxGeom).  One thread per 32-weight block of a row.
 __global__ void mx_pack_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scales,
@@ -96,6 +121,14 @@ cudaError_t launch_dequant(const Layer &L, int expert, int proj, float *out, cud
         long long units = (long long)v.N * (v.K / 32);
         dequant_mxfp4_kernel<<<(unsigned)((units + threads - 1) / threads), threads, 0, s>>>(
             v.codes + (size_t)expert * g.expert_bytes(), g, out);
+    } else if (is_gvq1(L.d.fmt)) {
+        long long units = (long long)v.N * (v.K / 8);
+        const uint8_t *c12 = v.code12 + (size_t)expert * v.N * v.K * 3 / 16;
+        const uint8_t *h1 = v.hi1 + (size_t)expert * v.N * v.K / 64;
+        const uint8_t *i8 = v.idx8 ? v.idx8 + (size_t)expert * v.N * (v.K / 8) : nullptr;
+        const uint16_t *g = v.gain ? v.gain + (size_t)expert * v.N : nullptr;
+        dequant_gvq1_kernel<<<(unsigned)((units + threads - 1) / threads), threads, 0, s>>>(
+            c12, h1, i8, v.gbook13, v.gbook8, v.gs13, v.gs8, g, v.N, v.K, out);
     } else {
         long long units = (long long)v.N * (v.K / 8);
         const uint8_t *i13 = v.idx13 + (size_t)expert * v.N * (v.K / 8) * 13 / 8;

@@ -19,7 +19,7 @@ namespace {
 constexpr int kRowsPerCta = 8;          // one row per warp
 constexpr int kTok = 4;                 // tokens per pass over a row
 
-enum { FMT_MX = 0, FMT_VQ = 1 };
+enum { FMT_MX = 0, FMT_VQ = 1, FMT_G = 2 };
 
 // Exact f32 values of weights 32u .. 32u+31 of row n of expert e.
 template <int FMT>
@@ -35,6 +35,25 @@ __device__ __forceinline__ void decode_unit(const ProjView &v, int e, int n, int
         for (int a = 0; a < 4; ++a)
 #pragma unroll
             for (int i = 0; i < 8; ++i) w[a * 8 + i] = __fmul_rn(e2m1_to_f32((q[a] >> (4 * i)) & 0xFu), sc);
+    } else if constexpr (FMT == FMT_G) {
+        const uint8_t *c12 = v.code12 + row * (size_t)v.K * 3 / 16, *h1 = v.hi1 + row * (size_t)v.K / 64;
+        float g = v.gain ? f16_bits_to_f32(__ldg(v.gain + row)) : 1.0f;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int j = 4 * u + a;
+            const uint32_t c = gvq1_idx_at(c12, h1, j);
+            const uint2 b = __ldg(reinterpret_cast<const uint2 *>(v.gbook13) + c);
+            uint2 r = make_uint2(0u, 0u);
+            if (v.idx8) r = __ldg(reinterpret_cast<const uint2 *>(v.gbook8) + __ldg(v.idx8 + row * (v.K / 8) + j));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t bb = ((i < 4 ? b.x : b.y) >> (8 * (i & 3))) & 0xFFu;
+                float val = __fmul_rn(e4m3_to_f32(bb), v.gs13);
+                if (v.idx8) val = __fadd_rn(val, __fmul_rn(e4m3_to_f32(((i < 4 ? r.x : r.y) >> (8 * (i & 3))) & 0xFFu), v.gs8));
+                if (v.gain) val = __fmul_rn(val, g);
+                w[a * 8 + i] = val;
+            }
+        }
     } else {
         const uint8_t *row13 = v.idx13 + row * (size_t)(v.K / 8) * 13 / 8;
         float g = v.gain ? f16_bits_to_f32(__ldg(v.gain + row)) : 1.0f;
@@ -217,6 +236,9 @@ cudaError_t launch_ffn_simt(const Layer &L, const void *x, const float *topk_w, 
     const bool bf = L.d.act == MOEQ_ACT_BF16;
     if (mx) return bf ? run<FMT_MX, true>(L, x, topk_w, n_tokens, out, s, ev)
                       : run<FMT_MX, false>(L, x, topk_w, n_tokens, out, s, ev);
+    if (is_gvq1(L.d.fmt))
+        return bf ? run<FMT_G, true>(L, x, topk_w, n_tokens, out, s, ev)
+                  : run<FMT_G, false>(L, x, topk_w, n_tokens, out, s, ev);
     return bf ? run<FMT_VQ, true>(L, x, topk_w, n_tokens, out, s, ev)
               : run<FMT_VQ, false>(L, x, topk_w, n_tokens, out, s, ev);
 }

@@ -35,6 +35,12 @@ struct DevWeights {
     uint16_t *gain[3] = {nullptr, nullptr, nullptr};
     uint16_t *book13 = nullptr;
     uint16_t *book8 = nullptr;
+    // GVQ1: 12-bit code streams, bit-12 planes, E4M3 books and their scales
+    uint8_t *code12[3] = {nullptr, nullptr, nullptr};
+    uint8_t *hi1[3] = {nullptr, nullptr, nullptr};
+    uint8_t *gbook13 = nullptr;
+    uint8_t *gbook8 = nullptr;
+    float gscale[2] = {0.f, 0.f};
     bool has_gain = false;
 };
 
@@ -54,8 +60,17 @@ struct ProjView {
     const uint16_t *gain;   // f16 row gains          [E][N] or null
     const uint16_t *book13; // bf16 [8192][8]
     const uint16_t *book8;  // bf16 [256][8] or null
+    const uint8_t *code12;  // GVQ1 12-bit stream     [E][N][K*3/16]
+    const uint8_t *hi1;     // GVQ1 bit-12 plane      [E][N][K/64]
+    const uint8_t *gbook13; // E4M3 [8192][8]
+    const uint8_t *gbook8;  // E4M3 [256][8] or null
+    float gs13, gs8;        // their scales
     int32_t N, K;
 };
+
+inline bool is_gvq1(int fmt) { return fmt == MOEQ_FMT_GVQ1 || fmt == MOEQ_FMT_GVQ1_R8; }
+inline bool is_vq13(int fmt) { return fmt == MOEQ_FMT_VQ13 || fmt == MOEQ_FMT_VQ13_R8; }
+inline bool has_r8(int fmt) { return fmt == MOEQ_FMT_VQ13_R8 || fmt == MOEQ_FMT_GVQ1_R8; }
 
 // Prefill path for MXFP4 (prefill_mx.cu): a second copy of the weights in the
 // logical layout for tensor copies, scale atoms, activation workspaces and the
@@ -132,10 +147,16 @@ struct Layer {
         v.codes = w.codes[p];
         v.scales = w.scales[p];
         v.idx13 = w.idx13[p];
-        v.idx8 = (d.fmt == MOEQ_FMT_VQ13_R8) ? w.idx8[p] : nullptr;
+        v.idx8 = has_r8(d.fmt) ? w.idx8[p] : nullptr;
         v.gain = w.has_gain ? w.gain[p] : nullptr;
         v.book13 = w.book13;
         v.book8 = (d.fmt == MOEQ_FMT_VQ13_R8) ? w.book8 : nullptr;
+        v.code12 = w.code12[p];
+        v.hi1 = w.hi1[p];
+        v.gbook13 = w.gbook13;
+        v.gbook8 = (d.fmt == MOEQ_FMT_GVQ1_R8) ? w.gbook8 : nullptr;
+        v.gs13 = w.gscale[0];
+        v.gs8 = w.gscale[1];
         v.N = (p == MOEQ_DOWN) ? d.hidden : d.inter;
         v.K = (p == MOEQ_DOWN) ? d.inter : d.hidden;
         return v;
@@ -281,5 +302,23 @@ __device__ __forceinline__ uint32_t idx13_at(const uint8_t *row, int j) {
 }
 
 __device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + expf(-g)); }
+
+// E4M3 byte -> f32, exact (sign, 4 exponent bits with bias 7, 3 mantissa
+// bits; exponent 0 is subnormal; 0x7F / 0xFF are NaN, rejected at upload):
+// a normal value's f32 pattern is (e + 120) << 23 | m << 20.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u, s = (b & 0x80u) << 24;
+    const float mag = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;   // m * 2^-9
+    return __uint_as_float(__float_as_uint(mag) | s);
+}
+
+// GVQ1 index j of a row: low 12 bits from the 12-bit stream, bit 12 from
+// the plane.  Reads the second byte of a code only when the field reaches it.
+__device__ __forceinline__ uint32_t gvq1_idx_at(const uint8_t *code_row, const uint8_t *hi_row, int j) {
+    const uint32_t bit = 12u * (uint32_t)j;
+    const uint8_t *p = code_row + (bit >> 3);
+    const uint32_t lo = (((uint32_t)p[0] | ((uint32_t)p[1] << 8)) >> (bit & 7u)) & 0xFFFu;
+    return lo | ((uint32_t)((hi_row[j >> 3] >> (j & 7)) & 1u) << 12);
+}
 
 }  // namespace moeq

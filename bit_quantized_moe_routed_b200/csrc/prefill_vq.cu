@@ -559,12 +559,12 @@ size_t dn_smem() { return (size_t)kDNStages * kDNStage + kBook13 + kBook8 + 1024
 }  // namespace
 
 bool prefill_vq_supported(const Layer &L, int T) {
-    return L.pv != nullptr && L.pv->ready && T >= 1 && L.d.fmt != MOEQ_FMT_MXFP4 && L.d.act == MOEQ_ACT_BF16;
+    return L.pv != nullptr && L.pv->ready && T >= 1 && is_vq13(L.d.fmt) && L.d.act == MOEQ_ACT_BF16;
 }
 
 cudaError_t prefill_vq_create(Layer &L) {
     const moeq_layer_desc &d = L.d;
-    if (d.fmt == MOEQ_FMT_MXFP4 || d.act != MOEQ_ACT_BF16) return cudaSuccess;
+    if (!is_vq13(d.fmt) || d.act != MOEQ_ACT_BF16) return cudaSuccess;
     if (d.hidden % kT || d.inter % kT) return cudaSuccess;
     PrefillVq *pv = new (std::nothrow) PrefillVq();
     if (!pv) return cudaErrorMemoryAllocation;

@@ -23,7 +23,7 @@ if not os.path.exists(LIB_PATH):
 _lib = C.CDLL(LIB_PATH)
 
 OK, INVALID_ARGUMENT, UNSUPPORTED, OUT_OF_MEMORY, CUDA, NOT_UPLOADED, ROUTE_OUT_OF_RANGE, TIMEOUT = range(8)
-FMT = {"mxfp4": 0, "vq13": 1, "vq13r8": 2}
+FMT = {"mxfp4": 0, "vq13": 1, "vq13r8": 2, "gvq1": 3, "gvq1r8": 4}
 ACT = {"f32": 0, "bf16": 1}
 GATE, UP, DOWN = 0, 1, 2
 
@@ -44,7 +44,8 @@ class LayerDesc(C.Structure):
 class Weights(C.Structure):
     _fields_ = [("codes", C.c_void_p * 3), ("scales", C.c_void_p * 3), ("idx13", C.c_void_p * 3),
                 ("idx8", C.c_void_p * 3), ("book13", C.c_void_p), ("book8", C.c_void_p),
-                ("gain", C.c_void_p * 3)]
+                ("gain", C.c_void_p * 3), ("code12", C.c_void_p * 3), ("hi1", C.c_void_p * 3),
+                ("gbook13", C.c_void_p), ("gbook8", C.c_void_p), ("gscale", C.c_float * 2)]
 
 
 _lib.moeq_layer_create.argtypes = [C.POINTER(LayerDesc), C.POINTER(C.c_void_p)]
@@ -169,19 +170,25 @@ class Layer:
 
     def upload(self, w, stream=None):
         """``w``: host arrays with the attributes codes, scales, idx13, idx8,
-        book13, book8, gain (per-projection lists), logical layout."""
+        gain, code12, hi1 (per-projection lists), book13, book8 (bf16),
+        gbook13, gbook8 (E4M3) and gscale, logical layout; missing
+        attributes count as absent."""
         ws = Weights()
         keep = []
         for p in range(3):
             for name, dt in (("codes", np.uint8), ("scales", np.uint8), ("idx13", np.uint8),
-                             ("idx8", np.uint8), ("gain", np.uint16)):
-                arr, ptr = _host(getattr(w, name)[p], dt)
+                             ("idx8", np.uint8), ("gain", np.uint16), ("code12", np.uint8), ("hi1", np.uint8)):
+                arrs = getattr(w, name, None)
+                arr, ptr = _host(arrs[p] if arrs is not None else None, dt)
                 keep.append(arr)
                 getattr(ws, name)[p] = ptr
-        for name in ("book13", "book8"):
-            arr, ptr = _host(getattr(w, name), np.uint16)
+        for name, dt in (("book13", np.uint16), ("book8", np.uint16), ("gbook13", np.uint8), ("gbook8", np.uint8)):
+            arr, ptr = _host(getattr(w, name, None), dt)
             keep.append(arr)
             setattr(ws, name, ptr)
+        gs = getattr(w, "gscale", None)
+        if gs is not None:
+            ws.gscale[0], ws.gscale[1] = float(gs[0]), float(gs[1])
         _check(_lib.moeq_upload_weights(self._h, C.byref(ws), _stream_ptr(stream)), "moeq_upload_weights")
         del keep
 

@@ -65,7 +65,13 @@ typedef enum {
     MOEQ_ERR_TIMEOUT = 7            /* device flag: a bounded wait gave up     */
 } moeq_status;
 
-typedef enum { MOEQ_FMT_MXFP4 = 0, MOEQ_FMT_VQ13 = 1, MOEQ_FMT_VQ13_R8 = 2 } moeq_format;
+typedef enum {
+    MOEQ_FMT_MXFP4 = 0,
+    MOEQ_FMT_VQ13 = 1,      /* 13-bit stream, bf16 books                              */
+    MOEQ_FMT_VQ13_R8 = 2,   /* ... plus the 8-bit residual stage                      */
+    MOEQ_FMT_GVQ1 = 3,      /* 12-bit stream + bit-12 plane, 1-byte E4M3 book entries */
+    MOEQ_FMT_GVQ1_R8 = 4    /* ... plus the 8-bit residual stage                      */
+} moeq_format;
 typedef enum { MOEQ_ACT_F32 = 0, MOEQ_ACT_BF16 = 1 } moeq_dtype;
 typedef enum { MOEQ_GATE = 0, MOEQ_UP = 1, MOEQ_DOWN = 2 } moeq_proj;
 /* Routing weights of the router (moeq_router_upload). */
@@ -108,6 +114,26 @@ typedef struct moeq_layer *moeq_layer_t;
  *   gain[p]    uint16 f16 [E][N] or NULL (gain 1)
  *   weight[n][8j+i] = (book13[idx13][i] + book8[idx8][i]) * gain[n], each
  *   operation IEEE f32 round-to-nearest-even, in that order.
+ * GVQ1 / GVQ1_R8 (same page, "Recipe": "the 12-bit code stream plus a 1-bit
+ * plane"; "Why 13 bits plus an 8-bit residual": 1-byte book entries, 64 KiB
+ * + 2 KiB of books.  The byte layout and the entry type are not on the
+ * page; this library reads them as follows):
+ *   code12[p]  uint8 [E][N][K*3/16]  per row, the low 12 bits of the K/8
+ *                                 indices as one little-endian bitstream
+ *                                 (index j: bits 12j..12j+11)
+ *   hi1[p]     uint8 [E][N][K/64] per row, bit 12 of index j is bit j
+ *                                 (bit j%8 of byte j/8)
+ *   idx8[p]    as for VQ13_R8 (GVQ1_R8 only)
+ *   gbook13    uint8 [8192][8]    E4M3 entries (the OCP 8-bit float without
+ *                                 infinities: sign, 4 exponent bits with
+ *                                 bias 7, 3 mantissa bits); 0x7F / 0xFF
+ *                                 (NaN) are rejected
+ *   gbook8     uint8 [256][8]     E4M3 residual entries (GVQ1_R8 only)
+ *   gscale[2]  the f32 scales of gbook13 and gbook8 (finite)
+ *   gain[p]    as for VQ13
+ *   weight[n][8j+i] = (e4m3(gbook13[c][i]) * gscale[0]
+ *                      + e4m3(gbook8[r][i]) * gscale[1]) * gain[n],
+ *   each operation IEEE f32 round-to-nearest-even, in that order.
  * Arrays not used by the format must be NULL.
  */
 typedef struct {
@@ -118,6 +144,11 @@ typedef struct {
     const uint16_t *book13;
     const uint16_t *book8;
     const uint16_t *gain[3];
+    const uint8_t *code12[3];
+    const uint8_t *hi1[3];
+    const uint8_t *gbook13;
+    const uint8_t *gbook8;
+    float gscale[2];
 } moeq_weights;
 
 /* Create a layer on desc->device and allocate, on that device, its weight
@@ -125,14 +156,16 @@ typedef struct {
  * of it until moeq_layer_destroy.
  * Errors: INVALID_ARGUMENT (NULL pointer; a non-positive size; top_k > E or
  * > 64; E > 1024; for MXFP4 hidden or inter not a multiple of 128, or
- * above 1024 and not a multiple of 1024; for VQ not a multiple of 64;
+ * above 1024 and not a multiple of 1024; for VQ13 / GVQ1 not a multiple of
+ * 64;
  * unknown fmt/act), CUDA (bad device), OUT_OF_MEMORY.  On error *out
  * is set to NULL and nothing is left allocated. */
 MOEQ_API moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out);
 
 /* Copy the host arrays of w into the layer (the library may store them in a
  * different internal order).  Validates first: every array the format needs
- * is non-NULL, arrays it does not use are NULL, no E8M0 byte is 255.  Uses
+ * is non-NULL, arrays it does not use are NULL, no E8M0 byte is 255, no
+ * E4M3 book entry is NaN, the GVQ1 book scales are finite.  Uses
  * `stream` for the copies and synchronizes it before returning, so the
  * caller may free w's arrays as soon as the call returns.
  * Errors: INVALID_ARGUMENT (validation), CUDA. */

@@ -55,7 +55,7 @@ def _desc(moeq, **kw):
     dict(hidden=0), dict(inter=-1), dict(n_experts=0), dict(top_k=0), dict(max_tokens=0),
     dict(top_k=17), dict(n_experts=2048, top_k=2), dict(top_k=65, n_experts=128),
     dict(hidden=250), dict(inter=100), dict(hidden=320), dict(inter=96), dict(hidden=1152), dict(fmt=1, hidden=288), dict(fmt=2, inter=96),
-    dict(fmt=3), dict(act=2),
+    dict(fmt=5), dict(fmt=3, hidden=288), dict(fmt=4, inter=96), dict(act=2),
 ])
 def test_create_rejects_bad_descriptors_on_the_host(moeq, bad):
     lib = moeq.lib()
