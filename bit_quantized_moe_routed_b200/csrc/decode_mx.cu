@@ -9,20 +9,24 @@
 //
 // Work: a unit is one expert's 16 gate + 16 up rows (gate/up kernel) or 32
 // down rows (down kernel) over the full K; each CTA (one per SM) takes a
-// contiguous, balanced range of units.  The 16 consumer warps form one group
+// contiguous, balanced range of units.  The 8 consumer warps form one group
 // per 1024-column chunk of K, so every chunk of a unit is in compute at
 // once; inside a group each warp takes a share of the chunk's 32-weight
 // block columns for both halves (gate and up, or the two 16-row down tiles),
 // i.e. two independent accumulator chains.  A warp reads the fragments of
 // its next group while it computes the current one.  Per unit the warps
-// hand their partial fragments to two epilogue warps through a two-slot
+// hand their partial fragments to four epilogue warps through a four-slot
 // ring (full/empty mbarriers), which sum them (SwiGLU and h for gate/up),
-// so the consumers never wait for one another.
+// so the consumers never wait for one another and run up to four units
+// ahead of the hand-off.  Eight consumer warps keep every register a warp
+// needs (up to 153, no spills); sixteen did not fit without spilling.
 //
 // Memory: the device layout (MxGeom) keeps each (16-row tile, 1024-column
 // chunk) block contiguous, so a producer warp streams a chunk of a unit as
 // two 8.7 KB bulk copies (TMA) into a ring of shared-memory stages with
-// full/empty mbarriers, unit by unit and chunk by chunk; the activations
+// full/empty mbarriers, unit by unit and chunk by chunk (one chunk per stage
+// where the stage count allows it, so a chunk's warps start as soon as it
+// lands); the activations
 // arrive first, one bulk copy per token.  Bulk copies of several KB are what
 // keep HBM busy; the layout also makes the fragment and scale reads
 // bank-conflict free.  The gate/up kernel lets the down kernel launch as its
@@ -135,7 +139,7 @@ __device__ __forceinline__ uint32_t u4get(const uint4 &v, int j) {
     return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
 
-constexpr int kCW = 16;   // consumer warps per CTA
+constexpr int kCW = 8;    // consumer warps per CTA (at up to 153 registers: no spills)
 
 // Barrier among the kCW consumer warps (id 1; the producer warp does not join).
 __device__ __forceinline__ void named_sync_consumers() {
@@ -345,8 +349,8 @@ struct GateUpArgs {
 };
 
 // Partial-sum slots between the consumer warps and the epilogue warps.
-constexpr int kRedSlots = 2;
-constexpr int kEpiWarps = 2;
+constexpr int kRedSlots = 4;
+constexpr int kEpiWarps = 4;
 constexpr int kGUThreads = 32 * (kCW + 1 + kEpiWarps);
 constexpr int kEpiWarp0 = kCW + 1;
 
@@ -878,8 +882,19 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
         __threadfence();
         for (int idx = tid; idx < n_last * 32 * T; idx += 32 * kCW) {
             const int row = idx & 31, col = (idx >> 5) % T, m0 = last_tiles[(idx >> 5) / T] * 32;
+            const float *yb = a.ybuf + (size_t)col * H + m0 + row;
+            // the experts' slices 16 loads at a time (independent, so they
+            // overlap), added in expert order
             float sum = 0.f;
-            for (int dd = 0; dd < tb.D; ++dd) sum += __ldcg(a.ybuf + ((size_t)dd * kMaxT + col) * H + m0 + row);
+            for (int d0 = 0; d0 < tb.D; d0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    v[i] = d0 + i < tb.D ? __ldcg(yb + (size_t)(d0 + i) * kMaxT * H) : 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (d0 + i < tb.D) sum += v[i];
+            }
             __nv_bfloat16 o = __float2bfloat16_rn(sum);
             a.out[(size_t)col * H + m0 + row] = *reinterpret_cast<uint16_t *>(&o);
         }
@@ -904,15 +919,16 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 
 // Stages and chunks per stage (cps, a divisor of the unit's nch chunks) for
 // a kernel whose other shared memory takes `fixed` bytes: of the choices
-// with at least three stages, the one with the most bytes in flight (larger
-// pieces on a tie), else one chunk per stage.
+// with at least three stages, the one with the most bytes in flight
+// (smaller pieces on a tie: the warps of a chunk start on it as soon as it
+// has landed), else one chunk per stage.
 struct StagePlan {
     int S, cps;
 };
 StagePlan plan_stages(int nch, size_t fixed) {
     StagePlan best{0, 1};
     long long best_bytes = -1;
-    for (int cps = nch; cps >= 1; cps /= 2) {
+    for (int cps = 1; cps <= nch; cps *= 2) {
         long long s = ((long long)kMaxDynSmem - (long long)fixed) / (long long)piece_bytes(cps);
         if (s > kMaxStages) s = kMaxStages;
         if (s < 3 && cps != 1) continue;
