@@ -272,8 +272,12 @@ __device__ __forceinline__ bool wait_piece(uint64_t *full, FastDiv S, int p, vol
 // the epilogue warps) and are summed in warp order.  A unit has at most
 // Tc = min(T, 8) columns, so only those are kept.
 __host__ __device__ inline int red_cols(int T) { return T < kMaxT ? T : kMaxT; }
+// Partial-sum slots between the consumer warps and the epilogue warps.
+constexpr int kRedSlots = 4;
+constexpr int kEpiWarps = 4;
+// red: [slot][consumer warp][half][16 rows][Tc columns] f32
 __host__ __device__ inline size_t red_bytes(int T) {
-    return 2 * (size_t)kCW * 2 * 16 * red_cols(T) * sizeof(float);
+    return (size_t)kRedSlots * kCW * 2 * 16 * red_cols(T) * sizeof(float);
 }
 
 __device__ __forceinline__ void put_partials(float *rb, int Tc, int warp, int g, int t, const float a0[4],
@@ -348,9 +352,6 @@ struct GateUpArgs {
     int T, k, E, H, I, cps;
 };
 
-// Partial-sum slots between the consumer warps and the epilogue warps.
-constexpr int kRedSlots = 4;
-constexpr int kEpiWarps = 4;
 constexpr int kGUThreads = 32 * (kCW + 1 + kEpiWarps);
 constexpr int kEpiWarp0 = kCW + 1;
 
