@@ -47,9 +47,10 @@
 // overflow, and the scale is undone in f32.
 //
 // Combine: the down kernel writes each expert's contribution, prescale
-// undone, to its own slice of a scratch buffer; the last unit to finish a
-// 32-row tile (per-tile arrival counter) sums the experts in a fixed order
-// and writes bf16 out, so the result does not depend on timing.
+// undone, to its own slice of a scratch buffer; a third, small kernel (one
+// output element per thread, launched as a programmatic dependent) sums the
+// slices in expert order and writes bf16 out, so the result does not depend
+// on timing and the sum is spread over the whole GPU.
 #include <mutex>
 
 #include "async.cuh"
@@ -612,7 +613,7 @@ struct DownArgs {
     const int32_t *ids;
     const float *topk_w;
     float *ybuf;                    // [kMaxR expert slots][kMaxT][H]
-    int *counters;                  // [H/32], zero between calls
+    int *n_routed;                  // out: number of experts with routes in this call (for the combine)
     uint16_t *out;                  // bf16 [T][H]
     uint32_t *status;
     long long wait_cycles;          // limit of every wait but the final drains
@@ -646,8 +647,7 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
     __shared__ int slot_d[kMaxBSlots], slot_t[kMaxBSlots];
     __shared__ unsigned slot_max[kMaxBSlots];
     __shared__ float slot_scale[kMaxBSlots], slot_inv[kMaxBSlots];
-    __shared__ int n_slots, n_last;
-    __shared__ int last_tiles[kMaxTiles];
+    __shared__ int n_slots;
     const int H = a.H, I = a.I, T = a.T, k = a.k, S = (int)a.S.d, cps = a.cps, Tc = red_cols(a.T);
     uint8_t *stages = smem_raw;
     uint16_t *bs = reinterpret_cast<uint16_t *>(smem_raw + (size_t)S * piece_bytes(cps));   // [slot][I+pad] f16
@@ -672,7 +672,6 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
         mbar_fence_init();
         issued = 0;
         abort_flag = 0;
-        n_last = 0;
     }
     const long long lim = a.wait_cycles;
     if (tid < kMaxBSlots) slot_max[tid] = 0u;
@@ -682,10 +681,9 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
     // this grid's completion before touching memory this kernel uses)
     pdl_launch_dependents();
     const int n_units = tb.D * tiles;
-    if (tb.D == 0) {   // no valid route at all: every output is zero
-        for (int i = blockIdx.x * kDNThreads + tid; i < T * H; i += gridDim.x * kDNThreads) a.out[i] = 0;
-        return;
-    }
+    // the combine kernel sums this many slices (it runs after this grid completes)
+    if (blockIdx.x == 0 && tid == 0) *a.n_routed = tb.D;
+    if (tb.D == 0) return;   // no valid route at all: the combine writes zeros
     int u0, u1;
     my_range(n_units, u0, u1);
     const int n_mine = u1 - u0;
@@ -869,42 +867,37 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
         if (lane == 0) mbar_arrive(&red_full[slot]);
     }
     if ((timed_out || abort_flag) && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
-    // Combine: once every expert's slice of a 32-row tile is in, the CTA
-    // whose unit completed it sums the slices in expert order and writes
-    // bf16; the order of the sum does not depend on timing.  The epilogue
-    // warps fenced their slices before this barrier.
-    asm volatile("bar.sync 3, %0;" ::"r"(32 * (kCW + kEpiWarps)) : "memory");
-    for (int j = tid; j < n_mine; j += 32 * kCW) {
-        const int tile = (u0 + j) & (tiles - 1);
-        if (atomicAdd(a.counters + tile, 1) == tb.D - 1) last_tiles[atomicAdd(&n_last, 1)] = tile;
-    }
-    named_sync_consumers();
-    if (n_last > 0) {
-        __threadfence();
-        for (int idx = tid; idx < n_last * 32 * T; idx += 32 * kCW) {
-            const int row = idx & 31, col = (idx >> 5) % T, m0 = last_tiles[(idx >> 5) / T] * 32;
-            const float *yb = a.ybuf + (size_t)col * H + m0 + row;
-            // the experts' slices 16 loads at a time (independent, so they
-            // overlap), added in expert order
-            float sum = 0.f;
-            for (int d0 = 0; d0 < tb.D; d0 += 16) {
-                float v[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    v[i] = d0 + i < tb.D ? __ldcg(yb + (size_t)(d0 + i) * kMaxT * H) : 0.f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (d0 + i < tb.D) sum += v[i];
-            }
-            __nv_bfloat16 o = __float2bfloat16_rn(sum);
-            a.out[(size_t)col * H + m0 + row] = *reinterpret_cast<uint16_t *>(&o);
-        }
-        for (int li = tid; li < n_last; li += 32 * kCW) a.counters[last_tiles[li]] = 0;
-    }
 }
 
-template <typename K, typename A>
-cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, A args) {
+// Combine (one output element per thread): the experts' f32 slices of the
+// down kernel summed in expert order, rounded once to bf16.  Launched as a
+// programmatic dependent of the down kernel, whose completion it waits for;
+// the order of the sum does not depend on timing.
+constexpr int kCombineThreads = 256;
+__global__ void __launch_bounds__(kCombineThreads) dec_combine_kernel(const float *ybuf, const int *n_routed,
+                                                                       uint16_t *out, int T, int H) {
+    pdl_wait_primary();
+    pdl_launch_dependents();
+    const int D = __ldcg(n_routed);
+    const int i = blockIdx.x * kCombineThreads + threadIdx.x;
+    if (i >= T * H) return;
+    const float *yb = ybuf + i;   // [d][col][m]: element i = col * H + m of slice d at d * kMaxT * H
+    // the slices 16 loads at a time (independent, so they overlap), added in expert order
+    float sum = 0.f;
+    for (int d0 = 0; d0 < D; d0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) v[q] = d0 + q < D ? __ldcg(yb + (size_t)(d0 + q) * kMaxT * H) : 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            if (d0 + q < D) sum += v[q];
+    }
+    __nv_bfloat16 o = __float2bfloat16_rn(sum);
+    out[i] = *reinterpret_cast<uint16_t *>(&o);
+}
+
+template <typename K, typename... A>
+cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, A... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -915,7 +908,7 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, args);
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 // Stages and chunks per stage (cps, a divisor of the unit's nch chunks) for
@@ -981,7 +974,7 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     const StagePlan gp = gu_plan(T, H);
     ga.S = make_fastdiv((uint32_t)gp.S);
     ga.cps = gp.cps;
-    L.count_launches(2);
+    L.count_launches(3);
     if (ev) record_phase(ev[1], s);   // routing is fused into both kernels' prologues
     cudaError_t e = launch_ex(dec_gateup_mx_kernel<NCU>, dim3(grid), dim3(kGUThreads),
                               gu_bytes(gp.S, ga.cps, T, H), s, ev == nullptr, ga);
@@ -993,7 +986,7 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     da.ids = ids;
     da.topk_w = topk_w;
     da.ybuf = L.dec_ybuf;
-    da.counters = L.dec_counters;
+    da.n_routed = L.dec_counters;
     da.out = reinterpret_cast<uint16_t *>(out);
     da.status = L.status;
     da.wait_cycles = L.wait_cycles;
@@ -1011,10 +1004,12 @@ cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const 
     e = launch_ex(dec_down_mx_kernel<NCD>, dim3(grid), dim3(kDNThreads), dn_bytes(dp.S, da.cps, T, I), s, ev == nullptr,
                   da);
     if (e != cudaSuccess) return e;
-    if (ev) {
-        record_phase(ev[3], s);
-        record_phase(ev[4], s);
-    }
+    if (ev) record_phase(ev[3], s);
+    const int n_out = T * H;
+    e = launch_ex(dec_combine_kernel, dim3((n_out + kCombineThreads - 1) / kCombineThreads), dim3(kCombineThreads), 0,
+                  s, ev == nullptr, (const float *)L.dec_ybuf, (const int *)L.dec_counters, (uint16_t *)out, T, H);
+    if (e != cudaSuccess) return e;
+    if (ev) record_phase(ev[4], s);
     return cudaSuccess;
 }
 

@@ -54,15 +54,12 @@ def test_wait_runs_out_and_the_device_stays_usable(family, limit, monkeypatch):
         st = short.status(clear=True)
         assert st in (moeq.OK, moeq.TIMEOUT)
         n_timeout += st == moeq.TIMEOUT
-    if family.startswith("decode"):
-        # the decode kernels have no waits between warps in their main loop
-        # (the VQ kernels wait once for the books, which usually have landed
-        # by then): whenever no wait ran out, the result is exact
+    if family == "decode_vq13r8":
+        # the VQ decode kernels wait once, for the books, which usually have
+        # landed by then: whenever no wait ran out, the result is exact
         out = run(short, cfg, x, ids, w)
         if short.status(clear=True) == moeq.OK:
             assert_close(out, oracle_ref(L, x, ids, w), "bf16", "decode under a short limit")
-        if family == "decode_mxfp4":
-            assert n_timeout == 0
     elif limit == 1:
         assert n_timeout == 3                  # a 1-cycle limit cannot be met
     torch.cuda.synchronize()                   # the context is intact
