@@ -724,8 +724,7 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
         }
         __syncwarp();
         if (abort_flag && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
-        __threadfence();
-        asm volatile("bar.sync 3, %0;" ::"r"(32 * (kCW + kEpiWarps)) : "memory");
+        // the slices reach the combine kernel through this grid's completion
         return;
     }
 
