@@ -15,10 +15,10 @@
 // block columns for both halves (gate and up, or the two 16-row down tiles),
 // i.e. two independent accumulator chains.  A warp reads the fragments of
 // its next group while it computes the current one.  Per unit the warps
-// hand their partial fragments to four epilogue warps through a four-slot
+// hand their partial fragments to two epilogue warps through a two-slot
 // ring (full/empty mbarriers), which sum them (SwiGLU and h for gate/up),
-// so the consumers never wait for one another and run up to four units
-// ahead of the hand-off.  Eight consumer warps keep every register a warp
+// so the consumers never wait for one another.  (Four slots took shared
+// memory from the stage ring and measured slower at T = 8.)  Eight consumer warps keep every register a warp
 // needs (up to 153, no spills); sixteen did not fit without spilling.
 //
 // Memory: the device layout (MxGeom) keeps each (16-row tile, 1024-column
@@ -274,8 +274,8 @@ __device__ __forceinline__ bool wait_piece(uint64_t *full, FastDiv S, int p, vol
 // Tc = min(T, 8) columns, so only those are kept.
 __host__ __device__ inline int red_cols(int T) { return T < kMaxT ? T : kMaxT; }
 // Partial-sum slots between the consumer warps and the epilogue warps.
-constexpr int kRedSlots = 4;
-constexpr int kEpiWarps = 4;
+constexpr int kRedSlots = 2;
+constexpr int kEpiWarps = 2;
 // red: [slot][consumer warp][half][16 rows][Tc columns] f32
 __host__ __device__ inline size_t red_bytes(int T) {
     return (size_t)kRedSlots * kCW * 2 * 16 * red_cols(T) * sizeof(float);
