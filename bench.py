@@ -73,6 +73,8 @@ WORKLOADS = {
     "decode_vq_t4": ("decode_vq", dict(T=4)),
     "decode_vq_t8": ("decode_vq", dict(T=8)),
     "decode_vq_t1_r0": ("decode_vq", dict(T=1, fmt="vq13")),
+    "decode_gvq1_t1": ("decode_vq", dict(T=1, fmt="gvq1r8")),
+    "decode_gvq1_t8": ("decode_vq", dict(T=8, fmt="gvq1r8")),
     "decode_vq_t8_r0": ("decode_vq", dict(T=8, fmt="vq13")),
     "prefill_mxfp4_zipf": ("prefill_mxfp4_zipf", {}),
     "prefill_vq_overflow": ("prefill_vq_overflow", {}),
@@ -99,8 +101,11 @@ def proj_bytes(cfg, p):
     N, K = cfg.shape(p)
     if cfg.fmt == "mxfp4":
         return N * (K // 2 + K // 32)
-    b = N * synth.idx13_row_bytes(K)
-    if cfg.fmt == "vq13r8":
+    if cfg.fmt.startswith("gvq1"):
+        b = N * (synth.gvq1_code_row_bytes(K) + K // 64)   # 12-bit stream + bit-12 plane: 13 bits per 8 weights
+    else:
+        b = N * synth.idx13_row_bytes(K)
+    if cfg.fmt in ("vq13r8", "gvq1r8"):
         b += N * (K // 8)
     if cfg.gains:
         b += 2 * N
@@ -108,7 +113,11 @@ def proj_bytes(cfg, p):
 
 
 def book_bytes(cfg):
-    return 0 if cfg.fmt == "mxfp4" else 8192 * 16 + (256 * 16 if cfg.fmt == "vq13r8" else 0)
+    if cfg.fmt == "mxfp4":
+        return 0
+    if cfg.fmt.startswith("gvq1"):   # 1-byte entries
+        return 8192 * 8 + (256 * 8 if cfg.fmt == "gvq1r8" else 0)
+    return 8192 * 16 + (256 * 16 if cfg.fmt == "vq13r8" else 0)
 
 
 def flops(cfg, n_routes):
@@ -288,7 +297,8 @@ def cpu_baseline(cfg, L, xs, ids, w, seconds=12.0):
 # Workloads the default run times after the headline one, one layer at a
 # time (each layer is freed before the next is built): the prefill
 # micro-batches and the VQ decode batch sizes.
-EXTRA_WORKLOADS = ("prefill_mxfp4_zipf", "prefill_vq_overflow", "decode_vq_t1", "decode_vq_t4", "decode_vq_t8")
+EXTRA_WORKLOADS = ("decode_mxfp4_t8", "prefill_mxfp4_zipf", "prefill_vq_overflow", "decode_vq_t1", "decode_vq_t4",
+                   "decode_vq_t8", "decode_gvq1_t1", "decode_gvq1_t8")
 
 
 def load_peaks():

@@ -32,7 +32,9 @@
 // finishes last casts the accumulator to bf16 and clears it for the next
 // call.
 #include <algorithm>
+#include <cmath>
 #include <mutex>
+#include <type_traits>
 
 #include "async.cuh"
 #include "decode_common.cuh"
@@ -66,6 +68,13 @@ struct VqdArgs {
     int *done;                 // arrival counter of the down kernel's CTAs, zero between calls
     uint32_t *status;
     long long wait_cycles;
+    // GVQ1 layers
+    const uint8_t *code12[3];  // [E][N][K*3/16] 12-bit code streams
+    const uint8_t *hi1[3];     // [E][N][K/64] bit-12 planes
+    const uint8_t *gbook13;    // E4M3 [8192][8]
+    const uint8_t *gbook8;     // E4M3 [256][8] (R8 only)
+    float gs13;                // base book scale
+    uint32_t rho2;             // (residual scale / base scale) as an f16 pair
     int T, k, E, H, I;
 };
 
@@ -141,6 +150,59 @@ struct Idx8 {
     __device__ __forceinline__ uint32_t get(int m) const { return (w[m >> 2] >> (8 * (m & 3))) & 0xFFu; }
 };
 
+// GVQ1: the lane's stretch of one row's 12-bit code stream (12 VPL / 8
+// bytes at byte 12 VPL l / 8: whole words) and its VPL bits of the bit-12
+// plane.
+template <int VPL>
+struct Idx12 {
+    static constexpr int NW = 12 * VPL / 32;                 // 6 or 3
+    uint32_t w[NW];
+    uint32_t hi;
+    __device__ __forceinline__ void load(const uint8_t *code_row, const uint8_t *hi_row, int lane) {
+        const uint32_t *p = reinterpret_cast<const uint32_t *>(code_row) + NW * lane;
+#pragma unroll
+        for (int q = 0; q < NW; ++q) w[q] = __ldcs(reinterpret_cast<const unsigned int *>(p + q));
+        if constexpr (VPL == 16) hi = __ldcs(reinterpret_cast<const unsigned short *>(hi_row) + lane);
+        else hi = __ldcs(reinterpret_cast<const unsigned char *>(hi_row) + lane);
+    }
+    __device__ __forceinline__ void align() {}
+    __device__ __forceinline__ uint32_t get(int m) const {
+        const int p = 12 * m, q = p >> 5, s = p & 31;
+        const int q1 = q + 1 < NW ? q + 1 : NW - 1;
+        const uint32_t lo = (s + 12 <= 32 ? (w[q] >> s) : __funnelshift_r(w[q], w[q1], s)) & 0xFFFu;
+        return lo | (((hi >> m) & 1u) << 12);
+    }
+};
+template <int VPL, bool G1>
+using IdxT = typename std::conditional<G1, Idx12<VPL>, Idx13<VPL>>::type;
+
+// Eight E4M3 bytes -> four f16 pairs, exact (byte i lands in element i).
+__device__ __forceinline__ uint4 e4m3x8_to_f16x2(uint2 v) {
+    uint4 r;
+    asm("{\n\t.reg .b16 a0, a1, a2, a3;\n\t"
+        "mov.b32 {a0, a1}, %4;\n\tmov.b32 {a2, a3}, %5;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a0;\n\tcvt.rn.f16x2.e4m3x2 %1, a1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %2, a2;\n\tcvt.rn.f16x2.e4m3x2 %3, a3;\n\t}"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "r"(v.x), "r"(v.y));
+    return r;
+}
+__device__ __forceinline__ uint32_t hfma2_f16(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+// (acc0, acc1) += (f32(w.lo), f32(w.hi)) * (x.lo, x.hi) for an f16 pair w and
+// a bf16 pair x, in f32.
+__device__ __forceinline__ void dot2h(float &acc0, float &acc1, uint32_t w, uint32_t x) {
+    asm("{\n\t.reg .b16 h0, h1;\n\t.reg .f32 f0, f1;\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b32 {h0, h1}, %2;\n\tcvt.f32.f16 f0, h0;\n\tcvt.f32.f16 f1, h1;\n\t"
+        "mov.b64 ra, {f0, f1};\n\tmov.b64 rb, {%3, %4};\n\tmov.b64 rc, {%0, %1};\n\t"
+        "fma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(w), "r"(x << 16), "r"(x & 0xFFFF0000u));
+}
+
 __device__ __forceinline__ uint32_t hadd2_bf16(uint32_t a, uint32_t b) {
     uint32_t r;
     asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -154,11 +216,21 @@ __device__ __forceinline__ void dot2(float &acc0, float &acc1, uint32_t a, uint3
         : "+f"(acc0), "+f"(acc1)
         : "r"(a << 16), "r"(a & 0xFFFF0000u), "r"(b << 16), "r"(b & 0xFFFF0000u));
 }
+// The dot product of a vector's 8 weights (bf16 pairs, or f16 pairs for
+// GVQ1) with 8 bf16 activations, into two f32 partial sums.
+template <bool G1 = false>
 __device__ __forceinline__ void dot8(float acc[2], const uint4 &w, const uint4 &x) {
-    dot2(acc[0], acc[1], w.x, x.x);
-    dot2(acc[0], acc[1], w.y, x.y);
-    dot2(acc[0], acc[1], w.z, x.z);
-    dot2(acc[0], acc[1], w.w, x.w);
+    if constexpr (G1) {
+        dot2h(acc[0], acc[1], w.x, x.x);
+        dot2h(acc[0], acc[1], w.y, x.y);
+        dot2h(acc[0], acc[1], w.z, x.z);
+        dot2h(acc[0], acc[1], w.w, x.w);
+    } else {
+        dot2(acc[0], acc[1], w.x, x.x);
+        dot2(acc[0], acc[1], w.y, x.y);
+        dot2(acc[0], acc[1], w.z, x.z);
+        dot2(acc[0], acc[1], w.w, x.w);
+    }
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -179,43 +251,75 @@ __device__ __forceinline__ void warp_range(int n, int &i0, int &i1) {
 // Shared-memory bytes of the books; with RI the residual book is stored 8
 // times, copy q in 16-byte bank group q only (entry r of copy q at
 // (8 r + q) * 16), and lane l reads copy l % 8: the 8 lanes of a quarter
-// warp then never share a bank group, however random their indices.
-template <bool R8, bool RI>
-constexpr int books_bytes() { return kB13Bytes + (R8 ? (RI ? 8 * kB8Bytes : kB8Bytes) : 0); }
+// warp then never share a bank group, however random their indices.  GVQ1
+// entries are 8 bytes: the base book takes 64 KB, and the interleaved
+// residual book 16 copies (8-byte slots, a half warp per phase).
+constexpr int kG13Bytes = kBook13Rows * 8, kG8Bytes = kBook8Rows * 8;
+template <bool R8, bool RI, bool G1 = false>
+constexpr int books_bytes() {
+    if constexpr (G1) return kG13Bytes + (R8 ? (RI ? 16 * kG8Bytes : kG8Bytes) : 0);
+    else return kB13Bytes + (R8 ? (RI ? 8 * kB8Bytes : kB8Bytes) : 0);
+}
 // Staged-operand bytes of each kernel for K = 256 VPL.
 constexpr int gu_stage_bytes(int TB, int VPL) { return TB * (256 * VPL + 256) * 2; }
 constexpr int dn_stage_bytes(int TB, int VPL) { return 2 * TB * (256 * VPL + 256) * 2; }
 // The residual book interleaved when it and the staged operands fit.
-template <int VPL, bool R8, int TB, bool DOWN>
+template <int VPL, bool R8, int TB, bool DOWN, bool G1 = false>
 constexpr bool use_ri() {
-    return R8 && books_bytes<true, true>() + (DOWN ? dn_stage_bytes(TB, VPL) : gu_stage_bytes(TB, VPL)) <= kVMaxSmem;
+    return R8 &&
+           books_bytes<true, true, G1>() + (DOWN ? dn_stage_bytes(TB, VPL) : gu_stage_bytes(TB, VPL)) <= kVMaxSmem;
 }
 
 // Both books into shared memory (warp 0): the base book by bulk copies on
 // `bar`; the residual book by the same copy, or, interleaved (RI), by the
 // whole CTA with plain loads (call fill_ri after the barrier's init).
-template <bool RI>
+template <bool RI, bool G1 = false>
 __device__ void load_books(uint8_t *b13, uint8_t *b8, const VqdArgs &a, uint64_t *bar) {
     const int lane = threadIdx.x & 31;
-    const bool copy8 = a.book8 && !RI;
-    if (lane == 0) mbar_arrive_expect_tx(bar, kB13Bytes + (copy8 ? kB8Bytes : 0));
+    const uint8_t *src13 = G1 ? a.gbook13 : reinterpret_cast<const uint8_t *>(a.book13);
+    const uint8_t *src8 = G1 ? a.gbook8 : reinterpret_cast<const uint8_t *>(a.book8);
+    constexpr int n13 = G1 ? kG13Bytes : kB13Bytes, n8 = G1 ? kG8Bytes : kB8Bytes;
+    const bool copy8 = src8 && !RI;
+    if (lane == 0) mbar_arrive_expect_tx(bar, n13 + (copy8 ? n8 : 0));
     __syncwarp();
-    if (lane < 4)
-        bulk_g2s(b13 + lane * (kB13Bytes / 4), reinterpret_cast<const uint8_t *>(a.book13) + lane * (kB13Bytes / 4),
-                 kB13Bytes / 4, bar);
-    if (lane == 4 && copy8) bulk_g2s(b8, a.book8, kB8Bytes, bar);
+    if (lane < 4) bulk_g2s(b13 + lane * (n13 / 4), src13 + lane * (n13 / 4), n13 / 4, bar);
+    if (lane == 4 && copy8) bulk_g2s(b8, src8, n8, bar);
     __syncwarp();
 }
-__device__ void fill_ri(uint8_t *b8, const uint16_t *book8) {
-    for (int i = threadIdx.x; i < kBook8Rows * 8; i += kVThreads) {
-        const int r = i >> 3, q = i & 7;
-        reinterpret_cast<uint4 *>(b8)[8 * r + q] = __ldg(reinterpret_cast<const uint4 *>(book8) + r);
+template <bool G1 = false>
+__device__ void fill_ri(uint8_t *b8, const VqdArgs &a) {
+    if constexpr (G1) {
+        for (int i = threadIdx.x; i < kBook8Rows * 16; i += kVThreads) {
+            const int r = i >> 4, q = i & 15;
+            reinterpret_cast<uint2 *>(b8)[16 * r + q] = __ldg(reinterpret_cast<const uint2 *>(a.gbook8) + r);
+        }
+    } else {
+        for (int i = threadIdx.x; i < kBook8Rows * 8; i += kVThreads) {
+            const int r = i >> 3, q = i & 7;
+            reinterpret_cast<uint4 *>(b8)[8 * r + q] = __ldg(reinterpret_cast<const uint4 *>(a.book8) + r);
+        }
     }
 }
 
-// The 8 weights of a vector: base (+ residual) as bf16 pairs.
-template <bool R8, bool RI>
-__device__ __forceinline__ uint4 codeword2(const uint8_t *b13, const uint8_t *b8, uint32_t c, uint32_t r, int q8) {
+// The 8 weights of a vector: base (+ residual) as bf16 pairs; for GVQ1 as
+// f16 pairs of base + rho * residual (both E4M3 values exact in f16; the
+// base scale and the gain are applied to the row's sum).
+template <bool R8, bool RI, bool G1 = false>
+__device__ __forceinline__ uint4 codeword2(const uint8_t *b13, const uint8_t *b8, uint32_t c, uint32_t r, int lane,
+                                           uint32_t rho2 = 0u) {
+    if constexpr (G1) {
+        uint4 v = e4m3x8_to_f16x2(*reinterpret_cast<const uint2 *>(b13 + 8u * c));
+        if constexpr (R8) {
+            const uint4 q = e4m3x8_to_f16x2(
+                *reinterpret_cast<const uint2 *>(b8 + 8u * (RI ? 16u * r + (uint32_t)(lane & 15) : r)));
+            v.x = hfma2_f16(q.x, rho2, v.x);
+            v.y = hfma2_f16(q.y, rho2, v.y);
+            v.z = hfma2_f16(q.z, rho2, v.z);
+            v.w = hfma2_f16(q.w, rho2, v.w);
+        }
+        return v;
+    }
+    const int q8 = lane & 7;
     uint4 v = lds128(b13 + 16u * c);
     if constexpr (R8) {
         const uint4 q = lds128(b8 + 16u * (RI ? 8u * r + (uint32_t)q8 : r));
@@ -229,9 +333,9 @@ __device__ __forceinline__ uint4 codeword2(const uint8_t *b13, const uint8_t *b8
 
 // ---------------------------------------------------------------- gate/up
 
-template <int VPL, bool R8>
+template <int VPL, bool R8, bool G1>
 struct GURow {
-    Idx13<VPL> g13, u13;
+    IdxT<VPL, G1> g13, u13;
     Idx8<VPL> g8, u8;
 };
 
@@ -246,11 +350,11 @@ struct VqdShared {
 // Columns j0 .. j0 + NC - 1 (at most four per pass: more would not fit the
 // registers; a fifth to eighth column takes a second pass over the row).
 // The index words must be aligned (Idx13::align) before the first pass.
-template <int VPL, bool R8, bool RI, int NC>
+template <int VPL, bool R8, bool RI, int NC, bool G1>
 __device__ __forceinline__ void gu_row(const VqdArgs &a, const VqdShared &s, const uint8_t *b13, const uint8_t *b8,
                                        const uint16_t *xs, int xstride, int chunk, int d, int n, int j0,
-                                       const GURow<VPL, R8> &r) {
-    const int lane = threadIdx.x & 31, q8 = lane & 7, I = a.I;
+                                       const GURow<VPL, R8, G1> &r) {
+    const int lane = threadIdx.x & 31, I = a.I;
     float ag[NC][2], au[NC][2];
     const uint16_t *xr[NC];
 #pragma unroll
@@ -265,18 +369,19 @@ __device__ __forceinline__ void gu_row(const VqdArgs &a, const VqdShared &s, con
             rg = r.g8.get(m);
             ru = r.u8.get(m);
         }
-        const uint4 wg = codeword2<R8, RI>(b13, b8, r.g13.get(m), rg, q8);
-        const uint4 wu = codeword2<R8, RI>(b13, b8, r.u13.get(m), ru, q8);
+        const uint4 wg = codeword2<R8, RI, G1>(b13, b8, r.g13.get(m), rg, lane, a.rho2);
+        const uint4 wu = codeword2<R8, RI, G1>(b13, b8, r.u13.get(m), ru, lane, a.rho2);
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
             const uint4 xv = lds128(xr[j] + 8 * m);
-            dot8(ag[j], wg, xv);
-            dot8(au[j], wu, xv);
+            dot8<G1>(ag[j], wg, xv);
+            dot8<G1>(au[j], wu, xv);
         }
     }
     const size_t row = (size_t)s.tb.expert[d] * I + n;
-    const float gg = a.gain[0] ? f16_bits_to_f32(__ldg(a.gain[0] + row)) : 1.f;
-    const float gu = a.gain[1] ? f16_bits_to_f32(__ldg(a.gain[1] + row)) : 1.f;
+    const float bs = G1 ? a.gs13 : 1.f;   // the GVQ1 base scale
+    const float gg = (a.gain[0] ? f16_bits_to_f32(__ldg(a.gain[0] + row)) : 1.f) * bs;
+    const float gu = (a.gain[1] ? f16_bits_to_f32(__ldg(a.gain[1] + row)) : 1.f) * bs;
 #pragma unroll
     for (int j = 0; j < NC; ++j) {
         const float g = warp_sum(ag[j][0] + ag[j][1]) * gg;
@@ -291,12 +396,12 @@ __device__ __forceinline__ void gu_row(const VqdArgs &a, const VqdShared &s, con
     }
 }
 
-template <int VPL, bool R8, int TB>   // VPL = H / 256; TB >= tokens
+template <int VPL, bool R8, int TB, bool G1>   // VPL = H / 256; TB >= tokens; G1: GVQ1 format
 __global__ void __launch_bounds__(kVThreads, 1) vqd_gateup_kernel(VqdArgs a) {
-    constexpr bool RI = use_ri<VPL, R8, TB, false>();
+    constexpr bool RI = use_ri<VPL, R8, TB, false, G1>();
     extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t *b13 = smem, *b8 = smem + kB13Bytes;
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem + books_bytes<R8, RI>());
+    uint8_t *b13 = smem, *b8 = smem + (G1 ? kG13Bytes : kB13Bytes);
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem + books_bytes<R8, RI, G1>());
     __shared__ VqdShared s;
     __shared__ __align__(8) uint64_t bar;
     const int H = a.H, I = a.I, T = a.T;
@@ -308,8 +413,8 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_gateup_kernel(VqdArgs a) {
     }
     __syncthreads();
     // the books are weights: fetch them before waiting for the previous kernel
-    if (warp == 0) load_books<RI>(b13, b8, a, &bar);
-    if constexpr (RI) fill_ri(b8, a.book8);
+    if (warp == 0) load_books<RI, G1>(b13, b8, a, &bar);
+    if constexpr (RI) fill_ri<G1>(b8, a);
     pdl_wait_primary();
     if (warp == 0) {
         build_route_table(s.tb, a.ids, a.topk_w, T * a.k, a.k, a.E, a.status, blockIdx.x == 0);
@@ -336,34 +441,39 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_gateup_kernel(VqdArgs a) {
     int i0, i1;
     warp_range(s.tb.D * I, i0, i1);
     const int chunk = skew_pos<VPL>(lane * 8 * VPL);   // this lane's columns in a staged row
-    auto load = [&](int i, GURow<VPL, R8> &r) {
+    auto load = [&](int i, GURow<VPL, R8, G1> &r) {
         const size_t row = (size_t)s.tb.expert[i >> lI] * I + (i & (I - 1));
-        r.g13.load(a.idx13[0] + row * RB13, lane);
-        r.u13.load(a.idx13[1] + row * RB13, lane);
+        if constexpr (G1) {
+            r.g13.load(a.code12[0] + row * (H * 3 / 16), a.hi1[0] + row * (H / 64), lane);
+            r.u13.load(a.code12[1] + row * (H * 3 / 16), a.hi1[1] + row * (H / 64), lane);
+        } else {
+            r.g13.load(a.idx13[0] + row * RB13, lane);
+            r.u13.load(a.idx13[1] + row * RB13, lane);
+        }
         if constexpr (R8) {
             r.g8.load(a.idx8[0] + row * RB8, lane);
             r.u8.load(a.idx8[1] + row * RB8, lane);
         }
     };
-    auto compute = [&](int i, GURow<VPL, R8> &r) {
+    auto compute = [&](int i, GURow<VPL, R8, G1> &r) {
         const int d = i >> lI, n = i & (I - 1);
         r.g13.align();
         r.u13.align();
         // the expert's column count, a compile-time constant inside
         const int nc = s.ct.ncol[d];
         if (nc > 4) {
-            if constexpr (TB >= 8) gu_row<VPL, R8, RI, 4>(a, s, b13, b8, xs, xstride, chunk, d, n, 0, r);
+            if constexpr (TB >= 8) gu_row<VPL, R8, RI, 4, G1>(a, s, b13, b8, xs, xstride, chunk, d, n, 0, r);
         }
         const int j0 = nc > 4 ? 4 : 0;
         switch (nc - j0) {
-            case 1: gu_row<VPL, R8, RI, 1>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
-            case 2: if constexpr (TB >= 2) gu_row<VPL, R8, RI, 2>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
-            case 3: if constexpr (TB >= 4) gu_row<VPL, R8, RI, 3>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
-            case 4: if constexpr (TB >= 4) gu_row<VPL, R8, RI, 4>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
+            case 1: gu_row<VPL, R8, RI, 1, G1>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
+            case 2: if constexpr (TB >= 2) gu_row<VPL, R8, RI, 2, G1>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
+            case 3: if constexpr (TB >= 4) gu_row<VPL, R8, RI, 3, G1>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
+            case 4: if constexpr (TB >= 4) gu_row<VPL, R8, RI, 4, G1>(a, s, b13, b8, xs, xstride, chunk, d, n, j0, r); break;
             default: break;
         }
     };
-    GURow<VPL, R8> ra, rb;
+    GURow<VPL, R8, G1> ra, rb;
     if (i0 < i1) load(i0, ra);
     for (int i = i0; i < i1; i += 2) {
         if (i + 1 < i1) load(i + 1, rb);
@@ -376,18 +486,19 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_gateup_kernel(VqdArgs a) {
 
 // ---------------------------------------------------------------- down
 
-template <int VPL, bool R8>
+template <int VPL, bool R8, bool G1>
 struct DNRow {
-    Idx13<VPL> c13;
+    IdxT<VPL, G1> c13;
     Idx8<VPL> c8;
 };
 
 // One output row m of expert slot d (staged columns at vr) for NC columns:
 // the dot products, the warp sums, one atomic per (row, token).
-template <int VPL, bool R8, bool RI, int NC>
+template <int VPL, bool R8, bool RI, int NC, bool G1>
 __device__ __forceinline__ void dn_row(const VqdArgs &a, const VqdShared &s, const uint8_t *b13, const uint8_t *b8,
-                                       const uint16_t *vr, int vstride, int d, int m, int j0, const DNRow<VPL, R8> &r) {
-    const int lane = threadIdx.x & 31, q8 = lane & 7, H = a.H;
+                                       const uint16_t *vr, int vstride, int d, int m, int j0,
+                                       const DNRow<VPL, R8, G1> &r) {
+    const int lane = threadIdx.x & 31, H = a.H;
     vr += (size_t)j0 * vstride;
     float ay[NC][2];
 #pragma unroll
@@ -396,12 +507,12 @@ __device__ __forceinline__ void dn_row(const VqdArgs &a, const VqdShared &s, con
     for (int mm = 0; mm < VPL; ++mm) {
         uint32_t rr = 0;
         if constexpr (R8) rr = r.c8.get(mm);
-        const uint4 wv = codeword2<R8, RI>(b13, b8, r.c13.get(mm), rr, q8);
+        const uint4 wv = codeword2<R8, RI, G1>(b13, b8, r.c13.get(mm), rr, lane, a.rho2);
 #pragma unroll
-        for (int j = 0; j < NC; ++j) dot8(ay[j], wv, lds128(vr + (size_t)j * vstride + 8 * mm));
+        for (int j = 0; j < NC; ++j) dot8<G1>(ay[j], wv, lds128(vr + (size_t)j * vstride + 8 * mm));
     }
     const size_t row = (size_t)s.tb.expert[d] * H + m;
-    const float gd = a.gain[2] ? f16_bits_to_f32(__ldg(a.gain[2] + row)) : 1.f;
+    const float gd = (a.gain[2] ? f16_bits_to_f32(__ldg(a.gain[2] + row)) : 1.f) * (G1 ? a.gs13 : 1.f);
 #pragma unroll
     for (int j = 0; j < NC; ++j) {
         const float y = warp_sum(ay[j][0] + ay[j][1]) * gd;
@@ -409,12 +520,12 @@ __device__ __forceinline__ void dn_row(const VqdArgs &a, const VqdShared &s, con
     }
 }
 
-template <int VPL, bool R8, int TB>   // VPL = I / 256
+template <int VPL, bool R8, int TB, bool G1>   // VPL = I / 256; G1: GVQ1 format
 __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
-    constexpr bool RI = use_ri<VPL, R8, TB, true>();
+    constexpr bool RI = use_ri<VPL, R8, TB, true, G1>();
     extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t *b13 = smem, *b8 = smem + kB13Bytes;
-    uint16_t *vs = reinterpret_cast<uint16_t *>(smem + books_bytes<R8, RI>());   // [2][TB][skewed I] bf16
+    uint8_t *b13 = smem, *b8 = smem + (G1 ? kG13Bytes : kB13Bytes);
+    uint16_t *vs = reinterpret_cast<uint16_t *>(smem + books_bytes<R8, RI, G1>());   // [2][TB][skewed I] bf16
     __shared__ VqdShared s;
     __shared__ __align__(8) uint64_t bar;
     __shared__ int is_last;
@@ -427,12 +538,12 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
     }
     __syncthreads();
     if (warp == 0) {
-        load_books<RI>(b13, b8, a, &bar);
+        load_books<RI, G1>(b13, b8, a, &bar);
         build_route_table(s.tb, a.ids, a.topk_w, T * a.k, a.k, a.E, nullptr, false);
         __syncwarp();
         build_cols(s.ct, s.tb);
     }
-    if constexpr (RI) fill_ri(b8, a.book8);
+    if constexpr (RI) fill_ri<G1>(b8, a);
     __syncthreads();
     // this CTA's items (expert slot, output row) span at most two experts
     // (the grid has at least as many CTAs as there are experts)
@@ -479,29 +590,30 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
         const int w0 = c0 + (int)((long long)(c1 - c0) * warp / kVWarps);
         const int w1 = c0 + (int)((long long)(c1 - c0) * (warp + 1) / kVWarps);
         const int chunk = skew_pos<VPL>(lane * 8 * VPL);
-        auto load = [&](int i, DNRow<VPL, R8> &r) {
+        auto load = [&](int i, DNRow<VPL, R8, G1> &r) {
             const size_t row = (size_t)s.tb.expert[i >> lH] * H + (i & (H - 1));
-            r.c13.load(a.idx13[2] + row * RB13, lane);
+            if constexpr (G1) r.c13.load(a.code12[2] + row * (I * 3 / 16), a.hi1[2] + row * (I / 64), lane);
+            else r.c13.load(a.idx13[2] + row * RB13, lane);
             if constexpr (R8) r.c8.load(a.idx8[2] + row * RB8, lane);
         };
-        auto compute = [&](int i, DNRow<VPL, R8> &r) {
+        auto compute = [&](int i, DNRow<VPL, R8, G1> &r) {
             const int d = i >> lH, m = i & (H - 1);
             const uint16_t *vr = vs + (size_t)(d - d_lo) * TB * vstride + chunk;
             r.c13.align();
             const int nc = s.ct.ncol[d];
             if (nc > 4) {
-                if constexpr (TB >= 8) dn_row<VPL, R8, RI, 4>(a, s, b13, b8, vr, vstride, d, m, 0, r);
+                if constexpr (TB >= 8) dn_row<VPL, R8, RI, 4, G1>(a, s, b13, b8, vr, vstride, d, m, 0, r);
             }
             const int j0 = nc > 4 ? 4 : 0;
             switch (nc - j0) {
-                case 1: dn_row<VPL, R8, RI, 1>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
-                case 2: if constexpr (TB >= 2) dn_row<VPL, R8, RI, 2>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
-                case 3: if constexpr (TB >= 4) dn_row<VPL, R8, RI, 3>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
-                case 4: if constexpr (TB >= 4) dn_row<VPL, R8, RI, 4>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
+                case 1: dn_row<VPL, R8, RI, 1, G1>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
+                case 2: if constexpr (TB >= 2) dn_row<VPL, R8, RI, 2, G1>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
+                case 3: if constexpr (TB >= 4) dn_row<VPL, R8, RI, 3, G1>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
+                case 4: if constexpr (TB >= 4) dn_row<VPL, R8, RI, 4, G1>(a, s, b13, b8, vr, vstride, d, m, j0, r); break;
                 default: break;
             }
         };
-        DNRow<VPL, R8> ra, rb;
+        DNRow<VPL, R8, G1> ra, rb;
         if (w0 < w1) load(w0, ra);
         for (int i = w0; i < w1; i += 2) {
             if (i + 1 < w1) load(i + 1, rb);
@@ -535,10 +647,10 @@ __global__ void __launch_bounds__(kVThreads, 1) vqd_down_kernel(VqdArgs a) {
 
 // ---------------------------------------------------------------- host
 
-template <int VPL, bool R8, int TB>
-size_t gu_smem() { return books_bytes<R8, use_ri<VPL, R8, TB, false>()>() + gu_stage_bytes(TB, VPL); }
-template <int VPL, bool R8, int TB>
-size_t dn_smem() { return books_bytes<R8, use_ri<VPL, R8, TB, true>()>() + dn_stage_bytes(TB, VPL); }
+template <int VPL, bool R8, int TB, bool G1>
+size_t gu_smem() { return books_bytes<R8, use_ri<VPL, R8, TB, false, G1>(), G1>() + gu_stage_bytes(TB, VPL); }
+template <int VPL, bool R8, int TB, bool G1>
+size_t dn_smem() { return books_bytes<R8, use_ri<VPL, R8, TB, true, G1>(), G1>() + dn_stage_bytes(TB, VPL); }
 
 int tokens_bound(int T) { return T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8)); }
 
@@ -557,27 +669,28 @@ cudaError_t launch_pdl(K kernel, int grid, size_t smem, cudaStream_t s, bool pdl
     return cudaLaunchKernelEx(&cfg, kernel, args);
 }
 
-template <int VPLG, int VPLD, bool R8, int TB>
+template <int VPLG, int VPLD, bool R8, int TB, bool G1>
 cudaError_t run(const Layer &L, const VqdArgs &a, cudaStream_t s, const cudaEvent_t *ev) {
     const int dev = L.d.device;
     static std::once_flag once[64];
     static cudaError_t err[64];
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&] {
-        cudaError_t e = cudaFuncSetAttribute(vqd_gateup_kernel<VPLG, R8, TB>,
+        cudaError_t e = cudaFuncSetAttribute(vqd_gateup_kernel<VPLG, R8, TB, G1>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kVMaxSmem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(vqd_down_kernel<VPLD, R8, TB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            e = cudaFuncSetAttribute(vqd_down_kernel<VPLD, R8, TB, G1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kVMaxSmem);
         err[dev] = e;
     });
     if (err[dev] != cudaSuccess) return err[dev];
     L.count_launches(2);
     if (ev) record_phase(ev[1], s);
-    cudaError_t e = launch_pdl(vqd_gateup_kernel<VPLG, R8, TB>, L.sm_count, gu_smem<VPLG, R8, TB>(), s, ev == nullptr, a);
+    cudaError_t e = launch_pdl(vqd_gateup_kernel<VPLG, R8, TB, G1>, L.sm_count, gu_smem<VPLG, R8, TB, G1>(), s,
+                               ev == nullptr, a);
     if (e != cudaSuccess) return e;
     if (ev) record_phase(ev[2], s);
-    e = launch_pdl(vqd_down_kernel<VPLD, R8, TB>, L.sm_count, dn_smem<VPLD, R8, TB>(), s, ev == nullptr, a);
+    e = launch_pdl(vqd_down_kernel<VPLD, R8, TB, G1>, L.sm_count, dn_smem<VPLD, R8, TB, G1>(), s, ev == nullptr, a);
     if (e != cudaSuccess) return e;
     if (ev) {
         record_phase(ev[3], s);
@@ -586,30 +699,45 @@ cudaError_t run(const Layer &L, const VqdArgs &a, cudaStream_t s, const cudaEven
     return cudaSuccess;
 }
 
-template <int VPLG, int VPLD, bool R8>
+template <int VPLG, int VPLD, bool R8, bool G1>
 cudaError_t run_tb(const Layer &L, const VqdArgs &a, cudaStream_t s, const cudaEvent_t *ev) {
     switch (tokens_bound(a.T)) {
-        case 1: return run<VPLG, VPLD, R8, 1>(L, a, s, ev);
-        case 2: return run<VPLG, VPLD, R8, 2>(L, a, s, ev);
-        case 4: return run<VPLG, VPLD, R8, 4>(L, a, s, ev);
-        default: return run<VPLG, VPLD, R8, 8>(L, a, s, ev);
+        case 1: return run<VPLG, VPLD, R8, 1, G1>(L, a, s, ev);
+        case 2: return run<VPLG, VPLD, R8, 2, G1>(L, a, s, ev);
+        case 4: return run<VPLG, VPLD, R8, 4, G1>(L, a, s, ev);
+        default: return run<VPLG, VPLD, R8, 8, G1>(L, a, s, ev);
     }
 }
 
-template <bool R8>
+template <bool R8, bool G1>
 cudaError_t run_shape(const Layer &L, const VqdArgs &a, cudaStream_t s, const cudaEvent_t *ev) {
-    if (a.H == 4096 && a.I == 2048) return run_tb<16, 8, R8>(L, a, s, ev);
-    if (a.H == 2048 && a.I == 2048) return run_tb<8, 8, R8>(L, a, s, ev);
-    if (a.H == 4096 && a.I == 4096) return run_tb<16, 16, R8>(L, a, s, ev);
-    if (a.H == 2048 && a.I == 4096) return run_tb<8, 16, R8>(L, a, s, ev);
+    if (a.H == 4096 && a.I == 2048) return run_tb<16, 8, R8, G1>(L, a, s, ev);
+    if (a.H == 2048 && a.I == 2048) return run_tb<8, 8, R8, G1>(L, a, s, ev);
+    if (a.H == 4096 && a.I == 4096) return run_tb<16, 16, R8, G1>(L, a, s, ev);
+    if (a.H == 2048 && a.I == 4096) return run_tb<8, 16, R8, G1>(L, a, s, ev);
     return cudaErrorInvalidValue;
+}
+
+// The GVQ1 residual term is folded into the base entries as an f16 pair
+// multiple: the ratio of the book scales must be an f16 value (normal, or
+// zero without a residual stage), and the base scale nonzero.
+bool gvq1_ratio(const Layer &L, uint32_t *rho2) {
+    const float s13 = L.w.gscale[0], s8 = has_r8(L.d.fmt) ? L.w.gscale[1] : 0.f;
+    if (!(s13 != 0.f) || !std::isfinite(s13)) return false;
+    const float rho = s8 / s13;
+    if (!std::isfinite(rho) || (rho != 0.f && (std::fabs(rho) > 65504.f || std::fabs(rho) < 6.103515625e-05f)))
+        return false;
+    const uint16_t b = __half_as_ushort(__float2half_rn(rho));
+    if (rho2) *rho2 = (uint32_t)b | ((uint32_t)b << 16);
+    return true;
 }
 
 }  // namespace
 
 bool decode_vq_supported(const Layer &L, int T) {
     const moeq_layer_desc &d = L.d;
-    if ((d.fmt != MOEQ_FMT_VQ13 && d.fmt != MOEQ_FMT_VQ13_R8) || d.act != MOEQ_ACT_BF16) return false;
+    if (!(is_vq13(d.fmt) || is_gvq1(d.fmt)) || d.act != MOEQ_ACT_BF16) return false;
+    if (is_gvq1(d.fmt) && !gvq1_ratio(L, nullptr)) return false;
     if (!L.vq_acc || !L.vq_done) return false;
     if (T < 1 || T > kVMaxT || T * d.top_k > dec::kMaxR) return false;
     if (!((d.hidden == 2048 || d.hidden == 4096) && (d.inter == 2048 || d.inter == 4096))) return false;
@@ -629,9 +757,16 @@ cudaError_t launch_decode_vq(const Layer &L, const void *x, const int32_t *ids, 
         a.idx13[p] = v.idx13;
         a.idx8[p] = v.idx8;
         a.gain[p] = v.gain;
+        a.code12[p] = v.code12;
+        a.hi1[p] = v.hi1;
     }
+    const bool g1 = is_gvq1(L.d.fmt), r8 = has_r8(L.d.fmt);
     a.book13 = L.w.book13;
     a.book8 = L.d.fmt == MOEQ_FMT_VQ13_R8 ? L.w.book8 : nullptr;
+    a.gbook13 = L.w.gbook13;
+    a.gbook8 = L.d.fmt == MOEQ_FMT_GVQ1_R8 ? L.w.gbook8 : nullptr;
+    a.gs13 = L.w.gscale[0];
+    if (g1 && !gvq1_ratio(L, &a.rho2)) return cudaErrorInvalidValue;
     a.x = reinterpret_cast<const uint16_t *>(x);
     a.ids = ids;
     a.topk_w = topk_w;
@@ -646,7 +781,8 @@ cudaError_t launch_decode_vq(const Layer &L, const void *x, const int32_t *ids, 
     a.E = L.d.n_experts;
     a.H = L.d.hidden;
     a.I = L.d.inter;
-    return a.book8 ? run_shape<true>(L, a, s, ev) : run_shape<false>(L, a, s, ev);
+    if (g1) return r8 ? run_shape<true, true>(L, a, s, ev) : run_shape<false, true>(L, a, s, ev);
+    return r8 ? run_shape<true, false>(L, a, s, ev) : run_shape<false, false>(L, a, s, ev);
 }
 
 }  // namespace moeq
