@@ -308,26 +308,38 @@ def load_peaks():
 
 
 def roofline(cfg, workload, ids_h, warmup, n_total, launch_ms, ms_step, peaks, peak_src, phase_how):
-    """The dominant kernel's roofline (gate/up + SwiGLU) and whole-step figures.
+    """The dominant kernel's roofline and whole-step figures.
 
-    Decode: algorithmic bytes = distinct experts per step x compressed
-    gate+up bytes per expert (+ codebooks), against the measured HBM copy
-    bandwidth.  Prefill: 2 x routes x 2 x H x I flop, against the measured
+    Decode: algorithmic bytes = distinct experts per step x compressed bytes
+    per expert of the projections the kernel streams (all three for the
+    one-launch MXFP4 step; gate+up, + codebooks, for VQ), against the
+    measured HBM copy bandwidth.  Prefill: 2 x routes x 2 x H x I flop, against the measured
     burst bf16 GEMM rate (the kernel runs for milliseconds inside a
     sub-second graph, not under a seconds-long power-capped load)."""
     n_steps = n_total - warmup
     if is_decode(cfg):
         d_mean = float(np.mean([len(np.unique(ids_h[i][(ids_h[i] >= 0) & (ids_h[i] < cfg.E)]))
                                 for i in range(warmup, n_total)]))
-        bytes_gu = d_mean * (proj_bytes(cfg, 0) + proj_bytes(cfg, 1)) + book_bytes(cfg)
-        achieved = bytes_gu / (launch_ms / 1e3) / 1e9
+        if cfg.fmt == "mxfp4":
+            # one kernel does the whole step: its bytes are all three
+            # projections, and its average duration is the step's device time
+            # over the K replayed launches (gaps between launches included)
+            kernel = "decode step (one launch: routing, gate/up + SwiGLU, down, combine)"
+            bytes_k = d_mean * sum(proj_bytes(cfg, p) for p in range(3))
+            per_unit = "compressed gate+up+down bytes of one expert"
+            launch_ms = ms_step
+            phase_how = "one launch per step: CUDA events around the K replayed steps, divided by K"
+        else:
+            kernel = "gate/up + SwiGLU"
+            bytes_k = d_mean * (proj_bytes(cfg, 0) + proj_bytes(cfg, 1)) + book_bytes(cfg)
+            per_unit = "compressed gate+up bytes of one expert (+ codebooks once per launch)"
+        achieved = bytes_k / (launch_ms / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
         traffic, traffic_src = ncu_traffic(workload)
-        roof = {"kernel": "gate/up + SwiGLU", "bound": "hbm", "achieved": achieved, "peak": peak,
+        roof = {"kernel": kernel, "bound": "hbm", "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                "peak_source": f"{peak_src} hbm_gbs", "per_launch_bytes": bytes_gu,
-                "per_unit": "compressed gate+up bytes of one expert (+ codebooks once per launch)",
-                "units_per_launch": d_mean, "launch_ms": launch_ms, "timing": phase_how}
+                "peak_source": f"{peak_src} hbm_gbs", "per_launch_bytes": bytes_k,
+                "per_unit": per_unit, "units_per_launch": d_mean, "launch_ms": launch_ms, "timing": phase_how}
         if traffic_src:
             roof["traffic_source"] = traffic_src
         step_bytes = d_mean * sum(proj_bytes(cfg, p) for p in range(3)) + book_bytes(cfg)
@@ -461,6 +473,125 @@ def measure(workload, steps, warmup, world, rank, local, barrier, cpu_seconds, w
     return res
 
 
+# f32 FMA peak of the CUDA cores: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz (the recipe's unit
+# counts and maximum SM clock), for kernels bound by plain ALU arithmetic
+ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def time_graph(fn, steps, warmup, dev):
+    """Device time (ms) of `steps` calls of fn captured in one CUDA graph,
+    after `warmup` eager calls; CUDA events on the replaying stream."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream(device=dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for _ in range(steps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del g
+    return ms
+
+
+def measure_router(T, steps, warmup, local, peaks, peak_src):
+    """The router kernel (moeq_router, sigmoid weights) on the MiMo shape:
+    tokens/s, and its roofline -- the f32 router matrix (E x H x 4 bytes,
+    the algorithmic bytes; the kernel reads it as three bf16 terms) at one
+    token, 2 T E H flop at prefill sizes."""
+    import torch
+    from bit_quantized_moe_routed_b200 import moeq
+    cfg = synth.get_cfg("decode_mxfp4", T=T)
+    dev = torch.device("cuda", local)
+    lay = moeq.Layer(cfg.H, cfg.I, cfg.E, cfg.k, T, "mxfp4", "bf16", device=local)
+    lay.router_upload(synth.gen_router(cfg), "sigmoid")
+    x = torch.from_numpy(synth.gen_activations(cfg).view(np.int16)).view(torch.bfloat16).to(dev)
+    ids = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+    n0 = lay.kernel_launches()
+    ms = time_graph(lambda: moeq.lib().moeq_router(lay.handle, moeq.C.c_void_p(x.data_ptr()), T,
+                                                  moeq.C.c_void_p(ids.data_ptr()), moeq.C.c_void_p(w.data_ptr()),
+                                                  None, moeq._stream_ptr(None)), steps, warmup, dev)
+    launches = (lay.kernel_launches() - n0) // (steps + warmup)
+    per = ms / steps / 1e3
+    if T <= 8:
+        nbytes = cfg.E * cfg.H * 4 + T * cfg.H * 2
+        roof = {"kernel": "router (logits, top-k, weights)", "bound": "hbm", "achieved": nbytes / per / 1e9,
+                "peak": float(peaks["hbm_gbs"]), "unit": "GB/s", "traffic": None,
+                "per_unit": "the f32 router matrix (E x H x 4 bytes) and the step's activations",
+                "peak_source": f"{peak_src} hbm_gbs"}
+    else:
+        fl = 2.0 * T * cfg.E * cfg.H
+        roof = {"kernel": "router (logits, top-k, weights)", "bound": "tensor", "achieved": fl / per / 1e12,
+                "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s", "traffic": None,
+                "per_unit": "2 x E x H flop per token (the kernel issues three bf16 MMAs per product)",
+                "peak_source": f"{peak_src} bf16_tflops (burst)"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    lay.close()
+    return {"metric": "router tokens/s", "value": T / per, "unit": "tokens/s", "steps": steps, "warmup": warmup,
+            "ms_per_step": ms / steps, "dtype": "bf16 x, f32 router", "config": {"workload": f"router_t{T}",
+            "hidden": cfg.H, "experts": cfg.E, "top_k": cfg.k, "tokens_per_step": T, "score": "sigmoid"},
+            "roofline": roof, "gpu_launches": int(launches * steps)}
+
+
+def measure_encoder(steps, warmup, local, with_cpu):
+    """The VQ encoder (moeq_vq_encode, VQ13+R8, unit column weights) on one
+    MiMo expert's three matrices: weights/s, against the f32 FMA peak with
+    the algorithmic flops 16 x (8192 + 256) per 8-vector (the expanded
+    distance's dot product over both books)."""
+    import torch
+    from bit_quantized_moe_routed_b200 import moeq
+    cfg = synth.get_cfg("decode_vq", E=1)
+    L = synth.gen_layer(cfg, seed=7)
+    dev = torch.device("cuda", local)
+    rng = np.random.default_rng(7)
+    mats = []
+    for p in range(3):
+        N, K = cfg.shape(p)
+        W = torch.from_numpy(rng.normal(0.0, 0.02, size=(N, K)).astype(np.float32)).to(dev)
+        mats.append((W, torch.empty((N, K * 13 // 64), dtype=torch.uint8, device=dev),
+                     torch.empty((N, K // 8), dtype=torch.uint8, device=dev)))
+    b13 = torch.from_numpy(L.book13.view(np.int16)).to(dev)
+    b8 = torch.from_numpy(L.book8.view(np.int16)).to(dev)
+    P = moeq.C.c_void_p
+
+    def fn():
+        for W, o13, o8 in mats:
+            moeq.lib().moeq_vq_encode(P(W.data_ptr()), W.shape[0], W.shape[1], None, None, P(b13.data_ptr()),
+                                      P(b8.data_ptr()), P(o13.data_ptr()), P(o8.data_ptr()), moeq._stream_ptr(None))
+    ms = time_graph(fn, steps, warmup, dev)
+    n_w = sum(W.numel() for W, _, _ in mats)
+    per = ms / steps / 1e3
+    fl = 16.0 * (8192 + 256) * (n_w / 8)
+    roof = {"kernel": "vq_encode_kernel", "bound": "alu", "achieved": fl / per / 1e12, "peak": ALU_F32_TFLOPS,
+            "unit": "TFLOP/s", "frac": fl / per / 1e12 / ALU_F32_TFLOPS, "traffic": None,
+            "per_unit": "16 x (8192 + 256) flop per 8-weight vector",
+            "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz"}
+    line = {"metric": "VQ encode weights/s", "value": n_w / per, "unit": "weights/s", "steps": steps,
+            "warmup": warmup, "ms_per_step": ms / steps, "dtype": "f32", "config": {
+                "workload": "vq_encode_expert", "matrices": "gate, up [2048][4096], down [4096][2048]",
+                "format": "vq13r8", "weights": "N(0, 0.02^2)", "column_weights": None},
+            "roofline": roof, "gpu_launches": 3 * steps}
+    if with_cpu:
+        import oracle.vq_encode as ve
+        W0 = mats[0][0][:2].cpu().numpy()
+        t0 = time.perf_counter()
+        ve.encode_rows(W0, L.book13, L.book8)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": W0.size / dt, "unit": "weights/s", "cores": os.cpu_count(),
+                                "kind": "oracle", "sample": f"2 rows of the gate matrix ({W0.size} weights), "
+                                f"{dt:.1f} s"}
+    return line
+
+
 def summarize(args, workload, r, world, steps, warmup, peaks, peak_src):
     """The contract's fields for one measured workload (times already reduced over ranks)."""
     cfg = r["cfg"]
@@ -539,6 +670,16 @@ def main():
                 lx.pop(key, None)
             extra[name] = lx
         torch.cuda.empty_cache()
+
+    if extra_names:
+        # the steps on either side of the layer: the router and the VQ encoder
+        for T in (1, 2048):
+            rr = measure_router(T, args.extra_steps, args.warmup, local, peaks, peak_src)
+            if rank == 0:
+                extra[f"router_t{T}"] = rr
+        re_ = measure_encoder(3, 3, local, with_cpu)
+        if rank == 0:
+            extra["vq_encode_expert"] = re_
 
     if rank == 0:
         if extra:

@@ -223,7 +223,7 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     ALLOC(L->h, sizeof(float) * M * k * I);
     ALLOC(L->acc, sizeof(float) * M * H);
     ALLOC(L->dec_ybuf, sizeof(float) * kDecMaxRoutes * kDecMaxTokens * H);
-    ALLOC(L->dec_counters, sizeof(int) * (H / 32 + 1));
+    ALLOC(L->dec_counters, sizeof(int) * 2);
     ALLOC(L->status, sizeof(uint32_t));
     ALLOC(L->x_stage, (size_t)L->elem_bytes() * M * H);
     ALLOC(L->out_stage, (size_t)L->elem_bytes() * M * H);
@@ -233,7 +233,7 @@ moeq_status moeq_layer_create(const moeq_layer_desc *desc, moeq_layer_t *out) {
     if (e == cudaSuccess) e = prefill_mx_create(*L);
     if (e == cudaSuccess) e = prefill_vq_create(*L);
     if (e == cudaSuccess) e = cudaMemset(L->status, 0, sizeof(uint32_t));
-    if (e == cudaSuccess) e = cudaMemset(L->dec_counters, 0, sizeof(int) * (H / 32 + 1));
+    if (e == cudaSuccess) e = cudaMemset(L->dec_counters, 0, sizeof(int) * 2);
     if (e == cudaSuccess && L->vq_acc) e = cudaMemset(L->vq_acc, 0, sizeof(float) * kDecMaxTokens * H);
     if (e == cudaSuccess && L->vq_done) e = cudaMemset(L->vq_done, 0, sizeof(int));
     if (e != cudaSuccess) {
@@ -470,10 +470,10 @@ moeq_status moeq_layer_status(moeq_layer_t L, int32_t clear) {
     uint32_t v = 0;
     cudaError_t e = cudaMemcpy(&v, L->status, sizeof(v), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && clear) e = cudaMemset(L->status, 0, sizeof(uint32_t));
-    // a kernel that gave up on a wait may have left the decode combine's
-    // per-tile arrival counters part-way: clearing the status resets them
+    // a decode step that gave up on a wait may have left its grid barrier
+    // part-way: clearing the status resets it
     if (e == cudaSuccess && clear && (v & FLAG_TIMEOUT))
-        e = cudaMemset(L->dec_counters, 0, sizeof(int) * (L->d.hidden / 32 + 1));
+        e = cudaMemset(L->dec_counters, 0, sizeof(int) * 2);
     if (e != cudaSuccess) return from_cuda(e);
     if (v & FLAG_ROUTE_RANGE) return MOEQ_ERR_ROUTE_OUT_OF_RANGE;
     if (v & FLAG_TIMEOUT) return MOEQ_ERR_TIMEOUT;

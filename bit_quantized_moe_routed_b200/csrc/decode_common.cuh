@@ -44,6 +44,7 @@ __device__ inline void build_route_table(RouteTable &tb, const int32_t *__restri
     const bool bad = (r0 < R && !v0 && id0 != -1) || (r1 < R && !v1 && id1 != -1);
     if (report && __any_sync(full, bad) && lane == 0) atomicOr(status, FLAG_ROUTE_RANGE);
     int rank0 = 0, rank1 = 0;
+#pragma unroll 8
     for (int q = 0; q < R; ++q) {
         const int idq = __shfl_sync(full, q < 32 ? id0 : id1, q & 31);
         if (idq >= 0 && idq < E) {

@@ -1,39 +1,39 @@
 // decode_mx.cu -- MXFP4 routed-expert FFN at decode sizes (1..8 tokens,
 // bf16 activations): a grouped GEMV that streams each selected expert's
-// packed codes from HBM once.
+// packed codes from HBM once, the whole step in one kernel launch.
 //
 // Layer: out[t] = sum_s w[t,s] W_down,e (silu(W_gate,e x_t) * (W_up,e x_t))
 // ("MiMo-V2.6-Flash-RL GGUF for a single DGX Spark", "Architecture notes":
 // top-8 of 256 routed experts, MXFP4 experts with one E8M0 exponent per 32
 // values; "Recipe": expert intermediates stay in a type with f32's range).
 //
-// Work: a unit is one expert's 16 gate + 16 up rows (gate/up kernel) or 32
-// down rows (down kernel) over the full K; each CTA (one per SM) takes a
-// contiguous, balanced range of units.  The 8 consumer warps form one group
-// per 1024-column chunk of K, so every chunk of a unit is in compute at
-// once; inside a group each warp takes a share of the chunk's 32-weight
-// block columns for both halves (gate and up, or the two 16-row down tiles),
-// i.e. two independent accumulator chains.  A warp reads the fragments of
-// its next group while it computes the current one.  Per unit the warps
-// hand their partial fragments to two epilogue warps through a two-slot
-// ring (full/empty mbarriers), which sum them (SwiGLU and h for gate/up),
-// so the consumers never wait for one another.  (Four slots took shared
-// memory from the stage ring and measured slower at T = 8.)  Eight consumer warps keep every register a warp
-// needs (up to 153, no spills); sixteen did not fit without spilling.
+// One cooperative launch, one CTA per SM, all co-resident: phase 1 computes
+// h for the gate/up units, phase 2 the down units, phase 3 the combine; two
+// grid barriers (bounded waits) separate them.  The route table is built
+// once per CTA.  A gate/up unit is one expert's 16 gate + 16 up rows over
+// the full K, a down unit 32 down rows; each CTA takes a contiguous,
+// balanced range of units in each phase.  The 8 consumer warps form one
+// group per 1024-column chunk of K, so every chunk of a unit is in compute
+// at once; inside a group each warp takes a share of the chunk's 32-weight
+// block columns for both halves (gate and up, or the two 16-row down
+// tiles), i.e. two independent accumulator chains.  A warp reads the
+// fragments of its next group while it computes the current one.  Per unit
+// the warps hand their partial fragments to two epilogue warps through a
+// two-slot ring (full/empty mbarriers), which sum them (SwiGLU and h in
+// phase 1, the expert's f32 output slice in phase 2), so the consumers
+// never wait for one another.  Eight consumer warps keep every register a
+// warp needs (up to 161, no spills).
 //
 // Memory: the device layout (MxGeom) keeps each (16-row tile, 1024-column
 // chunk) block contiguous, so a producer warp streams a chunk of a unit as
 // two 8.7 KB bulk copies (TMA) into a ring of shared-memory stages with
-// full/empty mbarriers, unit by unit and chunk by chunk (one chunk per stage
-// where the stage count allows it, so a chunk's warps start as soon as it
-// lands); the activations
-// arrive first, one bulk copy per token.  Bulk copies of several KB are what
-// keep HBM busy; the layout also makes the fragment and scale reads
-// bank-conflict free.  The gate/up kernel lets the down kernel launch as its
-// CTAs finish (programmatic dependent launch): the down weights stream in
-// while gate/up drains, and only the down consumers wait for h.  The down
-// kernel does the same for the next gate/up launch, which waits for it
-// before reading anything.
+// full/empty mbarriers.  The ring serves both weight phases (a piece is the
+// same pair of blocks in both), and the producer runs on from the last
+// gate/up piece into the down pieces: the down weights stream in while
+// phase 1 drains and while the CTA waits at the barrier.  The activations
+// arrive first, one bulk copy per token, issued before the routing is read.
+// Bulk copies of several KB are what keep HBM busy; the layout also makes
+// the fragment and scale reads bank-conflict free.
 //
 // Math: warp-level mma.sync.m16n8k16 (f16 in, f32 accumulate).  Each thread
 // reads its A-fragment slice of four 32-weight blocks (bytes 4t..4t+3 of
@@ -46,11 +46,10 @@
 // (expert, token) column of w * h for the down projection.  f16 cannot
 // overflow, and the scale is undone in f32.
 //
-// Combine: the down kernel writes each expert's contribution, prescale
-// undone, to its own slice of a scratch buffer; a third, small kernel (one
-// output element per thread, launched as a programmatic dependent) sums the
-// slices in expert order and writes bf16 out, so the result does not depend
-// on timing and the sum is spread over the whole GPU.
+// Combine: phase 2 writes each expert's contribution, prescale undone, to
+// its own slice of a scratch buffer; after the second barrier every CTA sums
+// the slices of its share of the outputs in expert order and writes bf16,
+// so the result does not depend on timing.
 #include <mutex>
 
 #include "async.cuh"
@@ -339,30 +338,10 @@ __device__ __forceinline__ void compute_group(const GroupFrags &f, const uint4 x
     }
 }
 
-// ---------------------------------------------------------------- gate/up
-
-struct GateUpArgs {
-    const uint8_t *codes_g, *codes_u;   // gate, up projections in the device layout (MxGeom)
-    const uint16_t *x;                  // bf16 [T][H]
-    const int32_t *ids;                 // [T][k]
-    const float *topk_w;                // [T][k]
-    float *h;                           // [T*k][I] f32, by route id
-    uint32_t *status;
-    long long wait_cycles;              // limit of every wait but the final drains
-    FastDiv S;                          // stages
-    int T, k, E, H, I, cps;
-};
+// ---------------------------------------------------------------- units
 
 constexpr int kGUThreads = 32 * (kCW + 1 + kEpiWarps);
 constexpr int kEpiWarp0 = kCW + 1;
-
-__host__ __device__ inline size_t gu_xs_off(int n_stages, int cps) { return (size_t)n_stages * piece_bytes(cps); }
-__host__ __device__ inline size_t gu_red_off(int n_stages, int cps, int T, int H) {
-    return gu_xs_off(n_stages, cps) + sizeof(uint16_t) * (size_t)T * (H + kXPad);
-}
-__host__ __device__ inline size_t gu_bytes(int n_stages, int cps, int T, int H) {
-    return gu_red_off(n_stages, cps, T, H) + red_bytes(T);
-}
 
 // Unit i -> (expert slot d, column chunk, 16-row tile): an expert's routes
 // are taken Tc = min(T, 8) columns per pass (the width of the partial-sum
@@ -378,37 +357,217 @@ __device__ __forceinline__ int unit_tile(uint32_t u) { return (int)((u >> 6) & 5
 __device__ __forceinline__ int unit_cb(uint32_t u) { return (int)((u >> 15) & 127u); }
 __device__ __forceinline__ int unit_ncol(uint32_t u) { return (int)(u >> 22); }
 
-template <int NCH>   // K chunks per unit = H / kKC
-__global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs a) {
-    static_assert(kCW % NCH == 0 && 8 % (kCW / NCH) == 0, "warps per chunk must divide the 8 K-groups of a chunk");
+// Staged (expert, token) B columns per CTA.  A CTA's contiguous range of
+// units is no longer than one expert's tiles when the grid has at least as
+// many CTAs as there are routed experts, so it touches at most two experts:
+// at most 2T columns.
+constexpr int kMaxBSlots = 16;
+constexpr int kMaxTiles = 128;   // H / 32 for H <= 4096
+__host__ __device__ inline int dn_slots(int T) { return 2 * T < kMaxBSlots ? 2 * T : kMaxBSlots; }
+
+// ---------------------------------------------------------------- one launch
+
+// The whole decode step as one cooperative launch (one CTA per SM, all
+// co-resident): phase 1 the gate/up units, phase 2 the down units, phase 3
+// the combine, separated by two grid barriers.  One ring of stages serves
+// both weight phases (a piece is the same pair of blocks of a chunk in
+// both), and the producer runs on from the last gate/up piece into the down
+// pieces, so the down weights stream in while gate/up drains and while the
+// CTA waits at the barrier; the route table is built once.  The region of
+// the staged activations holds the down B columns once phase 1 is over.
+
+// Grid barrier: bar[0] counts arrivals, bar[1] is a generation number that
+// the last arrival advances after it resets the count.  A CTA reads the
+// generation once before its first arrival (gen0) and has passed barrier b
+// (1 or 2) once the generation is gen0 + b.  Each CTA arrives once per
+// barrier, and at barrier 2 only after it passed barrier 1, so an arrival
+// is never counted at the wrong barrier.
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int *p, int v) {
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void red_add_release_gpu(int *p, int v) {
+    asm volatile("red.add.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// The arrival releases what this thread (and, through the CTA barrier before
+// it, its CTA) wrote; the last arrival acquires every other arrival's
+// release, resets the count and releases the new generation.
+__device__ __forceinline__ void grid_arrive(int *bar) {
+    if (atom_add_acq_rel_gpu(bar, 1) == (int)gridDim.x - 1) {
+        atomicExch(bar, 0);
+        red_add_release_gpu(bar + 1, 1);
+    }
+}
+__device__ __forceinline__ bool grid_wait(const int *bar, int gen0, int b, volatile int *abort, long long limit) {
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(bar + 1) - gen0 < b) {
+        if (*abort) return false;
+        if (clock64() - t0 > limit) {
+            *abort = 1;
+            return false;
+        }
+        __nanosleep(20);
+    }
+    return true;
+}
+
+// Barrier among the epilogue warps (id 2).
+__device__ __forceinline__ void named_sync_epilogue() {
+    asm volatile("bar.sync 2, %0;" ::"r"(32 * kEpiWarps) : "memory");
+}
+
+// The consumer warps' side of one weight phase: n units of NCH chunks each,
+// the phase's pieces numbered from p0 in the ring and its partial-sum
+// hand-offs from r0.  brow(j, live) is this lane's B row for unit j (f16,
+// offset by 8t).  Each warp releases a stage with NCH arrivals, so a piece
+// takes kCW * cps arrivals in either phase.  False if a wait gave up.
+template <int NCH, typename BRow>
+__device__ __forceinline__ bool consume_phase(const uint8_t *stages, uint64_t *full, uint64_t *empty,
+                                              uint64_t *red_full, uint64_t *red_empty, float *red, int Tc,
+                                              FastDiv S, int cps, int n, int p0, int r0, volatile int *issued,
+                                              volatile int *abort, long long lim, BRow brow) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    constexpr int WPC = kCW / NCH;   // warps per chunk
+    constexpr int NG = 8 / WPC;      // K-groups of this warp per unit
+    const int q = warp / WPC, wi = warp % WPC;
+    const int lcps = cps == 4 ? 2 : (cps == 2 ? 1 : 0);
+    bool ok = true;
+    const uint8_t *st0 = stages, *st1 = stages;
+    int s_cur = 0;
+    auto open_unit = [&](int j, const uint8_t *&b0, const uint8_t *&b1, int &s) {
+        const int c = j * NCH + q, pc = p0 + (c >> lcps);
+        if (!wait_piece(full, S, pc, issued, abort, lim)) ok = false;
+        s = pc - (int)(S.div((uint32_t)pc) * S.d);
+        b0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c & (cps - 1)) * kBlk;
+        b1 = b0 + (size_t)cps * kBlk;
+    };
+    GroupFrags cur;
+    if (n > 0) {
+        open_unit(0, st0, st1, s_cur);
+        load_group(st0, st1, g, t, wi * NG, cur);
+    }
+    for (int j = 0; j < n && ok; ++j) {
+        bool live;
+        const uint16_t *row = brow(j, live);
+        float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int p = 0; p < NG; ++p) {
+            const int gp = wi * NG + p;
+            const uint8_t *n0 = st0, *n1 = st1;
+            int ns = s_cur;
+            GroupFrags nxt;
+            if (p + 1 < NG) {
+                load_group(st0, st1, g, t, gp + 1, nxt);
+            } else {
+                // the unit's groups are all in registers: release its stage
+                // before waiting for the next unit's piece
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cnt(&empty[s_cur], NCH);
+                if (j + 1 < n) {
+                    open_unit(j + 1, n0, n1, ns);
+                    load_group(n0, n1, g, t, wi * NG, nxt);
+                }
+            }
+            const uint16_t *xq = row + q * kKC + gp * 128;
+            uint4 xb[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) xb[jj] = live ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
+            compute_group(cur, xb, a0, a1);
+            cur = nxt;
+            st0 = n0;
+            st1 = n1;
+            s_cur = ns;
+        }
+        const int jj = r0 + j, slot = jj % kRedSlots;
+        if (jj >= kRedSlots && !mbar_wait_abort(&red_empty[slot], (uint32_t)((jj / kRedSlots - 1) & 1), abort, lim))
+            ok = false;
+        put_partials(red + (size_t)slot * kCW * 2 * 16 * Tc, Tc, warp, g, t, a0, a1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_full[slot]);
+    }
+    return ok;
+}
+
+struct FusedArgs {
+    const uint8_t *codes_g, *codes_u, *codes_d;   // the three projections in the device layout (MxGeom)
+    const uint16_t *x;                            // bf16 [T][H]
+    const int32_t *ids;                           // [T][k]
+    const float *topk_w;                          // [T][k]
+    float *h;                                     // [T*k][I] f32, by route id
+    float *ybuf;                                  // [kMaxR expert slots][kMaxT][H]
+    int *gbar;                                    // grid barrier words (count, generation)
+    uint16_t *out;                                // bf16 [T][H]
+    uint32_t *status;
+    long long wait_cycles;                        // limit of every wait but the final drains
+    FastDiv S;                                    // stages
+    int T, k, E, H, I, cps;
+};
+
+// Shared memory: [stages][activations | down B columns][partial sums].
+__host__ __device__ inline size_t fu_xb_bytes(int T, int H, int I) {
+    const size_t xr = sizeof(uint16_t) * (size_t)T * (H + kXPad);
+    const size_t br = sizeof(uint16_t) * (size_t)dn_slots(T) * (I + kXPad);
+    return xr > br ? xr : br;
+}
+__host__ __device__ inline size_t fu_red_off(int n_stages, int cps, int T, int H, int I) {
+    return (size_t)n_stages * piece_bytes(cps) + fu_xb_bytes(T, H, I);
+}
+__host__ __device__ inline size_t fu_bytes(int n_stages, int cps, int T, int H, int I) {
+    return fu_red_off(n_stages, cps, T, H, I) + red_bytes(T);
+}
+
+template <int NCU, int NCD>   // K chunks of a gate/up unit (H / kKC) and of a down unit (I / kKC)
+__global__ void __launch_bounds__(kGUThreads, 1) dec_fused_mx_kernel(FusedArgs a) {
+    static_assert(kCW % NCU == 0 && 8 % (kCW / NCU) == 0 && kCW % NCD == 0 && 8 % (kCW / NCD) == 0,
+                  "warps per chunk must divide the 8 K-groups of a chunk");
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ RouteTable tb;
     __shared__ GUItems items;
     __shared__ uint32_t units[kMaxUnits];
     __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], xbar, red_full[kRedSlots],
         red_empty[kRedSlots];
-    __shared__ int issued;   // chunks issued by the producer (see produce)
-    __shared__ volatile int abort_flag;   // set by the first role that gives up on a wait
-    __shared__ int n_units, unit0;
+    __shared__ int issued;                 // pieces issued by the producer (see produce)
+    __shared__ volatile int abort_flag;    // set by the first role that gives up on a wait
+    __shared__ int n_gu, unit0, gen0;
     __shared__ float xinv[kMaxT];
+    __shared__ int slot_of[2][kMaxT];      // (expert slot - d_lo, token) -> staged B column, -1 none
+    __shared__ int slot_d[kMaxBSlots], slot_t[kMaxBSlots];
+    __shared__ unsigned slot_max[kMaxBSlots];
+    __shared__ float slot_scale[kMaxBSlots], slot_inv[kMaxBSlots];
+    __shared__ int n_slots;
     const int H = a.H, I = a.I, T = a.T, k = a.k, S = (int)a.S.d, cps = a.cps, Tc = red_cols(a.T);
     uint8_t *stages = smem_raw;
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw + gu_xs_off(S, cps));
-    float *red = reinterpret_cast<float *>(smem_raw + gu_red_off(S, cps, T, H));
-    const int xs_stride = H + kXPad;
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_raw + (size_t)S * piece_bytes(cps));   // phase 1
+    uint16_t *bs = xs;                                                                       // phase 2
+    float *red = reinterpret_cast<float *>(smem_raw + fu_red_off(S, cps, T, H, I));
+    const int xs_stride = H + kXPad, bs_stride = I + kXPad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int tiles = I / 16;
-    const MxGeom geo(I, H);
-    constexpr int WPC = kCW / NCH;   // warps per chunk
-    const int lcps = cps == 4 ? 2 : (cps == 2 ? 1 : 0);
+    const int gu_tiles = I / 16, dn_tiles = H / 32;
+    const MxGeom ggeo(I, H), dgeo(H, I);
 
+    // the activations do not depend on the routing: the producer warp
+    // starts their copies first thing (one bulk copy per token row)
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            mbar_init(&xbar, 1);
+            mbar_fence_init();
+            mbar_arrive_expect_tx(&xbar, (uint32_t)(T * H * 2));
+        }
+        __syncwarp();
+        if (lane < T) bulk_g2s(xs + (size_t)lane * xs_stride, a.x + (size_t)lane * H, H * 2, &xbar);
+    }
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], WPC * cps);
+            mbar_init(&empty[s], kCW * cps);
         }
-        mbar_init(&xbar, 1);
         for (int r = 0; r < kRedSlots; ++r) {
             mbar_init(&red_full[r], kCW);
             mbar_init(&red_empty[r], kEpiWarps);
@@ -417,33 +576,43 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
         issued = 0;
         abort_flag = 0;
     }
+    if (warp == kEpiWarp0 && lane == 0) gen0 = ld_acquire_gpu(a.gbar + 1);   // before this CTA's first arrival
+    if (tid < kMaxBSlots) slot_max[tid] = 0u;
     const long long lim = a.wait_cycles;
-    // launched as a programmatic dependent of the previous kernel in the
-    // stream: its outputs (these inputs, or h that kernel still reads) are
-    // ready and free only after this wait; the dependents this kernel lets
-    // launch below therefore see finished inputs as well
-    pdl_wait_primary();
     if (warp == 0) {
         build_route_table(tb, a.ids, a.topk_w, T * k, k, a.E, a.status, blockIdx.x == 0);
         __syncwarp();
-        if (lane == 0) {
-            int n = 0;
-            for (int d = 0; d < tb.D; ++d) {
-                items.beg[d] = n;
-                n += ((tb.col_beg[d + 1] - tb.col_beg[d] + Tc - 1) / Tc) * tiles;
+        // units per expert slot (lane d and d + 32), exclusive prefix sum over the warp
+        const int D = tb.D;
+        int c0 = 0, c1 = 0;
+        if (lane < D) c0 = ((tb.col_beg[lane + 1] - tb.col_beg[lane] + Tc - 1) / Tc) * gu_tiles;
+        if (lane + 32 < D) c1 = ((tb.col_beg[lane + 33] - tb.col_beg[lane + 32] + Tc - 1) / Tc) * gu_tiles;
+        int s0 = c0, s1 = c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v0 = __shfl_up_sync(0xffffffffu, s0, o), v1 = __shfl_up_sync(0xffffffffu, s1, o);
+            if (lane >= o) {
+                s0 += v0;
+                s1 += v1;
             }
-            items.beg[tb.D] = n;
+        }
+        const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+        if (lane < D) items.beg[lane] = s0 - c0;
+        if (lane + 32 < D) items.beg[lane + 32] = tot0 + s1 - c1;
+        const int n = tot0 + __shfl_sync(0xffffffffu, s1, 31);
+        if (lane == 0) {
+            items.beg[D] = n;
             items.n = n;
             int i0, i1;
             my_range(n, i0, i1);
             unit0 = i0;
-            n_units = min(i1 - i0, kMaxUnits);
+            n_gu = min(i1 - i0, kMaxUnits);
         }
         __syncwarp();
-        // this CTA's units, one per lane (tiles is a power of two; binary
-        // search for the expert slot: beg[d] <= i < beg[d + 1])
-        const int ltiles = 31 - __clz(tiles), D = tb.D;
-        for (int j = lane; j < n_units; j += 32) {
+        // this CTA's gate/up units, one per lane (binary search for the
+        // expert slot: beg[d] <= i < beg[d + 1])
+        const int ltiles = 31 - __clz(gu_tiles);
+        for (int j = lane; j < n_gu; j += 32) {
             const int i = unit0 + j;
             int lo = 0, hi = D - 1;
             while (lo < hi) {
@@ -451,40 +620,52 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
                 if (items.beg[mid] <= i) lo = mid;
                 else hi = mid - 1;
             }
-            const int d = lo, rel = i - items.beg[d], pass = rel >> ltiles, tile = rel & (tiles - 1);
+            const int d = lo, rel = i - items.beg[d], pass = rel >> ltiles, tile = rel & (gu_tiles - 1);
             const int cb = tb.col_beg[d] + pass * Tc, ncol = min(Tc, tb.col_beg[d + 1] - cb);
             units[j] = (uint32_t)d | ((uint32_t)tile << 6) | ((uint32_t)cb << 15) | ((uint32_t)ncol << 22);
         }
     }
     __syncthreads();
-    // the down kernel may take SMs as this grid's CTAs finish: it streams
-    // its weights at once and reads h only after this grid completes
-    pdl_launch_dependents();
-    const int n_mine = n_units;
+    // down units: unit u -> expert slot u / dn_tiles, 32-row tile u % dn_tiles
+    const int n_gu_units = n_gu;
+    const int ldt = 31 - __clz(dn_tiles);
+    int u0, u1;
+    my_range(tb.D * dn_tiles, u0, u1);
+    const int n_dn = u1 - u0;
+    const int d_lo = n_dn > 0 ? u0 >> ldt : 0;
+    const int n_gu_p = n_gu_units * NCU / cps;   // pieces of phase 1
 
     if (warp == kProducerWarp) {
-        // the activations first (one bulk copy per token row, into padded rows)
-        if (lane == 0) mbar_arrive_expect_tx(&xbar, (uint32_t)(T * H * 2));
-        __syncwarp();
-        if (lane < T) bulk_g2s(xs + (size_t)lane * xs_stride, a.x + (size_t)lane * H, H * 2, &xbar);
-        produce(stages, full, empty, a.S, cps, n_mine * NCH / cps, &abort_flag, lim, &issued,
+        produce(stages, full, empty, a.S, cps, n_gu_p + n_dn * NCD / cps, &abort_flag, lim, &issued,
                 [&](int p, const uint8_t *&b0, const uint8_t *&b1) {
-                    const int c = p * cps;
-                    const uint32_t u = units[c / NCH];
-                    const size_t off = (size_t)tb.expert[unit_d(u)] * geo.expert_bytes() +
-                                       geo.block_off(unit_tile(u), c % NCH);
-                    b0 = a.codes_g + off;
-                    b1 = a.codes_u + off;
+                    if (p < n_gu_p) {
+                        const int c = p * cps;
+                        const uint32_t u = units[c / NCU];
+                        const size_t off = (size_t)tb.expert[unit_d(u)] * ggeo.expert_bytes() +
+                                           ggeo.block_off(unit_tile(u), c % NCU);
+                        b0 = a.codes_g + off;
+                        b1 = a.codes_u + off;
+                    } else {
+                        const int c = (p - n_gu_p) * cps;
+                        const int u = u0 + c / NCD, d = u >> ldt, t32 = u & (dn_tiles - 1), qq = c % NCD;
+                        const uint8_t *eb = a.codes_d + (size_t)tb.expert[d] * dgeo.expert_bytes();
+                        b0 = eb + dgeo.block_off(2 * t32, qq);
+                        b1 = eb + dgeo.block_off(2 * t32 + 1, qq);
+                    }
                 });
         return;
     }
 
     if (warp >= kEpiWarp0) {
-        // epilogue: sum the 16 warps' partial fragments of a unit, SwiGLU, h
         const int e = warp - kEpiWarp0;
-        for (int j = 0; j < n_mine; ++j) {
+        bool ok = true;
+        // phase 1: sum the consumers' partial fragments of a unit, SwiGLU, h
+        for (int j = 0; j < n_gu_units && ok; ++j) {
             const int slot = j % kRedSlots;
-            if (!mbar_wait_abort(&red_full[slot], (uint32_t)((j / kRedSlots) & 1), &abort_flag, lim)) break;
+            if (!mbar_wait_abort(&red_full[slot], (uint32_t)((j / kRedSlots) & 1), &abort_flag, lim)) {
+                ok = false;
+                break;
+            }
             const uint32_t u = units[j];
             const int cb = unit_cb(u), ncol = unit_ncol(u), n0 = unit_tile(u) * 16;
             const float *rb = red + (size_t)slot * kCW * 2 * 16 * Tc;
@@ -498,14 +679,56 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
             __syncwarp();
             if (lane == 0) mbar_arrive(&red_empty[slot]);
         }
+        // this CTA's share of h is written: one arrival at barrier 1
+        named_sync_epilogue();
+        if (e == 0 && lane == 0 && ok && !abort_flag) grid_arrive(a.gbar);
+        // phase 2: undo the column prescale and store the expert's f32 slice
+        for (int j = 0; j < n_dn && ok; ++j) {
+            const int jj = n_gu_units + j, slot = jj % kRedSlots;
+            if (!mbar_wait_abort(&red_full[slot], (uint32_t)((jj / kRedSlots) & 1), &abort_flag, lim)) {
+                ok = false;
+                break;
+            }
+            const int u = u0 + j, d = u >> ldt, m0 = (u & (dn_tiles - 1)) * 32;
+            const float *rb = red + (size_t)slot * kCW * 2 * 16 * Tc;
+            for (int idx = lane + 32 * e; idx < 32 * T; idx += 32 * kEpiWarps) {
+                const int row = idx & 31, col = idx >> 5;
+                const int sl = slot_of[d - d_lo][col];
+                const float v = sl >= 0 ? sum_partials(rb, Tc, row >> 4, row & 15, col) * slot_inv[sl] : 0.f;
+                __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row, v);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_empty[slot]);
+        }
+        // the slices are written: one arrival at barrier 2, after barrier 1
+        named_sync_epilogue();
+        if (e == 0 && lane == 0 && ok && !abort_flag && grid_wait(a.gbar, gen0, 1, &abort_flag, lim))
+            grid_arrive(a.gbar);
         __syncwarp();
         if (abort_flag && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
         return;
     }
 
-    // ---- consumers: x -> f16 in place, with a per-token power-of-two
-    // prescale (warp w <-> token w)
-    bool timed_out = !mbar_wait_abort(&xbar, 0, &abort_flag, lim);
+    // ---- consumers.  The B columns of this CTA's down experts (the
+    // (expert, token) pairs with routes), while the weights stream in
+    if (tid == 0) {
+        int ns = 0;
+        const int d_hi = n_dn > 0 ? (u1 - 1) >> ldt : -1;
+        for (int dd = 0; dd < 2; ++dd)
+            for (int tk = 0; tk < kMaxT; ++tk) slot_of[dd][tk] = -1;
+        for (int d = d_lo; d <= d_hi && d < d_lo + 2; ++d)
+            for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) {
+                const int tk = tb.tok[tb.route[cc]];
+                if (ns < kMaxBSlots && slot_of[d - d_lo][tk] < 0) {
+                    slot_of[d - d_lo][tk] = ns;
+                    slot_d[ns] = d;
+                    slot_t[ns++] = tk;
+                }
+            }
+        n_slots = ns;
+    }
+    // x -> f16 in place, with a per-token power-of-two prescale (warp w <-> token w)
+    bool ok = mbar_wait_abort(&xbar, 0, &abort_flag, lim);
     if (warp < T) {
         uint4 *row = reinterpret_cast<uint4 *>(xs + (size_t)warp * xs_stride);
         float m = 0.f;
@@ -536,225 +759,29 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_gateup_mx_kernel(GateUpArgs
     }
     named_sync_consumers();
 
-    // Each warp walks its groups of every unit one ahead: the fragments of
-    // the next group (the next unit's first group at the end of a unit) are
-    // read from shared memory while the current group is computed.  A unit's
-    // stage is released once its last group is in registers, before the
-    // warp waits for the next unit's piece.
-    const int q = warp / WPC, wi = warp % WPC;   // this warp's chunk of every unit and its place in it
-    constexpr int NG = 8 / WPC;                  // groups of this warp per unit (8 per chunk)
-    const uint8_t *st0 = stages, *st1 = stages;
-    int s_cur = 0;
-    auto open_unit = [&](int j, const uint8_t *&b0, const uint8_t *&b1, int &s) {
-        const int c = j * NCH + q, pc = c >> lcps;
-        if (!wait_piece(full, a.S, pc, &issued, &abort_flag, lim)) timed_out = true;
-        s = pc - (int)(a.S.div((uint32_t)pc) * a.S.d);
-        // [gate blocks of the piece][up blocks of the piece]
-        b0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c & (cps - 1)) * kBlk;
-        b1 = b0 + (size_t)cps * kBlk;
-    };
-    GroupFrags cur;
-    if (n_mine > 0) {
-        open_unit(0, st0, st1, s_cur);
-        load_group(st0, st1, g, t, wi * NG, cur);
-    }
-    for (int j = 0; j < n_mine && !timed_out; ++j) {
-        const uint32_t u = units[j];
-        const int cb = unit_cb(u), ncol = unit_ncol(u);
-        const bool live = g < ncol;
-        const int tok = live ? tb.tok[tb.route[cb + g]] : 0;
-        const uint16_t *xrow = xs + (size_t)tok * xs_stride + 8 * t;
-        float aG[4] = {0.f, 0.f, 0.f, 0.f}, aU[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int p = 0; p < NG; ++p) {
-            const int gp = wi * NG + p;
-            const uint8_t *n0 = st0, *n1 = st1;
-            int ns = s_cur;
-            GroupFrags nxt;
-            if (p + 1 < NG) {
-                load_group(st0, st1, g, t, gp + 1, nxt);
-            } else {
-                // every group of this unit was read before the compute that
-                // precedes this step: release the stage before waiting for
-                // the next unit's piece (holding it could wait on itself)
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s_cur]);
-                if (j + 1 < n_mine) {
-                    open_unit(j + 1, n0, n1, ns);
-                    load_group(n0, n1, g, t, wi * NG, nxt);
-                }
-            }
-            const uint16_t *xq = xrow + (size_t)(q * (kKC / 32) + gp * 4) * 32;
-            uint4 xb[4];
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) xb[jj] = live ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
-            compute_group(cur, xb, aG, aU);
-            cur = nxt;
-            st0 = n0;
-            st1 = n1;
-            s_cur = ns;
-        }
-        // hand the partial fragments to the epilogue warps
-        const int slot = j % kRedSlots;
-        if (j >= kRedSlots && !mbar_wait_abort(&red_empty[slot], (uint32_t)((j / kRedSlots - 1) & 1), &abort_flag, lim))
-            timed_out = true;
-        put_partials(red + (size_t)slot * kCW * 2 * 16 * Tc, Tc, warp, g, t, aG, aU);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&red_full[slot]);
-    }
-    if ((timed_out || abort_flag) && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
-}
-
-// ---------------------------------------------------------------- down
-
-struct DownArgs {
-    const uint8_t *codes;           // down projection in the device layout (MxGeom)
-    const float *h;                 // [T*k][I]
-    const int32_t *ids;
-    const float *topk_w;
-    float *ybuf;                    // [kMaxR expert slots][kMaxT][H]
-    int *n_routed;                  // out: number of experts with routes in this call (for the combine)
-    uint16_t *out;                  // bf16 [T][H]
-    uint32_t *status;
-    long long wait_cycles;          // limit of every wait but the final drains
-    FastDiv S;                      // stages
-    int T, k, E, H, I, cps;
-};
-
-// Staged (expert, token) B columns per CTA.  A CTA's contiguous range of
-// units is no longer than one expert's tiles when the grid has at least as
-// many CTAs as there are routed experts, so it touches at most two experts:
-// at most 2T columns.
-constexpr int kMaxBSlots = 16;
-constexpr int kMaxTiles = 128;   // H / 32 for H <= 4096
-constexpr int kDNThreads = kGUThreads;
-__host__ __device__ inline int dn_slots(int T) { return 2 * T < kMaxBSlots ? 2 * T : kMaxBSlots; }
-__host__ __device__ inline size_t dn_red_off(int n_stages, int cps, int T, int I) {
-    return (size_t)n_stages * piece_bytes(cps) + sizeof(uint16_t) * (size_t)dn_slots(T) * (I + kXPad);
-}
-__host__ __device__ inline size_t dn_bytes(int n_stages, int cps, int T, int I) {
-    return dn_red_off(n_stages, cps, T, I) + red_bytes(T);
-}
-
-template <int NCH>   // K chunks per unit = I / kKC
-__global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ RouteTable tb;
-    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages], red_full[kRedSlots], red_empty[kRedSlots];
-    __shared__ int issued;   // chunks issued by the producer (see produce)
-    __shared__ volatile int abort_flag;   // set by the first role that gives up on a wait
-    __shared__ int slot_of[2][kMaxT];    // (expert slot - d_lo, token) -> staged B column, -1 none
-    __shared__ int slot_d[kMaxBSlots], slot_t[kMaxBSlots];
-    __shared__ unsigned slot_max[kMaxBSlots];
-    __shared__ float slot_scale[kMaxBSlots], slot_inv[kMaxBSlots];
-    __shared__ int n_slots;
-    const int H = a.H, I = a.I, T = a.T, k = a.k, S = (int)a.S.d, cps = a.cps, Tc = red_cols(a.T);
-    uint8_t *stages = smem_raw;
-    uint16_t *bs = reinterpret_cast<uint16_t *>(smem_raw + (size_t)S * piece_bytes(cps));   // [slot][I+pad] f16
-    float *red = reinterpret_cast<float *>(smem_raw + dn_red_off(S, cps, T, I));
-    const int bs_stride = I + kXPad;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int tiles = H / 32;
-    const MxGeom geo(H, I);
-    constexpr int WPC = kCW / NCH;   // warps per chunk
-    const int lcps = cps == 4 ? 2 : (cps == 2 ? 1 : 0);
-
-    if (tid == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], WPC * cps);
-        }
-        for (int r = 0; r < kRedSlots; ++r) {
-            mbar_init(&red_full[r], kCW);
-            mbar_init(&red_empty[r], kEpiWarps);
-        }
-        mbar_fence_init();
-        issued = 0;
-        abort_flag = 0;
-    }
-    const long long lim = a.wait_cycles;
-    if (tid < kMaxBSlots) slot_max[tid] = 0u;
-    if (warp == 0) build_route_table(tb, a.ids, a.topk_w, T * k, k, a.E, nullptr, false);
-    __syncthreads();
-    // the next kernel may take SMs as this grid's CTAs finish (it waits for
-    // this grid's completion before touching memory this kernel uses)
-    pdl_launch_dependents();
-    const int n_units = tb.D * tiles;
-    // the combine kernel sums this many slices (it runs after this grid completes)
-    if (blockIdx.x == 0 && tid == 0) *a.n_routed = tb.D;
-    if (tb.D == 0) return;   // no valid route at all: the combine writes zeros
-    int u0, u1;
-    my_range(n_units, u0, u1);
-    const int n_mine = u1 - u0;
-    // unit u -> expert slot u / tiles, 32-row tile u % tiles (tiles is a power of two)
-    const int ltiles = 31 - __clz(tiles);
-    const int d_lo = n_mine > 0 ? u0 >> ltiles : 0;
-
-    if (warp == kProducerWarp) {
-        // the weights do not depend on the gate/up kernel: stream them at once
-        produce(stages, full, empty, a.S, cps, n_mine * NCH / cps, &abort_flag, lim, &issued,
-                [&](int p, const uint8_t *&b0, const uint8_t *&b1) {
-                    const int c = p * cps;
-                    const int u = u0 + c / NCH, d = u >> ltiles, t32 = u & (tiles - 1), q = c % NCH;
-                    const uint8_t *eb = a.codes + (size_t)tb.expert[d] * geo.expert_bytes();
-                    b0 = eb + geo.block_off(2 * t32, q);
-                    b1 = eb + geo.block_off(2 * t32 + 1, q);
-                });
-        return;
-    }
-
-    if (warp >= kEpiWarp0) {
-        // epilogue: sum the 16 warps' partial fragments of a unit, undo the
-        // column's prescale and store the expert's f32 slice for the combine
-        const int e = warp - kEpiWarp0;
-        for (int j = 0; j < n_mine; ++j) {
-            const int slot = j % kRedSlots;
-            if (!mbar_wait_abort(&red_full[slot], (uint32_t)((j / kRedSlots) & 1), &abort_flag, lim)) break;
-            const int u = u0 + j, d = u >> ltiles, m0 = (u & (tiles - 1)) * 32;
-            const float *rb = red + (size_t)slot * kCW * 2 * 16 * Tc;
-            for (int idx = lane + 32 * e; idx < 32 * T; idx += 32 * kEpiWarps) {
-                const int row = idx & 31, col = idx >> 5;
-                const int sl = slot_of[d - d_lo][col];
-                const float v = sl >= 0 ? sum_partials(rb, Tc, row >> 4, row & 15, col) * slot_inv[sl] : 0.f;
-                __stcg(a.ybuf + ((size_t)d * kMaxT + col) * H + m0 + row, v);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&red_empty[slot]);
-        }
-        __syncwarp();
-        if (abort_flag && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
-        // the slices reach the combine kernel through this grid's completion
-        return;
-    }
-
-    // ---- consumers.  The (expert, token) columns of this CTA's experts
-    if (tid == 0) {
-        int ns = 0;
-        const int d_hi = n_mine > 0 ? (u1 - 1) >> ltiles : -1;
-        for (int dd = 0; dd < 2; ++dd)
-            for (int tk = 0; tk < kMaxT; ++tk) slot_of[dd][tk] = -1;
-        for (int d = d_lo; d <= d_hi && d < d_lo + 2; ++d)
-            for (int cc = tb.col_beg[d]; cc < tb.col_beg[d + 1]; ++cc) {
-                const int tk = tb.tok[tb.route[cc]];
-                if (ns < kMaxBSlots && slot_of[d - d_lo][tk] < 0) {
-                    slot_of[d - d_lo][tk] = ns;
-                    slot_d[ns] = d;
-                    slot_t[ns++] = tk;
-                }
-            }
-        n_slots = ns;
-    }
-    // h comes from the gate/up kernel
-    pdl_wait_primary();
+    // phase 1
+    if (ok)
+        ok = consume_phase<NCU>(stages, full, empty, red_full, red_empty, red, Tc, a.S, cps, n_gu_units, 0, 0,
+                                &issued, &abort_flag, lim, [&](int j, bool &live) {
+                                    const uint32_t u = units[j];
+                                    live = g < unit_ncol(u);
+                                    const int tok = live ? tb.tok[tb.route[unit_cb(u) + g]] : 0;
+                                    return xs + (size_t)tok * xs_stride + 8 * t;
+                                });
+    // every consumer is done with the activations (their region takes the B
+    // columns next), and every CTA's h is written
     named_sync_consumers();
+    if (tid == 0 && ok && !abort_flag) grid_wait(a.gbar, gen0, 1, &abort_flag, lim);
+    named_sync_consumers();
+    ok = ok && !abort_flag;
+
     // B column sl = (sum of w_r h_r over the token's routes to the expert,
     // in f32) * 2^s_sl in f16, the power of two putting the column's largest
     // magnitude in [2^14, 2^15): f16 cannot overflow and the epilogue undoes
     // the scale exactly.  Pass 1 finds the maxima with the values kept in
     // registers (two 8-value pieces per thread; larger layers build them
     // again in pass 2).
-    const int n_idx = n_slots * (I / 8);
+    const int n_idx = ok ? n_slots * (I / 8) : 0;
     auto col8 = [&](int idx, float *vv) {   // 8 values of B column idx / (I/8) from k = 8 (idx % (I/8))
         const int sl = idx / (I / 8), k8 = (idx % (I / 8)) * 8, d = slot_d[sl], tk = slot_t[sl];
 #pragma unroll
@@ -808,106 +835,44 @@ __global__ void __launch_bounds__(kDNThreads, 1) dec_down_mx_kernel(DownArgs a) 
     }
     named_sync_consumers();
 
-    // the units, one group ahead as in the gate/up kernel
-    const int q = warp / WPC, wi = warp % WPC;   // this warp's chunk of every unit and its place in it
-    constexpr int NG = 8 / WPC;
-    bool timed_out = false;
-    const uint8_t *st0 = stages, *st1 = stages;
-    int s_cur = 0;
-    auto open_unit = [&](int j, const uint8_t *&b0, const uint8_t *&b1, int &s) {
-        const int c = j * NCH + q, pc = c >> lcps;
-        if (!wait_piece(full, a.S, pc, &issued, &abort_flag, lim)) timed_out = true;
-        s = pc - (int)(a.S.div((uint32_t)pc) * a.S.d);
-        // [rows m0..+15: blocks of the piece][rows m0+16..+31: blocks of the piece]
-        b0 = stages + (size_t)s * piece_bytes(cps) + (size_t)(c & (cps - 1)) * kBlk;
-        b1 = b0 + (size_t)cps * kBlk;
-    };
-    GroupFrags cur;
-    if (n_mine > 0) {
-        open_unit(0, st0, st1, s_cur);
-        load_group(st0, st1, g, t, wi * NG, cur);
-    }
-    for (int j = 0; j < n_mine && !timed_out; ++j) {
-        const int d = (u0 + j) >> ltiles;
-        const int my_slot = (g < T) ? slot_of[d - d_lo][g] : -1;   // B column g = token g
-        const uint16_t *brow = bs + (size_t)(my_slot < 0 ? 0 : my_slot) * bs_stride + 8 * t;
-        float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+    // phase 2
+    if (ok)
+        ok = consume_phase<NCD>(stages, full, empty, red_full, red_empty, red, Tc, a.S, cps, n_dn, n_gu_p,
+                                n_gu_units, &issued, &abort_flag, lim, [&](int j, bool &live) {
+                                    const int d = (u0 + j) >> ldt;
+                                    const int sl = g < T ? slot_of[d - d_lo][g] : -1;   // column g = token g
+                                    live = sl >= 0;
+                                    return bs + (size_t)(live ? sl : 0) * bs_stride + 8 * t;
+                                });
+
+    // phase 3, after every CTA's slices are written: this CTA's share of
+    // the outputs, the experts' slices summed in expert order (16 loads in
+    // flight at a time), one bf16 rounding
+    named_sync_consumers();
+    if (tid == 0 && ok && !abort_flag) grid_wait(a.gbar, gen0, 2, &abort_flag, lim);
+    named_sync_consumers();
+    if (ok && !abort_flag) {
+        const int D = tb.D;
+        int o0, o1;
+        my_range(T * H, o0, o1);
+        for (int i = o0 + tid; i < o1; i += 32 * kCW) {
+            const float *yb = a.ybuf + i;   // element i = col * H + m of slice d at d * kMaxT * H
+            float sum = 0.f;
+            for (int d0 = 0; d0 < D; d0 += 16) {
+                float vv[16];
 #pragma unroll
-        for (int p = 0; p < NG; ++p) {
-            const int gp = wi * NG + p;
-            const uint8_t *n0 = st0, *n1 = st1;
-            int ns = s_cur;
-            GroupFrags nxt;
-            if (p + 1 < NG) {
-                load_group(st0, st1, g, t, gp + 1, nxt);
-            } else {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s_cur]);
-                if (j + 1 < n_mine) {
-                    open_unit(j + 1, n0, n1, ns);
-                    load_group(n0, n1, g, t, wi * NG, nxt);
-                }
+                for (int qq = 0; qq < 16; ++qq) vv[qq] = d0 + qq < D ? __ldcg(yb + (size_t)(d0 + qq) * kMaxT * H) : 0.f;
+#pragma unroll
+                for (int qq = 0; qq < 16; ++qq)
+                    if (d0 + qq < D) sum += vv[qq];
             }
-            const uint16_t *xq = brow + q * kKC + gp * 128;
-            uint4 xb[4];
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) xb[jj] = my_slot >= 0 ? lds128(xq + jj * 32) : make_uint4(0u, 0u, 0u, 0u);
-            compute_group(cur, xb, acc0, acc1);
-            cur = nxt;
-            st0 = n0;
-            st1 = n1;
-            s_cur = ns;
+            __nv_bfloat16 o = __float2bfloat16_rn(sum);
+            a.out[i] = *reinterpret_cast<uint16_t *>(&o);
         }
-        const int slot = j % kRedSlots;
-        if (j >= kRedSlots && !mbar_wait_abort(&red_empty[slot], (uint32_t)((j / kRedSlots - 1) & 1), &abort_flag, lim))
-            timed_out = true;
-        put_partials(red + (size_t)slot * kCW * 2 * 16 * Tc, Tc, warp, g, t, acc0, acc1);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&red_full[slot]);
+    } else {
+        ok = false;
     }
-    if ((timed_out || abort_flag) && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
-}
-
-// Combine (one output element per thread): the experts' f32 slices of the
-// down kernel summed in expert order, rounded once to bf16.  Launched as a
-// programmatic dependent of the down kernel, whose completion it waits for;
-// the order of the sum does not depend on timing.
-constexpr int kCombineThreads = 256;
-__global__ void __launch_bounds__(kCombineThreads) dec_combine_kernel(const float *ybuf, const int *n_routed,
-                                                                       uint16_t *out, int T, int H) {
-    pdl_wait_primary();
-    pdl_launch_dependents();
-    const int D = __ldcg(n_routed);
-    const int i = blockIdx.x * kCombineThreads + threadIdx.x;
-    if (i >= T * H) return;
-    const float *yb = ybuf + i;   // [d][col][m]: element i = col * H + m of slice d at d * kMaxT * H
-    // the slices 16 loads at a time (independent, so they overlap), added in expert order
-    float sum = 0.f;
-    for (int d0 = 0; d0 < D; d0 += 16) {
-        float v[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) v[q] = d0 + q < D ? __ldcg(yb + (size_t)(d0 + q) * kMaxT * H) : 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-            if (d0 + q < D) sum += v[q];
-    }
-    __nv_bfloat16 o = __float2bfloat16_rn(sum);
-    out[i] = *reinterpret_cast<uint16_t *>(&o);
-}
-
-template <typename K, typename... A>
-cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, A... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
+    if ((!ok || abort_flag) && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);
 }
 
 // Stages and chunks per stage (cps, a divisor of the unit's nch chunks) for
@@ -933,82 +898,68 @@ StagePlan plan_stages(int nch, size_t fixed) {
     }
     return best;
 }
-StagePlan gu_plan(int T, int H) { return plan_stages(H / kKC, gu_bytes(0, 1, T, H)); }
-StagePlan dn_plan(int T, int I) { return plan_stages(I / kKC, dn_bytes(0, 1, T, I)); }
+StagePlan fu_plan(int T, int H, int I) {
+    return plan_stages(std::min(H, I) / kKC, fu_bytes(0, 1, T, H, I));
+}
 
+// The one-launch decode step: a cooperative launch (all CTAs co-resident,
+// which the grid barriers need; the launch fails rather than hangs when they
+// cannot be).
 template <int NCU, int NCD>
-cudaError_t run_decode(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
-                       cudaStream_t s, const cudaEvent_t *ev) {
+cudaError_t run_fused(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
+                      cudaStream_t s, const cudaEvent_t *ev) {
     const int H = L.d.hidden, I = L.d.inter;
-    const int grid = L.sm_count;
-    // the kernels' shared-memory limit, once per device (the caller made the
-    // layer's device current); concurrent first calls from several host
-    // threads run it once
     static std::once_flag attr_once[64];
     static cudaError_t attr_err[64];
     const int dev = L.d.device;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(attr_once[dev], [&] {
-        cudaError_t e = cudaFuncSetAttribute(dec_gateup_mx_kernel<NCU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err[dev] = cudaFuncSetAttribute(dec_fused_mx_kernel<NCU, NCD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kMaxDynSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(dec_down_mx_kernel<NCD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-        attr_err[dev] = e;
     });
     if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-    GateUpArgs ga;
-    ga.codes_g = L.w.codes[MOEQ_GATE];
-    ga.codes_u = L.w.codes[MOEQ_UP];
-    ga.x = reinterpret_cast<const uint16_t *>(x);
-    ga.ids = ids;
-    ga.topk_w = topk_w;
-    ga.h = L.h;
-    ga.status = L.status;
-    ga.wait_cycles = L.wait_cycles;
-    ga.T = T;
-    ga.k = L.d.top_k;
-    ga.E = L.d.n_experts;
-    ga.H = H;
-    ga.I = I;
-    const StagePlan gp = gu_plan(T, H);
-    ga.S = make_fastdiv((uint32_t)gp.S);
-    ga.cps = gp.cps;
-    L.count_launches(3);
-    if (ev) record_phase(ev[1], s);   // routing is fused into both kernels' prologues
-    cudaError_t e = launch_ex(dec_gateup_mx_kernel<NCU>, dim3(grid), dim3(kGUThreads),
-                              gu_bytes(gp.S, ga.cps, T, H), s, ev == nullptr, ga);
+    FusedArgs fa;
+    fa.codes_g = L.w.codes[MOEQ_GATE];
+    fa.codes_u = L.w.codes[MOEQ_UP];
+    fa.codes_d = L.w.codes[MOEQ_DOWN];
+    fa.x = reinterpret_cast<const uint16_t *>(x);
+    fa.ids = ids;
+    fa.topk_w = topk_w;
+    fa.h = L.h;
+    fa.ybuf = L.dec_ybuf;
+    fa.gbar = L.dec_counters;
+    fa.out = reinterpret_cast<uint16_t *>(out);
+    fa.status = L.status;
+    fa.wait_cycles = L.wait_cycles;
+    fa.T = T;
+    fa.k = L.d.top_k;
+    fa.E = L.d.n_experts;
+    fa.H = H;
+    fa.I = I;
+    const StagePlan pl = fu_plan(T, H, I);
+    fa.S = make_fastdiv((uint32_t)pl.S);
+    fa.cps = pl.cps;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(L.sm_count);
+    cfg.blockDim = dim3(kGUThreads);
+    cfg.dynamicSmemBytes = fu_bytes(pl.S, pl.cps, T, H, I);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    L.count_launches(1);
+    // routing, gate/up, down and the combine are one kernel: their phase
+    // events are recorded back to back around it
+    if (ev) record_phase(ev[1], s);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, dec_fused_mx_kernel<NCU, NCD>, fa);
     if (e != cudaSuccess) return e;
-    if (ev) record_phase(ev[2], s);
-    DownArgs da;
-    da.codes = L.w.codes[MOEQ_DOWN];
-    da.h = L.h;
-    da.ids = ids;
-    da.topk_w = topk_w;
-    da.ybuf = L.dec_ybuf;
-    da.n_routed = L.dec_counters;
-    da.out = reinterpret_cast<uint16_t *>(out);
-    da.status = L.status;
-    da.wait_cycles = L.wait_cycles;
-    da.T = T;
-    da.k = L.d.top_k;
-    da.E = L.d.n_experts;
-    da.H = H;
-    da.I = I;
-    const StagePlan dp = dn_plan(T, I);
-    da.S = make_fastdiv((uint32_t)dp.S);
-    da.cps = dp.cps;
-    // programmatic dependent launch: the down kernel's producer streams
-    // weights while the gate/up kernel drains; its consumers wait for that
-    // grid before reading h.  Not with phase events between the launches.
-    e = launch_ex(dec_down_mx_kernel<NCD>, dim3(grid), dim3(kDNThreads), dn_bytes(dp.S, da.cps, T, I), s, ev == nullptr,
-                  da);
-    if (e != cudaSuccess) return e;
-    if (ev) record_phase(ev[3], s);
-    const int n_out = T * H;
-    e = launch_ex(dec_combine_kernel, dim3((n_out + kCombineThreads - 1) / kCombineThreads), dim3(kCombineThreads), 0,
-                  s, ev == nullptr, (const float *)L.dec_ybuf, (const int *)L.dec_counters, (uint16_t *)out, T, H);
-    if (e != cudaSuccess) return e;
-    if (ev) record_phase(ev[4], s);
+    if (ev) {
+        record_phase(ev[2], s);
+        record_phase(ev[3], s);
+        record_phase(ev[4], s);
+    }
     return cudaSuccess;
 }
 
@@ -1020,7 +971,7 @@ bool decode_mx_supported(const Layer &L, int T) {
     if (T < 1 || T > kMaxT || T * d.top_k > kMaxR) return false;
     if (!((d.hidden == 2048 || d.hidden == 4096) && (d.inter == 2048 || d.inter == 4096))) return false;
     for (int tt = 1; tt <= kMaxT; ++tt)
-        if (gu_plan(tt, d.hidden).S < 2 || dn_plan(tt, d.inter).S < 2) return false;
+        if (fu_plan(tt, d.hidden, d.inter).S < 3) return false;
     // a CTA's gate/up units fit its unit table
     const long long max_units = (long long)kMaxR * (d.inter / 16);   // passes <= routes
     if (L.sm_count <= 0 || (max_units + L.sm_count - 1) / L.sm_count > kMaxUnits) return false;
@@ -1033,10 +984,10 @@ bool decode_mx_supported(const Layer &L, int T) {
 cudaError_t launch_decode_mx(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T,
                              void *out, cudaStream_t s, const cudaEvent_t *ev) {
     const int H = L.d.hidden, I = L.d.inter;
-    if (H == 2048 && I == 2048) return run_decode<2, 2>(L, x, ids, topk_w, T, out, s, ev);
-    if (H == 2048 && I == 4096) return run_decode<2, 4>(L, x, ids, topk_w, T, out, s, ev);
-    if (H == 4096 && I == 2048) return run_decode<4, 2>(L, x, ids, topk_w, T, out, s, ev);
-    if (H == 4096 && I == 4096) return run_decode<4, 4>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 2048 && I == 2048) return run_fused<2, 2>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 2048 && I == 4096) return run_fused<2, 4>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 4096 && I == 2048) return run_fused<4, 2>(L, x, ids, topk_w, T, out, s, ev);
+    if (H == 4096 && I == 4096) return run_fused<4, 4>(L, x, ids, topk_w, T, out, s, ev);
     return cudaErrorInvalidValue;
 }
 

@@ -743,8 +743,9 @@ bool decode_vq_supported(const Layer &L, int T) {
     if (!((d.hidden == 2048 || d.hidden == 4096) && (d.inter == 2048 || d.inter == 4096))) return false;
     // the staged operands fit beside the books (without the interleaved residual copies)
     const int TB = tokens_bound(T);
-    if (books_bytes<true, false>() + gu_stage_bytes(TB, d.hidden / 256) > kVMaxSmem) return false;
-    if (books_bytes<true, false>() + dn_stage_bytes(TB, d.inter / 256) > kVMaxSmem) return false;
+    const int books = is_gvq1(d.fmt) ? books_bytes<true, false, true>() : books_bytes<true, false>();
+    if (books + gu_stage_bytes(TB, d.hidden / 256) > kVMaxSmem) return false;
+    if (books + dn_stage_bytes(TB, d.inter / 256) > kVMaxSmem) return false;
     // a down CTA's items span at most two experts: at least one CTA per routed expert
     return L.sm_count >= std::min(dec::kMaxR, d.n_experts) && L.sm_count <= 4096;
 }

@@ -105,6 +105,7 @@ struct PrefillVq {
 struct RouterState {
     uint4 *wfrag = nullptr;    // bf16 activations: three bf16 terms of Wr in tensor-core fragment order
     float *wt = nullptr;       // f32 activations: Wr transposed, [H][E]
+    float *wrow = nullptr;     // Wr as given, [E][H] f32 (the decode-size GEMV)
     float *part = nullptr;     // [K slices][T][E] partial logits
     int *counters = nullptr;   // [token tiles], zero between calls
     int score = 0;             // moeq_score
@@ -122,7 +123,7 @@ struct Layer {
     float *acc = nullptr;      // [max_tokens][H] f32 combine accumulator
     // decode fast path scratch
     float *dec_ybuf = nullptr;     // [kDecMaxRoutes][kDecMaxTokens][H] per-expert partial outputs
-    int *dec_counters = nullptr;   // [H/32] per-tile arrival counters, zero between calls
+    int *dec_counters = nullptr;   // [2] grid barrier of the one-launch MXFP4 decode (arrivals, generation)
     float *vq_acc = nullptr;       // VQ decode: [kDecMaxTokens][H] f32 combine accumulator, zero between calls
     int *vq_done = nullptr;        // VQ decode: CTA arrival counter of the down kernel, zero between calls
     uint32_t *status = nullptr;

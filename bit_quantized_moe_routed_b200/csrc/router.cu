@@ -29,6 +29,12 @@
 // logits [K slice][token][E], and the last CTA of a token tile to finish
 // (arrival counter) sums the slices in slice order -- so the logits do not
 // depend on timing -- selects and weights.
+// Decode sizes (up to 8 tokens, either activation type): a GEMV on the CUDA
+// cores instead, one CTA per expert row reading Wr as given ([E][H] f32,
+// coalesced 16-byte loads, each byte once per call) with f32 FMAs (each
+// product exact inside its FMA), the row's partial sums added in a fixed
+// order; the last CTA to finish selects.  The tensor-core path would spend
+// most of its work on the padding of a 32-token tile and read 1.5x the bytes.
 #include <algorithm>
 #include <cstring>
 #include <new>
@@ -99,15 +105,29 @@ __device__ void select_topk(float (&v)[kMaxPerLane], int E, int k, int score, in
     __syncwarp();
 }
 
-// The last CTA of a token tile: sum the K slices of every token's logits in
-// slice order, then select.  part: [nsplit][T][E].
-__device__ void finish_tile(const float *part, int nsplit, int T, int E, int k, int score, int t0, int32_t *topk_ids,
+// The last CTA of a token tile: the K slices of every logit of the tile
+// summed in slice order, then one warp per token selects.  part:
+// [nsplit][T][E].  With many slices (few token tiles) the whole CTA sums
+// them first, in place of slice 0; with a few, each warp sums its token's.
+__device__ void finish_tile(float *part, int nsplit, int T, int E, int k, int score, int t0, int32_t *topk_ids,
                             float *topk_w, float *logits, float (*sel)[kMaxTopK]) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nt = min(kTileTok, T - t0);
+    const bool presum = nsplit > 4;
+    if (presum) {
+        const size_t slice = (size_t)T * E;
+        for (int i = threadIdx.x; i < nt * E; i += kRThreads) {
+            float *p = part + (size_t)t0 * E + i;    // slice 0 of token t0 + i / E, expert i % E
+            float s = __ldcg(p);
+#pragma unroll 8
+            for (int q = 1; q < nsplit; ++q) s += __ldcg(p + q * slice);
+            __stcg(p, s);
+        }
+        __syncthreads();
+    }
     const int per = (E + 31) / 32;
-    for (int tt = warp; tt < kTileTok; tt += kRWarps) {
+    for (int tt = warp; tt < nt; tt += kRWarps) {
         const int t = t0 + tt;
-        if (t >= T) break;
         float v[kMaxPerLane];
 #pragma unroll
         for (int i = 0; i < kMaxPerLane; ++i) {
@@ -115,10 +135,11 @@ __device__ void finish_tile(const float *part, int nsplit, int T, int E, int k, 
             if (i >= per) continue;
             const int e = lane + 32 * i;
             if (e >= E) continue;
-            float s = 0.f;
-            for (int q = 0; q < nsplit; ++q) s += __ldcg(part + ((size_t)q * T + t) * E + e);
-            v[i] = s;
-            if (logits) logits[(size_t)t * E + e] = s;
+            float z = __ldcg(part + (size_t)t * E + e);
+            if (!presum)
+                for (int q = 1; q < nsplit; ++q) z += __ldcg(part + ((size_t)q * T + t) * E + e);
+            v[i] = z;
+            if (logits) logits[(size_t)t * E + e] = z;
         }
         select_topk(v, E, k, score, topk_ids + (size_t)t * k, topk_w + (size_t)t * k, sel[warp]);
     }
@@ -144,6 +165,7 @@ struct RouterArgs {
     const void *x;            // [T][H] bf16 or f32
     const uint4 *wfrag;       // bf16 terms in fragment order (bf16 activations)
     const float *wt;          // [H][E] f32 (f32 activations)
+    const float *wrow;        // [E][H] f32 (the GEMV)
     float *part;              // [nsplit][T][E]
     int *counters;            // [token tiles], zero between calls
     int32_t *topk_ids;
@@ -238,6 +260,98 @@ __global__ void __launch_bounds__(kRThreads, 2) router_bf16_kernel(RouterArgs a)
         finish_tile(a.part, a.nsplit, a.T, a.E, a.k, a.score, t0, a.topk_ids, a.topk_w, a.logits, sel);
 }
 
+// ------------------------------------------------------------ decode sizes
+
+constexpr int kGemvMaxT = 8;              // tokens per call served by the GEMV
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// CTA e computes logit row e for the call's T <= 8 tokens: warp w takes the
+// w-th eighth of the row's 16-byte groups, lane l every 32nd group from its
+// l-th, and accumulates one f32 FMA chain per token; the lanes' sums are
+// added by a butterfly, the warps' in warp order.  The last CTA to finish
+// selects, one warp per token.
+template <bool BF>
+__global__ void __launch_bounds__(kRThreads) router_gemv_kernel(RouterArgs a) {
+    __shared__ float red[kRWarps][kGemvMaxT];
+    __shared__ float sel[kRWarps][kMaxTopK];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x, T = a.T, H = a.H, n4 = H >> 2;
+    const int j0 = warp * n4 / kRWarps, j1 = (warp + 1) * n4 / kRWarps;
+    const float4 *wr = reinterpret_cast<const float4 *>(a.wrow + (size_t)e * H);
+    float acc[kGemvMaxT];
+#pragma unroll
+    for (int t = 0; t < kGemvMaxT; ++t) acc[t] = 0.f;
+    for (int jb = j0 + lane; jb < j1; jb += 4 * 32) {
+        float4 w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = jb + 32 * u;
+            w[u] = j < j1 ? __ldcs(wr + j) : make_float4(0.f, 0.f, 0.f, 0.f);   // read once: evict first
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = jb + 32 * u;
+            if (j >= j1) break;
+#pragma unroll
+            for (int t = 0; t < kGemvMaxT; ++t) {
+                if (t >= T) break;
+                float x0, x1, x2, x3;
+                if constexpr (BF) {
+                    // four bf16 at element 4j: two 4-byte words (x is 4-byte aligned)
+                    const uint32_t *xp =
+                        reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint16_t *>(a.x) + (size_t)t * H) +
+                        2 * j;
+                    const uint32_t p0 = __ldg(xp), p1 = __ldg(xp + 1);
+                    x0 = __uint_as_float(p0 << 16);
+                    x1 = __uint_as_float(p0 & 0xffff0000u);
+                    x2 = __uint_as_float(p1 << 16);
+                    x3 = __uint_as_float(p1 & 0xffff0000u);
+                } else {
+                    const float *xp = reinterpret_cast<const float *>(a.x) + (size_t)t * H + 4 * j;
+                    x0 = __ldg(xp);
+                    x1 = __ldg(xp + 1);
+                    x2 = __ldg(xp + 2);
+                    x3 = __ldg(xp + 3);
+                }
+                acc[t] = fmaf(x0, w[u].x, acc[t]);
+                acc[t] = fmaf(x1, w[u].y, acc[t]);
+                acc[t] = fmaf(x2, w[u].z, acc[t]);
+                acc[t] = fmaf(x3, w[u].w, acc[t]);
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < kGemvMaxT; ++t) {
+        if (t >= T) break;
+        const float v = warp_sum(acc[t]);
+        if (lane == 0) red[warp][t] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < T) {
+        const int t = threadIdx.x;
+        float z = 0.f;
+#pragma unroll
+        for (int w = 0; w < kRWarps; ++w) z += red[w][t];
+        __stcg(a.part + (size_t)t * a.E + e, z);
+        if (a.logits) a.logits[(size_t)t * a.E + e] = z;
+    }
+    if (last_of_tile(a.counters, gridDim.x) && warp < T) {
+        const int t = warp, per = (a.E + 31) / 32;
+        float v[kMaxPerLane];
+#pragma unroll
+        for (int i = 0; i < kMaxPerLane; ++i) {
+            const int ex = lane + 32 * i;
+            v[i] = (i < per && ex < a.E) ? __ldcg(a.part + (size_t)t * a.E + ex) : 0.f;
+        }
+        select_topk(v, a.E, a.k, a.score, a.topk_ids + (size_t)t * a.k, a.topk_w + (size_t)t * a.k, sel[warp]);
+    }
+}
+
 // ------------------------------------------------------------ f32 path
 
 __global__ void __launch_bounds__(kRThreads) router_f32_kernel(RouterArgs a) {
@@ -305,12 +419,17 @@ cudaError_t router_upload(Layer &L, const float *wr, int score, cudaStream_t s) 
         cudaError_t e = cudaSuccess;
         if (bf) e = dev_alloc((void **)&r->wfrag, mtiles * (H / 16) * 3 * 32 * sizeof(uint4));
         else e = dev_alloc((void **)&r->wt, sizeof(float) * (size_t)E * H);
+        if (e == cudaSuccess) e = dev_alloc((void **)&r->wrow, sizeof(float) * (size_t)E * H);
         if (e == cudaSuccess) e = dev_alloc((void **)&r->part, sizeof(float) * max_rows * E);
         if (e == cudaSuccess) e = dev_alloc((void **)&r->counters, sizeof(int) * (size_t)tiles);
         if (e == cudaSuccess) e = cudaMemset(r->counters, 0, sizeof(int) * (size_t)tiles);
         if (e != cudaSuccess) return e;
     }
     r->score = score;
+    {
+        cudaError_t e = cudaMemcpyAsync(r->wrow, wr, sizeof(float) * (size_t)E * H, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return e;
+    }
     // the host image: terms in fragment order, or the transpose
     if (bf) {
         const int n_ks = H / 16, mtiles = (E + 15) / 16;
@@ -367,6 +486,7 @@ void router_free(Layer &L) {
     if (!r) return;
     cudaFree(r->wfrag);
     cudaFree(r->wt);
+    cudaFree(r->wrow);
     cudaFree(r->part);
     cudaFree(r->counters);
     delete r;
@@ -380,6 +500,7 @@ cudaError_t launch_router(const Layer &L, const void *x, int T, int32_t *topk_id
     a.x = x;
     a.wfrag = r->wfrag;
     a.wt = r->wt;
+    a.wrow = r->wrow;
     a.part = r->part;
     a.counters = r->counters;
     a.topk_ids = topk_ids;
@@ -392,8 +513,13 @@ cudaError_t launch_router(const Layer &L, const void *x, int T, int32_t *topk_id
     a.score = r->score;
     a.nsplit = router_nsplit(T, a.H);
     a.kslice = a.H / a.nsplit;
-    const dim3 grid((T + kTileTok - 1) / kTileTok, a.nsplit);
     L.count_launches(1);
+    if (T <= kGemvMaxT) {
+        if (L.d.act == MOEQ_ACT_BF16) router_gemv_kernel<true><<<a.E, kRThreads, 0, s>>>(a);
+        else router_gemv_kernel<false><<<a.E, kRThreads, 0, s>>>(a);
+        return cudaGetLastError();
+    }
+    const dim3 grid((T + kTileTok - 1) / kTileTok, a.nsplit);
     if (L.d.act == MOEQ_ACT_BF16) {
         // two 16-expert tiles per warp: 8 warps cover 256 experts per pass
         router_bf16_kernel<2><<<grid, kRThreads, 0, s>>>(a);

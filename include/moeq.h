@@ -364,9 +364,11 @@ MOEQ_API moeq_status moeq_dequant(moeq_layer_t layer, int32_t expert, int32_t pr
  * gave up: the kernel stopped issuing work, waited for its own copies and
  * tensor-core operations in flight, released its on-chip memory and
  * returned, so the device stays usable, but that forward's output is
- * undefined.  Clearing the status after a timeout also resets the decode
- * path's workspace counters (per-tile arrival counts that a forward which
- * gave up part-way can leave behind).  Errors: INVALID_ARGUMENT, CUDA. */
+ * undefined.  Clearing the status after a timeout also resets the grid
+ * barrier of the one-launch MXFP4 decode step, which a forward that gave up
+ * part-way can leave behind; until the status is cleared, later MXFP4
+ * decode forwards on the layer are undefined too.  Errors:
+ * INVALID_ARGUMENT, CUDA. */
 MOEQ_API moeq_status moeq_layer_status(moeq_layer_t layer, int32_t clear);
 
 /* Number of kernels the layer has launched so far (a launch captured into

@@ -90,10 +90,11 @@ def test_router_prefill_micro_batch():
     np.testing.assert_allclose(w.cpu().numpy(), w_k, rtol=4e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("T", [5, 45])          # the GEMV (T <= 8) and the tiled path
 @pytest.mark.parametrize("act", ["f32", "bf16"])
-def test_router_small_and_ragged_expert_count(act):
+def test_router_small_and_ragged_expert_count(act, T):
     # E = 24 (not a whole number of 16-expert tiles), H = 256, k = 3
-    cfg = synth.get_cfg("tiny_mxfp4", act=act, E=24, k=3, T=45)
+    cfg = synth.get_cfg("tiny_mxfp4", act=act, E=24, k=3, T=T)
     lay, wr = _router_layer(cfg, "sigmoid", seed=91)
     x = synth.gen_activations(cfg, seed=91)
     xt, _, _ = to_dev_inputs(cfg, x, np.zeros((1, 3), np.int32), np.zeros((1, 3), np.float32))
