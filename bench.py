@@ -41,9 +41,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     "decode_mxfp4": (("bit_quantized_moe_routed_b200/csrc/decode_mx.cu",
                       "bit_quantized_moe_routed_b200/csrc/async.cuh",
-                      "bit_quantized_moe_routed_b200/csrc/internal.cuh"),
-                     "da02a205cbb6dd722b2c28527a5684af27b376e3b21fcaf2b688e9d4968283fd",
-                     71364352.0 + 997376.0, "profiles/dec_gateup_mx_decode_mxfp4.md"),
+                      "bit_quantized_moe_routed_b200/csrc/decode_common.cuh",
+                      "bit_quantized_moe_routed_b200/csrc/internal.cuh",
+                      "include/moeq.h"),
+                     "ed3e0254c76ef30a5157cc87547b790366a1657d5edf54c4933bb398946ff5ce",
+                     107049216.0 + 403456.0, "profiles/dec_fused_mx_decode_mxfp4.md"),
 }
 
 
