@@ -400,7 +400,9 @@ __device__ __forceinline__ void red_add_release_gpu(int *p, int v) {
 // release, resets the count and releases the new generation.
 __device__ __forceinline__ void grid_arrive(int *bar) {
     if (atom_add_acq_rel_gpu(bar, 1) == (int)gridDim.x - 1) {
-        atomicExch(bar, 0);
+        // every CTA has arrived and none touches the count again before the
+        // generation moves on: a plain store resets it, the release orders it
+        asm volatile("st.relaxed.gpu.global.s32 [%0], 0;" ::"l"(bar) : "memory");
         red_add_release_gpu(bar + 1, 1);
     }
 }
@@ -701,8 +703,9 @@ __global__ void __launch_bounds__(kGUThreads, 1) dec_fused_mx_kernel(FusedArgs a
             if (lane == 0) mbar_arrive(&red_empty[slot]);
         }
         // the slices are written: one arrival at barrier 2, after barrier 1
+        // (which a CTA with down units has passed before its first one)
         named_sync_epilogue();
-        if (e == 0 && lane == 0 && ok && !abort_flag && grid_wait(a.gbar, gen0, 1, &abort_flag, lim))
+        if (e == 0 && lane == 0 && ok && !abort_flag && (n_dn > 0 || grid_wait(a.gbar, gen0, 1, &abort_flag, lim)))
             grid_arrive(a.gbar);
         __syncwarp();
         if (abort_flag && lane == 0) atomicOr(a.status, FLAG_TIMEOUT);

@@ -68,11 +68,10 @@ constexpr int kAtom = 512;        // one scale-factor atom: 128 rows x 4 blocks 
 // gate/up stage: [A gate][A up][B q1][B q2][SF gate][SF up][SF x], padded to 1 KB
 constexpr int kGUStage = 2 * kTileA + 2 * kTileB + 3 * kAtom + 512;
 constexpr int kGUStages = 4;
-constexpr int kGUFill = 2;        // stages the producer fills per step
 // down stage: [A down][B q1][B q2][SF down][SF h]
 constexpr int kDNStage = kTileA + 2 * kTileB + 2 * kAtom;
 constexpr int kDNStages = 6;
-constexpr int kDNFill = 3;
+constexpr int kDNFill = 3;        // stages the producer fills per step
 
 // tensor memory: two accumulator buffers (the epilogue of one item overlaps
 // the MMAs of the next), then a scale-factor ring (4 columns per atom)
@@ -279,44 +278,42 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int n_items = rt.tb[E] * subs;
 
     if (warp == 0) {
-        // kGUFill stages per step: lanes g < kGUFill wait for and arm stage
-        // c0 + g, then lanes 7g + j issue copy j of it -- one producer step
-        // costs about the same however many copies it issues, so it issues many
-        const int my_items = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-        const int total = my_items * slabs;
-        const int g = lane / 7, j = lane % 7;
-        int c0 = 0;
-        for (; c0 < total; c0 += kGUFill) {
-            const int c = c0 + (lane < kGUFill ? lane : 0), s = c % kGUStages;
-            bool ok = true;
-            if (lane < kGUFill && c < total && c >= kGUStages)
-                ok = wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag, a.wait_cycles);
-            if (__any_sync(0xffffffffu, !ok)) break;
-            if (lane < kGUFill && c < total) mbar_arrive_expect_tx(&full[s], 2 * kBoxA + 2 * kTileB + 3 * kAtom);
-            __syncwarp();
-            const int cc = c0 + g;
-            if (g < kGUFill && cc < total) {
-                const int sc = cc % kGUStages, sl = cc % slabs;
-                const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (cc / slabs) * gridDim.x);
-                uint8_t *st = smem + (size_t)sc * kGUStage;
+        // Each work item's tile coordinates are decoded once; its slabs are
+        // then streamed stage by stage: lane 0 waits for the stage to be
+        // released and arms it, lanes 0..6 issue its seven copies at once.
+        int c = 0, s = 0;
+        uint32_t rp = 0;   // parity of the current round of the stage ring
+        bool ok = true;
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const Item m = decode_item(rt.off, rt.tb, E, subs, it);
+            const int wrow = m.e * I + m.sub * kT;
+            const size_t wsf = (size_t)(m.e * subs + m.sub) * slabs * kAtom, xsf = (size_t)m.tau * slabs * kAtom;
+            for (int sl = 0; sl < slabs; ++sl, ++c) {
+                if (lane == 0 && c >= kGUStages) ok = wait_or_abort(&empty[s], rp ^ 1u, &abort_flag, a.wait_cycles);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], 2 * kBoxA + 2 * kTileB + 3 * kAtom);
+                __syncwarp();
+                uint8_t *st = smem + (size_t)s * kGUStage;
                 uint8_t *sf = st + 2 * kTileA + 2 * kTileB;
-                const int wrow = m.e * I + m.sub * kT;
-                const size_t wsf = ((size_t)(m.e * subs + m.sub) * slabs + sl) * kAtom;
-                switch (j) {
-                    case 0: tma_load_2d(st, &tWg, sl * kT, wrow, &full[sc]); break;
-                    case 1: tma_load_2d(st + kTileA, &tWu, sl * kT, wrow, &full[sc]); break;
-                    case 2: tma_load_2d(st + 2 * kTileA, &tX1, sl * kT, m.row0, &full[sc]); break;
-                    case 3: tma_load_2d(st + 2 * kTileA + kTileB, &tX2, sl * kT, m.row0, &full[sc]); break;
-                    case 4: bulk_g2s(sf, a.sfa0 + wsf, kAtom, &full[sc]); break;
-                    case 5: bulk_g2s(sf + kAtom, a.sfa1 + wsf, kAtom, &full[sc]); break;
-                    default:
-                        bulk_g2s(sf + 2 * kAtom, a.sfb + ((size_t)m.tau * slabs + sl) * kAtom, kAtom, &full[sc]);
-                        break;
+                switch (lane) {
+                    case 0: tma_load_2d(st, &tWg, sl * kT, wrow, &full[s]); break;
+                    case 1: tma_load_2d(st + kTileA, &tWu, sl * kT, wrow, &full[s]); break;
+                    case 2: tma_load_2d(st + 2 * kTileA, &tX1, sl * kT, m.row0, &full[s]); break;
+                    case 3: tma_load_2d(st + 2 * kTileA + kTileB, &tX2, sl * kT, m.row0, &full[s]); break;
+                    case 4: bulk_g2s(sf, a.sfa0 + wsf + (size_t)sl * kAtom, kAtom, &full[s]); break;
+                    case 5: bulk_g2s(sf + kAtom, a.sfa1 + wsf + (size_t)sl * kAtom, kAtom, &full[s]); break;
+                    case 6: bulk_g2s(sf + 2 * kAtom, a.sfb + xsf + (size_t)sl * kAtom, kAtom, &full[s]); break;
+                    default: break;
+                }
+                __syncwarp();
+                if (++s == kGUStages) {
+                    s = 0;
+                    rp ^= 1u;
                 }
             }
-            __syncwarp();
         }
-        if (lane == 0) drain_stages(full, kGUStages, c0 < total ? c0 : total);
+        if (lane == 0) drain_stages(full, kGUStages, c);
     } else if (warp == 1) {
         if (lane == 0) {
             int c = 0, q = 0;
@@ -439,8 +436,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int n_items = rt.tb[E] * subs;
 
     if (warp == 0) {
-        // kDNFill stages per step (see the gate/up kernel): lanes 5g + j issue
-        // copy j of stage c0 + g
+        // kDNFill stages per step: lanes g < kDNFill wait for and arm stage
+        // c0 + g, then lanes 5g + j issue copy j of it.  A down stage carries
+        // half the MMAs of a gate/up stage, and refilling three stages per
+        // step measured faster here than one at a time.
         const int my_items = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
         const int total = my_items * slabs;
         const int g = lane / 5, j = lane % 5;
