@@ -44,8 +44,8 @@ NCU_TRAFFIC = {
                       "bit_quantized_moe_routed_b200/csrc/decode_common.cuh",
                       "bit_quantized_moe_routed_b200/csrc/internal.cuh",
                       "include/moeq.h"),
-                     "ed3e0254c76ef30a5157cc87547b790366a1657d5edf54c4933bb398946ff5ce",
-                     107049216.0 + 403456.0, "profiles/dec_fused_mx_decode_mxfp4.md"),
+                     "d97f70d647b24ddd486a1f973719227a7809593cffca4084aaaf6222246a0cc3",
+                     107049216.0 + 358144.0, "profiles/dec_fused_mx_decode_mxfp4.md"),
 }
 
 
@@ -84,6 +84,7 @@ WORKLOADS = {
     # counter captures of the tensor-core kernels; not bench lines
     "prefill_mxfp4_zipf_e64_t512": ("prefill_mxfp4_zipf", dict(E=64, T=512)),
     "prefill_vq_overflow_e64_t512": ("prefill_vq_overflow", dict(E=64, T=512)),
+    "prefill_gvq1_overflow": ("prefill_vq_overflow", dict(fmt="gvq1r8")),
 }
 
 
@@ -299,8 +300,8 @@ def cpu_baseline(cfg, L, xs, ids, w, seconds=12.0):
 # Workloads the default run times after the headline one, one layer at a
 # time (each layer is freed before the next is built): the prefill
 # micro-batches and the VQ decode batch sizes.
-EXTRA_WORKLOADS = ("decode_mxfp4_t8", "prefill_mxfp4_zipf", "prefill_vq_overflow", "decode_vq_t1", "decode_vq_t4",
-                   "decode_vq_t8", "decode_gvq1_t1", "decode_gvq1_t8")
+EXTRA_WORKLOADS = ("decode_mxfp4_t8", "prefill_mxfp4_zipf", "prefill_vq_overflow", "prefill_gvq1_overflow",
+                   "decode_vq_t1", "decode_vq_t4", "decode_vq_t8", "decode_gvq1_t1", "decode_gvq1_t8")
 
 
 def load_peaks():

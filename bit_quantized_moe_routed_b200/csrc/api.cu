@@ -351,6 +351,9 @@ moeq_status moeq_upload_weights(moeq_layer_t L, const moeq_weights *w, void *str
     if (gq) {
         L->w.gscale[0] = w->gscale[0];
         L->w.gscale[1] = r8 ? w->gscale[1] : 0.f;
+        // the books of the tensor-core path (layers created for more than 8 tokens)
+        e = prefill_vq_upload_gvq1_books(*L, w->gbook13, r8 ? w->gbook8 : nullptr, L->w.gscale);
+        if (e != cudaSuccess) return from_cuda(e);
     }
     L->uploaded = true;
     return MOEQ_OK;

@@ -97,7 +97,12 @@ struct PrefillVq {
     int32_t *tile_base = nullptr;  // [E+1]
     uint16_t *xg = nullptr;
     uint16_t *hg = nullptr;
+    // GVQ1 layers: the books as the kernels read them, bf16 of the f32
+    // products e4m3(entry) x book scale, filled at upload
+    uint16_t *gbook13 = nullptr;   // [8192][8]
+    uint16_t *gbook8 = nullptr;    // [256][8]
     bool ready = false;
+    bool books_ready = false;
 };
 
 // Router of a layer (router.cu): the router matrix in the kernels' layout,
@@ -195,6 +200,7 @@ cudaError_t launch_decode_vq(const Layer &L, const void *x, const int32_t *ids, 
 bool prefill_vq_supported(const Layer &L, int T);
 cudaError_t prefill_vq_create(Layer &L);
 void prefill_vq_free(Layer &L);
+cudaError_t prefill_vq_upload_gvq1_books(Layer &L, const uint8_t *book13, const uint8_t *book8, const float scale[2]);
 cudaError_t launch_prefill_vq(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
                               cudaStream_t s, const cudaEvent_t *ev);
 cudaError_t router_upload(Layer &L, const float *wr, int score, cudaStream_t s);

@@ -29,7 +29,10 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
+#include <cstring>
 #include <new>
+#include <vector>
 
 #include "async.cuh"
 #include "internal.cuh"
@@ -65,9 +68,11 @@ __device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uin
 }
 
 struct VqProj {
-    const uint8_t *idx13;   // [E*N][K*13/64]
+    const uint8_t *idx13;   // [E*N][K*13/64] (VQ13), or null
     const uint8_t *idx8;    // [E*N][K/8] or null
     const uint16_t *gain;   // [E*N] f16 or null
+    const uint8_t *code12;  // GVQ1: [E*N][K*3/16], the low 12 bits of the indices; null for VQ13
+    const uint8_t *hi1;     // GVQ1: [E*N][K/64], bit 12 of index j as bit j % 8 of byte j / 8
 };
 
 // The index data of one row for one 64-column slab, fetched ahead of its
@@ -75,19 +80,33 @@ struct VqProj {
 // 13-byte chunk of 13-bit indices as four aligned words (the allocation has
 // slack for the last row), the eight residual indices and the row gain.
 struct RowRaw {
-    uint32_t w[4];
-    uint32_t shift;   // bit offset of the chunk inside w
+    uint32_t w[4];    // the chunk (VQ13: 13 bytes in four aligned words; GVQ1: 12 bytes in w[0..2])
+    uint32_t shift;   // bit offset of the chunk inside w (VQ13)
+    uint32_t hi;      // GVQ1: the slab's byte of bit-12 flags
     uint32_t i8lo, i8hi;
     uint32_t gain;    // f16 bits, 0x3C00 (1.0) when the layer has no gains
 };
+template <bool G1>   // GVQ1 container (else VQ13)
 __device__ __forceinline__ RowRaw fetch_row(const VqProj &pj, int K, size_t grow, int sl) {
     RowRaw v;
-    const uint8_t *chunk = pj.idx13 + grow * (size_t)(K * 13 / 64) + (size_t)sl * (kKS / 8 * 13 / 8);
-    const uintptr_t ad = reinterpret_cast<uintptr_t>(chunk);
-    const uint32_t *wp = reinterpret_cast<const uint32_t *>(ad & ~uintptr_t(3));
+    if constexpr (G1) {
+        // 8 vectors x 12 bits = 12 bytes, 4-byte aligned (K * 3/16 and 12 are multiples of 4)
+        const uint32_t *wp = reinterpret_cast<const uint32_t *>(pj.code12 + grow * (size_t)(K * 3 / 16) +
+                                                                (size_t)sl * (kKS / 8 * 12 / 8));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v.w[i] = __ldg(wp + i);
-    v.shift = (uint32_t)(ad & 3) * 8;
+        for (int i = 0; i < 3; ++i) v.w[i] = __ldg(wp + i);
+        v.w[3] = 0u;
+        v.shift = 0u;
+        v.hi = __ldg(pj.hi1 + grow * (size_t)(K / 64) + (size_t)sl);
+    } else {
+        const uint8_t *chunk = pj.idx13 + grow * (size_t)(K * 13 / 64) + (size_t)sl * (kKS / 8 * 13 / 8);
+        const uintptr_t ad = reinterpret_cast<uintptr_t>(chunk);
+        const uint32_t *wp = reinterpret_cast<const uint32_t *>(ad & ~uintptr_t(3));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v.w[i] = __ldg(wp + i);
+        v.shift = (uint32_t)(ad & 3) * 8;
+        v.hi = 0u;
+    }
     if (pj.idx8) {
         const uint2 q = __ldg(reinterpret_cast<const uint2 *>(pj.idx8 + grow * (size_t)(K / 8) + (size_t)sl * (kKS / 8)));
         v.i8lo = q.x;
@@ -98,8 +117,25 @@ __device__ __forceinline__ RowRaw fetch_row(const VqProj &pj, int K, size_t grow
     v.gain = pj.gain ? (uint32_t)__ldg(pj.gain + grow) : 0x3C00u;
     return v;
 }
-// The eight 13-bit indices of a fetched row chunk (index j at bits 13j..).
+// The eight 13-bit indices of a fetched row chunk: VQ13 index j at bits
+// 13j..13j+12 of the chunk; GVQ1 index j = bits 12j..12j+11 of the chunk,
+// plus bit j of the slab's flag byte as bit 12.
+template <bool G1>
 __device__ __forceinline__ void row_indices(const RowRaw &v, uint32_t idx[8]) {
+    if constexpr (G1) {
+        const uint32_t w0 = v.w[0], w1 = v.w[1], w2 = v.w[2];
+        idx[0] = w0 & 0xFFFu;
+        idx[1] = (w0 >> 12) & 0xFFFu;
+        idx[2] = __funnelshift_r(w0, w1, 24) & 0xFFFu;
+        idx[3] = (w1 >> 4) & 0xFFFu;
+        idx[4] = (w1 >> 16) & 0xFFFu;
+        idx[5] = __funnelshift_r(w1, w2, 28) & 0xFFFu;
+        idx[6] = (w2 >> 8) & 0xFFFu;
+        idx[7] = (w2 >> 20) & 0xFFFu;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) idx[j] |= ((v.hi >> j) & 1u) << 12;
+        return;
+    }
     const uint32_t x0 = __funnelshift_r(v.w[0], v.w[1], v.shift), x1 = __funnelshift_r(v.w[1], v.w[2], v.shift);
     const uint32_t x2 = __funnelshift_r(v.w[2], v.w[3], v.shift), x3 = v.w[3] >> v.shift;
     idx[0] = x0 & 0x1FFFu;
@@ -146,11 +182,11 @@ __device__ __forceinline__ void expand_vec(uint32_t idx, uint32_t i8, uint32_t g
 }
 
 // Decode vectors [J0, J0 + NV) of one fetched row into tile row r.
-template <int J0, int NV>
+template <bool G1, int J0, int NV>
 __device__ __forceinline__ void expand_row(const RowRaw &v, bool r8, const uint8_t *book13, const uint8_t *book8,
                                            uint8_t *tile, int r) {
     uint32_t idx[8];
-    row_indices(v, idx);
+    row_indices<G1>(v, idx);
 #pragma unroll
     for (int jj = 0; jj < NV; ++jj) {
         const int j = J0 + jj;
@@ -199,6 +235,7 @@ __device__ __forceinline__ void load_books(uint8_t *b13, uint8_t *b8, const VqAr
 
 // ---------------------------------------------------------------- gate/up
 
+template <bool G1>   // GVQ1 container (else VQ13)
 __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_constant__ CUtensorMap tX, VqArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -298,7 +335,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
         auto fetch = [&](int c, RowRaw &dst) {
             if (c >= total) return;
             const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
-            dst = fetch_row(pj, H, (size_t)m.e * I + m.sub * kT + r, c % slabs);
+            dst = fetch_row<G1>(pj, H, (size_t)m.e * I + m.sub * kT + r, c % slabs);
         };
         RowRaw q0, q1, q2, q3;
         fetch(0, q0);
@@ -312,7 +349,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
             if (c >= kGUStages) ok = wait_or_abort(&empty[s], (uint32_t)((c / kGUStages - 1) & 1), &abort_flag, a.wait_cycles);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) return;
-            expand_row<0, 8>(q, r8, b13, b8, smem + (size_t)s * kGUStage + mat * kTileA, r);
+            expand_row<G1, 0, 8>(q, r8, b13, b8, smem + (size_t)s * kGUStage + mat * kTileA, r);
             fetch(c + 4, q);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
@@ -362,6 +399,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_gateup_kernel(const __grid_c
 
 // ---------------------------------------------------------------- down
 
+template <bool G1>
 __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_constant__ CUtensorMap tH, VqArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -452,7 +490,7 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_con
         auto fetch = [&](int c, RowRaw &dst) {
             if (c >= total) return;
             const Item m = decode_item(rt.off, rt.tb, E, subs, blockIdx.x + (c / slabs) * gridDim.x);
-            dst = fetch_row(a.w0, I, (size_t)m.e * H + m.sub * kT + r, c % slabs);
+            dst = fetch_row<G1>(a.w0, I, (size_t)m.e * H + m.sub * kT + r, c % slabs);
         };
         RowRaw q0, q1, q2, q3;   // four slabs ahead, as in the gate/up kernel
         fetch(0, q0);
@@ -467,8 +505,8 @@ __global__ void __launch_bounds__(kVqThreads, 1) vq_down_kernel(const __grid_con
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) return;
             uint8_t *tile = smem + (size_t)s * kDNStage;
-            if (j0 == 0) expand_row<0, 4>(q, r8, b13, b8, tile, r);
-            else expand_row<4, 4>(q, r8, b13, b8, tile, r);
+            if (j0 == 0) expand_row<G1, 0, 4>(q, r8, b13, b8, tile, r);
+            else expand_row<G1, 4, 4>(q, r8, b13, b8, tile, r);
             fetch(c + 4, q);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
@@ -559,12 +597,13 @@ size_t dn_smem() { return (size_t)kDNStages * kDNStage + kBook13 + kBook8 + 1024
 }  // namespace
 
 bool prefill_vq_supported(const Layer &L, int T) {
-    return L.pv != nullptr && L.pv->ready && T >= 1 && is_vq13(L.d.fmt) && L.d.act == MOEQ_ACT_BF16;
+    return L.pv != nullptr && L.pv->ready && T >= 1 && L.d.act == MOEQ_ACT_BF16 &&
+           (is_vq13(L.d.fmt) || (is_gvq1(L.d.fmt) && L.pv->books_ready));
 }
 
 cudaError_t prefill_vq_create(Layer &L) {
     const moeq_layer_desc &d = L.d;
-    if (!is_vq13(d.fmt) || d.act != MOEQ_ACT_BF16) return cudaSuccess;
+    if (!(is_vq13(d.fmt) || is_gvq1(d.fmt)) || d.act != MOEQ_ACT_BF16) return cudaSuccess;
     if (d.hidden % kT || d.inter % kT) return cudaSuccess;
     PrefillVq *pv = new (std::nothrow) PrefillVq();
     if (!pv) return cudaErrorMemoryAllocation;
@@ -573,14 +612,22 @@ cudaError_t prefill_vq_create(Layer &L) {
     cudaError_t e = dev_alloc((void **)&pv->tile_base, sizeof(int32_t) * (d.n_experts + 1));
     if (e == cudaSuccess) e = dev_alloc((void **)&pv->xg, R * d.hidden * 2);
     if (e == cudaSuccess) e = dev_alloc((void **)&pv->hg, R * d.inter * 2);
+    if (e == cudaSuccess && is_gvq1(d.fmt)) e = dev_alloc((void **)&pv->gbook13, sizeof(uint16_t) * kBook13Rows * 8);
+    if (e == cudaSuccess && is_gvq1(d.fmt) && has_r8(d.fmt))
+        e = dev_alloc((void **)&pv->gbook8, sizeof(uint16_t) * kBook8Rows * 8);
     // route positions past a tile's routes feed discarded MMA columns: keep them finite
     if (e == cudaSuccess) e = cudaMemset(pv->xg, 0, R * d.hidden * 2);
     if (e == cudaSuccess) e = cudaMemset(pv->hg, 0, R * d.inter * 2);
     if (e != cudaSuccess) return e;
     e = make_bf16_map(&pv->map_x, pv->xg, d.hidden, (long long)R);
     if (e == cudaSuccess) e = make_bf16_map(&pv->map_h, pv->hg, d.inter, (long long)R);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(vq_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu_smem());
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(vq_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn_smem());
+    const bool g1 = is_gvq1(d.fmt);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(g1 ? vq_gateup_kernel<true> : vq_gateup_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu_smem());
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(g1 ? vq_down_kernel<true> : vq_down_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn_smem());
     if (e == cudaSuccess) pv->ready = true;
     return e == cudaErrorNotSupported ? cudaSuccess : e;
 }
@@ -591,8 +638,45 @@ void prefill_vq_free(Layer &L) {
     cudaFree(pv->tile_base);
     cudaFree(pv->xg);
     cudaFree(pv->hg);
+    cudaFree(pv->gbook13);
+    cudaFree(pv->gbook8);
     delete pv;
     L.pv = nullptr;
+}
+
+// GVQ1 books for the tensor-core path: entry value e4m3(b) (the OCP 8-bit
+// float without infinities: sign, 4 exponent bits with bias 7, 3 mantissa
+// bits, subnormal below exponent 1) times the book's scale as an f32
+// product, rounded to nearest even bf16 -- the f32 weight formula's product,
+// one bf16 rounding.  NaN bytes were rejected at upload.
+namespace {
+float e4m3_value(uint8_t b) {
+    const int sgn = b >> 7, ex = (b >> 3) & 15, man = b & 7;
+    const float mag = ex ? std::ldexp(1.0f + man / 8.0f, ex - 7) : std::ldexp(man / 8.0f, -6);
+    return sgn ? -mag : mag;
+}
+uint16_t bf16_rne(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u) return (uint16_t)(u >> 16);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+}  // namespace
+
+cudaError_t prefill_vq_upload_gvq1_books(Layer &L, const uint8_t *book13, const uint8_t *book8, const float scale[2]) {
+    PrefillVq *pv = L.pv;
+    if (!pv || !pv->ready || !pv->gbook13) return cudaSuccess;
+    std::vector<uint16_t> h13((size_t)kBook13Rows * 8), h8;
+    for (size_t i = 0; i < h13.size(); ++i) h13[i] = bf16_rne(e4m3_value(book13[i]) * scale[0]);
+    cudaError_t e = cudaMemcpy(pv->gbook13, h13.data(), h13.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && pv->gbook8 && book8) {
+        h8.resize((size_t)kBook8Rows * 8);
+        for (size_t i = 0; i < h8.size(); ++i) h8[i] = bf16_rne(e4m3_value(book8[i]) * scale[1]);
+        e = cudaMemcpy(pv->gbook8, h8.data(), h8.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+    }
+    pv->books_ready = e == cudaSuccess;
+    return e;
 }
 
 cudaError_t launch_prefill_vq(const Layer &L, const void *x, const int32_t *ids, const float *topk_w, int T, void *out,
@@ -615,8 +699,9 @@ cudaError_t launch_prefill_vq(const Layer &L, const void *x, const int32_t *ids,
     a.tile_base = pv->tile_base;
     a.perm = L.b.perm;
     a.topk_w = topk_w;
-    a.book13 = reinterpret_cast<const uint8_t *>(L.w.book13);
-    a.book8 = L.d.fmt == MOEQ_FMT_VQ13_R8 ? reinterpret_cast<const uint8_t *>(L.w.book8) : nullptr;
+    const bool g1 = is_gvq1(L.d.fmt);
+    a.book13 = reinterpret_cast<const uint8_t *>(g1 ? pv->gbook13 : L.w.book13);
+    a.book8 = has_r8(L.d.fmt) ? reinterpret_cast<const uint8_t *>(g1 ? pv->gbook8 : L.w.book8) : nullptr;
     a.hg = pv->hg;
     a.acc = L.acc;
     a.status = L.status;
@@ -627,17 +712,19 @@ cudaError_t launch_prefill_vq(const Layer &L, const void *x, const int32_t *ids,
     a.k = k;
     auto proj = [&](int p) {
         const ProjView v = L.view(p);
-        return VqProj{v.idx13, v.idx8, v.gain};
+        return g1 ? VqProj{nullptr, v.idx8, v.gain, v.code12, v.hi1} : VqProj{v.idx13, v.idx8, v.gain, nullptr, nullptr};
     };
     a.w0 = proj(MOEQ_GATE);
     a.w1 = proj(MOEQ_UP);
-    vq_gateup_kernel<<<L.sm_count, kVqThreads, gu_smem(), s>>>(pv->map_x, a);
+    if (g1) vq_gateup_kernel<true><<<L.sm_count, kVqThreads, gu_smem(), s>>>(pv->map_x, a);
+    else vq_gateup_kernel<false><<<L.sm_count, kVqThreads, gu_smem(), s>>>(pv->map_x, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev) record_phase(ev[2], s);
     VqArgs b = a;
     b.w0 = proj(MOEQ_DOWN);
-    b.w1 = VqProj{nullptr, nullptr, nullptr};
-    vq_down_kernel<<<L.sm_count, kVqThreads, dn_smem(), s>>>(pv->map_h, b);
+    b.w1 = VqProj{nullptr, nullptr, nullptr, nullptr, nullptr};
+    if (g1) vq_down_kernel<true><<<L.sm_count, kVqThreads, dn_smem(), s>>>(pv->map_h, b);
+    else vq_down_kernel<false><<<L.sm_count, kVqThreads, dn_smem(), s>>>(pv->map_h, b);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev) record_phase(ev[3], s);
     const long long n = (long long)T * H;

@@ -35,6 +35,22 @@ def test_gvq1_forward_general_paths(fmt, act, T):
     assert_close(run(lay, cfg, x, ids, w), oracle_ref(L, x, ids, w), act, f"{fmt} {act} T={T}")
 
 
+@pytest.mark.parametrize("fmt", ["gvq1", "gvq1r8"])
+def test_gvq1_prefill_runs_the_tensor_core_path(fmt):
+    # more than 8 tokens: the VQ tensor-core kernels (route/bucket, route
+    # tiles, gather, gate/up, down, cast: 6 launches; the SIMT path takes 4)
+    # with the books expanded to bf16 at upload
+    cfg = synth.get_cfg("tiny_mxfp4", fmt=fmt, act="bf16", gains=True, H=1024, I=512, E=16, k=4, T=300)
+    L = synth.gen_layer(cfg, seed=113)
+    x = synth.gen_activations(cfg, seed=113)
+    ids, w = synth.gen_routing(cfg, seed=113)
+    lay = dev_layer(L)
+    n0 = lay.kernel_launches()
+    out = run(lay, cfg, x, ids, w)
+    assert lay.kernel_launches() - n0 == 6
+    assert_close(out, oracle_ref(L, x, ids, w), "bf16", f"{fmt} prefill")
+
+
 GVQ1_DECODE = [
     dict(H=2048, I=2048, E=16, k=8, T=1),
     dict(H=2048, I=2048, E=8, k=8, T=8),
