@@ -1,5 +1,5 @@
-// prefill_vq.cu -- VQ13(+R8) routed-expert FFN on the 5th-generation tensor
-// cores (bf16 activations, any token count).
+// prefill_vq.cu -- VQ13(+R8) and GVQ1(+R8) routed-expert FFN on the
+// 5th-generation tensor cores (bf16 activations, any token count).
 //
 // Format ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): every 8
 // consecutive weights of an expert row are one 13-bit index into the layer's
@@ -10,6 +10,10 @@
 // for the tensor cores; activations are bf16 already,
 // so the MMAs are tcgen05.mma kind::f16 (bf16 x bf16 -> f32).  The expansion
 // adds base and residual codewords and applies the gain in bf16 pairs.
+// The GVQ1 container (same page, "Recipe": the 12-bit code stream plus a
+// 1-bit plane, 1-byte book entries) runs the same kernels, instantiated for
+// its index layout, on bf16 images of its books made at upload (entry =
+// bf16(f32(e4m3(byte) x book scale))).
 //
 // Steps of one forward:
 //   route/bucket, route tiles (as for MXFP4: tiles of up to 64 routes)
