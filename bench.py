@@ -310,6 +310,24 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def gather_roofline(cfg, d_mean, launch_ms, peaks):
+    """The shared-memory bound of a VQ decode gate/up launch: the codeword
+    bytes it gathers from the resident books (per 8 weights one base entry,
+    plus one residual entry with R8; 16-byte bf16 entries for VQ13, 8-byte
+    E4M3 entries for GVQ1) over the launch's duration, against the shared-
+    memory bandwidth of all SMs (148 x 128 bytes per clock at the maximum SM
+    clock)."""
+    entry = 8 if cfg.fmt.startswith("gvq1") else 16
+    per_vec = entry * (2 if cfg.fmt.endswith("r8") else 1)
+    nbytes = d_mean * 2 * cfg.I * (cfg.H // 8) * per_vec
+    achieved = nbytes / (launch_ms / 1e3) / 1e9
+    peak = 148 * 128 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e9
+    return {"bound": "shared-memory gathers", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "per_launch_bytes": nbytes,
+            "per_unit": f"{per_vec} gathered bytes per 8 weights of gate and up",
+            "peak_source": "derived: 148 SMs x 128 B per clock x sm_max_mhz"}
+
+
 def roofline(cfg, workload, ids_h, warmup, n_total, launch_ms, ms_step, peaks, peak_src, phase_how):
     """The dominant kernel's roofline and whole-step figures.
 
@@ -343,6 +361,8 @@ def roofline(cfg, workload, ids_h, warmup, n_total, launch_ms, ms_step, peaks, p
                 "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                 "peak_source": f"{peak_src} hbm_gbs", "per_launch_bytes": bytes_k,
                 "per_unit": per_unit, "units_per_launch": d_mean, "launch_ms": launch_ms, "timing": phase_how}
+        if cfg.fmt != "mxfp4":
+            roof["gather"] = gather_roofline(cfg, d_mean, launch_ms, peaks)
         if traffic_src:
             roof["traffic_source"] = traffic_src
         step_bytes = d_mean * sum(proj_bytes(cfg, p) for p in range(3)) + book_bytes(cfg)

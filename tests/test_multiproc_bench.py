@@ -57,3 +57,19 @@ def test_traffic_record_follows_the_profiled_source(tmp_path, monkeypatch):
     path, sha, traffic, summary = bench.NCU_TRAFFIC["decode_mxfp4"]
     monkeypatch.setitem(bench.NCU_TRAFFIC, "decode_mxfp4", (path, "0" * 64, traffic, summary))
     assert bench.ncu_traffic("decode_mxfp4") == (None, None)
+
+
+def test_gather_roofline_of_the_vq_decode_kernels():
+    # VQ13+R8 at one token: 8 experts x gate and up x 2048 rows x 512 vectors,
+    # two 16-byte entries per vector; GVQ1+R8 gathers 8-byte entries
+    import bench
+    import synth
+    cfg = synth.get_cfg("decode_vq", T=1)
+    g = bench.gather_roofline(cfg, 8.0, 0.05, {"sm_max_mhz": 1965.0})
+    assert g["per_launch_bytes"] == 8 * 2 * 2048 * 512 * 32
+    assert g["achieved"] == pytest.approx(g["per_launch_bytes"] / 50e-6 / 1e9)
+    assert g["peak"] == pytest.approx(148 * 128 * 1.965)
+    g1 = bench.gather_roofline(cfg.replace(fmt="gvq1r8"), 8.0, 0.05, {"sm_max_mhz": 1965.0})
+    assert g1["per_launch_bytes"] * 2 == g["per_launch_bytes"]
+    g0 = bench.gather_roofline(cfg.replace(fmt="vq13"), 8.0, 0.05, {"sm_max_mhz": 1965.0})
+    assert g0["per_launch_bytes"] * 2 == g["per_launch_bytes"]
