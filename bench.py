@@ -682,27 +682,39 @@ def main():
     r["ms"], r["e2e_s"] = reduce_times(r["ms"], r["e2e_s"], world, dev)
     line = summarize(args, args.workload, r, world, args.steps, args.warmup, peaks, peak_src) if rank == 0 else None
 
+    # The extra workloads follow the headline one; a failure in one of them is
+    # reported in its entry and does not cost the headline line.
     extra = {}
-    extra_names = () if (args.no_extra or args.workload != "decode_mxfp4") else EXTRA_WORKLOADS
-    for name in extra_names:
+
+    def run_extra(name, fn):
+        try:
+            res = fn()
+        except Exception as exc:   # noqa: BLE001 -- reported, not hidden
+            res = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        torch.cuda.empty_cache()
+        if rank == 0 and res is not None:
+            extra[name] = res
+
+    def layer_extra(name):
         rx = measure(name, args.extra_steps, args.warmup, world, rank, local, barrier, 6.0, with_cpu)
         rx["ms"], rx["e2e_s"] = reduce_times(rx["ms"], rx["e2e_s"], world, dev)
-        if rank == 0:
-            lx = summarize(args, name, rx, world, args.extra_steps, args.warmup, peaks, peak_src)
-            for key in ("metric", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "data"):
-                lx.pop(key, None)
-            extra[name] = lx
-        torch.cuda.empty_cache()
+        if rank != 0:
+            return None
+        lx = summarize(args, name, rx, world, args.extra_steps, args.warmup, peaks, peak_src)
+        for key in ("metric", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "data"):
+            lx.pop(key, None)
+        return lx
+
+    extra_names = () if (args.no_extra or args.workload != "decode_mxfp4") else EXTRA_WORKLOADS
+    for name in extra_names:
+        run_extra(name, lambda name=name: layer_extra(name))
 
     if extra_names:
         # the steps on either side of the layer: the router and the VQ encoder
         for T in (1, 2048):
-            rr = measure_router(T, args.extra_steps, args.warmup, local, peaks, peak_src)
-            if rank == 0:
-                extra[f"router_t{T}"] = rr
-        re_ = measure_encoder(3, 3, local, with_cpu)
-        if rank == 0:
-            extra["vq_encode_expert"] = re_
+            run_extra(f"router_t{T}", lambda T=T: measure_router(T, args.extra_steps, args.warmup, local, peaks,
+                                                                  peak_src))
+        run_extra("vq_encode_expert", lambda: measure_encoder(3, 3, local, with_cpu))
 
     if rank == 0:
         if extra:

@@ -73,3 +73,36 @@ def test_gather_roofline_of_the_vq_decode_kernels():
     assert g1["per_launch_bytes"] * 2 == g["per_launch_bytes"]
     g0 = bench.gather_roofline(cfg.replace(fmt="vq13"), 8.0, 0.05, {"sm_max_mhz": 1965.0})
     assert g0["per_launch_bytes"] * 2 == g["per_launch_bytes"]
+
+
+def test_a_failing_extra_workload_keeps_the_headline_line(monkeypatch, capsys):
+    # main() with the GPU-facing steps stubbed: one extra workload raises,
+    # the JSON line still prints, with the error in that workload's entry
+    import json
+    import sys
+
+    import torch
+
+    import bench
+    monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "empty_cache", lambda *a, **k: None)
+    monkeypatch.setattr(bench, "load_peaks", lambda: ({"hbm_gbs": 1.0, "bf16_tflops": 1.0}, "test"))
+    monkeypatch.setattr(bench, "reduce_times", lambda ms, e2e, world, dev: (ms, e2e))
+
+    def fake_measure(name, *a, **k):
+        if name == "prefill_vq_overflow":
+            raise RuntimeError("injected failure")
+        return {"ms": 1.0, "e2e_s": 1.0, "name": name}
+
+    monkeypatch.setattr(bench, "measure", fake_measure)
+    monkeypatch.setattr(bench, "summarize", lambda args, name, r, *a, **k: {"workload": name, "value": 1.0})
+    monkeypatch.setattr(bench, "measure_router", lambda T, *a, **k: {"workload": f"router_t{T}"})
+    monkeypatch.setattr(bench, "measure_encoder", lambda *a, **k: {"workload": "vq_encode_expert"})
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--no-cpu-baseline"])
+    assert bench.main() == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["workload"] == "decode_mxfp4"
+    w = line["workloads"]
+    assert "injected failure" in w["prefill_vq_overflow"]["error"]
+    assert w["prefill_mxfp4_zipf"]["workload"] == "prefill_mxfp4_zipf"
+    assert set(w) == set(bench.EXTRA_WORKLOADS) | {"router_t1", "router_t2048", "vq_encode_expert"}
