@@ -27,7 +27,8 @@ def test_header_declares_the_entry_points():
     syms = declared_symbols()
     for s in ("moeq_layer_create", "moeq_upload_weights", "moeq_forward", "moeq_dequant",
               "moeq_layer_destroy", "moeq_layer_status", "moeq_status_string", "moeq_route",
-              "moeq_forward_host", "moeq_forward_profiled"):
+              "moeq_forward_host", "moeq_forward_profiled", "moeq_route_noalloc", "moeq_router_upload",
+              "moeq_router", "moeq_forward_routed", "moeq_vq_encode", "moeq_kernel_launches"):
         assert s in syms
 
 
