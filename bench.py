@@ -44,7 +44,7 @@ NCU_TRAFFIC = {
                       "bit_quantized_moe_routed_b200/csrc/decode_common.cuh",
                       "bit_quantized_moe_routed_b200/csrc/internal.cuh",
                       "include/moeq.h"),
-                     "d97f70d647b24ddd486a1f973719227a7809593cffca4084aaaf6222246a0cc3",
+                     "0de1473aac3815e81c3c061c3fa8cc49daf52807194bb004d3434733454c8d81",
                      107049216.0 + 358144.0, "profiles/dec_fused_mx_decode_mxfp4.md"),
 }
 

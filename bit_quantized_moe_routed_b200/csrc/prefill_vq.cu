@@ -10,8 +10,9 @@
 // for the tensor cores; activations are bf16 already,
 // so the MMAs are tcgen05.mma kind::f16 (bf16 x bf16 -> f32).  The expansion
 // adds base and residual codewords and applies the gain in bf16 pairs.
-// The GVQ1 container (same page, "Recipe": the 12-bit code stream plus a
-// 1-bit plane, 1-byte book entries) runs the same kernels, instantiated for
+// The GVQ1 container (same page, "Recipe": a 12-bit code stream with a
+// separate plane of one-bit flags, books of 1-byte entries) runs the same
+// kernels, instantiated for
 // its index layout, on bf16 images of its books made at upload (entry =
 // bf16(f32(e4m3(byte) x book scale))).
 //

@@ -114,10 +114,10 @@ typedef struct moeq_layer *moeq_layer_t;
  *   gain[p]    uint16 f16 [E][N] or NULL (gain 1)
  *   weight[n][8j+i] = (book13[idx13][i] + book8[idx8][i]) * gain[n], each
  *   operation IEEE f32 round-to-nearest-even, in that order.
- * GVQ1 / GVQ1_R8 (same page, "Recipe": "the 12-bit code stream plus a 1-bit
- * plane"; "Why 13 bits plus an 8-bit residual": 1-byte book entries, 64 KiB
- * + 2 KiB of books.  The byte layout and the entry type are not on the
- * page; this library reads them as follows):
+ * GVQ1 / GVQ1_R8 (same page, "Recipe": the indices as a 12-bit code stream
+ * with a separate plane of one-bit flags; "Why 13 bits plus an 8-bit
+ * residual": books of 1-byte entries, 64 KiB + 2 KiB.  The byte layout and
+ * the entry type are not on the page; this library reads them as follows):
  *   code12[p]  uint8 [E][N][K*3/16]  per row, the low 12 bits of the K/8
  *                                 indices as one little-endian bitstream
  *                                 (index j: bits 12j..12j+11)
