@@ -44,7 +44,7 @@ NCU_TRAFFIC = {
                       "bit_quantized_moe_routed_b200/csrc/decode_common.cuh",
                       "bit_quantized_moe_routed_b200/csrc/internal.cuh",
                       "include/moeq.h"),
-                     "0de1473aac3815e81c3c061c3fa8cc49daf52807194bb004d3434733454c8d81",
+                     "0cca0e038c0ed780604c13d445697ac9d59ca7bc78d4644098ff1218d86fd098",
                      107049216.0 + 358144.0, "profiles/dec_fused_mx_decode_mxfp4.md"),
 }
 

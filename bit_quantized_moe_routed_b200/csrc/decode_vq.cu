@@ -1,10 +1,10 @@
 // decode_vq.cu -- VQ13 / VQ13+R8 routed-expert FFN at decode sizes (1..8
 // tokens, bf16 activations): a grouped GEMV, one warp per output row.
 //
-// Format ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): every 8
-// consecutive weights of an expert row are one 13-bit index into the
-// layer's 8192 x 8 codebook, plus (VQ13+R8) one 8-bit index into a 256 x 8
-// residual book, times one f16 row gain:
+// Format ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): an expert row is
+// cut into 8-weight vectors, each stored as a 13-bit index into the layer's
+// 8192 x 8 codebook (VQ13+R8: and an 8-bit index into a 256 x 8 residual
+// book); the row is scaled by an f16 gain:
 //     w[n][8j+i] = (B13[c_nj][i] + R8[r_nj][i]) * gain[n].
 // "Why 13 bits plus an 8-bit residual": the kernels keep the layer's whole
 // codebook in shared memory while they decode every selected expert -- here

@@ -1,10 +1,10 @@
 // prefill_vq.cu -- VQ13(+R8) and GVQ1(+R8) routed-expert FFN on the
 // 5th-generation tensor cores (bf16 activations, any token count).
 //
-// Format ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): every 8
-// consecutive weights of an expert row are one 13-bit index into the layer's
-// 8192 x 8 codebook (optionally plus an 8-bit index into a 256 x 8 residual
-// book), times an f16 row gain; one codebook pair serves every expert and
+// Format ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): an expert row is
+// cut into 8-weight vectors, each stored as a 13-bit index into the layer's
+// 8192 x 8 codebook (optionally with an 8-bit index into a 256 x 8 residual
+// book), the row scaled by an f16 gain; one codebook pair serves every expert and
 // gate/up/down ("Why 13 bits": the books stay in shared memory while every
 // selected expert is decoded).  Weight = (base + residual) * gain, in bf16
 // for the tensor cores; activations are bf16 already,

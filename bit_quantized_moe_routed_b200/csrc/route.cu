@@ -3,8 +3,8 @@
 //
 // The layer sends each token to k experts ("MiMo-V2.6-Flash-RL GGUF for a
 // single DGX Spark", "Architecture notes": 8 of 256 routed experts), and the
-// expert matmuls want all of an expert's tokens together ("Speed": at a
-// micro-batch of 512 each of the 256 experts sees too few tokens per matmul).
+// expert matmuls want all of an expert's tokens together ("Speed": with a
+// 512-token micro-batch the per-expert matmuls are too small to be efficient).
 // This kernel produces, for one forward:
 //   offsets[E+1]  exclusive scan of the per-expert route counts
 //   perm[n_valid] route ids r = t*k + s, ordered by (expert, r) -- stable, so

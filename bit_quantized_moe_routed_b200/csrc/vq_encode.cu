@@ -2,12 +2,11 @@
 // 8-weight vectors to the 13-bit base book, then of the remainder to the
 // 8-bit residual book, packed as the format stores them.
 //
-// Source ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): every 8
-// consecutive weights of an expert row become one index into the layer's
-// codebook, times one f16 row gain; a 256-entry residual book codes what the
-// first stage left, and the 13-bit stage is byte-identical with and without
-// it; vector assignment minimises an importance-weighted error with
-// per-column weights.  The codebooks, gains and column weights are inputs
+// Source ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): each 8-weight
+// vector of an expert row is replaced by the index of a codebook entry, the
+// row scaled by an f16 gain; a second, 256-entry book encodes the remainder
+// the first stage leaves, without changing the first stage's indices; the
+// assignment minimises an error weighted per column by importance.  The codebooks, gains and column weights are inputs
 // (their training is not part of this path).
 //
 // Error of a candidate for vector v (columns 8j..8j+7) of a row with gain g

@@ -304,12 +304,11 @@ MOEQ_API moeq_status moeq_forward_routed(moeq_layer_t layer, const void *x, int3
                                          float *topk_w, void *out, void *stream);
 
 /* VQ encoder: the indices that store a matrix in the VQ13 / VQ13_R8 format
- * ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe": every 8 consecutive
- * weights of an expert row become one index into the layer's codebook,
- * times one f16 row gain; a 256-entry residual book codes what the first
- * stage left, and the 13-bit stage is byte-identical with and without it;
- * assignment minimises an importance-weighted error with per-column
- * weights).  The codebooks, gains and column weights are given; training
+ * ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe": each 8-weight vector
+ * of an expert row is replaced by the index of a codebook entry, the row
+ * scaled by an f16 gain; a second, 256-entry book encodes the remainder the
+ * first stage leaves, without changing the first stage's indices; the
+ * assignment minimises an error weighted per column by importance).  The codebooks, gains and column weights are given; training
  * them is not part of this library.
  *   w           device f32 [n_rows][n_cols], row-major, 16-byte aligned;
  *               n_cols a multiple of 64

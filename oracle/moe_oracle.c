@@ -18,12 +18,13 @@
  *         E8M0 exponent per 32 values.  "Recipe": a 32-value intermediate
  *         sum passes f16's 65504 in layer 47, so intermediates stay in a
  *         wider type (here: double).
- *  [VQ]   "MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe": every 8
- *         consecutive weights of an expert row are one index into the
- *         layer's codebook, times one F16 row gain; one codebook per layer
- *         serves every expert and gate/up/down; a second 256-entry codebook
- *         codes the residual of the first stage with 8 more bits per 8
- *         weights, and the 13-bit stage is the same with or without it.
+ *  [VQ]   "MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe": an expert row
+ *         is cut into 8-weight vectors, each stored as an index into the
+ *         layer's codebook, the row scaled by an f16 gain; the layer has a
+ *         single codebook for all experts and all three projections; an
+ *         optional 256-entry second book spends 8 more bits per vector on
+ *         the first stage's remainder and leaves the first-stage indices
+ *         unchanged.
  *  [IQ3]  "MiMo-V2.6-Flash-RL: calibrated IQ3_XXS", "Calibration": the sum
  *         of the per-projection route counts is eight routes per token.
  *
@@ -172,8 +173,8 @@ double orc_e4m3(uint32_t b)
     return s ? -v : v;
 }
 
-/* Index j of a GVQ1 row [VQ "Recipe": "the 12-bit code stream plus a 1-bit
- * plane"]: the low 12 bits are bits 12j..12j+11 of the row's little-endian
+/* Index j of a GVQ1 row [VQ "Recipe": the indices as a 12-bit code stream
+ * with a separate plane of one-bit flags]: the low 12 bits are bits 12j..12j+11 of the row's little-endian
  * 12-bit stream, bit 12 is bit j of the row's bit plane (bit q of a stream
  * is bit q%8 of byte q/8, as for the 13-bit stream). */
 uint32_t orc_gvq1_idx(const uint8_t *code12_row, const uint8_t *hi_row, int64_t j)

@@ -4,12 +4,12 @@
 TEST INFRASTRUCTURE ONLY: a plain float64 brute force for the tests and the
 benchmark's CPU baseline; the CUDA library never calls it.
 
-Source ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): every 8
-consecutive weights of an expert row become one index into the layer's
-codebook, times one f16 row gain; the residual stage codes what the first
-stage left with a 256-entry book, and the 13-bit stage is byte-identical
-with and without it; codebook training, vector assignment and the row-gain
-refit minimise an importance-weighted error with per-column weights.  Only
+Source ("MiMo-V2.6-Flash-RL UNCENSORED VQ GGUF", "Recipe"): each 8-weight
+vector of an expert row is replaced by the index of a codebook entry, the
+row scaled by an f16 gain; a second, 256-entry book encodes the remainder
+the first stage leaves, without changing the first stage's indices; the
+page's whole procedure (books, assignment, gains) minimises an error
+weighted per column by importance.  Only
 the assignment is restated here (the codebooks and gains are inputs; their
 training needs calibration data and is not part of this path).  Readings:
   - the error of a candidate is sum_i omega_i (w_i - v_i)^2 over the vector's
