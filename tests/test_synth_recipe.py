@@ -117,3 +117,40 @@ def test_draws_depend_on_seed_and_component_only():
     # the activations do not move when the routing config changes
     np.testing.assert_array_equal(synth.gen_activations(cfg, seed=5),
                                   synth.gen_activations(cfg.replace(routing="zipf"), seed=5))
+
+
+def test_gvq1_books_streams_and_scales():
+    # GVQ1 layers: N(0,1) books rounded to E4M3 (no NaN byte), the book
+    # scales carry sigma (and the overflow multiplier), 12-bit streams and
+    # bit planes of the right sizes; without the residual stage no residual
+    # book, indices or scale
+    import torch
+    from synth.gen import gvq1_code_row_bytes
+
+    def e4m3_values(b):
+        return torch.from_numpy(b).view(torch.float8_e4m3fn).to(torch.float32).numpy().astype(np.float64)
+
+    cfg = synth.get_cfg("decode_vq", H=256, I=128, E=4, fmt="gvq1r8")
+    L = synth.gen_layer(cfg)
+    assert L.gbook13.shape == (BOOK13_ROWS, 8) and L.gbook13.dtype == np.uint8
+    assert L.gbook8.shape == (BOOK8_ROWS, 8)
+    for book in (L.gbook13, L.gbook8):
+        assert not np.isin(book, (0x7F, 0xFF)).any()
+    v13 = e4m3_values(L.gbook13)
+    assert abs(v13.std() - 1) < 0.03 and abs(v13.mean()) < 0.03
+    assert L.gscale == (float(np.float32(0.02)), float(np.float32(0.005)))
+    for p in range(3):
+        N, K = cfg.shape(p)
+        assert gvq1_code_row_bytes(K) == K * 3 // 16
+        assert L.code12[p].shape == (cfg.E, N, K * 3 // 16)
+        assert L.hi1[p].shape == (cfg.E, N, K // 64)
+        assert L.idx8[p].shape == (cfg.E, N, K // 8)
+    # the overflow workload's multiplier goes into the base book's scale
+    ov = synth.get_cfg("prefill_vq_overflow", H=256, I=128, E=4, fmt="gvq1r8")
+    Lo = synth.gen_layer(ov)
+    np.testing.assert_array_equal(Lo.gbook13, L.gbook13)
+    assert Lo.gscale[0] == float(np.float32(0.02 * 64))
+    # no residual stage
+    L0 = synth.gen_layer(cfg.replace(fmt="gvq1"))
+    assert L0.gbook8 is None and all(a is None for a in L0.idx8) and L0.gscale[1] == 0.0
+    np.testing.assert_array_equal(L0.gbook13, L.gbook13)
